@@ -1,0 +1,184 @@
+"""Seeded synthetic inputs for HSTU causal pointwise aggregated attention.
+
+This module only draws random numbers and rounds them to the run's dtype.  It
+holds none of the attention arithmetic, so both the fp64 oracle (``oracle/``)
+and the CUDA path (``pointwise_attention_b200``) may use it without sharing
+any of the method's code.
+
+Shapes follow the HSTU model card ("HSTU (Generative Recommender)", Structure
+table and Exported PyTorch: embed 512, 4 heads, d_qk = d_v = 128, 1024 tokens)
+and the five named workloads below.  Every draw comes from one CPU
+``torch.Generator`` seeded per workload, in a fixed order:
+
+    lengths -> Q -> K -> V -> U -> timestamps -> rab_pos -> rab_time -> dY
+
+Floating values are drawn in fp32 with ``randn`` and rounded (round to nearest
+even) to bf16 for the bf16 workloads; the same rounded host tensors feed the
+oracle (widened exactly to fp64) and the GPU.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional, Sequence
+
+import torch
+
+__all__ = ["Spec", "Inputs", "WORKLOADS", "make_inputs", "workload", "causal_flops"]
+
+NUM_TIME_BUCKETS = 128
+TIME_T0 = 1_700_000_000      # first timestamp of every sequence (seconds)
+TIME_GAP_MEAN = 300.0        # mean of the exponential gaps between events (seconds)
+
+
+@dataclasses.dataclass(frozen=True)
+class Spec:
+    """Shape and distribution of one synthetic workload."""
+    name: str
+    dtype: str                      # "f32" or "bf16"
+    batch: int
+    heads: int
+    d_qk: int
+    d_v: int
+    seq_len: int = 0                # dense: every sequence has this length
+    len_range: Optional[tuple] = None   # jagged: inclusive (lo, hi) uniform integer lengths
+    lengths: Optional[tuple] = None     # explicit lengths (tests)
+    qk_std: float = 1.0
+    vu_std: float = 1.0
+    rab_pos_len: int = 0            # L of the position table [H, 2L-1]; 0 = no position bias
+    rab_time: bool = False          # per-head [H, 128] time-bucket table + int64 timestamps
+    rab_std: float = 0.02
+    norm: str = "fixed"             # "fixed": divide by norm_len; "own": each sequence's length
+    norm_len: int = 0               # for "fixed"; 0 means the (dense) sequence length
+    grad: bool = False              # also draw the upstream gradient dY
+    ts_sorted: bool = True          # timestamps increasing within a sequence
+
+
+def _spec_table() -> Dict[str, Spec]:
+    s = 1.0 / math.sqrt(128.0)
+    return {
+        # Tiny fp32 forward: 2 x 64 tokens, 2 heads, d = 32, no relative bias.
+        "tiny": Spec("tiny", "f32", batch=2, heads=2, d_qk=32, d_v=32, seq_len=64),
+        # Shape of the model card's block: 8 x 1024 tokens, 4 heads, d = 128.
+        "neurarch": Spec("neurarch", "bf16", batch=8, heads=4, d_qk=128, d_v=128,
+                         seq_len=1024, qk_std=s, rab_pos_len=1024),
+        # 64 jagged sequences of 256..4096 tokens with position and time bias.
+        "jagged": Spec("jagged", "bf16", batch=64, heads=8, d_qk=128, d_v=128,
+                       len_range=(256, 4096), qk_std=s, rab_pos_len=4096,
+                       rab_time=True, norm="own"),
+        # 4 x 8192 tokens with position and time bias; the position table must
+        # reach i - j = 8191, so it holds 2 * 8192 - 1 entries.
+        "long": Spec("long", "bf16", batch=4, heads=4, d_qk=128, d_v=128, seq_len=8192,
+                     qk_std=s, rab_pos_len=8192, rab_time=True),
+        # Training step: 16 x 2048 tokens, position bias, upstream gradient dY.
+        "train": Spec("train", "bf16", batch=16, heads=4, d_qk=128, d_v=128, seq_len=2048,
+                      qk_std=s, rab_pos_len=2048, grad=True),
+    }
+
+
+WORKLOADS: Dict[str, Spec] = _spec_table()
+
+
+def workload(name: str, **overrides) -> Spec:
+    """Named workload, optionally with fields replaced (smaller batch, other lengths...)."""
+    return dataclasses.replace(WORKLOADS[name], **overrides)
+
+
+@dataclasses.dataclass
+class Inputs:
+    """Host (CPU) tensors of one problem, already rounded to the run dtype."""
+    spec: Spec
+    offsets: torch.Tensor           # int32 [B+1]
+    q: torch.Tensor                 # [T, H, d_qk]
+    k: torch.Tensor                 # [T, H, d_qk]
+    v: torch.Tensor                 # [T, H, d_v]
+    u: torch.Tensor                 # [T, H*d_v]
+    timestamps: Optional[torch.Tensor]  # int64 [T]
+    rab_pos: Optional[torch.Tensor]     # fp32 [H, 2L-1]
+    rab_time: Optional[torch.Tensor]    # fp32 [H, 128]
+    dy: Optional[torch.Tensor]          # [T, H*d_v]
+    norm_len: int                   # >0: divide by it; 0: by each sequence's length
+    rab_pos_len: int                # L (0 if no position table)
+
+    @property
+    def lengths(self) -> List[int]:
+        o = self.offsets.tolist()
+        return [o[i + 1] - o[i] for i in range(len(o) - 1)]
+
+    @property
+    def total_tokens(self) -> int:
+        return int(self.offsets[-1])
+
+    @property
+    def max_seq_len(self) -> int:
+        ls = self.lengths
+        return max(ls) if ls else 0
+
+
+def _torch_dtype(name: str) -> torch.dtype:
+    return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
+
+
+def causal_flops(lengths: Sequence[int], heads: int, d_qk: int, d_v: int) -> int:
+    """Algorithmic forward FLOPs: 2 * sum n(n+1)/2 * H * (d_qk + d_v)."""
+    pairs = sum(n * (n + 1) // 2 for n in lengths)
+    return 2 * pairs * heads * (d_qk + d_v)
+
+
+def make_inputs(spec: Spec, seed: int = 0) -> Inputs:
+    """Draw one problem for ``spec`` from a CPU generator seeded with ``seed``."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    # lengths
+    if spec.lengths is not None:
+        lengths = [int(x) for x in spec.lengths]
+    elif spec.len_range is not None:
+        lo, hi = spec.len_range
+        lengths = torch.randint(lo, hi + 1, (spec.batch,), generator=g).tolist()
+    else:
+        lengths = [spec.seq_len] * spec.batch
+    offs = [0]
+    for n in lengths:
+        offs.append(offs[-1] + n)
+    offsets = torch.tensor(offs, dtype=torch.int32)
+    T, H = offs[-1], spec.heads
+    dt = _torch_dtype(spec.dtype)
+
+    def draw(shape, std):
+        return (torch.randn(shape, generator=g, dtype=torch.float32) * std).to(dt)
+
+    q = draw((T, H, spec.d_qk), spec.qk_std)
+    k = draw((T, H, spec.d_qk), spec.qk_std)
+    v = draw((T, H, spec.d_v), spec.vu_std)
+    u = draw((T, H * spec.d_v), spec.vu_std)
+
+    ts = None
+    if spec.rab_time:
+        parts = []
+        for n in lengths:
+            gaps = torch.empty(max(n - 1, 0), dtype=torch.float64).exponential_(
+                1.0 / TIME_GAP_MEAN, generator=g)
+            gaps = torch.clamp(torch.round(gaps), min=1.0).to(torch.int64)
+            seq = torch.empty(n, dtype=torch.int64)
+            if n:
+                seq[0] = TIME_T0
+                seq[1:] = TIME_T0 + torch.cumsum(gaps, 0)
+            if not spec.ts_sorted and n:
+                seq = seq[torch.randperm(n, generator=g)]
+            parts.append(seq)
+        ts = torch.cat(parts) if parts else torch.empty(0, dtype=torch.int64)
+
+    L = spec.rab_pos_len
+    rab_pos = None
+    if L > 0:
+        rab_pos = torch.randn((H, 2 * L - 1), generator=g, dtype=torch.float32) * spec.rab_std
+    rab_time = None
+    if spec.rab_time:
+        rab_time = torch.randn((H, NUM_TIME_BUCKETS), generator=g,
+                               dtype=torch.float32) * spec.rab_std
+    dy = draw((T, H * spec.d_v), 1.0) if spec.grad else None
+
+    if spec.norm == "own":
+        norm_len = 0
+    else:
+        norm_len = spec.norm_len if spec.norm_len > 0 else (spec.seq_len or max(lengths or [1]))
+    return Inputs(spec, offsets, q, k, v, u, ts, rab_pos, rab_time, dy, norm_len, L)

@@ -1,0 +1,180 @@
+"""fp64 CPU oracle for HSTU causal pointwise aggregated attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It wraps the plain C
+oracle ``hstu_ref.c`` (fp64, fixed summation order, OpenMP over rows) through
+ctypes and shares no code with the CUDA library.
+
+Inputs are the rounded host tensors from ``hstu_inputs``; they are widened
+exactly to fp64 before the call, so input rounding is not counted as error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hstu_ref.c")
+_LIB = os.path.join(_HERE, "libhstu_ref.so")
+_lib = None
+
+LN_EPS = 1e-5
+NUM_TIME_BUCKETS = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile hstu_ref.c into libhstu_ref.so beside it (gcc, OpenMP)."""
+    hdr = os.path.join(_HERE, "hstu_ref.h")
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(hdr))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fPIC",
+                               "-shared", "-Wall", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32),
+        ("d_qk", ctypes.c_int32),
+        ("d_v", ctypes.c_int32),
+        ("offsets", ctypes.c_void_p),
+        ("timestamps", ctypes.c_void_p),
+        ("rab_pos", ctypes.c_void_p),
+        ("rab_pos_len", ctypes.c_int32),
+        ("rab_time", ctypes.c_void_p),
+        ("num_time_buckets", ctypes.c_int32),
+        ("norm_len", ctypes.c_int32),
+        ("ln_eps", ctypes.c_double),
+    ]
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.POINTER(_Problem)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        lib.hstu_ref_time_bucket.argtypes = [ctypes.c_int64, ctypes.c_int32]
+        lib.hstu_ref_time_bucket.restype = ctypes.c_int32
+        lib.hstu_ref_fwd.argtypes = [P] + [vp] * 8 + [i32]
+        lib.hstu_ref_fwd.restype = ctypes.c_int
+        lib.hstu_ref_fwd_rows.argtypes = [P] + [vp] * 5 + [i64] + [vp] * 4 + [i32]
+        lib.hstu_ref_fwd_rows.restype = ctypes.c_int
+        lib.hstu_ref_bwd.argtypes = [P] + [vp] * 11 + [i32]
+        lib.hstu_ref_bwd.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> Optional[np.ndarray]:
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class _Args:
+    """Keeps the fp64 copies alive while the C call runs."""
+
+    def __init__(self, offsets, q, k, v, u, timestamps=None, rab_pos=None, rab_time=None,
+                 norm_len=0, rab_pos_len=0, ln_eps=LN_EPS):
+        self.offsets = np.ascontiguousarray(np.asarray(offsets), dtype=np.int32)
+        self.q, self.k, self.v, self.u = _f64(q), _f64(k), _f64(v), _f64(u)
+        T = int(self.offsets[-1])
+        self.H = self.q.shape[1] if self.q.ndim == 3 else 1
+        self.dqk = self.q.shape[-1]
+        self.dv = self.v.shape[-1]
+        self.T = T
+        self.D = self.H * self.dv
+        self.ts = None if timestamps is None else np.ascontiguousarray(
+            np.asarray(timestamps), dtype=np.int64)
+        self.rab_pos = _f64(rab_pos)
+        self.rab_time = _f64(rab_time)
+        if self.rab_pos is not None and rab_pos_len <= 0:
+            rab_pos_len = (self.rab_pos.shape[-1] + 1) // 2
+        self.prob = _Problem(
+            batch=len(self.offsets) - 1, num_heads=self.H, d_qk=self.dqk, d_v=self.dv,
+            offsets=_ptr(self.offsets), timestamps=_ptr(self.ts), rab_pos=_ptr(self.rab_pos),
+            rab_pos_len=int(rab_pos_len), rab_time=_ptr(self.rab_time),
+            num_time_buckets=(self.rab_time.shape[-1] if self.rab_time is not None
+                              else NUM_TIME_BUCKETS),
+            norm_len=int(norm_len), ln_eps=float(ln_eps))
+
+
+def _args_from_inputs(inp, **kw):
+    return _Args(inp.offsets.numpy(), inp.q, inp.k, inp.v, inp.u,
+                 None if inp.timestamps is None else inp.timestamps.numpy(),
+                 inp.rab_pos, inp.rab_time, inp.norm_len, inp.rab_pos_len, **kw)
+
+
+def time_bucket(dt: int, num_buckets: int = NUM_TIME_BUCKETS) -> int:
+    return int(_load().hstu_ref_time_bucket(int(dt), int(num_buckets)))
+
+
+def fwd_raw(a: _Args, threads: int = 0):
+    """Full forward: returns dict y, o [T,D], mean, rstd [T] (fp64)."""
+    lib = _load()
+    y = np.zeros((a.T, a.D)); o = np.zeros((a.T, a.D))
+    mean = np.zeros(a.T); rstd = np.zeros(a.T)
+    rc = lib.hstu_ref_fwd(ctypes.byref(a.prob), _ptr(a.q), _ptr(a.k), _ptr(a.v), _ptr(a.u),
+                          _ptr(y), _ptr(o), _ptr(mean), _ptr(rstd), int(threads))
+    if rc != 0:
+        raise ValueError("hstu_ref_fwd rejected the problem (code %d)" % rc)
+    return dict(y=y, o=o, mean=mean, rstd=rstd)
+
+
+def fwd_rows_raw(a: _Args, rows: Sequence[int], threads: int = 0):
+    """Forward on selected global token rows; outputs are compact [len(rows), ...]."""
+    lib = _load()
+    r = np.ascontiguousarray(np.asarray(rows), dtype=np.int64)
+    n = len(r)
+    y = np.zeros((n, a.D)); o = np.zeros((n, a.D)); mean = np.zeros(n); rstd = np.zeros(n)
+    rc = lib.hstu_ref_fwd_rows(ctypes.byref(a.prob), _ptr(a.q), _ptr(a.k), _ptr(a.v),
+                               _ptr(a.u), _ptr(r), n, _ptr(y), _ptr(o), _ptr(mean),
+                               _ptr(rstd), int(threads))
+    if rc != 0:
+        raise ValueError("hstu_ref_fwd_rows rejected the problem (code %d)" % rc)
+    return dict(y=y, o=o, mean=mean, rstd=rstd)
+
+
+def bwd_raw(a: _Args, dy, threads: int = 0):
+    """Backward: returns dict dq, dk [T,H,dqk], dv [T,H,dv], du [T,D], d_rab_pos, d_rab_time."""
+    lib = _load()
+    dyd = _f64(dy)
+    dq = np.zeros((a.T, a.H, a.dqk)); dk = np.zeros((a.T, a.H, a.dqk))
+    dv = np.zeros((a.T, a.H, a.dv)); du = np.zeros((a.T, a.D))
+    drp = None if a.rab_pos is None else np.zeros_like(a.rab_pos)
+    drt = None if a.rab_time is None else np.zeros_like(a.rab_time)
+    rc = lib.hstu_ref_bwd(ctypes.byref(a.prob), _ptr(a.q), _ptr(a.k), _ptr(a.v), _ptr(a.u),
+                          _ptr(dyd), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(du), _ptr(drp),
+                          _ptr(drt), int(threads))
+    if rc != 0:
+        raise ValueError("hstu_ref_bwd rejected the problem (code %d)" % rc)
+    return dict(dq=dq, dk=dk, dv=dv, du=du, d_rab_pos=drp, d_rab_time=drt)
+
+
+def fwd(inp, threads: int = 0):
+    """Forward of an ``hstu_inputs.Inputs`` problem."""
+    return fwd_raw(_args_from_inputs(inp), threads)
+
+
+def fwd_rows(inp, rows, threads: int = 0):
+    return fwd_rows_raw(_args_from_inputs(inp), rows, threads)
+
+
+def bwd(inp, threads: int = 0):
+    """Backward of an ``hstu_inputs.Inputs`` problem (uses ``inp.dy``)."""
+    return bwd_raw(_args_from_inputs(inp), inp.dy, threads)

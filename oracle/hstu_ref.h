@@ -1,0 +1,61 @@
+/*
+ * hstu_ref.h -- fp64 CPU oracle for HSTU causal pointwise aggregated attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path includes, links or
+ * calls this; only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg do.  It shares no code with the CUDA library.
+ *
+ * All floating inputs are fp64 host arrays holding the (already rounded) values
+ * of the run; every computation is plain fp64 loops in a fixed order.
+ */
+#ifndef HSTU_REF_H
+#define HSTU_REF_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+    int32_t batch;              /* B                                               */
+    int32_t num_heads;          /* H                                               */
+    int32_t d_qk, d_v;          /* per-head widths                                 */
+    const int32_t *offsets;     /* [B+1], offsets[0] = 0, non-decreasing, = T      */
+    const int64_t *timestamps;  /* [T] or NULL (no time bias)                      */
+    const double *rab_pos;      /* [H, 2L-1] or NULL                               */
+    int32_t rab_pos_len;        /* L                                               */
+    const double *rab_time;     /* [H, num_time_buckets] or NULL                   */
+    int32_t num_time_buckets;   /* 128 in the workloads                            */
+    int32_t norm_len;           /* >0: divide by it; 0: divide by each n_b         */
+    double ln_eps;              /* LayerNorm epsilon (1e-5)                        */
+} hstu_ref_problem;
+
+/* Time bucket of a timestamp difference: min(NB-1, floor(ln(max(1,|dt|))/0.301)). */
+int32_t hstu_ref_time_bucket(int64_t dt, int32_t num_time_buckets);
+
+/* Forward on every token.  q,k: [T,H,dqk]; v: [T,H,dv]; u: [T,H*dv].
+ * Writes y [T,H*dv]; o [T,H*dv], mean [T], rstd [T] when non-NULL.
+ * Returns 0 on success, a negative code on invalid arguments. */
+int hstu_ref_fwd(const hstu_ref_problem *p, const double *q, const double *k,
+                 const double *v, const double *u, double *y, double *o,
+                 double *mean, double *rstd, int num_threads);
+
+/* Forward on the listed global token rows only (rows[r] in [0,T)).  Outputs
+ * are compact: y [nrows, H*dv], o [nrows, H*dv], mean/rstd [nrows]. */
+int hstu_ref_fwd_rows(const hstu_ref_problem *p, const double *q, const double *k,
+                      const double *v, const double *u, const int64_t *rows,
+                      int64_t nrows, double *y, double *o, double *mean,
+                      double *rstd, int num_threads);
+
+/* Backward from dy [T,H*dv].  Writes dq, dk [T,H,dqk], dv [T,H,dv],
+ * du [T,H*dv]; d_rab_pos [H,2L-1] and d_rab_time [H,NB] are overwritten
+ * (not accumulated) when non-NULL.  The forward is recomputed internally. */
+int hstu_ref_bwd(const hstu_ref_problem *p, const double *q, const double *k,
+                 const double *v, const double *u, const double *dy,
+                 double *dq, double *dk, double *dv, double *du,
+                 double *d_rab_pos, double *d_rab_time, int num_threads);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

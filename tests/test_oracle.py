@@ -1,0 +1,285 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these tests needs a GPU.  Each pin is chosen so that a plausible slip in
+the oracle (a dropped bias term, a wrong sign or index, a transposed operand, a
+wrong normaliser, an off-by-one mask) fails at least one of them:
+
+* dense torch restatement of the model card's HSTUBlock.forward (matrix form,
+  library matmul / tril / layer_norm) -- forward to 1e-12;
+* torch.autograd of that restatement -- every gradient to 1e-10;
+* central finite differences of the oracle's own forward -- every gradient;
+* the closed form of the first position, O_0 = SiLU(q_0.k_0 + b_00)/N * v_0;
+* invariants: causality, linearity of O in V, zero output for K = 0 without
+  bias, the A read-out with V = I, packing (jagged = each sequence alone),
+  head permutation, LayerNorm row statistics;
+* time buckets against exp thresholds and the special cases 0, +-1, the cap.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import hstu_inputs as hi
+from tests.dense_torch import dense_forward
+
+
+def small_inputs(lengths=(5, 9, 1, 12), H=3, dqk=6, dv=4, rab_pos=True, rab_time=True,
+                 norm="own", norm_len=0, seed=0, qk_std=0.7, rab_std=0.5, grad=True,
+                 ts_sorted=True, L=None):
+    spec = hi.Spec("t", "f32", batch=len(lengths), heads=H, d_qk=dqk, d_v=dv,
+                   lengths=tuple(lengths), qk_std=qk_std, vu_std=1.0,
+                   rab_pos_len=(L or max(lengths)) if rab_pos else 0, rab_time=rab_time,
+                   rab_std=rab_std, norm=norm, norm_len=norm_len, grad=grad,
+                   ts_sorted=ts_sorted)
+    inp = hi.make_inputs(spec, seed=seed)
+    if rab_time:
+        # Spread the timestamps so that many buckets are reached in small cases.
+        g = torch.Generator().manual_seed(seed + 100)
+        gaps = torch.randint(0, 4000, (inp.total_tokens,), generator=g).to(torch.int64)
+        ts = []
+        for b, n in enumerate(inp.lengths):
+            s = int(inp.offsets[b])
+            seq = 1_700_000_000 + torch.cumsum(gaps[s:s + n], 0)
+            if not ts_sorted and n:
+                seq = seq[torch.randperm(n, generator=g)]
+            ts.append(seq)
+        inp.timestamps = torch.cat(ts)
+    return inp
+
+
+def torch_args(inp, requires_grad=False):
+    d = lambda x: None if x is None else x.to(torch.float64).clone().requires_grad_(requires_grad)
+    return dict(offsets=inp.offsets.tolist(), q=d(inp.q), k=d(inp.k), v=d(inp.v), u=d(inp.u),
+                ts=inp.timestamps, rab_pos=d(inp.rab_pos), rab_time=d(inp.rab_time),
+                norm_len=inp.norm_len)
+
+
+def rel_err(a, b):
+    a = np.asarray(a, dtype=np.float64); b = np.asarray(b, dtype=np.float64)
+    scale = max(np.abs(b).max(), 1e-300)
+    return float(np.abs(a - b).max() / scale)
+
+
+@pytest.mark.parametrize("case", [
+    dict(),
+    dict(norm="fixed", norm_len=17),
+    dict(rab_time=False),
+    dict(rab_pos=False, rab_time=False),
+    dict(ts_sorted=False),
+    dict(lengths=(0, 7, 0, 3), H=2),
+    dict(lengths=(16,), H=1, dqk=3, dv=5, qk_std=2.0, rab_std=2.0),
+    dict(L=20),
+])
+def test_forward_matches_dense_torch(oracle_lib, case):
+    inp = small_inputs(**case)
+    got = oracle_lib.fwd(inp)
+    Y, O = dense_forward(**torch_args(inp), return_o=True)
+    assert rel_err(got["o"], O.numpy()) < 1e-12
+    assert rel_err(got["y"], Y.numpy()) < 1e-12
+
+
+@pytest.mark.parametrize("case", [
+    dict(),
+    dict(norm="fixed", norm_len=11),
+    dict(ts_sorted=False),
+    dict(lengths=(0, 7, 0, 3), H=2),
+    dict(rab_pos=False, rab_time=False, lengths=(13,), H=2, qk_std=1.5),
+])
+def test_backward_matches_autograd(oracle_lib, case):
+    inp = small_inputs(**case)
+    ta = torch_args(inp, requires_grad=True)
+    Y = dense_forward(**ta)
+    Y.backward(inp.dy.to(torch.float64))
+    got = oracle_lib.bwd(inp)
+    assert rel_err(got["dq"], ta["q"].grad.numpy()) < 1e-10
+    assert rel_err(got["dk"], ta["k"].grad.numpy()) < 1e-10
+    assert rel_err(got["dv"], ta["v"].grad.numpy()) < 1e-10
+    assert rel_err(got["du"], ta["u"].grad.numpy()) < 1e-10
+    if inp.rab_pos is not None:
+        assert rel_err(got["d_rab_pos"], ta["rab_pos"].grad.numpy()) < 1e-10
+    if inp.rab_time is not None:
+        assert rel_err(got["d_rab_time"], ta["rab_time"].grad.numpy()) < 1e-10
+
+
+def test_backward_finite_differences(oracle_lib):
+    """<grad, R> from the oracle's backward equals the central difference of
+    sum(Y * dY) along a random direction R, for every differentiable input."""
+    inp = small_inputs(lengths=(6, 4), H=2, dqk=3, dv=3)
+    a = oracle_lib._args_from_inputs(inp)
+    dy = inp.dy.to(torch.float64).numpy()
+    grads = oracle_lib.bwd_raw(a, dy)
+    rng = np.random.default_rng(1)
+    h = 1e-6
+    fields = [("q", "dq"), ("k", "dk"), ("v", "dv"), ("u", "du"),
+              ("rab_pos", "d_rab_pos"), ("rab_time", "d_rab_time")]
+    for name, gname in fields:
+        base = getattr(a, name).copy()
+        R = rng.standard_normal(base.shape)
+        vals = []
+        for sgn in (+1, -1):
+            getattr(a, name)[...] = base + sgn * h * R
+            vals.append(float((oracle_lib.fwd_raw(a)["y"] * dy).sum()))
+        getattr(a, name)[...] = base
+        fd = (vals[0] - vals[1]) / (2 * h)
+        an = float((grads[gname] * R).sum())
+        assert abs(fd - an) <= 1e-6 * max(abs(an), 1e-3), (name, fd, an)
+
+
+def test_first_position_closed_form(oracle_lib):
+    """O_0 = SiLU(q_0 . k_0 + rab_pos[L-1] + rab_time[0]) / N * v_0 per head."""
+    inp = small_inputs(lengths=(8, 5), norm="fixed", norm_len=13)
+    got = oracle_lib.fwd(inp)
+    H, dv = inp.q.shape[1], inp.v.shape[2]
+    L = inp.rab_pos_len
+    for b in range(2):
+        t = int(inp.offsets[b])
+        for h in range(H):
+            s = float((inp.q[t, h].double() * inp.k[t, h].double()).sum())
+            s += float(inp.rab_pos[h, L - 1]) + float(inp.rab_time[h, 0])
+            a = s / (1.0 + math.exp(-s)) / 13.0
+            expect = a * inp.v[t, h].double().numpy()
+            np.testing.assert_allclose(got["o"][t, h * dv:(h + 1) * dv], expect,
+                                       rtol=1e-13, atol=1e-15)
+
+
+def test_causality(oracle_lib):
+    inp = small_inputs(lengths=(12,), H=2)
+    base = oracle_lib.fwd(inp)["y"]
+    i = 5
+    for name in ("q", "k", "v", "u"):
+        pert = small_inputs(lengths=(12,), H=2)
+        t = getattr(pert, name)
+        t[i + 1:] = t[i + 1:] * -3.0 + 1.0
+        if name == "v":
+            pert.timestamps[i + 1:] += 10_000_000
+        y = oracle_lib.fwd(pert)["y"]
+        assert np.array_equal(y[:i + 1], base[:i + 1]), name
+        assert not np.array_equal(y[i + 1:], base[i + 1:]), name
+
+
+def test_linearity_in_v(oracle_lib):
+    inp1 = small_inputs(seed=3)
+    inp2 = small_inputs(seed=3)
+    g = torch.Generator().manual_seed(9)
+    inp2.v = torch.randn(inp1.v.shape, generator=g)
+    comb = small_inputs(seed=3)
+    comb.v = (2.5 * inp1.v.double() - 0.75 * inp2.v.double())
+    o1, o2, oc = (oracle_lib.fwd(x)["o"] for x in (inp1, inp2, comb))
+    assert rel_err(oc, 2.5 * o1 - 0.75 * o2) < 1e-12
+
+
+def test_zero_keys_without_bias_give_zero(oracle_lib):
+    inp = small_inputs(rab_pos=False, rab_time=False)
+    inp.k = torch.zeros_like(inp.k)
+    got = oracle_lib.fwd(inp)
+    assert np.all(got["o"] == 0.0)
+    assert np.all(got["y"] == 0.0)
+
+
+def test_attention_readout_with_identity_values(oracle_lib):
+    """K = 0 and v_j = e_j make O_i[h][:n] row i of A, so each bias index,
+    bucket, mask and the normaliser are checked element by element."""
+    n, H, L = 7, 2, 9
+    inp = small_inputs(lengths=(n,), H=H, dqk=2, dv=n, L=L, norm="fixed", norm_len=5)
+    inp.k = torch.zeros_like(inp.k)
+    eye = torch.eye(n)
+    inp.v = eye[:, None, :].repeat(1, H, 1)
+    # distinct, recognisable table entries
+    inp.rab_pos = (torch.arange(H * (2 * L - 1), dtype=torch.float32).reshape(H, 2 * L - 1)
+                   * 0.01 - 0.3)
+    inp.rab_time = (torch.arange(H * 128, dtype=torch.float32).reshape(H, 128) * -0.002 + 0.1)
+    ts = inp.timestamps.tolist()
+    got = oracle_lib.fwd(inp)["o"]
+    for h in range(H):
+        for i in range(n):
+            for j in range(n):
+                val = got[i, h * n + j]
+                if j > i:
+                    assert val == 0.0
+                    continue
+                dt = abs(ts[i] - ts[j])
+                kb = min(127, int(math.floor(math.log(max(1, dt)) / 0.301)))
+                bias = float(inp.rab_pos[h, i - j + L - 1]) + float(inp.rab_time[h, kb])
+                expect = bias / (1 + math.exp(-bias)) / 5.0
+                assert abs(val - expect) <= 1e-15 + 1e-13 * abs(expect)
+
+
+def test_packing_invariance(oracle_lib):
+    inp = small_inputs(lengths=(5, 9, 3), norm="own")
+    full = oracle_lib.fwd(inp)
+    for b, n in enumerate(inp.lengths):
+        s = int(inp.offsets[b])
+        one = oracle_lib._Args([0, n], inp.q[s:s + n], inp.k[s:s + n], inp.v[s:s + n],
+                               inp.u[s:s + n], inp.timestamps[s:s + n].numpy(),
+                               inp.rab_pos, inp.rab_time, 0, inp.rab_pos_len)
+        alone = oracle_lib.fwd_raw(one)
+        assert np.array_equal(alone["y"], full["y"][s:s + n])
+
+
+def test_head_permutation(oracle_lib):
+    inp = small_inputs(H=3)
+    base = oracle_lib.fwd(inp)["y"]
+    perm = [2, 0, 1]
+    dv = inp.v.shape[2]
+    T = inp.total_tokens
+    p = small_inputs(H=3)
+    p.q, p.k, p.v = inp.q[:, perm], inp.k[:, perm], inp.v[:, perm]
+    p.u = inp.u.reshape(T, 3, dv)[:, perm].reshape(T, 3 * dv)
+    p.rab_pos, p.rab_time = inp.rab_pos[perm], inp.rab_time[perm]
+    y = oracle_lib.fwd(p)["y"].reshape(T, 3, dv)
+    assert rel_err(y, base.reshape(T, 3, dv)[:, perm]) < 1e-12
+
+
+def test_layernorm_rows(oracle_lib):
+    inp = small_inputs()
+    got = oracle_lib.fwd(inp)
+    o = got["o"]
+    xhat = (o - got["mean"][:, None]) * got["rstd"][:, None]
+    var = o.var(axis=1)
+    assert np.abs(xhat.mean(axis=1)).max() < 1e-12
+    np.testing.assert_allclose(xhat.var(axis=1), var / (var + 1e-5), rtol=1e-10)
+
+
+def test_time_bucket_thresholds(oracle_lib):
+    """bucket(x) >= k exactly from ceil(exp(0.301 k)) on (integer |dt|)."""
+    tb = oracle_lib.time_bucket
+    assert tb(0) == 0 and tb(1) == 0 and tb(-1) == 0
+    assert tb(2) == 2 and tb(-2) == 2      # ln 2 / 0.301 = 2.30
+    assert tb(3) == 3                       # ln 3 / 0.301 = 3.65
+    assert tb(300) == 18                    # ln 300 / 0.301 = 18.95
+    assert tb(10 ** 17) == 127 and tb(-(2 ** 63)) == 127 and tb(2 ** 63 - 1) == 127
+    for kk in range(1, 128):
+        x = math.exp(0.301 * kk)
+        lo = math.ceil(x)
+        if lo > 2 ** 52 or abs(lo - x) < 1e-9 * x or abs(lo - 1 - x) < 1e-9 * x:
+            continue
+        assert tb(lo) >= kk and tb(lo - 1) < kk, kk
+        assert tb(-lo) >= kk and tb(1 - lo) < kk
+    # and on a sweep of small values the bucket is the count of thresholds passed
+    for x in range(0, 5000, 7):
+        assert tb(x) == sum(1 for kk in range(1, 128) if max(1, x) >= math.exp(0.301 * kk))
+    assert tb(4, num_buckets=3) == 2
+
+
+def test_workload_shapes_follow_model_card():
+    """The Neurarch-shaped workload matches the model card's block:
+    embed 512 = 4 heads x 128, attention width 128, 1024 input tokens."""
+    import json, os
+    fx = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "model_card_shapes.json")))
+    w = hi.WORKLOADS["neurarch"]
+    assert w.heads == fx["num_heads"] and w.d_v == fx["linear_dim"] and w.d_qk == fx["attn_dim"]
+    assert w.heads * w.d_v == fx["embed_dim"] and w.seq_len == fx["input_tokens"]
+
+
+def test_golden_regression(oracle_lib):
+    """Values written by tests/golden/make_golden.py (which calls only the
+    oracle) still come out of the oracle, so an unintended change shows."""
+    import json, os
+    fx = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "oracle_small.json")))
+    inp = hi.make_inputs(hi.Spec(**fx["spec"]), seed=fx["seed"])
+    got = oracle_lib.fwd(inp)
+    np.testing.assert_allclose(got["y"][fx["rows"]], np.array(fx["y_rows"]), rtol=1e-12,
+                               atol=1e-14)
+    for dt, kb in fx["buckets"]:
+        assert oracle_lib.time_bucket(dt) == kb
