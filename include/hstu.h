@@ -1,0 +1,147 @@
+/*
+ * hstu.h -- C ABI of libhstu: HSTU causal pointwise aggregated attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (one HSTU layer's spatial aggregation and gated output; see
+ * "HSTU (Generative Recommender)" model card, Exported PyTorch,
+ * HSTUBlock.forward; "HSTU Hierarchical Sequential Transduction Units",
+ * §1 The key contribution and §3 How it works; the HSTU reproduction note's
+ * flowchart and key-formula section):
+ *
+ *   for every sequence b (tokens s..s+n_b-1 of the packed token axis), every
+ *   head h and every local row i, over local columns j <= i:
+ *     S_ij = q_i . k_j + rab_pos[h][(i-j)+L-1] + rab_time[h][bucket(t_i - t_j)]
+ *     A_ij = SiLU(S_ij) / N_b        (no softmax; N_b = norm_len or n_b)
+ *     O_i  = sum_{j<=i} A_ij v_j     (heads concatenated: width D = H*d_v)
+ *     Y_i  = LayerNorm_D(O_i) (unit affine, biased variance, eps) * SiLU(U_i)
+ *   bucket(dt) = min(NB-1, floor(ln(max(1,|dt|)) / 0.301)).
+ *
+ * Layouts (row-major, token-major, packed over the B sequences):
+ *   q, k  [T, H, d_qk]    v [T, H, d_v]    u, y, dy [T, H*d_v]
+ *   offsets int32 [B+1] (offsets[0] = 0, non-decreasing, offsets[B] = T)
+ *   timestamps int64 [T]; rab_pos fp32 [H, 2L-1]; rab_time fp32 [H, NB]
+ *
+ * Ownership: the caller owns every buffer.  Device pointers must point to
+ * memory of the current CUDA device; the library allocates nothing, and all
+ * work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ * legacy default stream).
+ *
+ * Errors: argument checks are synchronous and return HSTU_ERR_INVALID_ARG,
+ * HSTU_ERR_UNSUPPORTED or HSTU_ERR_WORKSPACE without enqueueing anything.  A
+ * failed launch returns HSTU_ERR_CUDA.  Problems found on the device (offsets
+ * that contradict the sizes, a bounded wait that ran out) are recorded in a
+ * status word at the start of the workspace and reported by hstu_attn_check.
+ * No C++ exception crosses this boundary.
+ */
+#ifndef HSTU_H
+#define HSTU_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HSTU_API __attribute__((visibility("default")))
+#else
+#define HSTU_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARG = 1,  /* NULL/misaligned pointer, bad sizes, bad offsets  */
+  HSTU_ERR_UNSUPPORTED = 2,  /* valid problem outside the implemented shapes     */
+  HSTU_ERR_CUDA = 3,         /* a CUDA call or launch failed                     */
+  HSTU_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out               */
+  HSTU_ERR_WORKSPACE = 5     /* workspace NULL or smaller than required          */
+} hstu_status_t;
+
+typedef enum { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype_t;
+
+/* Problem description, passed by const pointer; read during the call only. */
+typedef struct {
+  hstu_dtype_t dtype;         /* q, k, v, u, y, dy and the gradients dq..du       */
+  int32_t batch;              /* B >= 0                                           */
+  int32_t total_tokens;       /* T = offsets[B]                                   */
+  int32_t max_seq_len;        /* >= every n_b; sizes the launch grid              */
+  int32_t num_heads;          /* H >= 1                                           */
+  int32_t d_qk, d_v;          /* per-head widths                                  */
+  const int32_t *offsets;     /* device [B+1]                                     */
+  const int32_t *offsets_host;/* optional host copy of offsets: full validation   */
+  const int64_t *timestamps;  /* device [T], or NULL when rab_time is NULL        */
+  const float *rab_pos;       /* device [H, 2L-1] or NULL (no position bias)      */
+  int32_t rab_pos_len;        /* L >= max_seq_len when rab_pos is given           */
+  const float *rab_time;      /* device [H, NB] or NULL (no time bias)            */
+  int32_t num_time_buckets;   /* NB in [1, 128] when rab_time is given            */
+  int32_t norm_len;           /* > 0: divide by it; 0: divide by each n_b         */
+  float ln_eps;               /* LayerNorm epsilon, > 0 (1e-5)                    */
+} hstu_problem_t;
+
+/*
+ * Bytes of device workspace the call needs (is_bwd = 0: forward; 1: backward).
+ * The workspace must be 256-byte aligned and zero-filled before its first use;
+ * its first word is the device status that hstu_attn_check reads and re-arms.
+ */
+HSTU_API size_t hstu_attn_workspace_size(const hstu_problem_t *p, int is_bwd);
+
+/*
+ * Forward.  q, k, v, u: inputs (dtype, layouts above, 16-byte aligned).
+ * y: output [T, H*d_v] (dtype).  o_save [T, H*d_v], ln_mean [T], ln_rstd [T]:
+ * optional fp32 outputs kept for the backward (all three or none; NULL = skip).
+ * Supported: bf16 with d_qk = d_v = 128 and 1 <= H <= 8 (tcgen05 path);
+ * fp32 with d_qk, d_v <= 128 and H*d_v <= 1024 (true-fp32 SIMT path).
+ */
+HSTU_API hstu_status_t hstu_attn_fwd(const hstu_problem_t *p, const void *q, const void *k,
+                            const void *v, const void *u, void *y, float *o_save,
+                            float *ln_mean, float *ln_rstd, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
+ * Backward of hstu_attn_fwd.  dy [T, H*d_v] (dtype) is the upstream gradient;
+ * o_save, ln_mean, ln_rstd are the forward's saved fp32 outputs (required).
+ * Writes dq, dk [T,H,d_qk], dv [T,H,d_v], du [T,H*d_v] (dtype); d_rab_pos
+ * [H,2L-1] and d_rab_time [H,NB] (fp32) are overwritten, not accumulated,
+ * when non-NULL (entries with i-j < 0 are zero).
+ */
+HSTU_API hstu_status_t hstu_attn_bwd(const hstu_problem_t *p, const void *dy, const void *q,
+                            const void *k, const void *v, const void *u,
+                            const float *o_save, const float *ln_mean, const float *ln_rstd,
+                            void *dq, void *dk, void *dv, void *du, float *d_rab_pos,
+                            float *d_rab_time, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/*
+ * Waits for `stream`, reads the device status word of `workspace`, resets it
+ * to zero and returns it (HSTU_OK, HSTU_ERR_INVALID_ARG for offsets found
+ * inconsistent on the device, HSTU_ERR_TIMEOUT for an expired wait), or
+ * HSTU_ERR_CUDA when the stream itself reports an error.
+ */
+HSTU_API hstu_status_t hstu_attn_check(void *workspace, void *stream);
+
+/* Static, NUL-terminated description of a status code. */
+HSTU_API const char *hstu_status_string(hstu_status_t s);
+
+/*
+ * Host utility: writes the library's time-bucket thresholds, out[k-1] = the
+ * smallest |dt| with bucket(dt) >= k for k = 1..num_buckets-1.  Returns the
+ * number written, or -1 for num_buckets outside [1, 128].
+ */
+HSTU_API int32_t hstu_time_bucket_thresholds(int64_t *out, int32_t num_buckets);
+
+/*
+ * Self-test of the device error path: launches one thread that waits on an
+ * mbarrier nothing arrives on, with the library's bounded wait limited to
+ * budget_ns (1 ns .. 5 s).  When the budget runs out the kernel sets the
+ * timeout bit of the workspace status word and returns; hstu_attn_check then
+ * reports HSTU_ERR_TIMEOUT and the context remains usable.  Returns
+ * HSTU_ERR_WORKSPACE for a NULL or unaligned workspace (256 bytes suffice).
+ */
+HSTU_API hstu_status_t hstu_selftest_wait_timeout(void *workspace, uint64_t budget_ns,
+                                                  void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HSTU_H */

@@ -1,0 +1,239 @@
+"""ctypes binding of libhstu (include/hstu.h): argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module
+only checks tensor placement, builds the ``hstu_problem_t`` struct, allocates
+outputs and workspace with torch (device memory is plumbing) and forwards
+raw pointers.  There is no fallback: if libhstu.so is missing, or a tensor is
+not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhstu.so")
+
+HSTU_OK, HSTU_ERR_INVALID_ARG, HSTU_ERR_UNSUPPORTED = 0, 1, 2
+HSTU_ERR_CUDA, HSTU_ERR_TIMEOUT, HSTU_ERR_WORKSPACE = 3, 4, 5
+HSTU_F32, HSTU_BF16 = 0, 1
+
+EXPORTED = ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_attn_check",
+            "hstu_status_string", "hstu_time_bucket_thresholds", "hstu_selftest_wait_timeout")
+
+
+class HSTUError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__("%s: %s" % (what, status_string(code)))
+
+
+class hstu_problem_t(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int),
+        ("batch", ctypes.c_int32),
+        ("total_tokens", ctypes.c_int32),
+        ("max_seq_len", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32),
+        ("d_qk", ctypes.c_int32),
+        ("d_v", ctypes.c_int32),
+        ("offsets", ctypes.c_void_p),
+        ("offsets_host", ctypes.c_void_p),
+        ("timestamps", ctypes.c_void_p),
+        ("rab_pos", ctypes.c_void_p),
+        ("rab_pos_len", ctypes.c_int32),
+        ("rab_time", ctypes.c_void_p),
+        ("num_time_buckets", ctypes.c_int32),
+        ("norm_len", ctypes.c_int32),
+        ("ln_eps", ctypes.c_float),
+    ]
+
+
+_lib = None
+
+
+def load_library():
+    """Loads libhstu.so from the package directory (raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libhstu.so is not built (%s); run `python -m "
+                           "pointwise_attention_b200.build`" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(hstu_problem_t)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.hstu_attn_workspace_size.argtypes = [P, ctypes.c_int]
+    lib.hstu_attn_workspace_size.restype = sz
+    lib.hstu_attn_fwd.argtypes = [P] + [vp] * 5 + [vp] * 3 + [vp, sz, vp]
+    lib.hstu_attn_fwd.restype = ctypes.c_int
+    lib.hstu_attn_bwd.argtypes = [P] + [vp] * 5 + [vp] * 3 + [vp] * 4 + [vp] * 2 + [vp, sz, vp]
+    lib.hstu_attn_bwd.restype = ctypes.c_int
+    lib.hstu_attn_check.argtypes = [vp, vp]
+    lib.hstu_attn_check.restype = ctypes.c_int
+    lib.hstu_status_string.argtypes = [ctypes.c_int]
+    lib.hstu_status_string.restype = ctypes.c_char_p
+    lib.hstu_time_bucket_thresholds.argtypes = [vp, ctypes.c_int32]
+    lib.hstu_time_bucket_thresholds.restype = ctypes.c_int32
+    lib.hstu_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
+    lib.hstu_selftest_wait_timeout.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().hstu_status_string(int(code)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError("%s must be a CUDA tensor (the library runs on the GPU only)" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must have dtype %s, got %s" % (name, dtype, t.dtype))
+    return t
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_problem(q, v, offsets, max_seq_len, timestamps=None, rab_pos=None, rab_time=None,
+                 norm_len=0, eps=1e-5, offsets_host=None):
+    """hstu_problem_t for tensors q [T,H,dqk], v [T,H,dv] and int32 offsets [B+1]."""
+    if q.dtype == torch.bfloat16:
+        dt = HSTU_BF16
+    elif q.dtype == torch.float32:
+        dt = HSTU_F32
+    else:
+        raise ValueError("q must be bf16 or fp32")
+    T, H, dqk = q.shape
+    p = hstu_problem_t()
+    p.dtype = dt
+    p.batch = offsets.numel() - 1
+    p.total_tokens = T
+    p.max_seq_len = int(max_seq_len)
+    p.num_heads = H
+    p.d_qk = dqk
+    p.d_v = v.shape[-1]
+    p.offsets = offsets.data_ptr()
+    p.offsets_host = None if offsets_host is None else offsets_host.data_ptr()
+    p.timestamps = None if timestamps is None else timestamps.data_ptr()
+    p.rab_pos = None if rab_pos is None else rab_pos.data_ptr()
+    p.rab_pos_len = 0 if rab_pos is None else (rab_pos.shape[-1] + 1) // 2
+    p.rab_time = None if rab_time is None else rab_time.data_ptr()
+    p.num_time_buckets = 0 if rab_time is None else rab_time.shape[-1]
+    p.norm_len = int(norm_len)
+    p.ln_eps = float(eps)
+    return p
+
+
+def hstu_attn_workspace_size(problem: hstu_problem_t, is_bwd: bool = False) -> int:
+    return int(load_library().hstu_attn_workspace_size(ctypes.byref(problem), int(bool(is_bwd))))
+
+
+def new_workspace(problem: hstu_problem_t, is_bwd: bool, device) -> torch.Tensor:
+    n = hstu_attn_workspace_size(problem, is_bwd)
+    if n == 0:
+        raise HSTUError(HSTU_ERR_INVALID_ARG, "hstu_attn_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def hstu_attn_fwd(q, k, v, u, offsets, max_seq_len, *, timestamps=None, rab_pos=None,
+                  rab_time=None, norm_len=0, eps=1e-5, save_for_backward=False,
+                  offsets_host=None, y=None, saved=None, workspace=None, stream=None):
+    """Forward.  Returns (y, saved) with saved = (o_save, ln_mean, ln_rstd) or None."""
+    lib = load_library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("u", u)):
+        _dev(t, name, q.dtype)
+    _dev(offsets, "offsets", torch.int32)
+    _dev(timestamps, "timestamps", torch.int64)
+    _dev(rab_pos, "rab_pos", torch.float32)
+    _dev(rab_time, "rab_time", torch.float32)
+    T, H, _ = q.shape
+    D = H * v.shape[-1]
+    p = make_problem(q, v, offsets, max_seq_len, timestamps, rab_pos, rab_time, norm_len, eps,
+                     offsets_host)
+    if y is None:
+        y = torch.empty((T, D), dtype=q.dtype, device=q.device)
+    _dev(y, "y", q.dtype)
+    if save_for_backward and saved is None:
+        saved = (torch.empty((T, D), dtype=torch.float32, device=q.device),
+                 torch.empty((T,), dtype=torch.float32, device=q.device),
+                 torch.empty((T,), dtype=torch.float32, device=q.device))
+    if not save_for_backward:
+        saved = None
+    if workspace is None:
+        workspace = new_workspace(p, False, q.device)
+    o_save, mean, rstd = saved if saved is not None else (None, None, None)
+    rc = lib.hstu_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(y),
+                           _ptr(o_save), _ptr(mean), _ptr(rstd), _ptr(workspace),
+                           workspace.numel(), _stream_ptr(stream))
+    if rc != HSTU_OK:
+        raise HSTUError(rc, "hstu_attn_fwd")
+    return y, saved
+
+
+def hstu_attn_bwd(dy, q, k, v, u, offsets, max_seq_len, saved, *, timestamps=None,
+                  rab_pos=None, rab_time=None, norm_len=0, eps=1e-5, offsets_host=None,
+                  need_rab_grads=True, grads=None, workspace=None, stream=None):
+    """Backward.  Returns dict dq, dk, dv, du, d_rab_pos, d_rab_time."""
+    lib = load_library()
+    for name, t in (("dy", dy), ("q", q), ("k", k), ("v", v), ("u", u)):
+        _dev(t, name, q.dtype)
+    _dev(offsets, "offsets", torch.int32)
+    o_save, mean, rstd = saved
+    for name, t in (("o_save", o_save), ("ln_mean", mean), ("ln_rstd", rstd)):
+        _dev(t, name, torch.float32)
+    p = make_problem(q, v, offsets, max_seq_len, timestamps, rab_pos, rab_time, norm_len, eps,
+                     offsets_host)
+    if grads is None:
+        grads = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                     du=torch.empty_like(u),
+                     d_rab_pos=(torch.empty_like(rab_pos)
+                                if (rab_pos is not None and need_rab_grads) else None),
+                     d_rab_time=(torch.empty_like(rab_time)
+                                 if (rab_time is not None and need_rab_grads) else None))
+    if workspace is None:
+        workspace = new_workspace(p, True, q.device)
+    rc = lib.hstu_attn_bwd(ctypes.byref(p), _ptr(dy), _ptr(q), _ptr(k), _ptr(v), _ptr(u),
+                           _ptr(o_save), _ptr(mean), _ptr(rstd), _ptr(grads["dq"]),
+                           _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["du"]),
+                           _ptr(grads["d_rab_pos"]), _ptr(grads["d_rab_time"]),
+                           _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    if rc != HSTU_OK:
+        raise HSTUError(rc, "hstu_attn_bwd")
+    return grads
+
+
+def hstu_attn_check(workspace, stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status word."""
+    return int(load_library().hstu_attn_check(_ptr(workspace), _stream_ptr(stream)))
+
+
+def hstu_time_bucket_thresholds(num_buckets: int = 128):
+    import numpy as np
+    out = np.zeros(max(num_buckets - 1, 1), dtype=np.int64)
+    n = load_library().hstu_time_bucket_thresholds(out.ctypes.data_as(ctypes.c_void_p),
+                                                   int(num_buckets))
+    if n < 0:
+        raise HSTUError(HSTU_ERR_INVALID_ARG, "hstu_time_bucket_thresholds")
+    return out[:n]
+
+
+def hstu_selftest_wait_timeout(workspace, budget_ns: int = 50_000_000, stream=None) -> int:
+    """Runs the bounded-wait self-test kernel; returns the launch status."""
+    return int(load_library().hstu_selftest_wait_timeout(_ptr(workspace), int(budget_ns),
+                                                         _stream_ptr(stream)))

@@ -1,0 +1,332 @@
+// hstu_api.cu -- the C ABI of libhstu (declared in include/hstu.h): argument
+// validation, workspace layout, the time-bucket threshold table, TMA tensor
+// maps, and kernel dispatch.  No exception crosses the boundary.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "hstu.h"
+#include "internal.h"
+
+using namespace hstu;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------- time buckets
+// bucket(a) for a >= 1 without the cap: floor(ln(a) / 0.301) in fp64.
+int bucket_uncapped(long long a) {
+  double x = static_cast<double>(a);
+  if (x < 1.0) x = 1.0;
+  return static_cast<int>(std::floor(std::log(x) / 0.301));
+}
+
+// thr_all[k] = smallest a >= 1 with bucket_uncapped(a) >= k, k = 1..127, found by
+// binary search (the bucket is non-decreasing in a).
+struct Thresholds {
+  long long thr[kMaxBuckets];
+};
+
+const Thresholds& thresholds() {
+  static Thresholds t;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    t.thr[0] = 0;
+    for (int k = 1; k < kMaxBuckets; ++k) {
+      long long lo = 1, hi = 0x7FFFFFFFFFFFFFFFll;
+      while (lo < hi) {
+        const long long mid = lo + (hi - lo) / 2;
+        if (bucket_uncapped(mid) >= k) hi = mid; else lo = mid + 1;
+      }
+      t.thr[k] = lo;
+    }
+  });
+  return t;
+}
+
+void fill_bucket_table(BucketTable* bt, int nb) {
+  const Thresholds& t = thresholds();
+  for (int k = 0; k < kThrLen; ++k)
+    bt->thr[k] = (k < nb && k < kMaxBuckets) ? t.thr[k] : 0x7FFFFFFFFFFFFFFFll;
+  for (int e = 0; e < 64; ++e) {
+    const long long p = (e < 63) ? (1ll << e) : 0x7FFFFFFFFFFFFFFFll;
+    int k = 0;
+    while (k + 1 < nb && bt->thr[k + 1] <= p) ++k;
+    bt->first_k[e] = static_cast<signed char>(k);
+  }
+}
+
+// ---------------------------------------------------------- TMA tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [T, H, 128] bf16 viewed as a 3-D tensor (d, head, token); box = 64 x 1 x 128,
+// 128-byte swizzle: one box is one 128-row x 128-byte slab of a K-major tile.
+bool make_map_3d(CUtensorMap* map, const void* base, int T, int H, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(H) * 128 * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------- validation
+hstu_status_t check_problem(const hstu_problem_t* p) {
+  if (!p) return HSTU_ERR_INVALID_ARG;
+  if (p->dtype != HSTU_F32 && p->dtype != HSTU_BF16) return HSTU_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->total_tokens < 0 || p->max_seq_len < 0 || p->num_heads < 1 ||
+      p->d_qk < 1 || p->d_v < 1 || p->norm_len < 0)
+    return HSTU_ERR_INVALID_ARG;
+  if (!(p->ln_eps > 0.0f) || !std::isfinite(p->ln_eps)) return HSTU_ERR_INVALID_ARG;
+  if (p->batch > 0 && !p->offsets) return HSTU_ERR_INVALID_ARG;
+  if (p->batch == 0 && p->total_tokens != 0) return HSTU_ERR_INVALID_ARG;
+  if (p->rab_pos && (p->rab_pos_len < 1 || p->rab_pos_len < p->max_seq_len))
+    return HSTU_ERR_INVALID_ARG;
+  if (p->rab_pos && static_cast<int64_t>(p->rab_pos_len) * 2 - 1 > 0x7FFFFFFF)
+    return HSTU_ERR_INVALID_ARG;
+  if (p->rab_time && (!p->timestamps || p->num_time_buckets < 1 ||
+                      p->num_time_buckets > kMaxBuckets))
+    return HSTU_ERR_INVALID_ARG;
+  if (p->offsets_host) {
+    const int32_t* o = p->offsets_host;
+    if (o[0] != 0 || o[p->batch] != p->total_tokens) return HSTU_ERR_INVALID_ARG;
+    for (int b = 0; b < p->batch; ++b) {
+      const int64_t n = static_cast<int64_t>(o[b + 1]) - o[b];
+      if (n < 0 || n > p->max_seq_len) return HSTU_ERR_INVALID_ARG;
+      if (p->rab_pos && n > p->rab_pos_len) return HSTU_ERR_INVALID_ARG;
+    }
+  }
+  return HSTU_OK;
+}
+
+bool bf16_supported(const hstu_problem_t* p) {
+  return p->dtype == HSTU_BF16 && p->d_qk == 128 && p->d_v == 128 && p->num_heads <= 8;
+}
+
+bool f32_supported(const hstu_problem_t* p) {
+  return p->dtype == HSTU_F32 && p->d_qk <= 128 && p->d_v <= 128 &&
+         p->num_heads * p->d_v <= 1024;
+}
+
+// Workspace layout: [status 256 B][dO: T*H*dv dtype][dq_acc: T*H*dqk fp32]
+struct WsLayout {
+  size_t dO_off, dq_off, total;
+};
+
+WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
+  WsLayout l{};
+  size_t off = kStatusBytes;
+  if (is_bwd) {
+    const size_t T = static_cast<size_t>(p->total_tokens);
+    l.dO_off = off;
+    off += align_up(T * p->num_heads * p->d_v * (p->dtype == HSTU_BF16 ? 2 : 4));
+    l.dq_off = off;
+    if (p->dtype == HSTU_BF16) off += align_up(T * p->num_heads * p->d_qk * 4);
+  }
+  l.total = off;
+  return l;
+}
+
+hstu_status_t check_ws(const hstu_problem_t* p, int is_bwd, void* ws, size_t bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return HSTU_ERR_WORKSPACE;
+  if (bytes < ws_layout(p, is_bwd).total) return HSTU_ERR_WORKSPACE;
+  return HSTU_OK;
+}
+
+void fill_common(const hstu_problem_t* p, int* status, FwdArgs* a) {
+  a->offsets = p->offsets;
+  a->timestamps = p->timestamps;
+  a->rab_pos = p->rab_pos;
+  a->rab_time = p->rab_time;
+  a->status = status;
+  a->B = p->batch;
+  a->T = p->total_tokens;
+  a->H = p->num_heads;
+  a->d_qk = p->d_qk;
+  a->d_v = p->d_v;
+  a->max_seq_len = p->max_seq_len;
+  a->max_tiles = (p->max_seq_len + 127) / 128;
+  a->L = p->rab_pos ? p->rab_pos_len : 0;
+  a->nb = p->rab_time ? p->num_time_buckets : 0;
+  a->norm_len = p->norm_len;
+  a->eps = p->ln_eps;
+  fill_bucket_table(&a->bt, p->rab_time ? p->num_time_buckets : 1);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hstu_attn_workspace_size(const hstu_problem_t* p, int is_bwd) {
+  if (check_problem(p) != HSTU_OK) return 0;
+  return ws_layout(p, is_bwd ? 1 : 0).total;
+}
+
+const char* hstu_status_string(hstu_status_t s) {
+  switch (s) {
+    case HSTU_OK: return "HSTU_OK";
+    case HSTU_ERR_INVALID_ARG: return "HSTU_ERR_INVALID_ARG: invalid argument";
+    case HSTU_ERR_UNSUPPORTED: return "HSTU_ERR_UNSUPPORTED: shape or dtype not implemented";
+    case HSTU_ERR_CUDA: return "HSTU_ERR_CUDA: a CUDA call or launch failed";
+    case HSTU_ERR_TIMEOUT: return "HSTU_ERR_TIMEOUT: a bounded device wait ran out";
+    case HSTU_ERR_WORKSPACE: return "HSTU_ERR_WORKSPACE: workspace missing, misaligned or too small";
+  }
+  return "HSTU: unknown status";
+}
+
+int32_t hstu_time_bucket_thresholds(int64_t* out, int32_t num_buckets) {
+  if (!out || num_buckets < 1 || num_buckets > kMaxBuckets) return -1;
+  BucketTable bt;
+  fill_bucket_table(&bt, num_buckets);
+  for (int k = 1; k < num_buckets; ++k) out[k - 1] = bt.thr[k];
+  return num_buckets - 1;
+}
+
+hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* k, const void* v,
+                            const void* u, void* y, float* o_save, float* ln_mean,
+                            float* ln_rstd, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  hstu_status_t st = check_problem(p);
+  if (st != HSTU_OK) return st;
+  if (p->total_tokens > 0) {
+    if (!q || !k || !v || !u || !y) return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(y))
+      return HSTU_ERR_INVALID_ARG;
+  }
+  const int nsave = (o_save != nullptr) + (ln_mean != nullptr) + (ln_rstd != nullptr);
+  if (nsave != 0 && nsave != 3) return HSTU_ERR_INVALID_ARG;
+  if (o_save && !aligned16(o_save)) return HSTU_ERR_INVALID_ARG;
+  if (!bf16_supported(p) && !f32_supported(p)) return HSTU_ERR_UNSUPPORTED;
+  st = check_ws(p, 0, workspace, workspace_bytes);
+  if (st != HSTU_OK) return st;
+  if (p->total_tokens == 0 || p->batch == 0) return HSTU_OK;
+
+  FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  fill_common(p, static_cast<int*>(workspace), &a);
+  a.q = q; a.k = k; a.v = v; a.u = u; a.y = y;
+  a.o_save = o_save; a.ln_mean = ln_mean; a.ln_rstd = ln_rstd;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err;
+  if (p->dtype == HSTU_BF16) {
+    CUtensorMap tq, tk, tv;
+    if (!make_map_3d(&tq, q, p->total_tokens, p->num_heads, 128) ||
+        !make_map_3d(&tk, k, p->total_tokens, p->num_heads, 128) ||
+        !make_map_3d(&tv, v, p->total_tokens, p->num_heads, 128))
+      return HSTU_ERR_CUDA;
+    err = launch_fwd_bf16_sm100(a, tq, tk, tv, s);
+  } else {
+    err = launch_fwd_f32_simt(a, s);
+  }
+  return err == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void* q, const void* k,
+                            const void* v, const void* u, const float* o_save,
+                            const float* ln_mean, const float* ln_rstd, void* dq, void* dk,
+                            void* dv, void* du, float* d_rab_pos, float* d_rab_time,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  hstu_status_t st = check_problem(p);
+  if (st != HSTU_OK) return st;
+  if (p->total_tokens > 0) {
+    const void* ptrs[] = {dy, q, k, v, u, o_save, ln_mean, ln_rstd, dq, dk, dv, du};
+    for (const void* x : ptrs)
+      if (!x) return HSTU_ERR_INVALID_ARG;
+    const void* al[] = {dy, q, k, v, u, o_save, dq, dk, dv, du};
+    for (const void* x : al)
+      if (!aligned16(x)) return HSTU_ERR_INVALID_ARG;
+  }
+  if (d_rab_pos && !p->rab_pos) return HSTU_ERR_INVALID_ARG;
+  if (d_rab_time && !p->rab_time) return HSTU_ERR_INVALID_ARG;
+  if (!bf16_supported(p) && !f32_supported(p)) return HSTU_ERR_UNSUPPORTED;
+  st = check_ws(p, 1, workspace, workspace_bytes);
+  if (st != HSTU_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d_rab_pos &&
+      cudaMemsetAsync(d_rab_pos, 0,
+                      sizeof(float) * p->num_heads * (2 * static_cast<size_t>(p->rab_pos_len) - 1),
+                      s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (d_rab_time &&
+      cudaMemsetAsync(d_rab_time, 0, sizeof(float) * p->num_heads * p->num_time_buckets, s) !=
+          cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (p->total_tokens == 0 || p->batch == 0) return HSTU_OK;
+
+  const WsLayout l = ws_layout(p, 1);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  FwdArgs common;
+  std::memset(&common, 0, sizeof(common));
+  fill_common(p, reinterpret_cast<int*>(ws), &common);
+  BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.offsets = common.offsets; a.timestamps = common.timestamps;
+  a.rab_pos = common.rab_pos; a.rab_time = common.rab_time;
+  a.q = q; a.k = k; a.v = v; a.u = u; a.dy = dy;
+  a.o_save = o_save; a.ln_mean = ln_mean; a.ln_rstd = ln_rstd;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.du = du;
+  a.d_rab_pos = d_rab_pos; a.d_rab_time = d_rab_time;
+  a.dO = ws + l.dO_off;
+  a.dq_acc = p->dtype == HSTU_BF16 ? reinterpret_cast<float*>(ws + l.dq_off) : nullptr;
+  a.status = common.status;
+  a.B = common.B; a.T = common.T; a.H = common.H; a.d_qk = common.d_qk; a.d_v = common.d_v;
+  a.max_seq_len = common.max_seq_len; a.max_tiles = common.max_tiles;
+  a.L = common.L; a.nb = common.nb; a.norm_len = common.norm_len; a.eps = common.eps;
+  a.bt = common.bt;
+  cudaError_t err;
+  if (p->dtype == HSTU_BF16) {
+    err = launch_bwd_bf16_simt(a, s);
+  } else {
+    err = launch_bwd_f32_simt(a, s);
+  }
+  return err == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_attn_check(void* workspace, void* stream) {
+  if (!workspace) return HSTU_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(int), s) != cudaSuccess) return HSTU_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return HSTU_ERR_CUDA;
+  }
+  if (word & kStatusTimeout) return HSTU_ERR_TIMEOUT;
+  if (word & kStatusBadOffsets) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+}  // extern "C"

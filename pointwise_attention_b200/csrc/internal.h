@@ -1,0 +1,88 @@
+// internal.h -- declarations shared by the host API and the kernels of libhstu.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace hstu {
+
+// Bits of the device status word (first 4 bytes of the workspace).
+constexpr int kStatusBadOffsets = 1;   // offsets contradict T / max_seq_len / L
+constexpr int kStatusTimeout = 2;      // a bounded wait ran out
+
+constexpr int kMaxBuckets = 128;
+// thr[k] = smallest |dt| with bucket(dt) >= k (thr[0] = 0); entries k >= NB
+// hold INT64_MAX so the bucket search never passes NB-1.
+constexpr int kThrLen = kMaxBuckets + 4;
+
+struct BucketTable {
+  long long thr[kThrLen];
+  signed char first_k[64];   // bucket(2^e), e = 0..62
+};
+
+// Arguments common to the forward kernels (bf16 tcgen05 and fp32 SIMT).
+struct FwdArgs {
+  const int32_t* offsets;
+  const int64_t* timestamps;
+  const float* rab_pos;
+  const float* rab_time;
+  const void* q;     // used by the SIMT path (the tcgen05 path reads q/k/v via TMA)
+  const void* k;
+  const void* v;
+  const void* u;
+  void* y;
+  float* o_save;
+  float* ln_mean;
+  float* ln_rstd;
+  int* status;
+  int B, T, H, d_qk, d_v;
+  int max_seq_len;
+  int max_tiles;     // ceil(max_seq_len / 128)
+  int L;             // rab_pos_len (0 if no position table)
+  int nb;            // number of time buckets (0 if no time table)
+  int norm_len;
+  float eps;
+  BucketTable bt;
+};
+
+struct BwdArgs {
+  const int32_t* offsets;
+  const int64_t* timestamps;
+  const float* rab_pos;
+  const float* rab_time;
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* u;
+  const void* dy;
+  const float* o_save;
+  const float* ln_mean;
+  const float* ln_rstd;
+  void* dq;
+  void* dk;
+  void* dv;
+  void* du;
+  float* d_rab_pos;
+  float* d_rab_time;
+  void* dO;          // workspace: dO in the compute dtype [T, H*d_v]
+  float* dq_acc;     // workspace: fp32 [T, H, d_qk] (bf16 path)
+  int* status;
+  int B, T, H, d_qk, d_v;
+  int max_seq_len;
+  int max_tiles;
+  int L;
+  int nb;
+  int norm_len;
+  float eps;
+  BucketTable bt;
+};
+
+// Kernel launchers (return cudaSuccess or the launch error).
+cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, cudaStream_t stream);
+cudaError_t launch_fwd_f32_simt(const FwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd_f32_simt(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd_bf16_simt(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd_pre_bf16(const BwdArgs& a, cudaStream_t stream);
+
+}  // namespace hstu

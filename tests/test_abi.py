@@ -1,0 +1,185 @@
+"""CPU tests of the C-ABI library: it loads without a GPU, exports every symbol
+include/hstu.h declares, builds the same time-bucket thresholds as the oracle,
+and rejects bad arguments synchronously, before anything is enqueued.
+
+The rejection cases pass placeholder device addresses; every case violates one
+rule, so the library returns before it touches them (no CUDA call is made).
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from pointwise_attention_b200 import build
+    build.build()
+    import pointwise_attention_b200 as pa
+    return pa
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "hstu.h")).read()
+    return sorted(set(re.findall(r"HSTU_API\s+[\w\s\*]*?\b(hstu_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 7
+    so = lib.load_library()
+    for n in names:
+        assert hasattr(so, n), n
+    assert set(names) == set(lib.EXPORTED)
+
+
+def test_thresholds_match_oracle_golden(lib):
+    rows = [l.split() for l in open(os.path.join(ROOT, "tests", "golden",
+                                                 "time_bucket_thresholds.txt"))
+            if not l.startswith("#")]
+    golden = np.array([int(r[1]) for r in rows], dtype=np.int64)
+    got = lib.hstu_time_bucket_thresholds(128)
+    assert np.array_equal(got, golden)
+    # a capped table keeps the first NB-1 thresholds
+    assert np.array_equal(lib.hstu_time_bucket_thresholds(10), golden[:9])
+    with pytest.raises(lib.HSTUError):
+        lib.hstu_time_bucket_thresholds(129)
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.status_string(code).startswith("HSTU_")
+    assert "unknown" in lib.status_string(99)
+
+
+FAKE = 0x7F0000000000   # placeholder device address, 256-byte aligned; never dereferenced
+
+
+def problem(lib, **kw):
+    p = lib.hstu_problem_t()
+    host_off = kw.pop("offsets_host", None)
+    p.dtype = kw.pop("dtype", 1)
+    p.batch = kw.pop("batch", 2)
+    p.total_tokens = kw.pop("total_tokens", 300)
+    p.max_seq_len = kw.pop("max_seq_len", 200)
+    p.num_heads = kw.pop("num_heads", 4)
+    p.d_qk = kw.pop("d_qk", 128)
+    p.d_v = kw.pop("d_v", 128)
+    p.offsets = kw.pop("offsets", FAKE)
+    p.timestamps = kw.pop("timestamps", None)
+    p.rab_pos = kw.pop("rab_pos", None)
+    p.rab_pos_len = kw.pop("rab_pos_len", 0)
+    p.rab_time = kw.pop("rab_time", None)
+    p.num_time_buckets = kw.pop("num_time_buckets", 0)
+    p.norm_len = kw.pop("norm_len", 0)
+    p.ln_eps = kw.pop("ln_eps", 1e-5)
+    assert not kw, kw
+    keep = None
+    if host_off is not None:
+        keep = (ctypes.c_int32 * len(host_off))(*host_off)
+        p.offsets_host = ctypes.cast(keep, ctypes.c_void_p).value
+    return p, keep
+
+
+def call_fwd(lib, p, ws_bytes=None, ws=FAKE, q=FAKE, save=(None, None, None), y=FAKE):
+    so = lib.load_library()
+    if ws_bytes is None:
+        ws_bytes = 1 << 20
+    vp = ctypes.c_void_p
+    return so.hstu_attn_fwd(ctypes.byref(p), vp(q), vp(FAKE), vp(FAKE), vp(FAKE), vp(y),
+                            *(vp(x) if x else None for x in save), vp(ws) if ws else None,
+                            ws_bytes, None)
+
+
+@pytest.mark.parametrize("field,value", [
+    ("dtype", 7), ("num_heads", 0), ("d_qk", 0), ("batch", -1), ("ln_eps", 0.0),
+    ("ln_eps", float("nan")), ("norm_len", -3), ("offsets", None), ("max_seq_len", -1),
+])
+def test_fwd_rejects_bad_problem(lib, field, value):
+    p, keep = problem(lib, **{field: value})
+    assert call_fwd(lib, p) == 1
+
+
+@pytest.mark.parametrize("host", [
+    [0, 200, 100],          # decreasing
+    [1, 100, 300],          # offsets[0] != 0
+    [0, 100, 299],          # offsets[B] != T
+    [0, 50, 300],           # a length above max_seq_len
+])
+def test_fwd_rejects_bad_host_offsets(lib, host):
+    p, keep = problem(lib, offsets_host=host)
+    assert call_fwd(lib, p) == 1
+
+
+def test_fwd_rejects_bias_shapes(lib):
+    p, _ = problem(lib, rab_pos=FAKE, rab_pos_len=100)        # L < max_seq_len
+    assert call_fwd(lib, p) == 1
+    p, _ = problem(lib, rab_pos=FAKE, rab_pos_len=200, max_seq_len=200,
+                   offsets_host=[0, 99, 300])                   # n_b = 201 > max_seq_len
+    assert call_fwd(lib, p) == 1
+    p, _ = problem(lib, rab_time=FAKE, num_time_buckets=128)  # no timestamps
+    assert call_fwd(lib, p) == 1
+    p, _ = problem(lib, rab_time=FAKE, timestamps=FAKE, num_time_buckets=129)
+    assert call_fwd(lib, p) == 1
+
+
+def test_fwd_rejects_pointers(lib):
+    p, _ = problem(lib)
+    assert call_fwd(lib, p, q=None) == 1
+    assert call_fwd(lib, p, q=FAKE + 8) == 1                  # not 16-byte aligned
+    assert call_fwd(lib, p, y=FAKE + 2) == 1
+    assert call_fwd(lib, p, save=(FAKE, None, None)) == 1     # all three saved outputs or none
+
+
+@pytest.mark.parametrize("kw", [
+    dict(d_qk=64, d_v=64), dict(num_heads=9), dict(dtype=0, d_qk=256), dict(dtype=0, d_v=200),
+    dict(dtype=0, num_heads=16, d_v=128),
+])
+def test_fwd_unsupported(lib, kw):
+    p, _ = problem(lib, **kw)
+    assert call_fwd(lib, p) == 2
+
+
+def test_fwd_workspace(lib):
+    p, _ = problem(lib)
+    need = lib.hstu_attn_workspace_size(p, False)
+    assert need >= 256 and need % 256 == 0
+    assert call_fwd(lib, p, ws=None) == 5
+    assert call_fwd(lib, p, ws_bytes=need - 1) == 5
+    assert call_fwd(lib, p, ws=FAKE + 16) == 5
+
+
+def test_bwd_workspace_size_and_rejections(lib):
+    p, _ = problem(lib, total_tokens=300)
+    need = lib.hstu_attn_workspace_size(p, True)
+    # status + dO (bf16, T*H*dv) + dq accumulator (fp32, T*H*dqk)
+    assert need >= 256 + 300 * 4 * 128 * 2 + 300 * 4 * 128 * 4
+    so = lib.load_library()
+    vp = ctypes.c_void_p
+    args = [vp(FAKE)] * 12
+    # d_rab_pos requested without a position table
+    rc = so.hstu_attn_bwd(ctypes.byref(p), *args, vp(FAKE), None, vp(FAKE), need, None)
+    assert rc == 1
+    # missing saved statistics
+    a2 = list(args)
+    a2[6] = None
+    rc = so.hstu_attn_bwd(ctypes.byref(p), *a2, None, None, vp(FAKE), need, None)
+    assert rc == 1
+    rc = so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), need - 256, None)
+    assert rc == 5
+
+
+def test_check_and_selftest_reject_missing_workspace(lib):
+    so = lib.load_library()
+    assert so.hstu_attn_check(None, None) == 5
+    assert so.hstu_selftest_wait_timeout(None, 1000, None) == 5
+    assert so.hstu_selftest_wait_timeout(ctypes.c_void_p(FAKE), 0, None) == 1
+
+
+def test_empty_problem_is_a_no_op(lib):
+    p, _ = problem(lib, batch=0, total_tokens=0, max_seq_len=0, offsets=None)
+    assert call_fwd(lib, p) == 0

@@ -1,0 +1,66 @@
+"""GPU parity of the backward (through the C ABI) against the oracle's fp64
+analytic gradients: dQ, dK, dV, dU, d(rab_pos) and d(rab_time)."""
+import numpy as np
+import pytest
+
+import hstu_inputs as hi
+import oracle
+from tests.gpu_util import assert_close, np64, run_bwd, run_fwd
+
+pytestmark = pytest.mark.gpu
+
+
+def spec(lengths, H=4, d=128, dtype="bf16", pos=True, time=False, norm="own", norm_len=0,
+         qk_std=1 / np.sqrt(128), L=None):
+    return hi.Spec("case", dtype, batch=len(lengths), heads=H, d_qk=d, d_v=d,
+                   lengths=tuple(lengths), qk_std=qk_std, vu_std=1.0,
+                   rab_pos_len=(L or max(lengths)) if pos else 0, rab_time=time,
+                   norm=norm, norm_len=norm_len, grad=True)
+
+
+def check_bwd(inp, dtype, rows_of=None):
+    y, saved, dev = run_fwd(inp)
+    g = run_bwd(inp, dev, saved)
+    ref = oracle.bwd(inp)
+    for name in ("dq", "dk", "dv", "du"):
+        assert_close(np64(g[name]), ref[name], dtype, name)
+    if inp.rab_pos is not None:
+        assert_close(np64(g["d_rab_pos"]), ref["d_rab_pos"], dtype, "d_rab_pos")
+    if inp.rab_time is not None:
+        assert_close(np64(g["d_rab_time"]), ref["d_rab_time"], dtype, "d_rab_time")
+
+
+@pytest.mark.parametrize("case", [
+    dict(lengths=(40, 3), H=2, d=16, dtype="f32", time=True),
+    dict(lengths=(130,), H=3, d=64, dtype="f32", norm="fixed", norm_len=200),
+])
+def test_fp32_backward(case):
+    check_bwd(hi.make_inputs(spec(**case, qk_std=0.5), seed=11), "f32")
+
+
+@pytest.mark.parametrize("case", [
+    dict(lengths=(128,), H=1),
+    dict(lengths=(1, 200, 129), H=4, time=True),
+    dict(lengths=(300, 0, 64), H=2, norm="fixed", norm_len=300),
+])
+def test_bf16_backward_small(case):
+    check_bwd(hi.make_inputs(spec(**case), seed=12), "bf16")
+
+
+def test_train_reduced_batch():
+    """The training workload's shapes and distributions with 2 sequences."""
+    check_bwd(hi.make_inputs(hi.workload("train", batch=2), seed=0), "bf16")
+
+
+def test_train_full_size():
+    """Full training workload on the GPU; gradients of two whole sequences are
+    compared with the oracle run on those sequences alone (sequences are
+    independent), and d(rab_pos), a sum over all sequences, with the oracle
+    on the full problem."""
+    inp = hi.make_inputs(hi.WORKLOADS["train"], seed=0)
+    y, saved, dev = run_fwd(inp)
+    g = run_bwd(inp, dev, saved)
+    ref_full = oracle.bwd(inp)
+    for name in ("dq", "dk", "dv", "du"):
+        assert_close(np64(g[name]), ref_full[name], "bf16", name)
+    assert_close(np64(g["d_rab_pos"]), ref_full["d_rab_pos"], "bf16", "d_rab_pos")

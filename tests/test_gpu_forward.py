@@ -1,0 +1,156 @@
+"""GPU parity of the forward (CUDA path through the C ABI) against the fp64 oracle.
+
+Small problems span several 128-row tiles and ragged tails and are compared
+element by element on every output; the named workloads run at full size in
+the launch configuration the benchmark times, compared in full where the oracle
+is quick (tiny, neurarch) and on sampled rows otherwise (jagged, long, train).
+"""
+import numpy as np
+import pytest
+import torch
+
+import hstu_inputs as hi
+import oracle
+import pointwise_attention_b200 as pa
+from tests.gpu_util import assert_close, np64, run_fwd, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def spec(lengths, H=4, d=128, dtype="bf16", pos=True, time=False, norm="own", norm_len=0,
+         qk_std=1 / np.sqrt(128), rab_std=0.02, L=None, ts_sorted=True):
+    return hi.Spec("case", dtype, batch=len(lengths), heads=H, d_qk=d, d_v=d,
+                   lengths=tuple(lengths), qk_std=qk_std, vu_std=1.0,
+                   rab_pos_len=(L or max(max(lengths), 1)) if pos else 0, rab_time=time,
+                   rab_std=rab_std, norm=norm, norm_len=norm_len, ts_sorted=ts_sorted)
+
+
+def check_full(inp, dtype):
+    y, saved, _ = run_fwd(inp)
+    ref = oracle.fwd(inp)
+    assert_close(np64(y), ref["y"], dtype, "y")
+    assert_close(np64(saved[0]), ref["o"], dtype, "o_save")
+    return y, saved, ref
+
+
+def test_tiny_fp32_workload():
+    inp = hi.make_inputs(hi.WORKLOADS["tiny"], seed=0)
+    y, saved, ref = check_full(inp, "f32")
+    np.testing.assert_allclose(np64(saved[1]), ref["mean"], rtol=0, atol=1e-5 * np.abs(ref["mean"]).max() + 1e-12)
+    np.testing.assert_allclose(np64(saved[2]), ref["rstd"], rtol=1e-5)
+
+
+@pytest.mark.parametrize("case", [
+    dict(lengths=(128,), H=1),
+    dict(lengths=(256,), H=2, pos=False),
+    dict(lengths=(1, 127, 128, 129, 300), H=4),
+    dict(lengths=(513, 77), H=8, time=True),
+    dict(lengths=(200, 0, 385), H=4, time=True, norm="fixed", norm_len=500),
+    dict(lengths=(640,), H=3, time=True, L=1000),
+    dict(lengths=(260, 131), H=2, time=True, ts_sorted=False),
+    dict(lengths=(300, 257), H=4, qk_std=1.0, rab_std=1.0, time=True),   # stress: large logits
+])
+def test_bf16_small(case):
+    inp = hi.make_inputs(spec(**case), seed=1)
+    check_full(inp, "bf16")
+
+
+@pytest.mark.parametrize("case", [
+    dict(lengths=(5, 70, 130), H=2, d=32, dtype="f32", time=True),
+    dict(lengths=(64, 1), H=4, d=100, dtype="f32", pos=False, norm="fixed", norm_len=64),
+])
+def test_fp32_small(case):
+    inp = hi.make_inputs(spec(**case, qk_std=0.5), seed=2)
+    check_full(inp, "f32")
+
+
+def test_neurarch_full():
+    inp = hi.make_inputs(hi.WORKLOADS["neurarch"], seed=0)
+    check_full(inp, "bf16")
+
+
+def sampled_rows(inp, per_seq=3, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = []
+    for b, n in enumerate(inp.lengths):
+        s = int(inp.offsets[b])
+        if n == 0:
+            continue
+        picks = {0, n - 1} | set(rng.integers(0, n, size=per_seq).tolist())
+        rows += [s + i for i in sorted(picks)]
+    return np.array(rows, dtype=np.int64)
+
+
+@pytest.mark.parametrize("name", ["jagged", "long", "train"])
+def test_full_size_sampled(name):
+    inp = hi.make_inputs(hi.WORKLOADS[name], seed=0)
+    y, saved, _ = run_fwd(inp)
+    rows = sampled_rows(inp, per_seq=4 if name == "jagged" else 24)
+    ref = oracle.fwd_rows(inp, rows)
+    got = np64(y)[rows]
+    assert_close(got, ref["y"], "bf16", "y[%s]" % name)
+    assert_close(np64(saved[0])[rows], ref["o"], "bf16", "o[%s]" % name)
+    # LayerNorm statistics of the sampled rows
+    np.testing.assert_allclose(np64(saved[2])[rows], ref["rstd"], rtol=2e-2)
+
+
+def test_causality_on_gpu():
+    inp = hi.make_inputs(spec((700,), H=4, time=True), seed=3)
+    y0 = np64(run_fwd(inp, save=False)[0])
+    cut = 333
+    for name in ("q", "k", "v", "u"):
+        pert = hi.make_inputs(spec((700,), H=4, time=True), seed=3)
+        t = getattr(pert, name)
+        t[cut + 1:] = -t[cut + 1:]
+        y1 = np64(run_fwd(pert, save=False)[0])
+        assert np.array_equal(y1[:cut + 1], y0[:cut + 1]), name
+        assert not np.array_equal(y1[cut + 1:], y0[cut + 1:]), name
+
+
+def test_deterministic():
+    inp = hi.make_inputs(spec((900, 300), H=4, time=True), seed=4)
+    a = np64(run_fwd(inp)[0])
+    b = np64(run_fwd(inp)[0])
+    assert np.array_equal(a, b)
+
+
+def test_degenerate_shapes():
+    # empty sequences, single tokens, max_seq_len above every length
+    inp = hi.make_inputs(spec((0, 1, 0, 2, 129), H=2, time=True, L=400), seed=5)
+    dev = to_dev(inp)
+    y, saved = pa.hstu_attn_fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["offsets"], 400,
+                                timestamps=dev["timestamps"], rab_pos=dev["rab_pos"],
+                                rab_time=dev["rab_time"], save_for_backward=True)
+    torch.cuda.synchronize()
+    ref = oracle.fwd(inp)
+    assert_close(np64(y), ref["y"], "bf16", "y")
+    # a first token alone: O_0 = SiLU(q0.k0 + b)/1 * v0 exactly up to bf16 rounding of P
+    # all-empty problem: nothing to do
+    empty = hi.make_inputs(spec((0, 0), H=2), seed=6)
+    dev = to_dev(empty)
+    y, _ = pa.hstu_attn_fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["offsets"], 1,
+                            rab_pos=dev["rab_pos"])
+    torch.cuda.synchronize()
+    assert y.numel() == 0
+
+
+def test_bad_device_offsets_reported():
+    """Offsets that contradict max_seq_len, given without a host copy, are found
+    by the kernel: the sequence is skipped and the status word says so."""
+    inp = hi.make_inputs(spec((300, 100), H=2), seed=7)
+    dev = to_dev(inp)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    pa.hstu_attn_fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["offsets"], 200,
+                     rab_pos=None, workspace=ws)
+    assert pa.hstu_attn_check(ws) == 1
+    assert pa.hstu_attn_check(ws) == 0          # re-armed
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives():
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    assert pa.hstu_selftest_wait_timeout(ws, budget_ns=20_000_000) == 0
+    assert pa.hstu_attn_check(ws) == 4
+    assert pa.hstu_attn_check(ws) == 0
+    inp = hi.make_inputs(spec((200,), H=2), seed=8)
+    y, saved, _ = run_fwd(inp)
+    assert_close(np64(y), oracle.fwd(inp)["y"], "bf16", "y after timeout")
