@@ -96,7 +96,8 @@ __device__ __forceinline__ int time_bucket(long long dt, const long long* thr,
   int e = 63 - __clzll(static_cast<long long>(a));
   if (e > 62) e = 62;
   int k = first_k[e];
-  const long long aa = static_cast<long long>(a > 0x7FFFFFFFFFFFFFFFull ? 0x7FFFFFFFFFFFFFFFull : a);
+  // Clamp below the INT64_MAX sentinels that close the table after bucket NB-1.
+  const long long aa = static_cast<long long>(a > 0x7FFFFFFFFFFFFFFEull ? 0x7FFFFFFFFFFFFFFEull : a);
   k += (aa >= thr[k + 1]);
   k += (aa >= thr[k + 1]);
   k += (aa >= thr[k + 1]);
@@ -296,6 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_bar_sync(1, 128);
       if (ok) ok = mbar_wait(bar(B_SFULL + x), (n >> 1) & 1, abort_flag);
       if (ok && n >= 2) ok = mbar_wait(bar(B_PFREE + x), ((n - 2) >> 1) & 1, abort_flag);
+      // The TMEM loads/stores below are warp-collective: keep the decision warp-uniform.
+      ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
       const bool diag = (n == m);
@@ -332,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------- LayerNorm over heads + gate
     if (ok) ok = mbar_wait(bar(B_OFULL), 0, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
     if (!ok) {
       set_status(a.status, kStatusTimeout);
       *abort_flag = 1;
@@ -380,40 +384,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int hh = 0; hh < H; ++hh) totsq += red1[hh * 128 + r];
     const float var = totsq / static_cast<float>(D);
     const float rstd = 1.0f / sqrtf(var + a.eps);
-    // pass 3: normalise, gate, store
-    if (row_ok) {
-      const size_t rowD = static_cast<size_t>(t_row) * D + static_cast<size_t>(h) * 128;
-      const __nv_bfloat16* urow = reinterpret_cast<const __nv_bfloat16*>(a.u) + rowD;
-      __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(a.y) + rowD;
-      for (int cc = 0; cc < 4; ++cc) {
-        float v[32];
-        tmem_ld32(o_addr + 32u * cc, v);
-        tmem_wait_ld();
-        if (a.o_save) {
-          float4* od = reinterpret_cast<float4*>(a.o_save + rowD + 32 * cc);
+    // pass 3: normalise, gate, store.  The TMEM loads are warp-collective, so
+    // every lane issues them; only the global accesses depend on the row.
+    const size_t rowD = static_cast<size_t>(t_row) * D + static_cast<size_t>(h) * 128;
+    const __nv_bfloat16* urow = reinterpret_cast<const __nv_bfloat16*>(a.u) + rowD;
+    __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(a.y) + rowD;
+    for (int cc = 0; cc < 4; ++cc) {
+      float v[32];
+      tmem_ld32(o_addr + 32u * cc, v);
+      tmem_wait_ld();
+      if (!row_ok) continue;
+      if (a.o_save) {
+        float4* od = reinterpret_cast<float4*>(a.o_save + rowD + 32 * cc);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            od[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        }
-        const uint4* us = reinterpret_cast<const uint4*>(urow + 32 * cc);
-        uint4* yd = reinterpret_cast<uint4*>(yrow + 32 * cc);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint4 uu = __ldg(us + i);
-          const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&uu);
-          uint4 out;
-          uint32_t* o32 = reinterpret_cast<uint32_t*>(&out);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 uf = __bfloat1622float2(u2[j]);
-            const float y0 = (v[8 * i + 2 * j] - mean) * rstd * silu_precise(uf.x);
-            const float y1 = (v[8 * i + 2 * j + 1] - mean) * rstd * silu_precise(uf.y);
-            __nv_bfloat162 pr = __floats2bfloat162_rn(y0, y1);
-            o32[j] = *reinterpret_cast<uint32_t*>(&pr);
-          }
-          yd[i] = out;
-        }
+        for (int i = 0; i < 8; ++i)
+          od[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
       }
+      const uint4* us = reinterpret_cast<const uint4*>(urow + 32 * cc);
+      uint4* yd = reinterpret_cast<uint4*>(yrow + 32 * cc);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 uu = __ldg(us + i);
+        const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&uu);
+        uint4 out;
+        uint32_t* o32 = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 uf = __bfloat1622float2(u2[j]);
+          const float y0 = (v[8 * i + 2 * j] - mean) * rstd * silu_precise(uf.x);
+          const float y1 = (v[8 * i + 2 * j + 1] - mean) * rstd * silu_precise(uf.y);
+          __nv_bfloat162 pr = __floats2bfloat162_rn(y0, y1);
+          o32[j] = *reinterpret_cast<uint32_t*>(&pr);
+        }
+        yd[i] = out;
+      }
+    }
+    if (row_ok) {
       if (h == 0 && a.ln_mean) {
         a.ln_mean[t_row] = mean;
         a.ln_rstd[t_row] = rstd;
