@@ -411,11 +411,13 @@ def run_gpu(args, spec):
     elapsed_max = reduce_max(elapsed, world, device)
     wl.check()
 
-    value = flops_step * world / elapsed_max / 1e12
+    value = flops_step * args.steps * world / elapsed_max / 1e12
     peaks, peak_kind = load_peaks()
     sec_per_step = elapsed / args.steps
     # Roofline of the dominant kernel (the forward for forward workloads).
     bytes_launch = algorithmic_bytes(inp)
+    # One forward launch per step, replayed back to back from the graph: the
+    # average launch duration is the timed region over the number of steps.
     t_launch = sec_per_step if not train else None
     roof = None
     if t_launch is not None:
