@@ -141,6 +141,33 @@ HSTU_API int32_t hstu_time_bucket_thresholds(int64_t *out, int32_t num_buckets);
 HSTU_API hstu_status_t hstu_selftest_wait_timeout(void *workspace, uint64_t budget_ns,
                                                   void *stream);
 
+/*
+ * Backward without a caller-provided workspace.  The pages define no such
+ * call; it exists for callers that cannot allocate device memory themselves
+ * (for example when another allocator already owns the free device memory,
+ * or a host framework forbids direct CUDA allocation).
+ *
+ * Same arguments, results and synchronous errors as hstu_attn_bwd, minus the
+ * workspace: the scratch lives in a fixed 16 MiB array in device global memory
+ * that the library reserves on every device it is loaded on and keeps until
+ * the process exits.  Problems whose backward workspace
+ * (hstu_attn_workspace_size(p, 1)) is larger return HSTU_ERR_WORKSPACE before
+ * anything is enqueued.  The function calls no allocation routine.  The first
+ * call on a device looks up the array's device address (with that device
+ * current) and caches it.  All calls share the one array: calls that may
+ * overlap on the GPU (different streams, no ordering between them) race on it
+ * and must be serialised by the caller.  Each call clears the device status
+ * word at the start of the array; device-side findings (offsets contradicting
+ * the sizes, an expired wait) stay in that word and are not reported by this
+ * entry point, so pass offsets_host to have the offsets checked on the host.
+ */
+HSTU_API hstu_status_t hstu_attn_bwd_noalloc(const hstu_problem_t *p, const void *dy,
+                                             const void *q, const void *k, const void *v,
+                                             const void *u, const float *o_save,
+                                             const float *ln_mean, const float *ln_rstd,
+                                             void *dq, void *dk, void *dv, void *du,
+                                             float *d_rab_pos, float *d_rab_time, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

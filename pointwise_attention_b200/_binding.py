@@ -22,7 +22,8 @@ HSTU_ERR_CUDA, HSTU_ERR_TIMEOUT, HSTU_ERR_WORKSPACE = 3, 4, 5
 HSTU_F32, HSTU_BF16 = 0, 1
 
 EXPORTED = ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_attn_check",
-            "hstu_status_string", "hstu_time_bucket_thresholds", "hstu_selftest_wait_timeout")
+            "hstu_status_string", "hstu_time_bucket_thresholds", "hstu_selftest_wait_timeout",
+            "hstu_attn_bwd_noalloc")
 
 
 class HSTUError(RuntimeError):
@@ -80,6 +81,8 @@ def load_library():
     lib.hstu_time_bucket_thresholds.restype = ctypes.c_int32
     lib.hstu_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
     lib.hstu_selftest_wait_timeout.restype = ctypes.c_int
+    lib.hstu_attn_bwd_noalloc.argtypes = [P] + [vp] * 5 + [vp] * 3 + [vp] * 4 + [vp] * 2 + [vp]
+    lib.hstu_attn_bwd_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
