@@ -288,7 +288,7 @@ class Workload:
                                   d_rab_time=(torch.empty_like(d["rab_time"])
                                               if d["rab_time"] is not None else None))
             self.sets.append(d)
-        self.launches_per_step = 1 if not train else 1 + 3   # forward; LN/gate, dQ, dK/dV backward
+        self.launches_per_step = 1 if not train else 1 + 3   # forward; LN/gate, dQ, dK/dV backward kernels
 
     def step(self, i: int, stream=None):
         d, inp, pa = self.sets[i % self.R], self.inp, self.pa

@@ -139,9 +139,9 @@ bool f32_supported(const hstu_problem_t* p) {
          p->num_heads * p->d_v <= 1024;
 }
 
-// Workspace layout: [status 256 B][dO: T*H*dv dtype][dq_acc: T*H*dqk fp32]
+// Workspace layout: [status 256 B][dO: T*H*dv in the input dtype] (backward)
 struct WsLayout {
-  size_t dO_off, dq_off, total;
+  size_t dO_off, total;
 };
 
 WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
@@ -151,8 +151,6 @@ WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
     const size_t T = static_cast<size_t>(p->total_tokens);
     l.dO_off = off;
     off += align_up(T * p->num_heads * p->d_v * (p->dtype == HSTU_BF16 ? 2 : 4));
-    l.dq_off = off;
-    if (p->dtype == HSTU_BF16) off += align_up(T * p->num_heads * p->d_qk * 4);
   }
   l.total = off;
   return l;
@@ -298,7 +296,6 @@ hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void*
   a.dq = dq; a.dk = dk; a.dv = dv; a.du = du;
   a.d_rab_pos = d_rab_pos; a.d_rab_time = d_rab_time;
   a.dO = ws + l.dO_off;
-  a.dq_acc = p->dtype == HSTU_BF16 ? reinterpret_cast<float*>(ws + l.dq_off) : nullptr;
   a.status = common.status;
   a.B = common.B; a.T = common.T; a.H = common.H; a.d_qk = common.d_qk; a.d_v = common.d_v;
   a.max_seq_len = common.max_seq_len; a.max_tiles = common.max_tiles;
@@ -306,7 +303,14 @@ hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void*
   a.bt = common.bt;
   cudaError_t err;
   if (p->dtype == HSTU_BF16) {
-    err = launch_bwd_bf16_simt(a, s);
+    CUtensorMap maps[4];
+    if (!make_map_3d(&maps[0], q, p->total_tokens, p->num_heads, 128) ||
+        !make_map_3d(&maps[1], k, p->total_tokens, p->num_heads, 128) ||
+        !make_map_3d(&maps[2], v, p->total_tokens, p->num_heads, 128) ||
+        !make_map_3d(&maps[3], a.dO, p->total_tokens, p->num_heads, 128))
+      return HSTU_ERR_CUDA;
+    err = launch_bwd_pre_bf16(a, s);                       // dU and dO (LayerNorm + gate)
+    if (err == cudaSuccess) err = launch_bwd_attn_bf16_sm100(a, maps, s);   // dQ, dK, dV, d_rab
   } else {
     err = launch_bwd_f32_simt(a, s);
   }

@@ -65,7 +65,6 @@ struct BwdArgs {
   float* d_rab_pos;
   float* d_rab_time;
   void* dO;          // workspace: dO in the compute dtype [T, H*d_v]
-  float* dq_acc;     // workspace: fp32 [T, H, d_qk] (bf16 path)
   int* status;
   int B, T, H, d_qk, d_v;
   int max_seq_len;
@@ -84,5 +83,7 @@ cudaError_t launch_fwd_f32_simt(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_f32_simt(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_bf16_simt(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_pre_bf16(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd_attn_bf16_sm100(const BwdArgs& a, const CUtensorMap* maps,
+                                       cudaStream_t stream);
 
 }  // namespace hstu
