@@ -64,13 +64,12 @@ __device__ __forceinline__ void mma_tile_tm(uint32_t d, uint32_t a_tmem, uint32_
            (accumulate || ks > 0) ? 1u : 0u);
 }
 
-// x = S + bias -> (P' = SiLU(x), G = SiLU'(x)) with one tanh.
-__device__ __forceinline__ void silu_and_grad(float x, float* p, float* g) {
-  const float hx = 0.5f * x;
-  const float t = tanh_approx(hx);
-  const float sg = fmaf(0.5f, t, 0.5f);             // sigma(x)
-  *p = hx + hx * t;                                 // x sigma(x)
-  *g = sg * fmaf(x, 1.0f - sg, 1.0f);               // sigma(x) (1 + x (1 - sigma(x)))
+// From hx = (S + bias)/2 and t = tanh(hx):
+//   sigma(x) = (1 + t)/2,  P' = SiLU(x) = hx (1 + t),
+//   SiLU'(x) = sigma(x) (1 + x (1 - sigma(x))) = sigma(x) (1 + hx (1 - t)).
+__device__ __forceinline__ float silu_grad_h(float hx, float t) {
+  const float sg = fmaf(t, 0.5f, 0.5f);
+  return sg * fmaf(hx, 1.0f - t, 1.0f);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -79,7 +78,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 // Per-warp staging of one 32 x 32 block: 63 position-bias diagonals (fp32,
-// full value) and the 32 column timestamps.
+// halved) and the 32 column timestamps.
 struct Stage {
   float w[64];
   long long ts[32];
@@ -129,6 +128,100 @@ __device__ __forceinline__ ChunkT chunk_time(long long my_ts, const long long* k
     }
   }
   return c;
+}
+
+// dS' of one 32-column chunk of the dQ kernel (rows = queries, columns =
+// keys), its bf16 packing, and the bias-gradient accumulation.  MASK: the
+// tile holds the diagonal or rows past the sequence end.
+template <bool POS, bool TIME, bool MASK>
+__device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
+                                         const Stage* stg, int lane, int r, int c0, bool diag,
+                                         bool row_ok, const ChunkT& ct, bool generic,
+                                         long long my_ts, const long long* thr,
+                                         const signed char* first, const float* rabt, float* win,
+                                         float* s_dt, uint32_t (&packed)[16], float& t_lo,
+                                         float& t_hi) {
+  // Diagonal sums of the warp's 32 x 32 block without per-element atomics:
+  // at column cl lane L reads column cl of lane (L + cl) mod 32, so every
+  // element of diagonal L (row - column = L) or L - 32 passes through lane L.
+  float dpos = 0.f, dneg = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float ds2[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int cl = 2 * i + hh;
+      const int c = c0 + cl;
+      float hb = POS ? stg->w[lane - cl + 31] : 0.f;
+      int kb = 0;
+      if (TIME) {
+        kb = generic ? time_bucket(my_ts - stg->ts[cl], thr, first)
+                     : ((cl < ct.split) ? ct.klo : ct.khi);
+        hb += rabt[kb];
+      }
+      const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
+      const float t = tanh_approx(hx);
+      float ds = __uint_as_float(dav[cl]) * silu_grad_h(hx, t);
+      if (MASK && ((diag && c > r) || !row_ok)) ds = 0.f;
+      ds2[hh] = ds;
+      if (POS) {
+        const float v = __shfl_sync(0xffffffffu, ds, (lane + cl) & 31);
+        if (lane + cl < 32) dpos += v; else dneg += v;
+      }
+      if (TIME) {
+        if (!generic) {
+          if (cl < ct.split) t_lo += ds; else t_hi += ds;
+        } else {
+          atomicAdd(&s_dt[kb], ds);
+        }
+      }
+    }
+    packed[i] = pack_bf16(ds2[0], ds2[1]);
+  }
+  if (POS) {
+    // lane L holds diagonal L (window index r - c0 + 127 for this row's lane)
+    // and diagonal L - 32 (index 32 lower); the latter is empty for lane 0.
+    atomicAdd(&win[r - c0 + 127], dpos);
+    if (lane > 0) atomicAdd(&win[r - c0 + 95], dneg);
+  }
+}
+
+// P'^T and dS'^T of one 32-column chunk of the dK/dV kernel (rows = keys,
+// columns = queries).  MASK: the diagonal tile or the sequence's last query tile.
+template <bool POS, bool TIME, bool MASK>
+__device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
+                                          const Stage* stg, int lane, int r, int c0, bool diag,
+                                          int qlim, const ChunkT& ct, bool generic,
+                                          long long my_ts, const long long* thr,
+                                          const signed char* first, const float* rabt,
+                                          uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float p2[2], d2[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int cl = 2 * i + hh;
+      const int c = c0 + cl;
+      float hb = POS ? stg->w[cl - lane + 31] : 0.f;
+      if (TIME) {
+        const int kb = generic ? time_bucket(stg->ts[cl] - my_ts, thr, first)
+                               : ((cl < ct.split) ? ct.klo : ct.khi);
+        hb += rabt[kb];
+      }
+      const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
+      const float t = tanh_approx(hx);
+      float p = fmaf(hx, t, hx);
+      float ds = __uint_as_float(dav[cl]) * silu_grad_h(hx, t);
+      if (MASK && ((diag && c < r) || c >= qlim)) {
+        p = 0.f;
+        ds = 0.f;
+      }
+      p2[hh] = p;
+      d2[hh] = ds;
+    }
+    pk[i] = pack_bf16(p2[0], p2[1]);
+    dk[i] = pack_bf16(d2[0], d2[1]);
+  }
 }
 
 // ===================================================================== dQ
@@ -212,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (TIME) {
       for (int i = et; i < kThrLen; i += kEpi) s_thr[i] = a.bt.thr[i];
       if (et < 64) s_first[et] = a.bt.first_k[et];
-      if (et < a.nb) s_rabt[et] = __ldg(a.rab_time + static_cast<size_t>(h) * a.nb + et);
+      if (et < a.nb) s_rabt[et] = 0.5f * __ldg(a.rab_time + static_cast<size_t>(h) * a.nb + et);
       if (et < 128) s_dt[et] = 0.f;
     }
   }
@@ -329,8 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool sorted = true;
     auto stage = [&]() {
       if (POS) {
-        stg->w[lane] = pw0;
-        stg->w[32 + lane] = pw1;
+        stg->w[lane] = 0.5f * pw0;
+        stg->w[32 + lane] = 0.5f * pw1;
       }
       if (TIME) {
         stg->ts[lane] = pt;
@@ -365,40 +458,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float t_lo = 0.f, t_hi = 0.f;      // d_rab_time partial sums (simple path)
         uint32_t packed[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float ds2[2];
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int cl = 2 * i + hh;
-            const int c = 32 * cq + cl;
-            float x = __uint_as_float(sv[cl]);
-            if (POS) x += stg->w[lane - cl + 31];
-            int kb = 0;
-            if (TIME) {
-              if (!generic) {
-                kb = (cl < ct.split) ? ct.klo : ct.khi;
-              } else {
-                kb = time_bucket(my_ts - stg->ts[cl], s_thr, s_first);
-              }
-              x += s_rabt[kb];
-            }
-            float p, g;
-            silu_and_grad(x, &p, &g);
-            float ds = __uint_as_float(dav[cl]) * g;
-            if ((diag && c > r) || !row_ok) ds = 0.f;
-            ds2[hh] = ds;
-            if (POS) atomicAdd(&win[r - c + 127], ds);
-            if (TIME) {
-              if (!generic) {
-                if (cl < ct.split) t_lo += ds; else t_hi += ds;
-              } else {
-                atomicAdd(&s_dt[kb], ds);
-              }
-            }
-          }
-          packed[i] = pack_bf16(ds2[0], ds2[1]);
-        }
+        if (diag || !__all_sync(0xffffffffu, row_ok))
+          dq_chunk<POS, TIME, true>(sv, dav, stg, lane, r, 32 * cq, diag, row_ok, ct, generic,
+                                    my_ts, s_thr, s_first, s_rabt, win, s_dt, packed, t_lo, t_hi);
+        else
+          dq_chunk<POS, TIME, false>(sv, dav, stg, lane, r, 32 * cq, diag, row_ok, ct, generic,
+                                     my_ts, s_thr, s_first, s_rabt, win, s_dt, packed, t_lo,
+                                     t_hi);
         if (TIME && !generic) {
           if (t_lo != 0.f) atomicAdd(&s_dt[ct.klo], t_lo);
           if (t_hi != 0.f) atomicAdd(&s_dt[ct.khi], t_hi);
@@ -532,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 64;
     for (int i = et; i < kThrLen; i += kEpi) s_thr[i] = a.bt.thr[i];
     if (et < 64) s_first[et] = a.bt.first_k[et];
-    if (et < a.nb) s_rabt[et] = __ldg(a.rab_time + static_cast<size_t>(h) * a.nb + et);
+    if (et < a.nb) s_rabt[et] = 0.5f * __ldg(a.rab_time + static_cast<size_t>(h) * a.nb + et);
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
@@ -642,8 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool sorted = true;
     auto stage = [&]() {
       if (POS) {
-        stg->w[lane] = pw0;
-        stg->w[32 + lane] = pw1;
+        stg->w[lane] = 0.5f * pw0;
+        stg->w[32 + lane] = 0.5f * pw1;
       }
       if (TIME) {
         stg->ts[lane] = pt;
@@ -676,34 +742,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ct = chunk_time<+1>(my_ts, stg->ts, sorted, s_thr, s_first);
           generic = !__all_sync(0xffffffffu, ct.simple);
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float p2[2], d2[2];
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int cl = 2 * i + hh;
-            const int c = 32 * cq + cl;
-            float x = __uint_as_float(sv[cl]);
-            if (POS) x += stg->w[cl - lane + 31];
-            if (TIME) {
-              int kb;
-              if (!generic) kb = (cl < ct.split) ? ct.klo : ct.khi;
-              else kb = time_bucket(stg->ts[cl] - my_ts, s_thr, s_first);
-              x += s_rabt[kb];
-            }
-            float p, g;
-            silu_and_grad(x, &p, &g);
-            float ds = __uint_as_float(dav[cl]) * g;
-            if ((diag && c < r) || c >= qlim) {
-              p = 0.f;
-              ds = 0.f;
-            }
-            p2[hh] = p;
-            d2[hh] = ds;
-          }
-          pk[i] = pack_bf16(p2[0], p2[1]);
-          dk[i] = pack_bf16(d2[0], d2[1]);
-        }
+        if (diag || qlim < 128)
+          dkv_chunk<POS, TIME, true>(sv, dav, stg, lane, r, 32 * cq, diag, qlim, ct, generic,
+                                     my_ts, s_thr, s_first, s_rabt, pk, dk);
+        else
+          dkv_chunk<POS, TIME, false>(sv, dav, stg, lane, r, 32 * cq, diag, qlim, ct, generic,
+                                      my_ts, s_thr, s_first, s_rabt, pk, dk);
       }
       // Every warp has read its S^T / dA^T columns before any is overwritten.
       named_bar_sync(1, kEpi);
