@@ -83,6 +83,10 @@ typedef struct {
  * Bytes of device workspace the call needs (is_bwd = 0: forward; 1: backward).
  * The workspace must be 256-byte aligned and zero-filled before its first use;
  * its first word is the device status that hstu_attn_check reads and re-arms.
+ * Words 16 and 17 hold the bf16 forward's work counters: each launch hands its
+ * (sequence, query tile) items out through them and the last cluster to
+ * finish returns them to zero.  Calls that share a workspace must therefore
+ * run one after another (same stream or ordered by events), never overlapped.
  */
 HSTU_API size_t hstu_attn_workspace_size(const hstu_problem_t *p, int is_bwd);
 
@@ -90,8 +94,9 @@ HSTU_API size_t hstu_attn_workspace_size(const hstu_problem_t *p, int is_bwd);
  * Forward.  q, k, v, u: inputs (dtype, layouts above, 16-byte aligned).
  * y: output [T, H*d_v] (dtype).  o_save [T, H*d_v], ln_mean [T], ln_rstd [T]:
  * optional fp32 outputs kept for the backward (all three or none; NULL = skip).
- * Supported: bf16 with d_qk = d_v = 128 and 1 <= H <= 8 (tcgen05 path);
- * fp32 with d_qk, d_v <= 128 and H*d_v <= 1024 (true-fp32 SIMT path).
+ * Supported: bf16 with d_qk = d_v = 128, 1 <= H <= 8 and batch times
+ * ceil(max_seq_len / 128) below 2^31 - 256 (tcgen05 path); fp32 with
+ * d_qk, d_v <= 128 and H*d_v <= 1024 (true-fp32 SIMT path).
  */
 HSTU_API hstu_status_t hstu_attn_fwd(const hstu_problem_t *p, const void *q, const void *k,
                             const void *v, const void *u, void *y, float *o_save,

@@ -1,7 +1,7 @@
 // fwd_sm100.cu -- bf16 forward of HSTU causal pointwise aggregated attention
 // on sm_100a: TMA-staged Q/K/V tiles, tcgen05 MMAs with TMEM accumulators,
-// a register epilogue for bias + SiLU + 1/N + causal mask between the two
-// MMAs, and the LayerNorm-over-heads + SiLU(U) gate fused into the store.
+// a register epilogue for bias + SiLU + causal mask between the two MMAs,
+// and the LayerNorm-over-heads + SiLU(U) gate fused into the store.
 //
 // Operation: "HSTU (Generative Recommender)" model card, Exported PyTorch,
 // HSTUBlock.forward (silu(q k^T)/t, tril, attn @ v, gate by silu(u));
@@ -9,32 +9,45 @@
 // Units", §1 and §3; post-pooling normalisation then U gate: the HSTU
 // reproduction note's flowchart.
 //
-// Work decomposition.  One CTA computes one (sequence b, query tile m, head h):
-// 128 query rows against key tiles n = 0..m (tiles above the diagonal are
-// skipped; only the diagonal tile is masked).  The H CTAs of one (b, m) form a
-// thread-block cluster so the LayerNorm over the concatenated heads can
-// exchange per-row partial sums through distributed shared memory (st.async).
-// Clusters enumerate (m descending, b), so the CTAs with the most key tiles are
-// dispatched first (the cost of a tile depends on m only).
+// Work decomposition.  A work item is one (sequence b, query tile m): 128
+// query rows against key tiles n = 0..m (tiles above the diagonal are skipped;
+// only the diagonal tile is masked), for all H heads.  The H CTAs of a
+// thread-block cluster take one head each, so the LayerNorm over the
+// concatenated heads exchanges per-row statistics through distributed shared
+// memory.  The kernel is persistent: the grid holds as many clusters as can
+// be resident, and each cluster loops over items that its leader CTA (rank 0)
+// claims from a work counter in global memory.  Items are numbered from the
+// most expensive (largest m) down, so the claims form a longest-first list
+// schedule; slots whose tile lies past the end of its sequence are skipped in
+// runs of up to 32 per claim.  The leader claims the next item once its loads
+// for the current item are issued and hands it to every CTA of the cluster
+// through an 8-entry ring in shared memory.  While the epilogue normalises
+// item j, the TMA and MMA warps already load and multiply item j+1.
 //
-// Roles (576 threads): warp 0 issues TMA, warp 1 allocates TMEM and issues the
-// MMAs (one thread), warps 2..17 form the epilogue in two teams of 8 warps:
-// team t = (w-2)/8 turns the S tiles n = t, t+2, t+4, ... (S buffer t) into P,
-// so the two teams overlap each other's waits; warp w owns TMEM lane quarter
-// w%4 (rows 32*(w%4) ..) and column half ((w-2)/4)%2 (64 columns) of its team's
-// tiles.  Each warp stages the position-bias diagonals and key timestamps of
-// its own 32x64 block in a private buffer, fetched from global memory one tile
-// ahead.  Waiting on S(n) also covers P buffer reuse: the MMA thread commits
-// S(n) after issuing P(n-2).V, and a commit tracks every earlier MMA.
+// Roles (640 threads): warp 0 issues TMA (and, in the leader, claims items);
+// warp 1 allocates TMEM and issues the S = Q K^T MMAs; warp 18 issues the
+// O += P V MMAs; warps 2..17 form the epilogue: warp w owns TMEM lane quarter
+// w%4 (rows 32*(w%4) ..) and the 32 columns (w-2)/4 of every tile.  Each warp
+// stages the position-bias diagonals and key timestamps of its own 32x32
+// block in a private buffer, fetched from global memory one tile ahead.  A
+// tcgen05.mma instruction costs its issuing thread about 110 cycles whatever
+// its N up to 128, about as long as the tensor core needs for 128x128x16, so
+// the two GEMMs of a tile are issued by two threads in parallel.
 //
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O [256,384) P0 [384,448)
-// P1 [448,512).  S = Q K^T is fp32; P' = SiLU(S+bias) is packed bf16 pairs and
-// is the A operand (from TMEM) of O' += P' V; O = O' / N in the epilogue.
+// TMEM (512 columns): three S/P buffers [0,128) [128,256) [256,384) and O
+// [384,512).  S(x) = Q K^T lands in buffer x % 3 in fp32; the epilogue writes
+// P' = SiLU(S+bias) over it as packed bf16 pairs (each warp only over columns
+// it has already read: its 32 keys take 16 columns), and P' is the A operand
+// (from TMEM) of O' += P' V; O = O' / N in the epilogue.  S(x+3) reuses the
+// buffer once P(x).V has completed; with three buffers S(x+1) and S(x+2) are
+// computed while the epilogue is on tile x.
 //
 // Every tcgen05.ld/st is warp-collective (.sync.aligned): they are issued by
 // all 32 lanes with warp-uniform control flow; only global accesses are
 // predicated per row.
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -43,7 +56,7 @@
 namespace hstu {
 namespace {
 
-constexpr int kThreads = 576;
+constexpr int kThreads = 640;
 constexpr int kEpiThreads = 512;
 constexpr int kColGroups = 4;               // epilogue warpgroups, 32 columns each
 constexpr int kRows = 128;                  // query rows per tile
@@ -52,38 +65,57 @@ constexpr int kHalf = 16384;                // 128 rows x 64 bf16 (one 128B-swiz
 constexpr int kTile = 2 * kHalf;            // 128 x 128 bf16
 constexpr int kKStages = 3;                 // K tiles in flight (S = Q K^T needs them first)
 constexpr int kVStages = 2;                 // V tiles in flight (P.V comes a tile later)
+constexpr int kRing = 8;                    // claimed items handed to the cluster, in flight
+constexpr int kMaxHeads = 8;
 
 // shared-memory map (byte offsets from a 1024-aligned base)
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kTile;                    // kKStages tiles
 constexpr int kOffV = kOffK + kKStages * kTile;         // kVStages tiles
-// Per epilogue warp: 96 fp32 half position-bias values (the 95 diagonals its
-// 32x64 block touches) and 64 int64 key timestamps.
-constexpr int kWarpStage = 96 * 4 + 64 * 8;             // bytes per warp
+// Per epilogue warp: the half position bias of the 63 diagonals its 32x32
+// block touches, as 64 overlapping bf16 pairs (entry k holds diagonals k and
+// k-1, the two an element pair needs), and 32 int64 key timestamps.
+constexpr int kWarpStage = 64 * 4 + 32 * 8;             // bytes per warp
 constexpr int kOffWarp = kOffV + kVStages * kTile;
+// LayerNorm partials of the four column groups, [4][128] (sum, M2) pairs.  They
+// alias the staging buffers, which are idle between an item's last tile and
+// the next item's first.
+constexpr int kOffLoc = kOffWarp;
 constexpr int kOffThr = kOffWarp + 16 * kWarpStage;     // kThrLen int64 thresholds
 constexpr int kOffFirst = kOffThr + kThrLen * 8;        // 64 int8 first bucket per octave
 constexpr int kOffRabT = kOffFirst + 64;                // 128 fp32 half time-bias row
-// LayerNorm reduction: per round, [4 column groups][128 rows] local partials
-// and [8 heads][128 rows] cluster exchange slots.
+// Cluster exchange slots of the per-head row statistics: [2 item parities]
+// [kMaxHeads][128 rows] (sum, M2) pairs.
 constexpr int kOffRed = kOffRabT + 128 * 4;
-constexpr int kRedBytes = 2 * (kColGroups * 128 + 8 * 128) * 4;
-constexpr int kOffBar = kOffRed + kRedBytes;            // mbarriers (8 B each)
-constexpr int kNumBars = 16;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;        // tmem base, abort flag, 2 LN barriers
+constexpr int kRedBytes = 2 * kMaxHeads * 128 * 8;
+constexpr int kOffRing = kOffRed + kRedBytes;           // kRing (m, b) pairs
+constexpr int kOffBar = kOffRing + kRing * 8;           // mbarriers (8 B each)
+constexpr int kNumBars = 41;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;        // tmem base, abort flag
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;        // + alignment slack
+static_assert(16 * kWarpStage >= kColGroups * 128 * 8, "LayerNorm partials must fit the staging");
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 // barrier indices
 constexpr int B_QFULL = 0;
-constexpr int B_KFULL = 1;    // +K stage
-constexpr int B_KEMPTY = 4;   // +K stage
-constexpr int B_VFULL = 7;    // +V stage
-constexpr int B_VEMPTY = 9;   // +V stage
-constexpr int B_SFULL = 11;   // +buffer
-constexpr int B_PFULL = 13;   // +buffer
-constexpr int B_OFULL = 15;
+constexpr int B_QEMPTY = 1;
+constexpr int B_KFULL = 2;    // +K stage
+constexpr int B_KEMPTY = 5;   // +K stage
+constexpr int B_VFULL = 8;    // +V stage
+constexpr int B_VEMPTY = 10;  // +V stage
+constexpr int kSBufs = 3;     // S/P buffers in TMEM
+constexpr int B_SFULL = 12;   // +buffer: S(x) computed
+constexpr int B_PFULL = 15;   // +buffer: P(x) written over S(x)
+constexpr int B_PVDONE = 18;  // +buffer: P(x).V completed, the buffer may be rewritten
+constexpr int B_OFULL = 21;
+constexpr int B_DONE = 22;    // every MMA of both issuers has completed
+constexpr int B_RED = 23;     // +item parity: LayerNorm statistics of all heads arrived
+constexpr int B_RFULL = 25;   // +ring slot: item written
+constexpr int B_REMPTY = 33;  // +ring slot (leader only): every CTA has read the item
+static_assert(B_REMPTY + kRing <= kNumBars, "barrier count");
 constexpr int kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColP0 = 384;
+constexpr uint32_t kColS0 = 0, kColO = 384;
+constexpr int kWarpPV = 18;   // warp of the P.V issuer
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);   // Q (K-major) x K (K-major)
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);   // P (TMEM) x V (MN-major)
@@ -93,7 +125,8 @@ __device__ __forceinline__ void set_status(int* status, int bit) {
 }
 
 struct EpiCtx {
-  const float* win;           // warp's half position bias: element (lane, cl) -> win[lane - cl + 31]
+  const uint32_t* wpk;        // warp's half position bias pairs: element pair (lane, 2i, 2i+1)
+                              // -> wpk[lane - 2i] = (diag of col 2i, diag of col 2i+1)
   const long long* kts;       // warp's 32 key timestamps
   const long long* thr;       // bucket thresholds
   const signed char* first;   // first bucket per octave
@@ -165,11 +198,16 @@ __device__ __forceinline__ void chunk_to_p(const uint32_t (&sraw)[32], int c0, c
                                            const ChunkTime& ct, uint32_t (&packed)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    float hx[2];
+    float hx[2], hbp[2] = {0.f, 0.f};
+    if (POS) {
+      const uint32_t w = e.wpk[e.lane - 2 * i];
+      hbp[0] = __uint_as_float(w << 16);
+      hbp[1] = __uint_as_float(w & 0xFFFF0000u);
+    }
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int cl = 2 * i + hh;
-      float hb = POS ? e.win[e.lane - cl + 31] : 0.f;
+      float hb = hbp[hh];
       if (MODE == 1) hb += ct.lo;
       if (MODE == 2) hb += (cl < ct.split) ? ct.hi : ct.lo;
       if (MODE == 3) hb += e.rabt[time_bucket(e.my_ts - e.kts[cl], e.thr, e.first)];
@@ -204,30 +242,75 @@ __device__ __forceinline__ void chunk_p(const uint32_t (&sv)[32], int c0, const 
   }
 }
 
-// This thread's 64 columns (col0 .. col0+63) of the S tile -> P in TMEM.
-// `wv` holds the warp's 96 staged diagonals, `kts` its 64 key timestamps.
+// This thread's 32 columns (col0 .. col0+31) of the S tile -> P in TMEM,
+// packed into columns col0 .. col0+15 of the same buffer (already read).
+// `wpk` holds the warp's 64 staged diagonal pairs, `kts` its 32 key timestamps.
 template <bool POS, bool TIME, bool DIAG>
-__device__ __forceinline__ void tile_to_p(uint32_t s_addr, uint32_t p_addr, int col0,
-                                          EpiCtx& e, const float* wv, const long long* kts,
-                                          bool sorted0, bool sorted1) {
+__device__ __forceinline__ void chunk_to_tmem(uint32_t s_addr, int col0, EpiCtx& e,
+                                              const uint32_t* wpk, const long long* kts,
+                                              bool sorted) {
   uint32_t sv[32];
   uint32_t packed[16];
-  // chunk 0: element (lane, cl) uses diagonal index lane - cl + 63
   tmem_ld32_nowait(s_addr + col0, sv);
   tmem_wait_ld_dep(sv);
-  e.win = wv + 32;
+  // element (lane, cl) uses diagonal index lane - cl + 31
+  e.wpk = wpk + 31;
   e.kts = kts;
-  e.chunk_sorted = sorted0;
+  e.chunk_sorted = sorted;
   chunk_p<POS, TIME, DIAG>(sv, col0, e, packed);
-  tmem_st16(p_addr + col0 / 2, packed);
-  // chunk 1: index lane - cl + 31
-  tmem_ld32_nowait(s_addr + col0 + 32, sv);
-  tmem_wait_ld_dep(sv);
-  e.win = wv;
-  e.kts = kts + 32;
-  e.chunk_sorted = sorted1;
-  chunk_p<POS, TIME, DIAG>(sv, col0 + 32, e, packed);
-  tmem_st16(p_addr + col0 / 2 + 16, packed);
+  tmem_st16(s_addr + col0, packed);
+}
+
+// SiLU of the gate input through tanh: x/2 (1 + tanh(x/2)).
+__device__ __forceinline__ float silu_gate(float x) {
+  const float hx = 0.5f * x;
+  return fmaf(hx, tanh_approx(hx), hx);
+}
+
+// Start and length of sequence b; inconsistent offsets give length -1.
+__device__ __forceinline__ int2 load_seq(const FwdArgs& a, int b, bool pos) {
+  const int s = __ldg(a.offsets + b);
+  const int e = __ldg(a.offsets + b + 1);
+  const int n = e - s;
+  if (s < 0 || n < 0 || e > a.T || n > a.max_seq_len || (pos && n > a.L)) return make_int2(0, -1);
+  return make_int2(s, n);
+}
+
+// Claims this cluster's next item (warp-collective; leader CTA's warp 0).
+// Slot k of the launch is the item (m = M-1 - k/B, b = k mod B), so the most
+// expensive query tiles come first.  The counter holds the next free slot and
+// an atomic add claims one.  A slot whose tile lies past its sequence end
+// holds no work: the warp then tests the 31 slots after it and raises the
+// counter past the empty ones among them (atomicMax; every skipped slot was
+// seen empty, and no slot is handed out twice), then claims again.  Returns
+// (-1, -1) once the slots are exhausted.
+template <bool POS>
+__device__ int2 claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots, int lane) {
+  const unsigned B = static_cast<unsigned>(a.B);
+  const int M = a.max_tiles;
+  for (;;) {
+    unsigned k = 0;
+    if (lane == 0) k = atomicAdd(counter, 1u);
+    k = __shfl_sync(0xffffffffu, k, 0);
+    if (k >= nslots) return make_int2(-1, -1);
+    const unsigned slot = k + static_cast<unsigned>(lane);
+    bool valid = false;
+    if (slot < nslots) {
+      const int m = M - 1 - static_cast<int>(slot / B);
+      const int b = static_cast<int>(slot % B);
+      const int2 sq = load_seq(a, b, POS);
+      if (sq.y < 0) {
+        if (m == 0) set_status(a.status, kStatusBadOffsets);
+      } else {
+        valid = kRows * m < sq.y;
+      }
+    }
+    const unsigned vb = __ballot_sync(0xffffffffu, valid);
+    if (vb & 1u) return make_int2(M - 1 - static_cast<int>(k / B), static_cast<int>(k % B));
+    const unsigned rest = vb & ~1u;
+    const unsigned skip_to = rest ? k + static_cast<unsigned>(__ffs(rest) - 1) : k + 32u;
+    if (lane == 0 && skip_to > k + 1) atomicMax(counter, min(skip_to, nslots));
+  }
 }
 
 template <bool POS, bool TIME>
@@ -242,41 +325,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // blockIdx.x = (cluster index) * H + head; the head is the rank in the cluster.
-  const int h = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.H));
-  const int idx = static_cast<int>(blockIdx.x / static_cast<unsigned>(a.H));
-  const int m = a.max_tiles - 1 - idx / a.B;
-  const int b = idx % a.B;
-
-  // Sequence bounds; inconsistent offsets make the sequence empty and are reported.
-  int s = __ldg(a.offsets + b);
-  int e = __ldg(a.offsets + b + 1);
-  int n_b = e - s;
-  if (s < 0 || n_b < 0 || e > a.T || n_b > a.max_seq_len || (POS && n_b > a.L)) {
-    if (threadIdx.x == 0 && h == 0 && m == 0) set_status(a.status, kStatusBadOffsets);
-    n_b = 0;
-  }
-  if (kRows * m >= n_b) return;               // whole cluster leaves together
-  const int nt = m + 1;                       // key tiles 0..m
+  const int H = a.H;
+  const int h = static_cast<int>(cluster_ctarank());   // head = rank in the cluster
+  const bool leader = (h == 0);
 
   auto bar = [&](int i) { return sbase + kOffBar + 8u * i; };
+  auto ring_addr = [&](int slot) { return sbase + kOffRing + 8u * slot; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-  const uint32_t bar_red0 = sbase + kOffMisc + 16;   // 8-byte aligned slots in misc
-  const uint32_t bar_red1 = sbase + kOffMisc + 24;
 
   long long* s_thr = reinterpret_cast<long long*>(smem + kOffThr);
   signed char* s_first = reinterpret_cast<signed char*>(smem + kOffFirst);
   float* s_rabt = reinterpret_cast<float*>(smem + kOffRabT);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i)
-      mbar_init(bar(i), (i == B_PFULL || i == B_PFULL + 1)
-                            ? static_cast<uint32_t>(kEpiThreads / 2)   // one team
-                            : 1u);
-    mbar_init(bar_red0, 1);
-    mbar_init(bar_red1, 1);
+    for (int i = 0; i < kNumBars; ++i) {
+      uint32_t count = 1;
+      if (i >= B_PFULL && i < B_PFULL + kSBufs) count = kEpiThreads;
+      if (i == B_DONE) count = 2;                                        // both issuers
+      if (i >= B_REMPTY && i < B_REMPTY + kRing) count = static_cast<uint32_t>(H);
+      mbar_init(bar(i), count);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -284,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(sbase + kOffMisc, kTmemCols);
     tmem_relinquish();
   }
-  if (TIME && warp >= 2) {
+  if (TIME && warp >= 2 && warp < kWarpPV) {
     const int et = threadIdx.x - 64;
     for (int i = et; i < kThrLen; i += kEpiThreads) s_thr[i] = a.bt.thr[i];
     if (et < 64) s_first[et] = a.bt.first_k[et];
@@ -303,285 +372,440 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_wait();
   const uint32_t tmem = misc[0];
 
+  // Item j of this cluster sits in ring slot j % kRing; every role reads it in order.
+  auto wait_item = [&](int j) -> bool {
+    return mbar_wait<true>(bar(B_RFULL + j % kRing), (j / kRing) & 1, abort_flag);
+  };
+  auto read_item = [&](int j) -> int2 {
+    int2 v;
+    asm volatile("ld.shared.v2.s32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(ring_addr(j % kRing))
+                 : "memory");
+    return v;
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const int row0 = s + kRows * m;
-      mbar_arrive_expect_tx(bar(B_QFULL), kTile);
-      tma_load_3d(sbase + kOffQ, &tm_q, bar(B_QFULL), 0, h, row0);
-      tma_load_3d(sbase + kOffQ + kHalf, &tm_q, bar(B_QFULL), 64, h, row0);
-      // K runs one tile ahead of V: K(n+1) is requested before V(n), whose
-      // stage frees only when P(n-2).V completes.
-      int k_last[kKStages] = {-1, -1, -1}, v_last[kVStages] = {-1, -1};
-      bool ok = true;
-      auto load_k = [&](int n) -> bool {
-        const int st = n % kKStages, use = n / kKStages;
-        if (use > 0 && !mbar_wait(bar(B_KEMPTY + st), (use - 1) & 1, abort_flag)) return false;
-        const int krow = s + kCols * n;
-        mbar_arrive_expect_tx(bar(B_KFULL + st), kTile);
-        tma_load_3d(sbase + kOffK + st * kTile, &tm_k, bar(B_KFULL + st), 0, h, krow);
-        tma_load_3d(sbase + kOffK + st * kTile + kHalf, &tm_k, bar(B_KFULL + st), 64, h, krow);
-        k_last[st] = use;
-        return true;
-      };
-      auto load_v = [&](int n) -> bool {
-        const int st = n % kVStages, use = n / kVStages;
-        if (use > 0 && !mbar_wait(bar(B_VEMPTY + st), (use - 1) & 1, abort_flag)) return false;
-        const int krow = s + kCols * n;
-        mbar_arrive_expect_tx(bar(B_VFULL + st), kTile);
-        tma_load_3d(sbase + kOffV + st * kTile, &tm_v, bar(B_VFULL + st), 0, h, krow);
-        tma_load_3d(sbase + kOffV + st * kTile + kHalf, &tm_v, bar(B_VFULL + st), 64, h, krow);
-        v_last[st] = use;
-        return true;
-      };
-      ok = load_k(0);
-      for (int n = 0; n < nt && ok; ++n) {
-        if (n + 1 < nt) ok = load_k(n + 1);
-        if (ok) ok = load_v(n);
+    unsigned* counter = reinterpret_cast<unsigned*>(a.status) + kSchedCounterWord;
+    unsigned* done = reinterpret_cast<unsigned*>(a.status) + kSchedDoneWord;
+    const unsigned nslots = static_cast<unsigned>(a.B) * static_cast<unsigned>(a.max_tiles);
+    // Leader: claim item j and hand it to every CTA of the cluster (warp-collective).
+    auto fetch = [&](int j) -> int2 {
+      bool okf = true;
+      int2 it = make_int2(-1, -1);
+      if (leader) {
+        // The slot's previous item (j - kRing) must have been read by every CTA.
+        if (lane == 0 && j >= kRing)
+          okf = mbar_wait<true>(bar(B_REMPTY + j % kRing), ((j / kRing) - 1) & 1, abort_flag);
+        okf = __shfl_sync(0xffffffffu, okf, 0);
+        if (okf) {
+          it = claim_item<POS>(a, counter, nslots, lane);
+          if (lane == 0) {
+            for (int pr = 0; pr < H; ++pr) {
+              st_cluster_v2_s32(mapa_shared(ring_addr(j % kRing), pr), it.x, it.y);
+              mbar_arrive_cluster(mapa_shared(bar(B_RFULL + j % kRing), pr));
+            }
+          }
+        }
+      } else {
+        if (lane == 0) {
+          okf = wait_item(j);
+          if (okf) it = read_item(j);
+        }
+        okf = __shfl_sync(0xffffffffu, okf, 0);
+        it.x = __shfl_sync(0xffffffffu, it.x, 0);
+        it.y = __shfl_sync(0xffffffffu, it.y, 0);
       }
+      __syncwarp();
+      return okf ? it : make_int2(-2, -2);
+    };
+
+    int k_last[kKStages] = {-1, -1, -1}, v_last[kVStages] = {-1, -1};
+    int q_last = -1;
+    bool ok = true;
+    int j = 0, g = 0;
+    int2 it = fetch(0);
+    while (it.x >= 0) {
+      if (lane == 0) {
+        const int m = it.x, nt = m + 1;
+        const int s = __ldg(a.offsets + it.y);
+        if (j > 0) ok = mbar_wait(bar(B_QEMPTY), (j - 1) & 1, abort_flag);
+        if (ok) {
+          const int row0 = s + kRows * m;
+          mbar_arrive_expect_tx(bar(B_QFULL), kTile);
+          tma_load_3d(sbase + kOffQ, &tm_q, bar(B_QFULL), 0, h, row0);
+          tma_load_3d(sbase + kOffQ + kHalf, &tm_q, bar(B_QFULL), 64, h, row0);
+          q_last = j;
+        }
+        // K runs one tile ahead of V: K(x+1) is requested before V(x), whose
+        // stage frees only when P(x-2).V completes.  x is the running tile index.
+        auto load_k = [&](int x, int n) -> bool {
+          const int st = x % kKStages, use = x / kKStages;
+          if (use > 0 && !mbar_wait(bar(B_KEMPTY + st), (use - 1) & 1, abort_flag)) return false;
+          const int krow = s + kCols * n;
+          mbar_arrive_expect_tx(bar(B_KFULL + st), kTile);
+          tma_load_3d(sbase + kOffK + st * kTile, &tm_k, bar(B_KFULL + st), 0, h, krow);
+          tma_load_3d(sbase + kOffK + st * kTile + kHalf, &tm_k, bar(B_KFULL + st), 64, h, krow);
+          k_last[st] = use;
+          return true;
+        };
+        auto load_v = [&](int x, int n) -> bool {
+          const int st = x % kVStages, use = x / kVStages;
+          if (use > 0 && !mbar_wait(bar(B_VEMPTY + st), (use - 1) & 1, abort_flag)) return false;
+          const int krow = s + kCols * n;
+          mbar_arrive_expect_tx(bar(B_VFULL + st), kTile);
+          tma_load_3d(sbase + kOffV + st * kTile, &tm_v, bar(B_VFULL + st), 0, h, krow);
+          tma_load_3d(sbase + kOffV + st * kTile + kHalf, &tm_v, bar(B_VFULL + st), 64, h, krow);
+          v_last[st] = use;
+          return true;
+        };
+        if (ok) ok = load_k(g, 0);
+        for (int n = 0; n < nt && ok; ++n) {
+          if (n + 1 < nt) ok = load_k(g + n + 1, n + 1);
+          if (ok) ok = load_v(g + n, n);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      g += it.x + 1;
+      ++j;
+      it = fetch(j);
+    }
+    if (it.x == -2) ok = false;
+    if (lane == 0) {
       if (!ok) {
         set_status(a.status, kStatusTimeout);
         *abort_flag = 1;
         // Let the copies already issued land before shared memory goes away.
-        mbar_wait(bar(B_QFULL), 0, nullptr);
+        if (q_last >= 0) mbar_wait(bar(B_QFULL), q_last & 1, nullptr);
         for (int st = 0; st < kKStages; ++st)
           if (k_last[st] >= 0) mbar_wait(bar(B_KFULL + st), k_last[st] & 1, nullptr);
         for (int st = 0; st < kVStages; ++st)
           if (v_last[st] >= 0) mbar_wait(bar(B_VFULL + st), v_last[st] & 1, nullptr);
       }
+      if (leader) {
+        // The last cluster to finish returns the work counter to zero for the next launch.
+        __threadfence();
+        const unsigned clusters = gridDim.x / static_cast<unsigned>(H);
+        if (atomicAdd(done, 1u) == clusters - 1) {
+          atomicExch(counter, 0u);
+          atomicExch(done, 0u);
+        }
+      }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer
     if (lane == 0) {
-      bool ok = mbar_wait(bar(B_QFULL), 0, abort_flag);
-      auto issue_s = [&](int n) -> bool {
-        const int st = n % kKStages;
-        if (!mbar_wait(bar(B_KFULL + st), (n / kKStages) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + kColS0 + 128u * (n & 1);
-        const uint32_t qa = sbase + kOffQ, ka = sbase + kOffK + st * kTile;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-          mma_ss(d, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), kIdescS,
-                 ks > 0);
-        }
-        mma_commit(bar(B_KEMPTY + st));
-        mma_commit(bar(B_SFULL + (n & 1)));
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      if (ok && nt > 1) ok = issue_s(1);
-      for (int n = 0; n < nt && ok; ++n) {
-        const int x = n & 1, st = n % kVStages;
-        ok = mbar_wait(bar(B_PFULL + x), (n >> 1) & 1, abort_flag);
+      bool ok = true;
+      int j = 0, g = 0;
+      for (;;) {
+        ok = wait_item(j);
         if (!ok) break;
-        ok = mbar_wait(bar(B_VFULL + st), (n / kVStages) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t va = sbase + kOffV + st * kTile;
+        const int2 it = read_item(j);
+        if (it.x < 0) break;
+        const int nt = it.x + 1;
+        ok = mbar_wait(bar(B_QFULL), j & 1, abort_flag);
+        for (int n = 0; n < nt && ok; ++n) {
+          const int x = g + n, st = x % kKStages, buf = x % kSBufs;
+          // The buffer's previous tile x-3 has been consumed by its P.V.
+          if (x >= kSBufs)
+            ok = mbar_wait(bar(B_PVDONE + buf), ((x - kSBufs) / kSBufs) & 1, abort_flag);
+          if (ok) ok = mbar_wait(bar(B_KFULL + st), (x / kKStages) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t d = tmem + kColS0 + 128u * buf;
+          const uint32_t qa = sbase + kOffQ, ka = sbase + kOffK + st * kTile;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          // 16 keys per step: rows 16ks.. of the V tile; the two 64-column
-          // halves of d_v are 16 KB apart (leading byte offset).
-          mma_ts(tmem + kColO, tmem + kColP0 + 64u * x + 8u * ks,
-                 sw128_desc(va + ks * 2048, kHalf, 1024), kIdescPV, (n > 0 || ks > 0));
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+            mma_ss(d, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), kIdescS,
+                   ks > 0);
+          }
+          mma_commit(bar(B_KEMPTY + st));
+          mma_commit(bar(B_SFULL + buf));
         }
-        mma_commit(bar(B_VEMPTY + st));
-        if (n + 2 < nt) ok = issue_s(n + 2);
+        if (!ok) break;
+        mma_commit(bar(B_QEMPTY));   // Q may be replaced by the next item's
+        g += nt;
+        ++j;
       }
       if (!ok) {
         set_status(a.status, kStatusTimeout);
         *abort_flag = 1;
       }
-      mma_commit(bar(B_OFULL));   // also marks every issued MMA as finished
+      mma_commit(bar(B_DONE));   // arrives once every MMA it issued has finished
     }
-  } else {
+  } else if (warp == kWarpPV) {
+    // ------------------------------------------------------------ P.V issuer
+    if (lane == 0) {
+      bool ok = true;
+      int j = 0, g = 0;
+      for (;;) {
+        ok = wait_item(j);
+        if (!ok) break;
+        const int2 it = read_item(j);
+        if (it.x < 0) break;
+        const int nt = it.x + 1;
+        for (int n = 0; n < nt && ok; ++n) {
+          const int x = g + n, st = x % kVStages, buf = x % kSBufs;
+          ok = mbar_wait(bar(B_PFULL + buf), (x / kSBufs) & 1, abort_flag);
+          if (ok) ok = mbar_wait(bar(B_VFULL + st), (x / kVStages) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t va = sbase + kOffV + st * kTile;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            // 16 keys per step: rows 16ks.. of the V tile; the two 64-column
+            // halves of d_v are 16 KB apart (leading byte offset).
+            // P keys 16ks..16ks+15: column group ks/2 holds its 32 keys in 16 columns.
+            mma_ts(tmem + kColO, tmem + kColS0 + 128u * buf + 32u * (ks >> 1) + 8u * (ks & 1),
+                   sw128_desc(va + ks * 2048, kHalf, 1024), kIdescPV, (n > 0 || ks > 0));
+          }
+          mma_commit(bar(B_VEMPTY + st));
+          mma_commit(bar(B_PVDONE + buf));
+        }
+        if (!ok) break;
+        mma_commit(bar(B_OFULL));
+        g += nt;
+        ++j;
+      }
+      if (!ok) {
+        set_status(a.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      mma_commit(bar(B_DONE));
+    }
+  } else if (warp < kWarpPV) {
     // ------------------------------------------------------------ epilogue
     const int q4 = warp & 3;                      // TMEM lane quarter
-    const int cq = (warp - 2) >> 2;               // column quarter of the S/O tiles
+    const int cq = (warp - 2) >> 2;               // 32-column group of the S/P and O tiles
     const int r = q4 * 32 + lane;                 // row within the tile
     const int et = threadIdx.x - 64;              // 0..511 among epilogue threads
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-    const int i_loc = kRows * m + r;              // local row index in the sequence
-    const bool row_ok = i_loc < n_b;
-    const int t_row = s + (row_ok ? i_loc : 0);
-    const float nrm = a.norm_len > 0 ? static_cast<float>(a.norm_len) : static_cast<float>(n_b);
     const int Lw = 2 * a.L - 1;
+    const int D = H * 128;
     uint8_t* wstage = smem + kOffWarp + (warp - 2) * kWarpStage;
-    float* wv = reinterpret_cast<float*>(wstage);
-    long long* wts = reinterpret_cast<long long*>(wstage + 96 * 4);
-    const int team = (warp - 2) >> 3;             // S buffer / tile parity of this warp
-    const int ch = ((warp - 2) >> 2) & 1;         // column half within the team's tiles
+    uint32_t* wpk = reinterpret_cast<uint32_t*>(wstage);
+    long long* wts = reinterpret_cast<long long*>(wstage + 64 * 4);
+    float2* loc = reinterpret_cast<float2*>(smem + kOffLoc);   // [4][128]
+    float2* red = reinterpret_cast<float2*>(smem + kOffRed);   // [2][kMaxHeads][128]
+    const uint32_t rempty_leader = mapa_shared(bar(B_REMPTY), 0);
     EpiCtx ec;
     ec.thr = s_thr;
     ec.first = s_first;
     ec.rabt = s_rabt;
-    ec.my_ts = TIME ? a.timestamps[t_row] : 0;
-    ec.inv_n = 1.0f / nrm;
     ec.r = r;
     ec.lane = lane;
     bool ok = true;
+    int j = 0, g = 0;
 
-    // Staging of this warp's 32 x 64 block of tile n: half position bias of
-    // the 95 diagonals d = r - c in [32 q4 - 64 ch - 63, 32 q4 - 64 ch + 31]
-    // (table index 128 (m - n) + d + L - 1), and the timestamps of its 64 keys
-    // (keys past the sequence end repeat its last timestamp, which keeps them
-    // non-decreasing; those keys are masked anyway).
-    const int dbase = 32 * q4 - 64 * ch - 63;
-    float pre_w0 = 0.f, pre_w1 = 0.f, pre_w2 = 0.f;
-    long long pre_t0 = 0, pre_t1 = 0;
-    auto prefetch = [&](int n) {
-      if (POS) {
-        const int t0 = kRows * (m - n) + dbase + lane + a.L - 1;
-        const float* tab = a.rab_pos + static_cast<size_t>(h) * Lw;
-        pre_w0 = (t0 >= 0 && t0 < Lw) ? __ldg(tab + t0) : 0.f;
-        pre_w1 = (t0 + 32 >= 0 && t0 + 32 < Lw) ? __ldg(tab + t0 + 32) : 0.f;
-        pre_w2 = (lane < 31 && t0 + 64 >= 0 && t0 + 64 < Lw) ? __ldg(tab + t0 + 64) : 0.f;
+    // Named barriers cannot time out, so every epilogue warp leaves the loop
+    // at the same point: the decisions to stop are OR-reduced over all of them.
+    for (;;) {
+      const bool got = __all_sync(0xffffffffu, wait_item(j));
+      const int2 it = got ? read_item(j) : make_int2(-2, -2);
+      if (named_bar_or(2, kEpiThreads, !ok || it.x < 0)) {
+        if (it.x == -2) ok = false;
+        break;
       }
-      if (TIME) {
-        const int j = kCols * n + 64 * ch + lane;
-        pre_t0 = a.timestamps[s + (j < n_b ? j : n_b - 1)];
-        pre_t1 = a.timestamps[s + (j + 32 < n_b ? j + 32 : n_b - 1)];
-      }
-    };
-    bool sorted0 = true, sorted1 = true;
-    auto stage = [&]() {   // previous users of the buffer (this warp) are done
-      if (POS) {
-        wv[lane] = 0.5f * pre_w0;
-        wv[32 + lane] = 0.5f * pre_w1;
-        wv[64 + lane] = 0.5f * pre_w2;
-      }
-      if (TIME) {
-        wts[lane] = pre_t0;
-        wts[32 + lane] = pre_t1;
-        const long long n0 = __shfl_down_sync(0xffffffffu, pre_t0, 1);
-        const long long n1 = __shfl_down_sync(0xffffffffu, pre_t1, 1);
-        sorted0 = !__any_sync(0xffffffffu, lane < 31 && n0 < pre_t0);
-        sorted1 = !__any_sync(0xffffffffu, lane < 31 && n1 < pre_t1);
-      }
-      __syncwarp();
-    };
-    if (team < nt) {
-      prefetch(team);
+      const int m = it.x, nt = m + 1;
+      const int s = __ldg(a.offsets + it.y);
+      const int n_b = __ldg(a.offsets + it.y + 1) - s;
+      const int i_loc = kRows * m + r;            // local row index in the sequence
+      const bool row_ok = i_loc < n_b;
+      const int t_row = s + (row_ok ? i_loc : 0);
+      const float nrm = a.norm_len > 0 ? static_cast<float>(a.norm_len) : static_cast<float>(n_b);
+      ec.my_ts = TIME ? a.timestamps[t_row] : 0;
+      ec.inv_n = 1.0f / nrm;
+
+      // Staging of this warp's 32 x 32 block of tile n: half position bias of
+      // the 63 diagonals d = r - c in [32 q4 - 32 cq - 31, 32 q4 - 32 cq + 31]
+      // (table index 128 (m - n) + d + L - 1), entry k as the bf16 pair
+      // (diagonal k, diagonal k-1), and the timestamps of its 32 keys (keys
+      // past the sequence end repeat its last timestamp, which keeps them
+      // non-decreasing; those keys are masked anyway).
+      const int dbase = 32 * q4 - 32 * cq - 31;
+      float pre_w0 = 0.f, pre_w1 = 0.f;
+      long long pre_t = 0;
+      auto prefetch = [&](int n) {
+        if (POS) {
+          const int t0 = kRows * (m - n) + dbase + lane + a.L - 1;
+          const float* tab = a.rab_pos + static_cast<size_t>(h) * Lw;
+          pre_w0 = (t0 >= 0 && t0 < Lw) ? __ldg(tab + t0) : 0.f;
+          pre_w1 = (lane < 31 && t0 + 32 >= 0 && t0 + 32 < Lw) ? __ldg(tab + t0 + 32) : 0.f;
+        }
+        if (TIME) {
+          const int jj = kCols * n + 32 * cq + lane;
+          pre_t = a.timestamps[s + (jj < n_b ? jj : n_b - 1)];
+        }
+      };
+      bool sorted = true;
+      auto stage = [&]() {   // previous users of the buffer (this warp) are done
+        if (POS) {
+          const float v0 = 0.5f * pre_w0, v1 = 0.5f * pre_w1;
+          float p0 = __shfl_up_sync(0xffffffffu, v0, 1);
+          float p1 = __shfl_up_sync(0xffffffffu, v1, 1);
+          const float e0 = __shfl_sync(0xffffffffu, v0, 31);
+          if (lane == 0) {
+            p0 = 0.f;
+            p1 = e0;
+          }
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(v0, p0);   // .x (low) = diagonal k
+          __nv_bfloat162 b1 = __floats2bfloat162_rn(v1, p1);
+          wpk[lane] = *reinterpret_cast<uint32_t*>(&b0);
+          wpk[32 + lane] = *reinterpret_cast<uint32_t*>(&b1);
+        }
+        if (TIME) {
+          wts[lane] = pre_t;
+          const long long nx = __shfl_down_sync(0xffffffffu, pre_t, 1);
+          sorted = !__any_sync(0xffffffffu, lane < 31 && nx < pre_t);
+        }
+        __syncwarp();
+      };
+
+      prefetch(0);
       stage();
-    }
+      for (int n = 0; n < nt; ++n) {
+        const int x = g + n, buf = x % kSBufs;
+        if (n + 1 < nt) prefetch(n + 1);          // global loads overlap this tile
+        if (ok) ok = mbar_wait(bar(B_SFULL + buf), (x / kSBufs) & 1, abort_flag);
+        // The TMEM loads/stores below are warp-collective: keep the decision warp-uniform.
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;                           // on to the collective exit below
+        tc_fence_after();
+        const uint32_t s_addr = tmem + lane_addr + kColS0 + 128u * buf;
+        if (n == m)
+          chunk_to_tmem<POS, TIME, true>(s_addr, 32 * cq, ec, wpk, wts, sorted);
+        else
+          chunk_to_tmem<POS, TIME, false>(s_addr, 32 * cq, ec, wpk, wts, sorted);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL + buf));
+        if (n + 1 < nt) stage();
+      }
 
-    for (int n = team; n < nt; n += 2) {
-      if (n + 2 < nt) prefetch(n + 2);            // global loads overlap this tile
-      if (ok) ok = mbar_wait(bar(B_SFULL + team), (n >> 1) & 1, abort_flag);
-      // The TMEM loads/stores below are warp-collective: keep the decision warp-uniform.
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t s_addr = tmem + lane_addr + kColS0 + 128u * team;
-      const uint32_t p_addr = tmem + lane_addr + kColP0 + 64u * team;
-      if (n == m)
-        tile_to_p<POS, TIME, true>(s_addr, p_addr, 64 * ch, ec, wv, wts, sorted0, sorted1);
-      else
-        tile_to_p<POS, TIME, false>(s_addr, p_addr, 64 * ch, ec, wv, wts, sorted0, sorted1);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_PFULL + team));
-      if (n + 2 < nt) stage();
-    }
-
-    // ---------------------------------------------- LayerNorm over heads + gate
-    if (ok) ok = mbar_wait(bar(B_OFULL), 0, abort_flag);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) {
-      set_status(a.status, kStatusTimeout);
-      *abort_flag = 1;
-    }
-    tc_fence_after();
-    const int H = a.H;
-    const int D = H * 128;
-    float* loc0 = reinterpret_cast<float*>(smem + kOffRed);   // [4][128] local partials
-    float* loc1 = loc0 + kColGroups * 128;
-    float* red0 = loc1 + kColGroups * 128;                      // [8][128] cluster slots
-    float* red1 = red0 + 8 * 128;
-    const uint32_t o_addr = tmem + lane_addr + kColO + 32u * cq;
-    // The row's 32 values of this head and column quarter stay in registers.
-    float ov[32];
-    {
-      uint32_t o0[32];
-      tmem_ld32_nowait(o_addr, o0);
-      tmem_wait_ld_dep(o0);
-      // O accumulated N * SiLU(.) / N terms: apply 1/N here, in fp32.
+      // -------------------------------------------- LayerNorm over heads + gate
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), j & 1, abort_flag));
+      if (ok) tc_fence_after();
+      // The row's 32 values of this head and column quarter stay in registers.
+      float ov[32];
+      {
+        uint32_t o0[32];
+        if (ok) {
+          tmem_ld32_nowait(tmem + lane_addr + kColO + 32u * cq, o0);
+          tmem_wait_ld_dep(o0);
+        } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(o0[i]) * ec.inv_n;
-    }
-    const uint32_t lnbytes = static_cast<uint32_t>(H * 128 * 4);
-    // pass 1: row sums.  The four column groups add up in shared memory, then
-    // one thread per row sends this head's sum to every CTA of the cluster.
-    float part = 0.f;
+          for (int i = 0; i < 32; ++i) o0[i] = 0u;
+        }
+        // O accumulated SiLU(.) terms: apply 1/N here, in fp32.
 #pragma unroll
-    for (int i = 0; i < 32; ++i) part += ov[i];
-    loc0[cq * 128 + r] = part;
-    named_bar_sync(1, kEpiThreads);
-    if (cq == 0) {
-      const float hsum = loc0[r] + loc0[128 + r] + loc0[256 + r] + loc0[384 + r];
-      const uint32_t slot = smem_u32(red0 + h * 128 + r);
-      for (int pr = 0; pr < H; ++pr)
-        st_async_f32(mapa_shared(slot, pr), hsum, mapa_shared(bar_red0, pr));
-    }
-    if (et == 0) mbar_arrive_expect_tx(bar_red0, lnbytes);
-    if (!mbar_wait<true>(bar_red0, 0, nullptr)) set_status(a.status, kStatusTimeout);
-    float tot = 0.f;
-    for (int k = 0; k < H; ++k) tot += red0[k * 128 + r];
-    const float mean = tot / static_cast<float>(D);
-    // pass 2: centred sum of squares, same route
-    float sq = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float d0 = ov[i] - mean;
-      sq = fmaf(d0, d0, sq);
-    }
-    loc1[cq * 128 + r] = sq;
-    named_bar_sync(1, kEpiThreads);
-    if (cq == 0) {
-      const float hsq = loc1[r] + loc1[128 + r] + loc1[256 + r] + loc1[384 + r];
-      const uint32_t slot = smem_u32(red1 + h * 128 + r);
-      for (int pr = 0; pr < H; ++pr)
-        st_async_f32(mapa_shared(slot, pr), hsq, mapa_shared(bar_red1, pr));
-    }
-    if (et == 0) mbar_arrive_expect_tx(bar_red1, lnbytes);
-    if (!mbar_wait<true>(bar_red1, 0, nullptr)) set_status(a.status, kStatusTimeout);
-    float totsq = 0.f;
-    for (int k = 0; k < H; ++k) totsq += red1[k * 128 + r];
-    const float var = totsq / static_cast<float>(D);
-    const float rstd = 1.0f / sqrtf(var + a.eps);
-    // pass 3: normalise, gate, store this thread's 32 columns
-    if (row_ok) {
+        for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(o0[i]) * ec.inv_n;
+      }
       const size_t rowD = static_cast<size_t>(t_row) * D + static_cast<size_t>(h) * 128 + 32 * cq;
-      if (a.o_save) {
+      // The gate input is requested now; its latency hides behind the exchange.
+      uint4 uu[4];
+      {
+        const uint4* us =
+            reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.u) + rowD);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) uu[i] = row_ok ? __ldg(us + i) : make_uint4(0, 0, 0, 0);
+      }
+      if (ok && row_ok && a.o_save) {
         float4* od = reinterpret_cast<float4*>(a.o_save + rowD);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           od[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
       }
-      const uint4* us = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.u) + rowD);
-      uint4* yd = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.y) + rowD);
+      // Row statistics of the 32 values: sum and sum of squared deviations.
+      {
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sum += ov[i];
+        const float mu = sum * (1.0f / 32.0f);
+        float m2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float d0 = ov[i] - mu;
+          m2 = fmaf(d0, d0, m2);
+        }
+        loc[cq * 128 + r] = make_float2(sum, m2);
+      }
+      tc_fence_before();
+      if (named_bar_or(1, kEpiThreads, !ok)) {
+        ok = false;
+        break;
+      }
+      // Every role of this CTA has read item j: release its ring slot.
+      if (et == 0) mbar_arrive_cluster(rempty_leader + 8u * (j % kRing));
+      const int pj = j & 1;
+      if (cq == 0) {
+        // Combine the four 32-column groups (equal counts) into this head's
+        // (sum, M2) and send it to every CTA of the cluster.
+        const float2 p0 = loc[r], p1 = loc[128 + r], p2 = loc[256 + r], p3 = loc[384 + r];
+        const float hs = (p0.x + p1.x) + (p2.x + p3.x);
+        const float mh = hs * (1.0f / 128.0f);
+        const float e0 = p0.x * (1.0f / 32.0f) - mh, e1 = p1.x * (1.0f / 32.0f) - mh;
+        const float e2 = p2.x * (1.0f / 32.0f) - mh, e3 = p3.x * (1.0f / 32.0f) - mh;
+        const float hm2 = (p0.y + p1.y) + (p2.y + p3.y) +
+                          32.0f * ((e0 * e0 + e1 * e1) + (e2 * e2 + e3 * e3));
+        const uint32_t slot = smem_u32(red + (pj * kMaxHeads + h) * 128 + r);
+        for (int pr = 0; pr < H; ++pr)
+          st_async_v2_f32(mapa_shared(slot, pr), hs, hm2, mapa_shared(bar(B_RED + pj), pr));
+      }
+      if (et == 0) mbar_arrive_expect_tx(bar(B_RED + pj), static_cast<uint32_t>(H * 128 * 8));
+      // Gate values while the statistics travel.
+      float gate[32];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        uint4 uu = __ldg(us + i);
-        const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&uu);
-        uint4 out;
-        uint32_t* o32 = reinterpret_cast<uint32_t*>(&out);
+        const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&uu[i]);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 uf = __bfloat1622float2(u2[j]);
-          const float y0 = (ov[8 * i + 2 * j] - mean) * rstd * silu_precise(uf.x);
-          const float y1 = (ov[8 * i + 2 * j + 1] - mean) * rstd * silu_precise(uf.y);
-          __nv_bfloat162 pr = __floats2bfloat162_rn(y0, y1);
-          o32[j] = *reinterpret_cast<uint32_t*>(&pr);
+        for (int q = 0; q < 4; ++q) {
+          const float2 uf = __bfloat1622float2(u2[q]);
+          gate[8 * i + 2 * q] = silu_gate(uf.x);
+          gate[8 * i + 2 * q + 1] = silu_gate(uf.y);
         }
-        yd[i] = out;
       }
-      if (h == 0 && cq == 0 && a.ln_mean) {
-        a.ln_mean[t_row] = mean;
-        a.ln_rstd[t_row] = rstd;
+      if (!mbar_wait<true>(bar(B_RED + pj), (j >> 1) & 1, nullptr)) set_status(a.status, kStatusTimeout);
+      // Chan's combination of the H per-head (sum, M2) pairs of 128 values each.
+      const float2* rr = red + pj * kMaxHeads * 128 + r;
+      float tot = 0.f;
+      for (int k = 0; k < H; ++k) tot += rr[k * 128].x;
+      const float mean = tot / static_cast<float>(D);
+      float m2 = 0.f;
+      for (int k = 0; k < H; ++k) {
+        const float2 pk = rr[k * 128];
+        const float dk = pk.x * (1.0f / 128.0f) - mean;
+        m2 += pk.y + 128.0f * dk * dk;
       }
+      const float var = m2 / static_cast<float>(D);
+      const float rstd = 1.0f / sqrtf(var + a.eps);
+      if (row_ok) {
+        uint4* yd = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.y) + rowD);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint4 out;
+          uint32_t* o32 = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int c = 8 * i + 2 * q;
+            __nv_bfloat162 pr =
+                __floats2bfloat162_rn((ov[c] - mean) * rstd * gate[c],
+                                      (ov[c + 1] - mean) * rstd * gate[c + 1]);
+            o32[q] = *reinterpret_cast<uint32_t*>(&pr);
+          }
+          yd[i] = out;
+        }
+        if (h == 0 && cq == 0 && a.ln_mean) {
+          a.ln_mean[t_row] = mean;
+          a.ln_rstd[t_row] = rstd;
+        }
+      }
+      g += nt;
+      ++j;
+    }
+    if (!ok) {
+      set_status(a.status, kStatusTimeout);
+      *abort_flag = 1;
     }
     tc_fence_before();
   }
@@ -589,32 +813,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    // Every MMA has completed once B_OFULL fired; wait for it before freeing TMEM.
-    if (lane == 0) mbar_wait(bar(B_OFULL), 0, nullptr);
+    // Every MMA has completed once B_DONE fired; wait for it before freeing TMEM.
+    if (lane == 0) mbar_wait(bar(B_DONE), 0, nullptr);
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
   }
+  // No CTA leaves while another may still write into its shared memory.
+  cluster_arrive();
+  cluster_wait();
 }
 
 template <bool POS, bool TIME>
 cudaError_t launch_variant(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                            const CUtensorMap& tv, cudaStream_t stream) {
-  // The shared-memory opt-in is a per-device function attribute: set it once
-  // per device (not inside a stream capture of a later call).
+  // The shared-memory opt-in is a per-device function attribute, and the
+  // number of co-resident clusters a per-device, per-cluster-size property:
+  // both are taken once per device (not inside a stream capture of a later call).
   static bool configured[64] = {};
+  static int max_clusters[64][kMaxHeads + 1] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
     err = cudaFuncSetAttribute(hstu_fwd_bf16_sm100<POS, TIME>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
-    if (dev >= 0 && dev < 64) configured[dev] = true;
+    configured[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.H) * static_cast<unsigned>(a.B) *
-                         static_cast<unsigned>(a.max_tiles),
-                     1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
@@ -625,6 +852,17 @@ cudaError_t launch_variant(const FwdArgs& a, const CUtensorMap& tq, const CUtens
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  int& resident = max_clusters[dev][a.H];
+  if (resident == 0) {
+    cfg.gridDim = dim3(static_cast<unsigned>(a.H), 1, 1);
+    int n = 0;
+    err = cudaOccupancyMaxActiveClusters(&n, hstu_fwd_bf16_sm100<POS, TIME>, &cfg);
+    if (err != cudaSuccess) return err;
+    resident = n > 0 ? n : 1;
+  }
+  const long long nslots = static_cast<long long>(a.B) * a.max_tiles;
+  const long long clusters = std::min<long long>(resident, nslots);
+  cfg.gridDim = dim3(static_cast<unsigned>(clusters * a.H), 1, 1);
   return cudaLaunchKernelEx(&cfg, hstu_fwd_bf16_sm100<POS, TIME>, tq, tk, tv, a);
 }
 
@@ -633,6 +871,9 @@ cudaError_t launch_variant(const FwdArgs& a, const CUtensorMap& tq, const CUtens
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, cudaStream_t stream) {
   if (a.B == 0 || a.max_tiles == 0) return cudaSuccess;
+  if (a.H < 1 || a.H > kMaxHeads) return cudaErrorInvalidValue;
+  // Work slots are numbered in 32 bits (plus one claim window of 32).
+  if (static_cast<long long>(a.B) * a.max_tiles > 0x7FFFFF00LL) return cudaErrorInvalidValue;
   const bool pos = a.rab_pos != nullptr, tim = a.rab_time != nullptr;
   if (pos && tim) return launch_variant<true, true>(a, tq, tk, tv, stream);
   if (pos) return launch_variant<true, false>(a, tq, tk, tv, stream);

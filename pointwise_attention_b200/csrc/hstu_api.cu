@@ -131,7 +131,10 @@ hstu_status_t check_problem(const hstu_problem_t* p) {
 }
 
 bool bf16_supported(const hstu_problem_t* p) {
-  return p->dtype == HSTU_BF16 && p->d_qk == 128 && p->d_v == 128 && p->num_heads <= 8;
+  // The forward numbers its (sequence, query tile) work slots in 32 bits.
+  const int64_t slots = static_cast<int64_t>(p->batch) * ((p->max_seq_len + 127) / 128);
+  return p->dtype == HSTU_BF16 && p->d_qk == 128 && p->d_v == 128 && p->num_heads <= 8 &&
+         slots <= 0x7FFFFF00LL;
 }
 
 bool f32_supported(const hstu_problem_t* p) {

@@ -10,6 +10,13 @@ namespace hstu {
 constexpr int kStatusBadOffsets = 1;   // offsets contradict T / max_seq_len / L
 constexpr int kStatusTimeout = 2;      // a bounded wait ran out
 
+// The 256-byte head of the workspace: word 0 is the status word; words 16 and
+// 17 are the bf16 forward's work counter and finished-cluster counter.  The
+// forward leaves both counters at zero when it ends (the last cluster to
+// finish resets them), so a zero-filled workspace stays valid across calls.
+constexpr int kSchedCounterWord = 16;
+constexpr int kSchedDoneWord = 17;
+
 constexpr int kMaxBuckets = 128;
 // thr[k] = smallest |dt| with bucket(dt) >= k (thr[0] = 0); entries k >= NB
 // hold INT64_MAX so the bucket search never passes NB-1.

@@ -67,6 +67,34 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
+// Non-blocking probe: true once the phase with `parity` has completed.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Blocking probe that suspends for at most about `hint_ns` before reporting
+// an incomplete phase.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait; returns false when the budget ran out (or *abort was raised
 // by another role), true once the phase with `parity` has completed.
 template <bool kCluster = false>
@@ -145,6 +173,12 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// Copy a 128-row x 256-bit matrix (one K-step of 16 bf16 per row) from shared
+// memory, described like an MMA operand, into TMEM lanes 0..127, 8 columns.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
@@ -221,6 +255,29 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
                    remote_addr),
                "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
+
+// Store 8 bytes into another CTA's shared memory and count them on its mbarrier.
+__device__ __forceinline__ void st_async_v2_f32(uint32_t remote_addr, float a, float b,
+                                                uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+          remote_addr),
+      "f"(a), "f"(b), "r"(remote_bar)
+      : "memory");
+}
+
+// Plain 8-byte store through the cluster shared-memory window (any CTA of the cluster).
+__device__ __forceinline__ void st_cluster_v2_s32(uint32_t addr, int a, int b) {
+  asm volatile("st.shared::cluster.v2.s32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+
+// Arrive on an mbarrier of any CTA of the cluster; the thread's earlier memory
+// operations are released at cluster scope before the arrival.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   bar_cluster_addr)
                : "memory");
 }
 

@@ -134,6 +134,27 @@ def test_degenerate_shapes():
     assert y.numel() == 0
 
 
+def test_work_counters_return_to_zero_and_calls_repeat():
+    """The bf16 forward hands (sequence, query tile) items to its clusters from
+    a counter in the workspace head; the last cluster to finish zeroes it, so
+    back-to-back calls on one workspace (and a workspace first used with many
+    empty slots: long and short sequences mixed) all see every item."""
+    inp = hi.make_inputs(spec((1500, 3, 700, 1, 0, 1200), H=4, time=True), seed=31)
+    dev = to_dev(inp)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ref = oracle.fwd(inp)
+    for call in range(3):
+        y, _ = pa.hstu_attn_fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["offsets"],
+                                inp.max_seq_len, timestamps=dev["timestamps"],
+                                rab_pos=dev["rab_pos"], rab_time=dev["rab_time"],
+                                workspace=ws)
+        torch.cuda.synchronize()
+        words = ws.view(torch.int32).cpu().numpy()
+        assert words[16] == 0 and words[17] == 0, words[:20]
+        assert pa.hstu_attn_check(ws) == 0
+        assert_close(np64(y), ref["y"], "bf16", "y (call %d)" % call)
+
+
 def test_bad_device_offsets_reported():
     """Offsets that contradict max_seq_len, given without a host copy, are found
     by the kernel: the sequence is skipped and the status word says so."""
