@@ -616,6 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float nrm = a.norm_len > 0 ? static_cast<float>(a.norm_len) : static_cast<float>(n_b);
       ec.my_ts = TIME ? a.timestamps[t_row] : 0;
       ec.inv_n = 1.0f / nrm;
+      // The gate input of this row is read at the end of the item: ask L2 for it now.
+      if (row_ok)
+        prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(a.u) +
+                    static_cast<size_t>(t_row) * (H * 128) + h * 128 + 32 * cq);
 
       // Staging of this warp's 32 x 32 block of tile n: half position bias of
       // the 63 diagonals d = r - c in [32 q4 - 32 cq - 31, 32 q4 - 32 cq + 31]
@@ -703,18 +707,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const size_t rowD = static_cast<size_t>(t_row) * D + static_cast<size_t>(h) * 128 + 32 * cq;
       // The gate input is requested now; its latency hides behind the exchange.
+      // Each lane owns a row, so every access below touches 32 rows: 32-byte
+      // accesses (when aligned) halve the requests the load/store unit handles.
       uint4 uu[4];
       {
-        const uint4* us =
-            reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.u) + rowD);
+        const __nv_bfloat16* us = reinterpret_cast<const __nv_bfloat16*>(a.u) + rowD;
+        if (!row_ok) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) uu[i] = row_ok ? __ldg(us + i) : make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 4; ++i) uu[i] = make_uint4(0, 0, 0, 0);
+        } else if (a.vec32) {
+          uint32_t w0[8], w1[8];
+          ld_global_nc_v8(us, w0);
+          ld_global_nc_v8(us + 16, w1);
+          uu[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+          uu[1] = make_uint4(w0[4], w0[5], w0[6], w0[7]);
+          uu[2] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+          uu[3] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) uu[i] = __ldg(reinterpret_cast<const uint4*>(us) + i);
+        }
       }
       if (ok && row_ok && a.o_save) {
-        float4* od = reinterpret_cast<float4*>(a.o_save + rowD);
+        float* od = a.o_save + rowD;
+        if (a.vec32) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          od[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) w[q] = __float_as_uint(ov[8 * i + q]);
+            st_global_v8(od + 8 * i, w);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(od)[i] =
+                make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+        }
       }
       // Row statistics of the 32 values: sum and sum of squared deviations.
       {
@@ -780,20 +809,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float var = m2 / static_cast<float>(D);
       const float rstd = 1.0f / sqrtf(var + a.eps);
       if (row_ok) {
-        uint4* yd = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.y) + rowD);
+        __nv_bfloat16* yd = reinterpret_cast<__nv_bfloat16*>(a.y) + rowD;
+        uint32_t yw[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint4 out;
-          uint32_t* o32 = reinterpret_cast<uint32_t*>(&out);
+        for (int q = 0; q < 16; ++q) {
+          __nv_bfloat162 pr = __floats2bfloat162_rn((ov[2 * q] - mean) * rstd * gate[2 * q],
+                                                    (ov[2 * q + 1] - mean) * rstd * gate[2 * q + 1]);
+          yw[q] = *reinterpret_cast<uint32_t*>(&pr);
+        }
+        if (a.vec32) {
+          st_global_v8(yd, reinterpret_cast<const uint32_t(&)[8]>(yw[0]));
+          st_global_v8(yd + 16, reinterpret_cast<const uint32_t(&)[8]>(yw[8]));
+        } else {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int c = 8 * i + 2 * q;
-            __nv_bfloat162 pr =
-                __floats2bfloat162_rn((ov[c] - mean) * rstd * gate[c],
-                                      (ov[c + 1] - mean) * rstd * gate[c + 1]);
-            o32[q] = *reinterpret_cast<uint32_t*>(&pr);
-          }
-          yd[i] = out;
+          for (int i = 0; i < 4; ++i)
+            reinterpret_cast<uint4*>(yd)[i] =
+                make_uint4(yw[4 * i], yw[4 * i + 1], yw[4 * i + 2], yw[4 * i + 3]);
         }
         if (h == 0 && cq == 0 && a.ln_mean) {
           a.ln_mean[t_row] = mean;

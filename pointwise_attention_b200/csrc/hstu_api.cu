@@ -238,6 +238,8 @@ hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* 
   fill_common(p, static_cast<int*>(workspace), &a);
   a.q = q; a.k = k; a.v = v; a.u = u; a.y = y;
   a.o_save = o_save; a.ln_mean = ln_mean; a.ln_rstd = ln_rstd;
+  auto al32 = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 31u) == 0; };
+  a.vec32 = al32(u) && al32(y) && (!o_save || al32(o_save));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (p->dtype == HSTU_BF16) {

@@ -49,6 +49,7 @@ struct FwdArgs {
   int nb;            // number of time buckets (0 if no time table)
   int norm_len;
   float eps;
+  int vec32;         // u, y and o_save (if given) are 32-byte aligned
   BucketTable bt;
 };
 

@@ -155,6 +155,36 @@ def test_work_counters_return_to_zero_and_calls_repeat():
         assert_close(np64(y), ref["y"], "bf16", "y (call %d)" % call)
 
 
+def test_sixteen_byte_aligned_buffers():
+    """U, Y and the saved O at 16-byte (not 32-byte) aligned addresses take
+    the 16-byte access path and give the same result."""
+    inp = hi.make_inputs(spec((300, 170), H=2, time=True), seed=33)
+    dev = to_dev(inp)
+    T, D = inp.u.shape
+
+    def shifted(shape, dtype, like=None):
+        n = int(np.prod(shape))
+        esz = torch.tensor([], dtype=dtype).element_size()
+        big = torch.zeros(n + 64 // esz, dtype=dtype, device="cuda")
+        t = big[16 // esz:16 // esz + n].view(*shape)
+        assert t.data_ptr() % 32 == 16
+        if like is not None:
+            t.copy_(like)
+        return t
+
+    u = shifted((T, D), torch.bfloat16, dev["u"])
+    y = shifted((T, D), torch.bfloat16)
+    o_save = shifted((T, D), torch.float32)
+    saved = (o_save, torch.zeros(T, device="cuda"), torch.zeros(T, device="cuda"))
+    pa.hstu_attn_fwd(dev["q"], dev["k"], dev["v"], u, dev["offsets"], inp.max_seq_len,
+                     timestamps=dev["timestamps"], rab_pos=dev["rab_pos"],
+                     rab_time=dev["rab_time"], save_for_backward=True, y=y, saved=saved)
+    torch.cuda.synchronize()
+    ref = oracle.fwd(inp)
+    assert_close(np64(y), ref["y"], "bf16", "y")
+    assert_close(np64(o_save), ref["o"], "bf16", "o_save")
+
+
 def test_bad_device_offsets_reported():
     """Offsets that contradict max_seq_len, given without a host copy, are found
     by the kernel: the sequence is skipped and the status word says so."""
