@@ -43,7 +43,8 @@ METRIC = "causal HSTU-attention TFLOP/s (bf16) and % of B200 dense tensor peak"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
-    "fwd": ["pointwise_attention_b200/csrc/fwd_sm100.cu", "pointwise_attention_b200/csrc/ptx.cuh"],
+    "fwd": ["pointwise_attention_b200/csrc/fwd_sm100.cu", "pointwise_attention_b200/csrc/ptx.cuh",
+            "pointwise_attention_b200/csrc/tile_math.cuh", "pointwise_attention_b200/csrc/internal.h"],
 }
 
 
