@@ -19,8 +19,12 @@
 //  * hstu_bwd_dkdv_sm100 -- one CTA per (sequence, key tile, head); query
 //    tiles n..last: S^T = K Q^T and dA^T = V dO^T, the epilogue writes P'^T and
 //    dS'^T over them in TMEM, dV += P'^T dO and dK += dS'^T Q accumulate.
-// Roles as in the forward: warp 0 TMA, warp 1 TMEM + MMA issue, warps 2..17
-// the epilogue (warp w: TMEM lane quarter w%4, 32-column quarter (w-2)/4).
+// Roles: warp 0 TMA, warps 2..17 the epilogue (warp w: TMEM lane quarter w%4,
+// 32-column quarter (w-2)/4), and the MMAs issued by two or three threads in
+// warps 1, 18 and 19, one per independent accumulator chain: a tcgen05.mma
+// costs its issuing thread about 110 cycles whatever its N up to 128, as long
+// as the tensor core needs for the 128x128x16 step, so one thread issuing
+// every GEMM of a tile would leave the tensor core idle most of the time.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -30,8 +34,10 @@
 namespace hstu {
 namespace {
 
-constexpr int kThreads = 576;
+constexpr int kThreads = 640;
 constexpr int kEpi = 512;
+constexpr int kWarpB = 18;                   // second MMA issuer
+constexpr int kWarpC = 19;                   // third MMA issuer (dQ kernel)
 constexpr int kHalf = 16384;                 // 128 rows x 64 bf16
 constexpr int kTile = 2 * kHalf;             // 128 x 128 bf16
 constexpr int kTmemCols = 512;
@@ -243,13 +249,13 @@ constexpr int kSmem = kOffMisc + 64 + 1024;
 
 constexpr int B_QFULL = 0;     // Q and dO tiles
 constexpr int B_KFULL = 1;     // +stage
-constexpr int B_KEMPTY = 3;    // +stage
+constexpr int B_KEMPTY = 3;    // +stage (count 2: read by S and by dQ)
 constexpr int B_VFULL = 5;     // +stage
 constexpr int B_VEMPTY = 7;    // +stage
-constexpr int B_SFULL = 9;     // S and dA of the current tile in TMEM
+constexpr int B_SFULL = 9;     // S and dA of the current tile in TMEM (count 2)
 constexpr int B_SFREE = 10;    // epilogue has read them (count kEpi)
 constexpr int B_DSFULL = 11;   // +buffer, dS' written (count kEpi)
-constexpr int B_DQFULL = 13;   // every MMA done
+constexpr int B_DQFULL = 13;   // every MMA of the three issuers done (count 3)
 constexpr uint32_t kColS = 0, kColDA = 128, kColDQ = 256, kColDS = 384;
 
 template <bool POS, bool TIME>
@@ -290,7 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       const bool epi = (i == B_SFREE || i == B_DSFULL || i == B_DSFULL + 1);
-      mbar_init(bar(i), epi ? static_cast<uint32_t>(kEpi) : 1u);
+      uint32_t count = epi ? static_cast<uint32_t>(kEpi) : 1u;
+      if (i == B_KEMPTY || i == B_KEMPTY + 1 || i == B_SFULL) count = 2;
+      if (i == B_DQFULL) count = 3;
+      mbar_init(bar(i), count);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -299,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(sbase + kOffMisc, kTmemCols);
     tmem_relinquish();
   }
-  if (warp >= 2) {
+  if (warp >= 2 && warp < kWarpB) {
     const int et = threadIdx.x - 64;
     if (POS && et < 512) s_win[et] = 0.f;
     if (TIME) {
@@ -357,39 +366,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == kWarpB || warp == kWarpC) {
+    // ------------------------------------- MMA issuers: S (warp 1), dA, dQ
     if (lane == 0) {
-      bool ok = mbar_wait(bar(B_QFULL), 0, abort_flag);
-      auto issue_dq = [&](int n) -> bool {   // dQ += dS'(n) K_n
-        if (!mbar_wait(bar(B_DSFULL + (n & 1)), (n >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        mma_tile_tm(tmem + kColDQ, tmem + kColDS + 64u * (n & 1),
-                    sbase + kOffK + (n & 1) * kTile, n > 0);
-        mma_commit(bar(B_KEMPTY + (n & 1)));
-        return true;
-      };
-      for (int n = 0; n < nt && ok; ++n) {
-        const int st = n & 1, use = n >> 1;
-        ok = mbar_wait(bar(B_KFULL + st), use & 1, abort_flag) &&
-             mbar_wait(bar(B_VFULL + st), use & 1, abort_flag);
-        if (ok && n > 0) ok = mbar_wait(bar(B_SFREE), (n - 1) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        mma_tile_kk(tmem + kColS, sbase + kOffQ, sbase + kOffK + st * kTile, false);
-        mma_tile_kk(tmem + kColDA, sbase + kOffDO, sbase + kOffV + st * kTile, false);
-        mma_commit(bar(B_VEMPTY + st));
-        mma_commit(bar(B_SFULL));
-        if (n > 0) ok = issue_dq(n - 1);
+      bool ok = true;
+      if (warp == 1 || warp == kWarpB) {
+        ok = mbar_wait(bar(B_QFULL), 0, abort_flag);
+        for (int n = 0; n < nt && ok; ++n) {
+          const int st = n & 1, use = n >> 1;
+          ok = mbar_wait(bar((warp == 1 ? B_KFULL : B_VFULL) + st), use & 1, abort_flag);
+          // S and dA of the previous tile have been read by the epilogue.
+          if (ok && n > 0) ok = mbar_wait(bar(B_SFREE), (n - 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          if (warp == 1) {
+            mma_tile_kk(tmem + kColS, sbase + kOffQ, sbase + kOffK + st * kTile, false);
+            mma_commit(bar(B_KEMPTY + st));
+          } else {
+            mma_tile_kk(tmem + kColDA, sbase + kOffDO, sbase + kOffV + st * kTile, false);
+            mma_commit(bar(B_VEMPTY + st));
+          }
+          mma_commit(bar(B_SFULL));
+        }
+      } else {
+        for (int n = 0; n < nt && ok; ++n) {   // dQ += dS'(n) K_n
+          ok = mbar_wait(bar(B_DSFULL + (n & 1)), (n >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tile_tm(tmem + kColDQ, tmem + kColDS + 64u * (n & 1),
+                      sbase + kOffK + (n & 1) * kTile, n > 0);
+          mma_commit(bar(B_KEMPTY + (n & 1)));
+        }
       }
-      if (ok) ok = issue_dq(nt - 1);
       if (!ok) {
         set_status(a.status, kStatusTimeout);
         *abort_flag = 1;
       }
       mma_commit(bar(B_DQFULL));
     }
-  } else {
+  } else if (warp < kWarpB) {
     // ---------------------------------------------------------- epilogue
     const int q4 = warp & 3, cq = (warp - 2) >> 2;
     const int r = 32 * q4 + lane, et = threadIdx.x - 64;
@@ -546,11 +561,11 @@ constexpr int kSmem = kOffMisc + 64 + 1024;
 
 constexpr int B_KVFULL = 0;
 constexpr int B_QFULL = 1;     // +stage: Q and dO tiles
-constexpr int B_QEMPTY = 3;    // +stage
-constexpr int B_SFULL = 5;     // S^T and dA^T in TMEM
+constexpr int B_QEMPTY = 3;    // +stage (count 2: one per issuer)
+constexpr int B_SFULL = 5;     // S^T and dA^T in TMEM (count 2)
 constexpr int B_PFULL = 6;     // P'^T and dS'^T written over them (count kEpi)
-constexpr int B_PDDONE = 7;    // dV/dK MMAs of the tile done
-constexpr int B_OUT = 8;       // every MMA done
+constexpr int B_PDDONE = 7;    // dV/dK MMAs of the tile done (count 2)
+constexpr int B_OUT = 8;       // every MMA of both issuers done (count 2)
 // S^T at [0,128) with P'^T over [0,64); dA^T at [128,256) with dS'^T over [128,192)
 constexpr uint32_t kColS = 0, kColDA = 128, kColDV = 256, kColDK = 384;
 
@@ -586,7 +601,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_rabt = reinterpret_cast<float*>(smem + kOffRabT);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), i == B_PFULL ? static_cast<uint32_t>(kEpi) : 1u);
+    for (int i = 0; i < kNumBars; ++i) {
+      uint32_t count = i == B_PFULL ? static_cast<uint32_t>(kEpi) : 1u;
+      if (i == B_QEMPTY || i == B_QEMPTY + 1 || i == B_SFULL || i == B_PDDONE || i == B_OUT)
+        count = 2;
+      mbar_init(bar(i), count);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -594,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(sbase + kOffMisc, kTmemCols);
     tmem_relinquish();
   }
-  if (TIME && warp >= 2) {
+  if (TIME && warp >= 2 && warp < kWarpB) {
     const int et = threadIdx.x - 64;
     for (int i = et; i < kThrLen; i += kEpi) s_thr[i] = a.bt.thr[i];
     if (et < 64) s_first[et] = a.bt.first_k[et];
@@ -642,27 +662,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q_last[st] >= 0) mbar_wait(bar(B_QFULL + st), q_last[st] & 1, nullptr);
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == kWarpB) {
+    // ------------------- MMA issuers: S^T then dV (warp 1), dA^T then dK
     if (lane == 0) {
+      const bool first = (warp == 1);
       bool ok = mbar_wait(bar(B_KVFULL), 0, abort_flag);
       for (int it = 0; it < nq && ok; ++it) {
         const int st = it & 1;
         ok = mbar_wait(bar(B_QFULL + st), (it >> 1) & 1, abort_flag);
         // P'^T / dS'^T of the previous tile live in the S / dA columns: their
-        // dV / dK products must be finished before S^T / dA^T are rewritten.
+        // dV / dK products (both issuers') must be finished before S^T / dA^T
+        // are rewritten.
         if (ok && it > 0) ok = mbar_wait(bar(B_PDDONE), (it - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t qa = sbase + kOffQ + st * kTile, da = sbase + kOffDO + st * kTile;
-        mma_tile_kk(tmem + kColS, sbase + kOffK, qa, false);     // S^T = K Q^T
-        mma_tile_kk(tmem + kColDA, sbase + kOffV, da, false);    // dA^T = V dO^T
+        if (first)
+          mma_tile_kk(tmem + kColS, sbase + kOffK, qa, false);   // S^T = K Q^T
+        else
+          mma_tile_kk(tmem + kColDA, sbase + kOffV, da, false);  // dA^T = V dO^T
         mma_commit(bar(B_SFULL));
         ok = mbar_wait(bar(B_PFULL), it & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        mma_tile_tm(tmem + kColDV, tmem + kColS, da, it > 0);    // dV += P'^T dO
-        mma_tile_tm(tmem + kColDK, tmem + kColDA, qa, it > 0);   // dK += dS'^T Q
+        if (first)
+          mma_tile_tm(tmem + kColDV, tmem + kColS, da, it > 0);  // dV += P'^T dO
+        else
+          mma_tile_tm(tmem + kColDK, tmem + kColDA, qa, it > 0); // dK += dS'^T Q
         mma_commit(bar(B_QEMPTY + st));
         mma_commit(bar(B_PDDONE));
       }
@@ -672,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(bar(B_OUT));
     }
-  } else {
+  } else if (warp < kWarpB) {
     // ---------------------------------------------------------- epilogue
     const int q4 = warp & 3, cq = (warp - 2) >> 2;
     const int r = 32 * q4 + lane, et = threadIdx.x - 64;
