@@ -90,7 +90,7 @@ constexpr int kOffRed = kOffRabT + 128 * 4;
 constexpr int kRedBytes = 2 * kMaxHeads * 128 * 8;
 constexpr int kOffRing = kOffRed + kRedBytes;           // kRing (m, b) pairs
 constexpr int kOffBar = kOffRing + kRing * 8;           // mbarriers (8 B each)
-constexpr int kNumBars = 41;
+constexpr int kNumBars = 43;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;        // tmem base, abort flag
 constexpr int kSmemBytes = kOffMisc + 64 + 1024;        // + alignment slack
 static_assert(16 * kWarpStage >= kColGroups * 128 * 8, "LayerNorm partials must fit the staging");
@@ -112,7 +112,9 @@ constexpr int B_DONE = 22;    // every MMA of both issuers has completed
 constexpr int B_RED = 23;     // +item parity: LayerNorm statistics of all heads arrived
 constexpr int B_RFULL = 25;   // +ring slot: item written
 constexpr int B_REMPTY = 33;  // +ring slot (leader only): every CTA has read the item
-static_assert(B_REMPTY + kRing <= kNumBars, "barrier count");
+constexpr int B_ULOAD = 41;   // the item's U tile has landed in the LayerNorm buffer
+constexpr int B_LNFREE = 42;  // the LayerNorm is done with its buffer (a V stage)
+static_assert(B_LNFREE < kNumBars, "barrier count");
 constexpr int kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColO = 384;
 constexpr int kWarpPV = 18;   // warp of the P.V issuer
@@ -318,6 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     hstu_fwd_bf16_sm100(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_u,
+                        const __grid_constant__ CUtensorMap tm_y,
                         const __grid_constant__ FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -363,6 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_u);
+    tma_prefetch_desc(&tm_y);
   }
   tc_fence_before();
   __syncthreads();
@@ -461,6 +467,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = load_k(g, 0);
         for (int n = 0; n < nt && ok; ++n) {
           if (n + 1 < nt) ok = load_k(g + n + 1, n + 1);
+          // The previous item's LayerNorm borrows the V stage of this item's
+          // first tile: wait until its U load and Y store are done with it.
+          if (ok && n == 0 && j > 0) ok = mbar_wait(bar(B_LNFREE), (j - 1) & 1, abort_flag);
           if (ok) ok = load_v(g + n, n);
         }
       }
@@ -706,28 +715,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(o0[i]) * ec.inv_n;
       }
       const size_t rowD = static_cast<size_t>(t_row) * D + static_cast<size_t>(h) * 128 + 32 * cq;
-      // The gate input is requested now; its latency hides behind the exchange.
-      // Each lane owns a row, so every access below touches 32 rows: 32-byte
-      // accesses (when aligned) halve the requests the load/store unit handles.
-      uint4 uu[4];
-      {
-        const __nv_bfloat16* us = reinterpret_cast<const __nv_bfloat16*>(a.u) + rowD;
-        if (!row_ok) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) uu[i] = make_uint4(0, 0, 0, 0);
-        } else if (a.vec32) {
-          uint32_t w0[8], w1[8];
-          ld_global_nc_v8(us, w0);
-          ld_global_nc_v8(us + 16, w1);
-          uu[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-          uu[1] = make_uint4(w0[4], w0[5], w0[6], w0[7]);
-          uu[2] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-          uu[3] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) uu[i] = __ldg(reinterpret_cast<const uint4*>(us) + i);
-        }
+      // U and Y of the item travel by TMA through the V stage of the next
+      // item's first tile (every P.V of this item has completed; the producer
+      // waits for B_LNFREE before loading it again).  In that 128B-swizzled
+      // tile, 16-byte chunk c of row r sits at r * 128 + 16 (c ^ (r % 8)) of
+      // its 64-column half: a warp's 32 rows hit every bank once per 8 rows.
+      const uint32_t lnbuf = sbase + kOffV + ((g + nt) % kVStages) * kTile;
+      if (et == 0) {
+        const int row0 = s + kRows * m;
+        mbar_arrive_expect_tx(bar(B_ULOAD), kTile);
+        tma_load_3d(lnbuf, &tm_u, bar(B_ULOAD), 0, h, row0);
+        tma_load_3d(lnbuf + kHalf, &tm_u, bar(B_ULOAD), 64, h, row0);
       }
+      const uint32_t myrow = lnbuf + (cq >> 1) * kHalf + r * 128;
+      auto chunk_addr = [&](int i) {   // i-th 16-byte chunk of this thread's 32 columns
+        return myrow + 16u * static_cast<uint32_t>((4 * (cq & 1) + i) ^ (r & 7));
+      };
       if (ok && row_ok && a.o_save) {
         float* od = a.o_save + rowD;
         if (a.vec32) {
@@ -783,10 +786,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (et == 0) mbar_arrive_expect_tx(bar(B_RED + pj), static_cast<uint32_t>(H * 128 * 8));
       // Gate values while the statistics travel.
+      if (!mbar_wait(bar(B_ULOAD), j & 1, abort_flag)) set_status(a.status, kStatusTimeout);
       float gate[32];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&uu[i]);
+        const uint4 ui = ld_shared_v4(chunk_addr(i));
+        const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&ui);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float2 uf = __bfloat1622float2(u2[q]);
@@ -808,8 +813,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float var = m2 / static_cast<float>(D);
       const float rstd = 1.0f / sqrtf(var + a.eps);
-      if (row_ok) {
-        __nv_bfloat16* yd = reinterpret_cast<__nv_bfloat16*>(a.y) + rowD;
+      {
         uint32_t yw[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
@@ -817,18 +821,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                     (ov[2 * q + 1] - mean) * rstd * gate[2 * q + 1]);
           yw[q] = *reinterpret_cast<uint32_t*>(&pr);
         }
-        if (a.vec32) {
-          st_global_v8(yd, reinterpret_cast<const uint32_t(&)[8]>(yw[0]));
-          st_global_v8(yd + 16, reinterpret_cast<const uint32_t(&)[8]>(yw[8]));
-        } else {
+        // A tile whose 128 rows all belong to the sequence leaves by one TMA
+        // store; the last, partial tile of a sequence stores its rows directly.
+        const bool full = kRows * m + kRows <= n_b;
+        if (full) {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            reinterpret_cast<uint4*>(yd)[i] =
-                make_uint4(yw[4 * i], yw[4 * i + 1], yw[4 * i + 2], yw[4 * i + 3]);
+            st_shared_v4(chunk_addr(i), make_uint4(yw[4 * i], yw[4 * i + 1], yw[4 * i + 2],
+                                                   yw[4 * i + 3]));
+          fence_proxy_async_smem();
+        } else if (row_ok) {
+          __nv_bfloat16* yd = reinterpret_cast<__nv_bfloat16*>(a.y) + rowD;
+          if (a.vec32) {
+            st_global_v8(yd, reinterpret_cast<const uint32_t(&)[8]>(yw[0]));
+            st_global_v8(yd + 16, reinterpret_cast<const uint32_t(&)[8]>(yw[8]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              reinterpret_cast<uint4*>(yd)[i] =
+                  make_uint4(yw[4 * i], yw[4 * i + 1], yw[4 * i + 2], yw[4 * i + 3]);
+          }
         }
-        if (h == 0 && cq == 0 && a.ln_mean) {
+        if (row_ok && h == 0 && cq == 0 && a.ln_mean) {
           a.ln_mean[t_row] = mean;
           a.ln_rstd[t_row] = rstd;
+        }
+        // Every thread is done with the buffer (its U read, its Y written).
+        named_bar_sync(3, kEpiThreads);
+        if (et == 0) {
+          if (full) {
+            tma_store_3d(&tm_y, lnbuf, 0, h, s + kRows * m);
+            tma_store_3d(&tm_y, lnbuf + kHalf, 64, h, s + kRows * m);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+          mbar_arrive(bar(B_LNFREE));
         }
       }
       g += nt;
@@ -838,6 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       set_status(a.status, kStatusTimeout);
       *abort_flag = 1;
     }
+    if (et == 0) bulk_wait_group0();   // the last Y stores have landed
     tc_fence_before();
   }
 
@@ -856,7 +884,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <bool POS, bool TIME>
 cudaError_t launch_variant(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                           const CUtensorMap& tv, cudaStream_t stream) {
+                           const CUtensorMap& tv, const CUtensorMap& tu, const CUtensorMap& ty,
+                           cudaStream_t stream) {
   // The shared-memory opt-in is a per-device function attribute, and the
   // number of co-resident clusters a per-device, per-cluster-size property:
   // both are taken once per device (not inside a stream capture of a later call).
@@ -894,22 +923,23 @@ cudaError_t launch_variant(const FwdArgs& a, const CUtensorMap& tq, const CUtens
   const long long nslots = static_cast<long long>(a.B) * a.max_tiles;
   const long long clusters = std::min<long long>(resident, nslots);
   cfg.gridDim = dim3(static_cast<unsigned>(clusters * a.H), 1, 1);
-  return cudaLaunchKernelEx(&cfg, hstu_fwd_bf16_sm100<POS, TIME>, tq, tk, tv, a);
+  return cudaLaunchKernelEx(&cfg, hstu_fwd_bf16_sm100<POS, TIME>, tq, tk, tv, tu, ty, a);
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                                  const CUtensorMap& tv, cudaStream_t stream) {
+                                  const CUtensorMap& tv, const CUtensorMap& tu,
+                                  const CUtensorMap& ty, cudaStream_t stream) {
   if (a.B == 0 || a.max_tiles == 0) return cudaSuccess;
   if (a.H < 1 || a.H > kMaxHeads) return cudaErrorInvalidValue;
   // Work slots are numbered in 32 bits (plus one claim window of 32).
   if (static_cast<long long>(a.B) * a.max_tiles > 0x7FFFFF00LL) return cudaErrorInvalidValue;
   const bool pos = a.rab_pos != nullptr, tim = a.rab_time != nullptr;
-  if (pos && tim) return launch_variant<true, true>(a, tq, tk, tv, stream);
-  if (pos) return launch_variant<true, false>(a, tq, tk, tv, stream);
-  if (tim) return launch_variant<false, true>(a, tq, tk, tv, stream);
-  return launch_variant<false, false>(a, tq, tk, tv, stream);
+  if (pos && tim) return launch_variant<true, true>(a, tq, tk, tv, tu, ty, stream);
+  if (pos) return launch_variant<true, false>(a, tq, tk, tv, tu, ty, stream);
+  if (tim) return launch_variant<false, true>(a, tq, tk, tv, tu, ty, stream);
+  return launch_variant<false, false>(a, tq, tk, tv, tu, ty, stream);
 }
 
 }  // namespace hstu

@@ -243,12 +243,14 @@ hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (p->dtype == HSTU_BF16) {
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tu, ty;   // U and Y [T, H*128] seen as [T, H, 128]
     if (!make_map_3d(&tq, q, p->total_tokens, p->num_heads, 128) ||
         !make_map_3d(&tk, k, p->total_tokens, p->num_heads, 128) ||
-        !make_map_3d(&tv, v, p->total_tokens, p->num_heads, 128))
+        !make_map_3d(&tv, v, p->total_tokens, p->num_heads, 128) ||
+        !make_map_3d(&tu, u, p->total_tokens, p->num_heads, 128) ||
+        !make_map_3d(&ty, y, p->total_tokens, p->num_heads, 128))
       return HSTU_ERR_CUDA;
-    err = launch_fwd_bf16_sm100(a, tq, tk, tv, s);
+    err = launch_fwd_bf16_sm100(a, tq, tk, tv, tu, ty, s);
   } else {
     err = launch_fwd_f32_simt(a, s);
   }

@@ -86,7 +86,8 @@ struct BwdArgs {
 
 // Kernel launchers (return cudaSuccess or the launch error).
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                                  const CUtensorMap& tv, cudaStream_t stream);
+                                  const CUtensorMap& tv, const CUtensorMap& tu,
+                                  const CUtensorMap& ty, cudaStream_t stream);
 cudaError_t launch_fwd_f32_simt(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_f32_simt(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_bf16_simt(const BwdArgs& a, cudaStream_t stream);
