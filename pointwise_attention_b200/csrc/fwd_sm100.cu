@@ -16,10 +16,11 @@
 // concatenated heads exchanges per-row statistics through distributed shared
 // memory.  The kernel is persistent: the grid holds as many clusters as can
 // be resident, and each cluster loops over items that its leader CTA (rank 0)
-// claims from a work counter in global memory.  Items are numbered from the
-// most expensive (largest m) down, so the claims form a longest-first list
-// schedule; slots whose tile lies past the end of its sequence are skipped in
-// runs of up to 32 per claim.  The leader claims the next item once its loads
+// claims from a work counter in global memory (the first one, slot c for
+// cluster c, without a claim).  Items are numbered from the most expensive
+// (largest m) down, so the claims form a longest-first list schedule; slots
+// whose tile lies past the end of its sequence are skipped in runs of up to
+// 32 per claim.  The leader claims the next item once its loads
 // for the current item are issued and hands it to every CTA of the cluster
 // through an 8-entry ring in shared memory.  While the epilogue normalises
 // item j, the TMA and MMA warps already load and multiply item j+1.
@@ -280,24 +281,30 @@ __device__ __forceinline__ int2 load_seq(const FwdArgs& a, int b, bool pos) {
 
 // Claims this cluster's next item (warp-collective; leader CTA's warp 0).
 // Slot k of the launch is the item (m = M-1 - k/B, b = k mod B), so the most
-// expensive query tiles come first.  The counter holds the next free slot and
-// an atomic add claims one.  A slot whose tile lies past its sequence end
-// holds no work: the warp then tests the 31 slots after it and raises the
-// counter past the empty ones among them (atomicMax; every skipped slot was
-// seen empty, and no slot is handed out twice), then claims again.  Returns
-// (-1, -1) once the slots are exhausted.
+// expensive query tiles come first.  Cluster c takes slot c as its first
+// item without touching the counter (the first `base` slots, one per
+// cluster); every later claim takes slot base + the counter's old value from
+// an atomic add.  A slot whose tile lies past its sequence end holds no work:
+// the warp then tests the 31 slots after it and raises the counter past the
+// empty ones among them (atomicMax; every skipped slot was seen empty, and no
+// slot is handed out twice), then claims again.  Returns (-1, -1) once the
+// slots are exhausted.
 template <bool POS>
-__device__ int2 claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots, int lane) {
+__device__ int2 claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots, unsigned base,
+                           int first, int lane) {
   const unsigned B = static_cast<unsigned>(a.B);
   const int M = a.max_tiles;
+  bool fixed = first >= 0;
   for (;;) {
-    unsigned k = 0;
-    if (lane == 0) k = atomicAdd(counter, 1u);
-    k = __shfl_sync(0xffffffffu, k, 0);
+    unsigned k = static_cast<unsigned>(first);
+    if (!fixed) {
+      if (lane == 0) k = atomicAdd(counter, 1u) + base;
+      k = __shfl_sync(0xffffffffu, k, 0);
+    }
     if (k >= nslots) return make_int2(-1, -1);
     const unsigned slot = k + static_cast<unsigned>(lane);
     bool valid = false;
-    if (slot < nslots) {
+    if (slot < nslots && (!fixed || lane == 0)) {
       const int m = M - 1 - static_cast<int>(slot / B);
       const int b = static_cast<int>(slot % B);
       const int2 sq = load_seq(a, b, POS);
@@ -309,9 +316,13 @@ __device__ int2 claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots,
     }
     const unsigned vb = __ballot_sync(0xffffffffu, valid);
     if (vb & 1u) return make_int2(M - 1 - static_cast<int>(k / B), static_cast<int>(k % B));
+    if (fixed) {          // the cluster's own first slot is empty: claim from the counter
+      fixed = false;
+      continue;
+    }
     const unsigned rest = vb & ~1u;
     const unsigned skip_to = rest ? k + static_cast<unsigned>(__ffs(rest) - 1) : k + 32u;
-    if (lane == 0 && skip_to > k + 1) atomicMax(counter, min(skip_to, nslots));
+    if (lane == 0 && skip_to > k + 1) atomicMax(counter, min(skip_to, nslots) - base);
   }
 }
 
@@ -404,7 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           okf = mbar_wait<true>(bar(B_REMPTY + j % kRing), ((j / kRing) - 1) & 1, abort_flag);
         okf = __shfl_sync(0xffffffffu, okf, 0);
         if (okf) {
-          it = claim_item<POS>(a, counter, nslots, lane);
+          const unsigned clusters = gridDim.x / static_cast<unsigned>(H);
+          it = claim_item<POS>(a, counter, nslots, clusters,
+                               j == 0 ? static_cast<int>(blockIdx.x / static_cast<unsigned>(H)) : -1,
+                               lane);
           if (lane == 0) {
             for (int pr = 0; pr < H; ++pr) {
               st_cluster_v2_s32(mapa_shared(ring_addr(j % kRing), pr), it.x, it.y);

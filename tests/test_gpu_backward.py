@@ -42,6 +42,7 @@ def test_fp32_backward(case):
     dict(lengths=(128,), H=1),
     dict(lengths=(1, 200, 129), H=4, time=True),
     dict(lengths=(300, 0, 64), H=2, norm="fixed", norm_len=300),
+    dict(lengths=(257, 129), H=8, time=True),
 ])
 def test_bf16_backward_small(case):
     check_bwd(hi.make_inputs(spec(**case), seed=12), "bf16")

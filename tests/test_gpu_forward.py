@@ -49,6 +49,8 @@ def test_tiny_fp32_workload():
     dict(lengths=(640,), H=3, time=True, L=1000),
     dict(lengths=(260, 131), H=2, time=True, ts_sorted=False),
     dict(lengths=(300, 257), H=4, qk_std=1.0, rab_std=1.0, time=True),   # stress: large logits
+    dict(lengths=(257, 100, 33), H=5, time=True),                          # odd cluster sizes
+    dict(lengths=(129, 129, 129), H=7),
 ])
 def test_bf16_small(case):
     inp = hi.make_inputs(spec(**case), seed=1)
@@ -183,6 +185,15 @@ def test_sixteen_byte_aligned_buffers():
     ref = oracle.fwd(inp)
     assert_close(np64(y), ref["y"], "bf16", "y")
     assert_close(np64(o_save), ref["o"], "bf16", "o_save")
+
+
+def test_many_short_sequences():
+    """Hundreds of sequences of 0 to 300 tokens: most work slots of the
+    launch are empty and the clusters claim many small items."""
+    rng = np.random.default_rng(41)
+    lengths = tuple(int(x) for x in rng.integers(0, 301, size=180))
+    inp = hi.make_inputs(spec(lengths, H=2, time=True, L=300), seed=42)
+    check_full(inp, "bf16")
 
 
 def test_bad_device_offsets_reported():
