@@ -415,7 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float nrm = a.norm_len > 0 ? static_cast<float>(a.norm_len) : static_cast<float>(n_b);
     const float inv_n = 1.0f / nrm;
     const int Lw = 2 * a.L - 1;
-    const long long my_ts = TIME ? a.timestamps[t_row] : 0;
+    // Query rows past the sequence end (never stored) take the last token's
+    // timestamp, which keeps their chunk plans on the cheap path.
+    const long long my_ts = TIME ? a.timestamps[row_ok ? t_row : s + n_b - 1] : 0;
     Stage* stg = reinterpret_cast<Stage*>(smem + kOffStage) + (warp - 2);
     // This warp's block: rows 32 q4.., columns 32 cq..; diagonals
     // d = r - c in [32 q4 - 32 cq - 31, +31] (local index lane - cl + 31).

@@ -637,7 +637,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = i_loc < n_b;
       const int t_row = s + (row_ok ? i_loc : 0);
       const float nrm = a.norm_len > 0 ? static_cast<float>(a.norm_len) : static_cast<float>(n_b);
-      ec.my_ts = TIME ? a.timestamps[t_row] : 0;
+      // Rows past the sequence end (never stored) take the last token's
+      // timestamp: every key is then at or before them, the chunk plans stay
+      // on the cheap path, and no warp drops to the per-element search.
+      ec.my_ts = TIME ? a.timestamps[row_ok ? t_row : s + n_b - 1] : 0;
       ec.inv_n = 1.0f / nrm;
       // The gate input of this row is read at the end of the item: ask L2 for it now.
       if (row_ok)
