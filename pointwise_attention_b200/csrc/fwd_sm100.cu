@@ -279,9 +279,18 @@ __device__ __forceinline__ int2 load_seq(const FwdArgs& a, int b, bool pos) {
   return make_int2(s, n);
 }
 
-// Claims this cluster's next item (warp-collective; leader CTA's warp 0).
-// Slot k of the launch is the item (m = M-1 - k/B, b = k mod B), so the most
-// expensive query tiles come first.  Cluster c takes slot c as its first
+// Work slots: sequences are taken in groups of G whose keys and values fit in
+// L2 together; inside a group, slot r is the item (m = M-1 - r/G, b = group
+// * G + r mod G), so the most expensive query tiles of the group come first
+// (a longest-first list schedule), and the K/V tiles every query tile of a
+// sequence reads stay in L2 while the group is worked on.
+__device__ __forceinline__ int2 slot_item(unsigned k, unsigned G, int M) {
+  const unsigned per = G * static_cast<unsigned>(M);
+  const unsigned grp = k / per, r = k % per;
+  return make_int2(M - 1 - static_cast<int>(r / G), static_cast<int>(grp * G + r % G));
+}
+
+// Claims this cluster's next item (warp-collective; leader CTA's warp 0).  Cluster c takes slot c as its first
 // item without touching the counter (the first `base` slots, one per
 // cluster); every later claim takes slot base + the counter's old value from
 // an atomic add.  A slot whose tile lies past its sequence end holds no work:
@@ -292,7 +301,7 @@ __device__ __forceinline__ int2 load_seq(const FwdArgs& a, int b, bool pos) {
 template <bool POS>
 __device__ int2 claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots, unsigned base,
                            int first, int lane) {
-  const unsigned B = static_cast<unsigned>(a.B);
+  const unsigned G = static_cast<unsigned>(a.group);
   const int M = a.max_tiles;
   bool fixed = first >= 0;
   for (;;) {
@@ -305,17 +314,18 @@ __device__ int2 claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots,
     const unsigned slot = k + static_cast<unsigned>(lane);
     bool valid = false;
     if (slot < nslots && (!fixed || lane == 0)) {
-      const int m = M - 1 - static_cast<int>(slot / B);
-      const int b = static_cast<int>(slot % B);
-      const int2 sq = load_seq(a, b, POS);
-      if (sq.y < 0) {
-        if (m == 0) set_status(a.status, kStatusBadOffsets);
-      } else {
-        valid = kRows * m < sq.y;
+      const int2 it = slot_item(slot, G, M);
+      if (it.y < a.B) {   // the last group may be partial
+        const int2 sq = load_seq(a, it.y, POS);
+        if (sq.y < 0) {
+          if (it.x == 0) set_status(a.status, kStatusBadOffsets);
+        } else {
+          valid = kRows * it.x < sq.y;
+        }
       }
     }
     const unsigned vb = __ballot_sync(0xffffffffu, valid);
-    if (vb & 1u) return make_int2(M - 1 - static_cast<int>(k / B), static_cast<int>(k % B));
+    if (vb & 1u) return slot_item(k, G, M);
     if (fixed) {          // the cluster's own first slot is empty: claim from the counter
       fixed = false;
       continue;
@@ -404,7 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     unsigned* counter = reinterpret_cast<unsigned*>(a.status) + kSchedCounterWord;
     unsigned* done = reinterpret_cast<unsigned*>(a.status) + kSchedDoneWord;
-    const unsigned nslots = static_cast<unsigned>(a.B) * static_cast<unsigned>(a.max_tiles);
+    const unsigned nslots = static_cast<unsigned>((a.B + a.group - 1) / a.group) *
+                            static_cast<unsigned>(a.group) * static_cast<unsigned>(a.max_tiles);
     // Leader: claim item j and hand it to every CTA of the cluster (warp-collective).
     auto fetch = [&](int j) -> int2 {
       bool okf = true;
@@ -937,7 +948,8 @@ cudaError_t launch_variant(const FwdArgs& a, const CUtensorMap& tq, const CUtens
     if (err != cudaSuccess) return err;
     resident = n > 0 ? n : 1;
   }
-  const long long nslots = static_cast<long long>(a.B) * a.max_tiles;
+  const long long nslots = static_cast<long long>((a.B + a.group - 1) / a.group) * a.group *
+                           a.max_tiles;
   const long long clusters = std::min<long long>(resident, nslots);
   cfg.gridDim = dim3(static_cast<unsigned>(clusters * a.H), 1, 1);
   return cudaLaunchKernelEx(&cfg, hstu_fwd_bf16_sm100<POS, TIME>, tq, tk, tv, tu, ty, a);
@@ -951,7 +963,9 @@ cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const
   if (a.B == 0 || a.max_tiles == 0) return cudaSuccess;
   if (a.H < 1 || a.H > kMaxHeads) return cudaErrorInvalidValue;
   // Work slots are numbered in 32 bits (plus one claim window of 32).
-  if (static_cast<long long>(a.B) * a.max_tiles > 0x7FFFFF00LL) return cudaErrorInvalidValue;
+  if (a.group < 1 || a.group > a.B) return cudaErrorInvalidValue;
+  if ((static_cast<long long>(a.B) + a.group) * a.max_tiles > 0x7FFFFF00LL)
+    return cudaErrorInvalidValue;
   const bool pos = a.rab_pos != nullptr, tim = a.rab_time != nullptr;
   if (pos && tim) return launch_variant<true, true>(a, tq, tk, tv, tu, ty, stream);
   if (pos) return launch_variant<true, false>(a, tq, tk, tv, tu, ty, stream);

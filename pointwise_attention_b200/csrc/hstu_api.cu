@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -132,7 +133,7 @@ hstu_status_t check_problem(const hstu_problem_t* p) {
 
 bool bf16_supported(const hstu_problem_t* p) {
   // The forward numbers its (sequence, query tile) work slots in 32 bits.
-  const int64_t slots = static_cast<int64_t>(p->batch) * ((p->max_seq_len + 127) / 128);
+  const int64_t slots = 2 * static_cast<int64_t>(p->batch) * ((p->max_seq_len + 127) / 128);
   return p->dtype == HSTU_BF16 && p->d_qk == 128 && p->d_v == 128 && p->num_heads <= 8 &&
          slots <= 0x7FFFFF00LL;
 }
@@ -238,6 +239,14 @@ hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* 
   fill_common(p, static_cast<int*>(workspace), &a);
   a.q = q; a.k = k; a.v = v; a.u = u; a.y = y;
   a.o_save = o_save; a.ln_mean = ln_mean; a.ln_rstd = ln_rstd;
+  // Scheduling groups of the bf16 forward: as many sequences as keep their K
+  // and V (at max_seq_len) within about 40 MB of the 126 MB L2.
+  {
+    const double kv = static_cast<double>(p->max_seq_len) * p->num_heads *
+                      (p->d_qk + p->d_v) * 2.0;
+    const double g = kv > 0 ? std::floor(40.0e6 / kv) : p->batch;
+    a.group = static_cast<int>(std::max(1.0, std::min(static_cast<double>(p->batch), g)));
+  }
   auto al32 = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 31u) == 0; };
   a.vec32 = al32(u) && al32(y) && (!o_save || al32(o_save));
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -50,6 +50,7 @@ struct FwdArgs {
   int norm_len;
   float eps;
   int vec32;         // u, y and o_save (if given) are 32-byte aligned
+  int group;         // bf16 forward: sequences per scheduling group (>= 1)
   BucketTable bt;
 };
 
