@@ -188,54 +188,61 @@ __global__ void __launch_bounds__(kT) bwd_pre_simt(const BwdArgs a) {
 
 // The same LayerNorm/gate backward for bf16 with d_v = 128, one warp per
 // token row: lane l holds columns 128 c + 4 l .. +3 of every 128-column slice
-// c < H, so each load or store instruction of the warp covers one contiguous
-// 256-byte (bf16) or 512-byte (fp32) span, and the row stays in registers
-// between the two reductions and the dO pass.
+// c < NC = H, so each load or store instruction of the warp covers one
+// contiguous 256-byte (bf16) or 512-byte (fp32) span.  All loads of the row are
+// issued before any arithmetic or store (the argument pointers may alias as far
+// as the compiler knows, so it would not hoist a later slice's loads above an
+// earlier slice's dU store), and the row stays in registers between the two
+// reductions and the dO pass.
 constexpr int kRowsPerBlock = 8;
 
+template <int NC>
 __global__ void __launch_bounds__(32 * kRowsPerBlock) bwd_pre_rows_bf16(const BwdArgs a) {
   const int t = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= a.T) return;
-  const int D = a.H * 128;
-  const float mean = a.ln_mean[t], rstd = a.ln_rstd[t];
+  constexpr int D = NC * 128;
   const size_t base = static_cast<size_t>(t) * D + 4 * lane;
   const __nv_bfloat16* u = static_cast<const __nv_bfloat16*>(a.u);
   const __nv_bfloat16* dy = static_cast<const __nv_bfloat16*>(a.dy);
   __nv_bfloat16* du = static_cast<__nv_bfloat16*>(a.du);
   __nv_bfloat16* dO = static_cast<__nv_bfloat16*>(a.dO);
-  float xh[32], dx[32];
+  float4 ov[NC];
+  uint2 uv[NC], gv[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const size_t o = base + 128 * c;
+    ov[c] = __ldcs(reinterpret_cast<const float4*>(a.o_save + o));
+    uv[c] = __ldcs(reinterpret_cast<const uint2*>(u + o));
+    gv[c] = __ldcs(reinterpret_cast<const uint2*>(dy + o));
+  }
+  const float mean = __ldg(a.ln_mean + t), rstd = __ldg(a.ln_rstd + t);
+  float xh[4 * NC], dx[4 * NC];
   float m1 = 0.f, m2 = 0.f;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    if (c < a.H) {
-      const size_t o = base + 128 * c;
-      const float4 ov = *reinterpret_cast<const float4*>(a.o_save + o);
-      const uint2 uv = *reinterpret_cast<const uint2*>(u + o);
-      const uint2 gv = *reinterpret_cast<const uint2*>(dy + o);
-      const float2 u01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv.x));
-      const float2 u23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv.y));
-      const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.x));
-      const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.y));
-      const float ovs[4] = {ov.x, ov.y, ov.z, ov.w};
-      const float us[4] = {u01.x, u01.y, u23.x, u23.y};
-      const float gs[4] = {g01.x, g01.y, g23.x, g23.y};
-      float dus[4];
+  for (int c = 0; c < NC; ++c) {
+    const float2 u01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv[c].x));
+    const float2 u23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv[c].y));
+    const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv[c].x));
+    const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv[c].y));
+    const float ovs[4] = {ov[c].x, ov[c].y, ov[c].z, ov[c].w};
+    const float us[4] = {u01.x, u01.y, u23.x, u23.y};
+    const float gs[4] = {g01.x, g01.y, g23.x, g23.y};
+    float dus[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float x = (ovs[e] - mean) * rstd;
-        const float d = gs[e] * silu_f(us[e]);
-        dus[e] = gs[e] * x * silu_grad_f(us[e]);
-        xh[4 * c + e] = x;
-        dx[4 * c + e] = d;
-        m1 += d;
-        m2 = fmaf(d, x, m2);
-      }
-      __nv_bfloat162 d01 = __floats2bfloat162_rn(dus[0], dus[1]);
-      __nv_bfloat162 d23 = __floats2bfloat162_rn(dus[2], dus[3]);
-      *reinterpret_cast<uint2*>(du + o) = make_uint2(*reinterpret_cast<uint32_t*>(&d01),
-                                                     *reinterpret_cast<uint32_t*>(&d23));
+    for (int e = 0; e < 4; ++e) {
+      const float x = (ovs[e] - mean) * rstd;
+      const float d = gs[e] * silu_f(us[e]);
+      dus[e] = gs[e] * x * silu_grad_f(us[e]);
+      xh[4 * c + e] = x;
+      dx[4 * c + e] = d;
+      m1 += d;
+      m2 = fmaf(d, x, m2);
     }
+    __nv_bfloat162 d01 = __floats2bfloat162_rn(dus[0], dus[1]);
+    __nv_bfloat162 d23 = __floats2bfloat162_rn(dus[2], dus[3]);
+    __stcs(reinterpret_cast<uint2*>(du + base + 128 * c),
+           make_uint2(*reinterpret_cast<uint32_t*>(&d01), *reinterpret_cast<uint32_t*>(&d23)));
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -245,16 +252,14 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock) bwd_pre_rows_bf16(const Bw
   m1 /= static_cast<float>(D);
   m2 /= static_cast<float>(D);
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    if (c < a.H) {
-      float r4[4];
+  for (int c = 0; c < NC; ++c) {
+    float r4[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) r4[e] = rstd * (dx[4 * c + e] - m1 - xh[4 * c + e] * m2);
-      __nv_bfloat162 d01 = __floats2bfloat162_rn(r4[0], r4[1]);
-      __nv_bfloat162 d23 = __floats2bfloat162_rn(r4[2], r4[3]);
-      *reinterpret_cast<uint2*>(dO + base + 128 * c) =
-          make_uint2(*reinterpret_cast<uint32_t*>(&d01), *reinterpret_cast<uint32_t*>(&d23));
-    }
+    for (int e = 0; e < 4; ++e) r4[e] = rstd * (dx[4 * c + e] - m1 - xh[4 * c + e] * m2);
+    __nv_bfloat162 d01 = __floats2bfloat162_rn(r4[0], r4[1]);
+    __nv_bfloat162 d23 = __floats2bfloat162_rn(r4[2], r4[3]);
+    *reinterpret_cast<uint2*>(dO + base + 128 * c) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&d01), *reinterpret_cast<uint32_t*>(&d23));
   }
 }
 
@@ -394,7 +399,17 @@ cudaError_t launch_bwd_pre_bf16(const BwdArgs& a, cudaStream_t stream) {
   if (a.T == 0) return cudaSuccess;
   if (a.d_v == 128 && a.H >= 1 && a.H <= 8) {
     const unsigned blocks = static_cast<unsigned>((a.T + kRowsPerBlock - 1) / kRowsPerBlock);
-    bwd_pre_rows_bf16<<<blocks, 32 * kRowsPerBlock, 0, stream>>>(a);
+    const dim3 g(blocks), b(32 * kRowsPerBlock);
+    switch (a.H) {
+      case 1: bwd_pre_rows_bf16<1><<<g, b, 0, stream>>>(a); break;
+      case 2: bwd_pre_rows_bf16<2><<<g, b, 0, stream>>>(a); break;
+      case 3: bwd_pre_rows_bf16<3><<<g, b, 0, stream>>>(a); break;
+      case 4: bwd_pre_rows_bf16<4><<<g, b, 0, stream>>>(a); break;
+      case 5: bwd_pre_rows_bf16<5><<<g, b, 0, stream>>>(a); break;
+      case 6: bwd_pre_rows_bf16<6><<<g, b, 0, stream>>>(a); break;
+      case 7: bwd_pre_rows_bf16<7><<<g, b, 0, stream>>>(a); break;
+      default: bwd_pre_rows_bf16<8><<<g, b, 0, stream>>>(a); break;
+    }
   } else {
     bwd_pre_simt<__nv_bfloat16><<<a.T, kT, 0, stream>>>(a);
   }
