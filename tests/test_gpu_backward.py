@@ -11,11 +11,11 @@ pytestmark = pytest.mark.gpu
 
 
 def spec(lengths, H=4, d=128, dtype="bf16", pos=True, time=False, norm="own", norm_len=0,
-         qk_std=1 / np.sqrt(128), L=None):
+         qk_std=1 / np.sqrt(128), L=None, ts_sorted=True):
     return hi.Spec("case", dtype, batch=len(lengths), heads=H, d_qk=d, d_v=d,
                    lengths=tuple(lengths), qk_std=qk_std, vu_std=1.0,
                    rab_pos_len=(L or max(lengths)) if pos else 0, rab_time=time,
-                   norm=norm, norm_len=norm_len, grad=True)
+                   norm=norm, norm_len=norm_len, grad=True, ts_sorted=ts_sorted)
 
 
 def check_bwd(inp, dtype, rows_of=None):
@@ -43,6 +43,10 @@ def test_fp32_backward(case):
     dict(lengths=(1, 200, 129), H=4, time=True),
     dict(lengths=(300, 0, 64), H=2, norm="fixed", norm_len=300),
     dict(lengths=(257, 129), H=8, time=True),
+    # unsorted timestamps: both kernels take the per-element bucket search and
+    # the dQ kernel accumulates d(rab_time) per element
+    dict(lengths=(260, 131), H=2, time=True, ts_sorted=False),
+    dict(lengths=(200,), H=4, pos=False, time=True, ts_sorted=False),
 ])
 def test_bf16_backward_small(case):
     check_bwd(hi.make_inputs(spec(**case), seed=12), "bf16")
@@ -51,6 +55,12 @@ def test_bf16_backward_small(case):
 def test_train_reduced_batch():
     """The training workload's shapes and distributions with 2 sequences."""
     check_bwd(hi.make_inputs(hi.workload("train", batch=2), seed=0), "bf16")
+
+
+def test_train_shapes_with_time_bias():
+    """Training shapes (2 x 2048 tokens, H=4) with the time bias added: the
+    backward of both relative biases at once, d(rab_time) included."""
+    check_bwd(hi.make_inputs(hi.workload("train", batch=2, rab_time=True), seed=3), "bf16")
 
 
 def test_train_full_size():
