@@ -7,7 +7,7 @@ any of the method's code.
 
 Shapes follow the HSTU model card ("HSTU (Generative Recommender)", Structure
 table and Exported PyTorch: embed 512, 4 heads, d_qk = d_v = 128, 1024 tokens)
-and the five named workloads below.  Every draw comes from one CPU
+and the six named workloads below.  Every draw comes from one CPU
 ``torch.Generator`` seeded per workload, in a fixed order:
 
     lengths -> Q -> K -> V -> U -> timestamps -> rab_pos -> rab_time -> dY
@@ -73,6 +73,10 @@ def _spec_table() -> Dict[str, Spec]:
         # Training step: 16 x 2048 tokens, position bias, upstream gradient dY.
         "train": Spec("train", "bf16", batch=16, heads=4, d_qk=128, d_v=128, seq_len=2048,
                       qk_std=s, rab_pos_len=2048, grad=True),
+        # The training step with the time bias as well: timestamps as in the
+        # jagged and long workloads, and the backward of both bias tables.
+        "train_time": Spec("train_time", "bf16", batch=16, heads=4, d_qk=128, d_v=128,
+                           seq_len=2048, qk_std=s, rab_pos_len=2048, rab_time=True, grad=True),
     }
 
 
