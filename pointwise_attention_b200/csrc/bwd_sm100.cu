@@ -151,6 +151,12 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
   // at column cl lane L reads column cl of lane (L + cl) mod 32, so every
   // element of diagonal L (row - column = L) or L - 32 passes through lane L.
   float dpos = 0.f, dneg = 0.f;
+  // Per-element time buckets: the row's dS' is summed over runs of equal
+  // bucket (with sorted timestamps the bucket only falls along the row) and a
+  // run goes to the shared histogram when the bucket changes, instead of one
+  // contended shared atomic per element.
+  int run_k = -1;
+  float run_s = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float ds2[2];
@@ -168,7 +174,8 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
       const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
       const float t = tanh_approx(hx);
       float ds = __uint_as_float(dav[cl]) * silu_grad_h(hx, t);
-      if (MASK && ((diag && c > r) || !row_ok)) ds = 0.f;
+      const bool masked = MASK && ((diag && c > r) || !row_ok);
+      if (masked) ds = 0.f;
       ds2[hh] = ds;
       if (POS) {
         const float v = __shfl_sync(0xffffffffu, ds, (lane + cl) & 31);
@@ -177,13 +184,19 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
       if (TIME) {
         if (!generic) {
           if (cl < ct.split) t_lo += ds; else t_hi += ds;
-        } else {
-          atomicAdd(&s_dt[kb], ds);
+        } else if (!masked) {
+          if (kb != run_k) {
+            if (run_k >= 0) atomicAdd(&s_dt[run_k], run_s);
+            run_k = kb;
+            run_s = 0.f;
+          }
+          run_s += ds;
         }
       }
     }
     packed[i] = pack_bf16(ds2[0], ds2[1]);
   }
+  if (TIME && run_k >= 0) atomicAdd(&s_dt[run_k], run_s);
   if (POS) {
     // lane L holds diagonal L (window index r - c0 + 127 for this row's lane)
     // and diagonal L - 32 (index 32 lower); the latter is empty for lane 0.
