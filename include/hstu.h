@@ -94,8 +94,8 @@ HSTU_API size_t hstu_attn_workspace_size(const hstu_problem_t *p, int is_bwd);
  * Forward.  q, k, v, u: inputs (dtype, layouts above, 16-byte aligned).
  * y: output [T, H*d_v] (dtype).  o_save [T, H*d_v], ln_mean [T], ln_rstd [T]:
  * optional fp32 outputs kept for the backward (all three or none; NULL = skip).
- * Supported: bf16 with d_qk = d_v = 128, 1 <= H <= 8 and batch times
- * ceil(max_seq_len / 128) below 2^31 - 256 (tcgen05 path); fp32 with
+ * Supported: bf16 with d_qk = d_v = 128, 1 <= H <= 8 and
+ * 2 * batch * ceil(max_seq_len / 128) <= 2^31 - 256 (tcgen05 path); fp32 with
  * d_qk, d_v <= 128 and H*d_v <= 1024 (true-fp32 SIMT path).
  */
 HSTU_API hstu_status_t hstu_attn_fwd(const hstu_problem_t *p, const void *q, const void *k,
@@ -108,7 +108,8 @@ HSTU_API hstu_status_t hstu_attn_fwd(const hstu_problem_t *p, const void *q, con
  * o_save, ln_mean, ln_rstd are the forward's saved fp32 outputs (required).
  * Writes dq, dk [T,H,d_qk], dv [T,H,d_v], du [T,H*d_v] (dtype); d_rab_pos
  * [H,2L-1] and d_rab_time [H,NB] (fp32) are overwritten, not accumulated,
- * when non-NULL (entries with i-j < 0 are zero).
+ * when non-NULL (entries with i-j < 0 are zero).  Supported shapes are those
+ * of hstu_attn_fwd.
  */
 HSTU_API hstu_status_t hstu_attn_bwd(const hstu_problem_t *p, const void *dy, const void *q,
                             const void *k, const void *v, const void *u,
@@ -147,8 +148,9 @@ HSTU_API hstu_status_t hstu_selftest_wait_timeout(void *workspace, uint64_t budg
                                                   void *stream);
 
 /*
- * Backward without a caller-provided workspace.  The pages define no such
- * call; it exists for callers that cannot allocate device memory themselves
+ * Backward without a caller-provided workspace.  The HSTU model card and
+ * papers define no such call; it exists for callers that cannot allocate
+ * device memory themselves
  * (for example when another allocator already owns the free device memory,
  * or a host framework forbids direct CUDA allocation).
  *
