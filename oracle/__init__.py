@@ -10,6 +10,7 @@ exactly to fp64 before the call, so input rounding is not counted as error.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -26,14 +27,20 @@ LN_EPS = 1e-5
 NUM_TIME_BUCKETS = 128
 
 
+def compile_source(src: str, out: str) -> str:
+    """Compile one C source of the oracle (hstu_ref.h found beside this file)."""
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fPIC",
+                           "-shared", "-Wall", "-I", _HERE, "-o", out, src, "-lm"])
+    return out
+
+
 def build(force: bool = False) -> str:
     """Compile hstu_ref.c into libhstu_ref.so beside it (gcc, OpenMP)."""
     hdr = os.path.join(_HERE, "hstu_ref.h")
     newest = max(os.path.getmtime(_SRC), os.path.getmtime(hdr))
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + ".tmp%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fPIC",
-                               "-shared", "-Wall", "-o", tmp, _SRC, "-lm"])
+        compile_source(_SRC, tmp)
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -55,22 +62,40 @@ class _Problem(ctypes.Structure):
     ]
 
 
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(_Problem)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    lib.hstu_ref_time_bucket.argtypes = [ctypes.c_int64, ctypes.c_int32]
+    lib.hstu_ref_time_bucket.restype = ctypes.c_int32
+    lib.hstu_ref_fwd.argtypes = [P] + [vp] * 8 + [i32]
+    lib.hstu_ref_fwd.restype = ctypes.c_int
+    lib.hstu_ref_fwd_rows.argtypes = [P] + [vp] * 5 + [i64] + [vp] * 4 + [i32]
+    lib.hstu_ref_fwd_rows.restype = ctypes.c_int
+    lib.hstu_ref_bwd.argtypes = [P] + [vp] * 11 + [i32]
+    lib.hstu_ref_bwd.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        P = ctypes.POINTER(_Problem)
-        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
-        lib.hstu_ref_time_bucket.argtypes = [ctypes.c_int64, ctypes.c_int32]
-        lib.hstu_ref_time_bucket.restype = ctypes.c_int32
-        lib.hstu_ref_fwd.argtypes = [P] + [vp] * 8 + [i32]
-        lib.hstu_ref_fwd.restype = ctypes.c_int
-        lib.hstu_ref_fwd_rows.argtypes = [P] + [vp] * 5 + [i64] + [vp] * 4 + [i32]
-        lib.hstu_ref_fwd_rows.restype = ctypes.c_int
-        lib.hstu_ref_bwd.argtypes = [P] + [vp] * 11 + [i32]
-        lib.hstu_ref_bwd.restype = ctypes.c_int
-        _lib = lib
+        _lib = _bind(build())
     return _lib
+
+
+@contextlib.contextmanager
+def library(path: str):
+    """Route every call of this module to another build of the oracle (for the
+    tests that plant a mistake in a copy of hstu_ref.c and check that the pins
+    reject it); the regular library is restored on exit."""
+    global _lib
+    prev = _load()
+    _lib = _bind(path)
+    try:
+        yield
+    finally:
+        _lib = prev
 
 
 def _f64(x) -> Optional[np.ndarray]:

@@ -143,6 +143,53 @@ def test_first_position_closed_form(oracle_lib):
                                        rtol=1e-13, atol=1e-15)
 
 
+def test_first_position_closed_form_own_length(oracle_lib):
+    """With the normaliser taken as each sequence's own length (the jagged
+    workload's reading of the model card's division by the length),
+    O_0 = SiLU(q_0 . k_0 + rab_pos[L-1] + rab_time[0]) / n_b * v_0."""
+    inp = small_inputs(lengths=(8, 5), norm="own")
+    got = oracle_lib.fwd(inp)
+    H, dv = inp.q.shape[1], inp.v.shape[2]
+    L = inp.rab_pos_len
+    for b, n in enumerate(inp.lengths):
+        t = int(inp.offsets[b])
+        for h in range(H):
+            s = float((inp.q[t, h].double() * inp.k[t, h].double()).sum())
+            s += float(inp.rab_pos[h, L - 1]) + float(inp.rab_time[h, 0])
+            expect = s / (1.0 + math.exp(-s)) / n * inp.v[t, h].double().numpy()
+            np.testing.assert_allclose(got["o"][t, h * dv:(h + 1) * dv], expect,
+                                       rtol=1e-13, atol=1e-15)
+
+
+def test_query_row_locality(oracle_lib):
+    """q_i enters only row i's scores (S_ij = q_i . k_j), so changing it changes
+    row i of Y and no other row, bit for bit."""
+    base = small_inputs(lengths=(9,), H=2)
+    y0 = oracle_lib.fwd(base)["y"]
+    i = 4
+    pert = small_inputs(lengths=(9,), H=2)
+    pert.q[i] = pert.q[i] * -2.0 + 0.5
+    y1 = oracle_lib.fwd(pert)["y"]
+    rows = [r for r in range(9) if r != i]
+    assert np.array_equal(y1[rows], y0[rows])
+    assert not np.array_equal(y1[i], y0[i])
+
+
+def test_gate_limits(oracle_lib):
+    """SiLU(40) = 40 to within 1e-16 relative and SiLU(-40) is below 2e-16, so
+    with U = +40 the output is 40 x_hat and with U = -40 it vanishes; x_hat is
+    taken from the returned O, mean and rstd."""
+    for uval in (40.0, -40.0):
+        inp = small_inputs()
+        inp.u = torch.full_like(inp.u, uval)
+        got = oracle_lib.fwd(inp)
+        xhat = (got["o"] - got["mean"][:, None]) * got["rstd"][:, None]
+        if uval > 0:
+            np.testing.assert_allclose(got["y"], 40.0 * xhat, rtol=1e-14, atol=1e-14)
+        else:
+            assert np.abs(got["y"]).max() <= 2e-16 * max(np.abs(xhat).max(), 1.0)
+
+
 def test_causality(oracle_lib):
     inp = small_inputs(lengths=(12,), H=2)
     base = oracle_lib.fwd(inp)["y"]
