@@ -27,6 +27,8 @@
 // every GEMM of a tile would leave the tensor core idle most of the time.
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "internal.h"
 #include "ptx.cuh"
 #include "tile_math.cuh"
@@ -844,16 +846,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 }  // namespace dkv
 
+// `configured` caches, per device, that the kernel's shared-memory opt-in has
+// been set.  Host threads may launch concurrently: the flag is atomic, and two
+// threads that both see it clear just set the same attribute twice.
 template <typename K>
 cudaError_t launch_plain(K kernel, int smem, unsigned grid, const CUtensorMap* maps,
-                         const BwdArgs& a, cudaStream_t stream, bool* configured) {
+                         const BwdArgs& a, cudaStream_t stream, std::atomic<bool>* configured) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
+  const bool cached = dev >= 0 && dev < 64;
+  if (!cached || !configured[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    if (dev >= 0 && dev < 64) configured[dev] = true;
+    if (cached) configured[dev].store(true, std::memory_order_release);
   }
   kernel<<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], a);
   return cudaGetLastError();
@@ -861,7 +867,7 @@ cudaError_t launch_plain(K kernel, int smem, unsigned grid, const CUtensorMap* m
 
 template <bool POS, bool TIME>
 cudaError_t launch_variant(const BwdArgs& a, const CUtensorMap* maps, cudaStream_t stream) {
-  static bool conf_dq[64] = {}, conf_dkv[64] = {};
+  static std::atomic<bool> conf_dq[64], conf_dkv[64];   // zero-initialised: false
   const unsigned grid = static_cast<unsigned>(a.H) * static_cast<unsigned>(a.B) *
                         static_cast<unsigned>(a.max_tiles);
   cudaError_t err = launch_plain(dq::hstu_bwd_dq_sm100<POS, TIME>, dq::kSmem, grid, maps, a,
