@@ -4,9 +4,12 @@
 
 A step is one pass of the whole hot path over one batch of synthetic input:
 for the forward workloads the fused attention + LayerNorm + gate forward, for
-"train" the forward with saved statistics followed by the backward.  The
-default workload is the model card's block shape ("neurarch": 8 sequences of
-1024 tokens, 4 heads, d_qk = d_v = 128, position bias, bf16).
+the training workloads the forward with saved statistics followed by the
+backward.  The default workload is the jagged one: 64 sequences of 256..4096
+tokens (seed 0), 8 heads, d_qk = d_v = 128, position and time bias,
+normalisation by each sequence's own length, bf16 -- the largest
+configuration that fits one GPU.  After the main line's measurement the
+long-sequence forward and the training step are timed as well (``also``).
 
 Timing: inputs are resident in HBM; R input sets whose total size exceeds
 twice the 126 MB L2 are used in rotation, so no step reads its inputs from L2
@@ -42,10 +45,15 @@ import hstu_inputs as hi  # noqa: E402
 METRIC = "causal HSTU-attention TFLOP/s (bf16) and % of B200 dense tensor peak"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FWD_KERNEL = "hstu_fwd_bf16_sm100"
+BWD_KERNELS = "bwd_pre_rows_bf16, hstu_bwd_dq_sm100, hstu_bwd_dkdv_sm100"
 KERNEL_SOURCES = {
-    "fwd": ["pointwise_attention_b200/csrc/fwd_sm100.cu", "pointwise_attention_b200/csrc/ptx.cuh",
-            "pointwise_attention_b200/csrc/tile_math.cuh", "pointwise_attention_b200/csrc/internal.h"],
+    "hstu_fwd_bf16_sm100": ["pointwise_attention_b200/csrc/fwd_sm100.cu",
+                            "pointwise_attention_b200/csrc/ptx.cuh",
+                            "pointwise_attention_b200/csrc/tile_math.cuh",
+                            "pointwise_attention_b200/csrc/internal.h"],
 }
+BWD_FLOP_FACTOR = 2.5      # S recomputed, dA, dV, dQ, dK: five GEMM-equivalents
 
 
 # ----------------------------------------------------------------- host logic
@@ -95,6 +103,20 @@ def algorithmic_bytes(inp) -> int:
     return int(n)
 
 
+def set_bytes(inp, train: bool) -> int:
+    """Device bytes of one input set (plus the training step's saved outputs
+    and gradients)."""
+    n = algorithmic_bytes(inp)
+    if train:
+        n += inp.total_tokens * inp.q.shape[1] * inp.v.shape[2] * (4 + 2 * 5)
+    return n
+
+
+def n_sets(inp, train: bool) -> int:
+    """Input sets in rotation: together more than twice the L2."""
+    return max(2, int(math.ceil(2 * L2_BYTES / set_bytes(inp, train))))
+
+
 def source_digest(paths) -> str:
     h = hashlib.sha256()
     for p in paths:
@@ -103,24 +125,44 @@ def source_digest(paths) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_key: str, workload: str):
+def profiled_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "%s.%s.txt" % (kernel_key, workload))
-    if not os.path.exists(path):
+    path = os.path.join(ROOT, "profiles", "%s.%s.txt" % (kernel, workload))
+    srcs = KERNEL_SOURCES.get(kernel)
+    if not os.path.exists(path) or not srcs:
         return None
     fields = {}
     for line in open(path):
         if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             fields[k.strip()] = v.strip()
-    srcs = KERNEL_SOURCES.get("fwd")
     if fields.get("kernel_source_sha256") != source_digest(srcs):
         return None
     try:
         return int(float(fields["dram_bytes_per_launch"]))
     except (KeyError, ValueError):
         return None
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_threads() -> int:
+    """Threads the oracle's OpenMP runtime uses by default: the CPUs this
+    process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 class ClockSampler:
@@ -130,7 +172,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.01):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.samples, self.reasons, self.period = [], set(), period_s
         self.max_mhz = None
         self._stop = threading.Event()
@@ -143,16 +185,19 @@ class ClockSampler:
         except Exception:   # NVML unavailable: report no clocks rather than guess
             self.nv = None
 
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):
@@ -165,6 +210,8 @@ class ClockSampler:
         self._stop.set()
         if self.nv is not None:
             self.t.join()
+            if not self.samples:
+                self._sample()
 
     def summary(self):
         if not self.samples:
@@ -172,6 +219,27 @@ class ClockSampler:
                     "samples": 0}
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def bench_config(spec, inp, world: int) -> dict:
+    """The `config` object of both arms: the workload and how its inputs
+    relate to the L2 between steps (`inp` is rank 0's drawn problem)."""
+    c = {"workload": spec.name, "batch": spec.batch, "heads": spec.heads, "d_qk": spec.d_qk,
+         "d_v": spec.d_v,
+         "rab": "+".join(x for x, on in (("pos", spec.rab_pos_len > 0), ("time", spec.rab_time))
+                         if on) or "none",
+         "norm": "own_length" if spec.norm == "own" else "fixed"}
+    if spec.len_range:
+        c["seq_len"] = "U[%d,%d]" % spec.len_range
+    else:
+        c["seq_len"] = spec.seq_len
+    if spec.stochastic_length:
+        c["stochastic_length"] = "keep %d, p %.2f" % spec.stochastic_length
+    c["parallelism"] = "replicas" if world > 1 else "single"
+    R = n_sets(inp, spec.grad)
+    c["l2"] = "%d rotating input sets (%.0f MB each) > 2x 126 MB L2" % (
+        R, set_bytes(inp, spec.grad) / 1e6)
+    return c
 
 
 # ----------------------------------------------------------------- oracle arm
@@ -186,33 +254,50 @@ def _row_sample(inp, stride: int):
     return rows, fl
 
 
-def oracle_step_sample(inp, budget_s: float):
-    """Times the oracle forward on the host cores: the whole workload if it fits
-    in the budget, else every stride-th row (stride from a small probe); returns
-    (flops, seconds, description)."""
+def oracle_step_sample(inp, budget_s: float, threads: int):
+    """Times the oracle forward on `threads` host threads: the whole workload
+    if it fits in the budget, else every stride-th row (stride from a small
+    probe); returns (flops, seconds, description, extrapolated)."""
     import numpy as np
     import oracle
     oracle.build()
     flops_full = hi.causal_flops(inp.lengths, inp.q.shape[1], inp.q.shape[2], inp.v.shape[2])
-    probe_stride = max(1, int(math.ceil(flops_full / 2e9)))
+    probe_stride = max(1, int(math.ceil(flops_full / (2e9 if threads > 1 else 2e8))))
     rows, fl = _row_sample(inp, probe_stride)
     t0 = time.perf_counter()
-    oracle.fwd_rows(inp, np.array(rows, dtype=np.int64))
+    oracle.fwd_rows(inp, np.array(rows, dtype=np.int64), threads=threads)
     rate = fl / max(time.perf_counter() - t0, 1e-9)
     if flops_full / rate <= budget_s:
         reps, total = 0, 0.0
         while reps == 0 or total < budget_s * 0.5:
             t0 = time.perf_counter()
-            oracle.fwd(inp)
+            oracle.fwd(inp, threads=threads)
             total += time.perf_counter() - t0
             reps += 1
-        return flops_full * reps, total, "full workload forward x%d" % reps
+        return flops_full * reps, total, "full workload forward x%d" % reps, False
     stride = max(1, int(math.ceil(flops_full / rate / budget_s)))
     rows, fl = _row_sample(inp, stride)
     t0 = time.perf_counter()
-    oracle.fwd_rows(inp, np.array(rows, dtype=np.int64))
+    oracle.fwd_rows(inp, np.array(rows, dtype=np.int64), threads=threads)
     return fl, time.perf_counter() - t0, "every %d-th row of the workload (%d rows)" % (
-        stride, len(rows))
+        stride, len(rows)), True
+
+
+def cpu_baseline(inp, budget_all: float, budget_single: float) -> dict:
+    """The oracle on all host threads and on one, each on a bounded sample of
+    the workload; the full workload's time is extrapolated from the sample's
+    FLOP rate where only a sample was run."""
+    threads = host_threads()
+    flops_full = hi.causal_flops(inp.lengths, inp.q.shape[1], inp.q.shape[2], inp.v.shape[2])
+    f, s, desc, ext = oracle_step_sample(inp, budget_all, threads)
+    out = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+           "sample": desc, "cpu_model": cpu_model(),
+           ("full_forward_s_extrapolated" if ext else "full_forward_s"): flops_full / (f / s)}
+    f1, s1, desc1, ext1 = oracle_step_sample(inp, budget_single, 1)
+    out["single_thread"] = {
+        "value": f1 / s1 / 1e12, "unit": "TFLOP/s", "sample": desc1,
+        ("full_forward_s_extrapolated" if ext1 else "full_forward_s"): flops_full / (f1 / s1)}
+    return out
 
 
 def run_reference(args, spec):
@@ -220,13 +305,13 @@ def run_reference(args, spec):
     if rank != 0:
         return 0
     inp = hi.make_inputs(spec, seed=args.seed)
-    cores = os.cpu_count()
+    threads = host_threads()
     for _ in range(args.warmup):
-        oracle_step_sample(inp, budget_s=0.5)
+        oracle_step_sample(inp, 0.5, threads)
     flops, secs = 0, 0.0
     desc = ""
     for _ in range(args.steps):
-        f, s, desc = oracle_step_sample(inp, budget_s=args.ref_step_budget)
+        f, s, desc, _ = oracle_step_sample(inp, args.ref_step_budget, threads)
         flops += f
         secs += s
     value = flops / secs / 1e12
@@ -235,9 +320,10 @@ def run_reference(args, spec):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": spec.name, **workload_config(spec)},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+        "config": bench_config(spec, inp, world),
+        "timing": "host wall clock around each sampled oracle forward",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -246,28 +332,13 @@ def run_reference(args, spec):
 
 
 # ----------------------------------------------------------------- GPU arm
-def workload_config(spec):
-    c = {"batch": spec.batch, "heads": spec.heads, "d_qk": spec.d_qk, "d_v": spec.d_v,
-         "rab": "+".join(x for x, on in (("pos", spec.rab_pos_len > 0), ("time", spec.rab_time))
-                         if on) or "none",
-         "norm": "own_length" if spec.norm == "own" else "fixed"}
-    if spec.len_range:
-        c["seq_len"] = "U[%d,%d]" % spec.len_range
-    else:
-        c["seq_len"] = spec.seq_len
-    return c
-
-
 class Workload:
     """R device copies of one rank's inputs plus outputs and workspaces."""
 
     def __init__(self, inp, train: bool, device):
         import pointwise_attention_b200 as pa
         self.pa, self.inp, self.train = pa, inp, train
-        per_set = algorithmic_bytes(inp)
-        if train:
-            per_set += inp.total_tokens * inp.q.shape[1] * inp.v.shape[2] * (4 + 2 * 5)
-        self.R = max(2, int(math.ceil(2 * L2_BYTES / per_set)))
+        self.R = n_sets(inp, train)
         self.sets = []
         for _ in range(self.R):
             d = {k: (None if v is None else v.to(device).contiguous()) for k, v in dict(
@@ -289,20 +360,15 @@ class Workload:
                                   d_rab_time=(torch.empty_like(d["rab_time"])
                                               if d["rab_time"] is not None else None))
             self.sets.append(d)
-        self.launches_per_step = 1 if not train else 1 + 3   # forward; LN/gate, dQ, dK/dV backward kernels
+        # forward; the backward's LN/gate, dQ and dK/dV kernels
+        self.launches_per_step = 1 if not train else 1 + 3
 
-    def step(self, i: int, stream=None):
+    def forward(self, i: int, stream=None):
         d, inp, pa = self.sets[i % self.R], self.inp, self.pa
         pa.hstu_attn_fwd(d["q"], d["k"], d["v"], d["u"], d["offsets"], inp.max_seq_len,
                          timestamps=d["ts"], rab_pos=d["rab_pos"], rab_time=d["rab_time"],
                          norm_len=inp.norm_len, save_for_backward=self.train, y=d["y"],
                          saved=d.get("saved"), workspace=d["ws"], stream=stream)
-        if self.train:
-            pa.hstu_attn_bwd(d["dy"], d["q"], d["k"], d["v"], d["u"], d["offsets"],
-                             inp.max_seq_len, d["saved"], timestamps=d["ts"],
-                             rab_pos=d["rab_pos"], rab_time=d["rab_time"],
-                             norm_len=inp.norm_len, grads=d["grads"], workspace=d["ws"],
-                             stream=stream)
 
     def backward(self, i: int, stream=None):
         d, inp, pa = self.sets[i % self.R], self.inp, self.pa
@@ -312,12 +378,133 @@ class Workload:
                          norm_len=inp.norm_len, grads=d["grads"], workspace=d["ws"],
                          stream=stream)
 
+    def step(self, i: int, stream=None):
+        self.forward(i, stream)
+        if self.train:
+            self.backward(i, stream)
+
     def check(self):
         for d in self.sets:
             rc = self.pa.hstu_attn_check(d["ws"])
             if rc != 0:
                 raise RuntimeError("device status after the timed region: %s"
                                    % self.pa.status_string(rc))
+
+
+def graph_of(fn, count: int, stream):
+    """CUDA graph of fn(0) .. fn(count-1) on `stream`."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(count):
+                fn(i, stream=stream)
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graphs(steps: int, R: int, fn, stream, world: int, clock_index=None):
+    """Replays graphs of R steps (plus a tail graph) until exactly `steps` steps
+    ran; returns (seconds on the device, max over ranks, clock summary)."""
+    reps, rest = divmod(steps, R)
+    graph = graph_of(fn, R, stream)
+    tail = graph_of(fn, rest, stream) if rest else None
+    for _ in range(2):                      # graph warm-up
+        graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(clock_index) if clock_index is not None else None
+    if clk is not None:
+        clk.__enter__()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        if tail is not None:
+            tail.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if clk is not None:
+        clk.__exit__(None, None, None)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    elapsed = e0.elapsed_time(e1) / 1e3
+    return elapsed, clk.summary() if clk is not None else None
+
+
+def measure(spec, seed: int, steps: int, warmup: int, device, world: int, local: int,
+            clocks: bool):
+    """Times `steps` steps of one workload; returns the measurement and the
+    Workload (for the end-to-end leg)."""
+    inp = hi.make_inputs(spec, seed=seed)
+    train = spec.grad
+    wl = Workload(inp, train, device)
+    flops_fwd = hi.causal_flops(inp.lengths, spec.heads, spec.d_qk, spec.d_v)
+    flops_step = flops_fwd * (1 + (BWD_FLOP_FACTOR if train else 0.0))
+    for i in range(warmup):
+        wl.step(i)
+    torch.cuda.synchronize()
+    wl.check()
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        wl.step(0, stream=stream)           # warm the capture stream
+    torch.cuda.synchronize()
+    elapsed, clk = time_graphs(steps, wl.R, wl.step, stream, world,
+                               local if clocks else None)
+    elapsed_max = reduce_max(elapsed, world, device)
+    wl.check()
+    peaks, peak_kind = load_peaks()
+    res = {"inp": inp, "flops_fwd": flops_fwd, "flops_step": flops_step,
+           "elapsed": elapsed, "elapsed_max": elapsed_max, "clocks": clk,
+           "value": flops_step * steps * world / elapsed_max / 1e12,
+           "ms_per_step": elapsed_max / steps * 1e3, "launches_per_step": wl.launches_per_step}
+
+    if not train:
+        # One forward launch per step, replayed back to back from the graph:
+        # the average launch duration is the timed region over the steps.
+        t_launch = elapsed / steps
+        bytes_launch = algorithmic_bytes(inp)
+        t_hbm = bytes_launch / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops_fwd / (peaks["bf16_tflops"] * 1e12)
+        if t_hbm >= t_tc:
+            roof = {"bound": "hbm", "achieved": bytes_launch / t_launch / 1e9,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        else:
+            roof = {"bound": "tensor", "achieved": flops_fwd / t_launch / 1e12,
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = profiled_traffic(FWD_KERNEL, spec.name)
+        roof["peak_source"] = peak_kind + (" burst" if roof["bound"] == "tensor" else "")
+        roof["kernel"] = FWD_KERNEL if spec.dtype == "bf16" else "fwd_simt<float>"
+        roof["algorithmic_bytes"] = bytes_launch
+        roof["algorithmic_flops"] = flops_fwd
+        roof["us_per_launch"] = t_launch * 1e6
+    else:
+        # Training: the backward call (LN/gate, dQ and dK/dV kernels) is the
+        # dominant unit.  It is timed on its own: graphs of R backward calls,
+        # replayed, on the saved outputs the timed steps left behind.
+        bsteps = max(wl.R, steps)
+        t_b, _ = time_graphs(bsteps, wl.R, wl.backward, stream, world)
+        t_bwd = t_b / bsteps
+        flops_bwd = BWD_FLOP_FACTOR * flops_fwd
+        roof = {"bound": "tensor", "achieved": flops_bwd / t_bwd / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = None
+        roof["peak_source"] = peak_kind + " burst"
+        roof["kernel"] = "hstu_attn_bwd (%s)" % BWD_KERNELS
+        roof["algorithmic_flops"] = flops_bwd
+        roof["ms_per_call"] = t_bwd * 1e3
+        roof["flops_2x_fwd_tflops"] = 2.0 * flops_fwd / t_bwd / 1e12
+        wl.check()
+    res["roofline"] = roof
+    return res, wl
 
 
 def timed_e2e(wl, steps: int, device):
@@ -357,6 +544,14 @@ def timed_e2e(wl, steps: int, device):
     return e0.elapsed_time(e1) / 1e3, h2d, d2h
 
 
+def summary_of(spec, res, world):
+    roof = dict(res["roofline"])
+    return {"workload": spec.name, "value": res["value"], "unit": "TFLOP/s",
+            "ms_per_step": res["ms_per_step"], "steps_timed": res["steps"],
+            "pct_of_dense_bf16_peak": 100.0 * res["value"] / world / roof["peak"],
+            "roofline": roof}
+
+
 def run_gpu(args, spec):
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -369,156 +564,54 @@ def run_gpu(args, spec):
     import pointwise_attention_b200 as pa
     pa.load_library()
 
-    inp = hi.make_inputs(spec, seed=rank_seed(args.seed, rank))
-    train = spec.grad
-    wl = Workload(inp, train, device)
-    flops_fwd = hi.causal_flops(inp.lengths, spec.heads, spec.d_qk, spec.d_v)
-    flops_step = flops_fwd * (1 + (2.5 if train else 0.0))
-
-    for i in range(args.warmup):
-        wl.step(i)
-    torch.cuda.synchronize()
-    wl.check()
-
-    # CUDA graph of R consecutive steps (one per input set), replayed.
-    stream = torch.cuda.Stream()
-    stream.wait_stream(torch.cuda.current_stream())
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        wl.step(0, stream=stream)           # warm the capture stream
-        torch.cuda.current_stream().synchronize()
-        with torch.cuda.graph(graph, stream=stream):
-            for i in range(wl.R):
-                wl.step(i, stream=stream)
-    torch.cuda.synchronize()
-    reps, rest = divmod(args.steps, wl.R)
-    tail = None
-    if rest:
-        tail = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            with torch.cuda.graph(tail, stream=stream):
-                for i in range(rest):
-                    wl.step(i, stream=stream)
-        torch.cuda.synchronize()
-    for _ in range(2):                      # graph warm-up
-        graph.replay()
-    torch.cuda.synchronize()
-
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(reps):
-                graph.replay()
-            if tail is not None:
-                tail.replay()
-            e1.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    elapsed = e0.elapsed_time(e1) / 1e3
-    elapsed_max = reduce_max(elapsed, world, device)
-    wl.check()
-
-    value = flops_step * args.steps * world / elapsed_max / 1e12
-    peaks, peak_kind = load_peaks()
-    sec_per_step = elapsed / args.steps
-    # Roofline of the dominant kernel (the forward for forward workloads).
-    bytes_launch = algorithmic_bytes(inp)
-    # One forward launch per step, replayed back to back from the graph: the
-    # average launch duration is the timed region over the number of steps.
-    t_launch = sec_per_step if not train else None
-    roof = None
-    if t_launch is not None:
-        t_hbm = bytes_launch / (peaks["hbm_gbs"] * 1e9)
-        t_tc = flops_fwd / (peaks["bf16_tflops"] * 1e12)
-        if t_hbm >= t_tc:
-            roof = {"bound": "hbm", "achieved": bytes_launch / t_launch / 1e9,
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-        else:
-            roof = {"bound": "tensor", "achieved": flops_fwd / t_launch / 1e12,
-                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["traffic"] = profiled_traffic("hstu_fwd_bf16_sm100", spec.name)
-        roof["peak_source"] = peak_kind + (" burst" if roof["bound"] == "tensor" else "")
-        roof["kernel"] = "hstu_fwd_bf16_sm100" if spec.dtype == "bf16" else "fwd_simt<float>"
-        roof["algorithmic_bytes"] = bytes_launch
-        roof["algorithmic_flops"] = flops_fwd
-
-    if train:
-        # Training: the backward call (LN/gate, dQ and dK/dV kernels: two thirds
-        # of the step in the ncu launch list) is the dominant unit.  It is timed
-        # on its own: a graph of R backward calls, replayed, on the saved
-        # outputs the timed steps left behind.
-        bgraph = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            with torch.cuda.graph(bgraph, stream=stream):
-                for i in range(wl.R):
-                    wl.backward(i, stream=stream)
-        torch.cuda.synchronize()
-        for _ in range(2):
-            bgraph.replay()
-        torch.cuda.synchronize()
-        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        breps = max(1, reps)
-        with torch.cuda.stream(stream):
-            b0.record(stream)
-            for _ in range(breps):
-                bgraph.replay()
-            b1.record(stream)
-        torch.cuda.synchronize()
-        t_bwd = b0.elapsed_time(b1) / 1e3 / (breps * wl.R)
-        flops_bwd = 2.5 * flops_fwd
-        roof = {"bound": "tensor", "achieved": flops_bwd / t_bwd / 1e12,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["traffic"] = None
-        roof["peak_source"] = peak_kind + " burst"
-        roof["kernel"] = "hstu_attn_bwd (bwd_pre_simt, hstu_bwd_dq_sm100, hstu_bwd_dkdv_sm100)"
-        roof["algorithmic_flops"] = flops_bwd
-        roof["ms_per_call"] = t_bwd * 1e3
-        wl.check()
-
+    res, wl = measure(spec, rank_seed(args.seed, rank), args.steps, args.warmup, device, world,
+                      local, clocks=True)
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
     e2e_t, h2d, d2h = timed_e2e(wl, e2e_steps, device)
     e2e_t = reduce_max(e2e_t, world, device)
+    inp = res["inp"]
+    del wl
+
+    also = {}
+    for name in [x for x in args.also.split(",") if x and x != spec.name]:
+        sp = hi.WORKLOADS[name]
+        steps = args.also_steps
+        r2, wl2 = measure(sp, rank_seed(args.seed, rank), steps, 3, device, world, local,
+                          clocks=False)
+        r2["steps"] = steps
+        del wl2
+        torch.cuda.empty_cache()
+        also[name] = summary_of(sp, r2, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, s, desc = oracle_step_sample(inp, budget_s=args.cpu_budget)
-        cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
-               "kind": "oracle", "sample": desc}
+        cpu = cpu_baseline(inp, args.cpu_budget, args.cpu_budget_single)
 
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    tensor_peak = peaks["bf16_tflops"]
+    roof = res["roofline"]
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_max / args.steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
-        if spec.dtype == "bf16" else "f32", "data": "synthetic",
-        "pct_of_dense_bf16_peak": 100.0 * value / world / tensor_peak,
-        "config": {"workload": spec.name, **workload_config(spec),
-                   "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "%d rotating input sets (%.0f MB each) > 2x 126 MB L2" % (
-                       wl.R, algorithmic_bytes(inp) / 1e6),
-                   "timing": "CUDA graph of %d steps, CUDA events" % wl.R},
-        "gpu_launches": args.steps * wl.launches_per_step,
+        "metric": METRIC, "value": res["value"], "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if spec.dtype == "bf16" else "f32", "data": "synthetic",
+        "pct_of_dense_bf16_peak": 100.0 * res["value"] / world / roof["peak"],
+        "config": bench_config(spec, inp, world),
+        "timing": "CUDA graph of %d steps replayed, CUDA events on the launching stream" % (
+            n_sets(inp, spec.grad)),
+        "gpu_launches": args.steps * res["launches_per_step"],
         "roofline": roof,
         "cpu_baseline": cpu,
-        "clocks": clk.summary(),
+        "clocks": res["clocks"],
     }
-    line["e2e"] = {"value": flops_step * world * e2e_steps / e2e_t / 1e12, "unit": "TFLOP/s",
-                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+    line["e2e"] = {"value": res["flops_step"] * world * e2e_steps / e2e_t / 1e12,
+                   "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                    "steps": e2e_steps}
+    if also:
+        line["also"] = also
     print(json.dumps(line), flush=True)
     return 0
 
@@ -526,13 +619,17 @@ def run_gpu(args, spec):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="neurarch", choices=sorted(hi.WORKLOADS))
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="jagged", choices=sorted(hi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--also", default="long,train",
+                    help="comma-separated workloads timed after the main one ('' for none)")
+    ap.add_argument("--also-steps", type=int, default=50)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--cpu-budget-single", type=float, default=6.0)
     ap.add_argument("--ref-step-budget", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -7,10 +7,11 @@ any of the method's code.
 
 Shapes follow the HSTU model card ("HSTU (Generative Recommender)", Structure
 table and Exported PyTorch: embed 512, 4 heads, d_qk = d_v = 128, 1024 tokens)
-and the six named workloads below.  Every draw comes from one CPU
+and the named workloads below.  Every draw comes from one CPU
 ``torch.Generator`` seeded per workload, in a fixed order:
 
-    lengths -> Q -> K -> V -> U -> timestamps -> rab_pos -> rab_time -> dY
+    lengths [-> Stochastic Length draws] -> Q -> K -> V -> U -> timestamps
+    -> rab_pos -> rab_time -> dY
 
 Floating values are drawn in fp32 with ``randn`` and rounded (round to nearest
 even) to bf16 for the bf16 workloads; the same rounded host tensors feed the
@@ -24,7 +25,8 @@ from typing import Dict, List, Optional, Sequence
 
 import torch
 
-__all__ = ["Spec", "Inputs", "WORKLOADS", "make_inputs", "workload", "causal_flops"]
+__all__ = ["Spec", "Inputs", "WORKLOADS", "make_inputs", "workload", "causal_flops",
+           "stochastic_length", "stochastic_length_rows"]
 
 NUM_TIME_BUCKETS = 128
 TIME_T0 = 1_700_000_000      # first timestamp of every sequence (seconds)
@@ -52,6 +54,9 @@ class Spec:
     norm_len: int = 0               # for "fixed"; 0 means the (dense) sequence length
     grad: bool = False              # also draw the upstream gradient dY
     ts_sorted: bool = True          # timestamps increasing within a sequence
+    # Stochastic Length: (keep_len, prob).  Each drawn length above keep_len
+    # is cut to keep_len with probability prob (see stochastic_length).
+    stochastic_length: Optional[tuple] = None
 
 
 def _spec_table() -> Dict[str, Spec]:
@@ -77,6 +82,12 @@ def _spec_table() -> Dict[str, Spec]:
         # jagged and long workloads, and the backward of both bias tables.
         "train_time": Spec("train_time", "bf16", batch=16, heads=4, d_qk=128, d_v=128,
                            seq_len=2048, qk_std=s, rab_pos_len=2048, rab_time=True, grad=True),
+        # Training step on jagged histories shortened by Stochastic Length:
+        # lengths U{256..4096}, histories above 2048 events cut to their
+        # latest 2048 with probability 1/2; position and time bias.
+        "train_sl": Spec("train_sl", "bf16", batch=16, heads=4, d_qk=128, d_v=128,
+                         len_range=(256, 4096), qk_std=s, rab_pos_len=4096, rab_time=True,
+                         norm="own", grad=True, stochastic_length=(2048, 0.5)),
     }
 
 
@@ -129,6 +140,40 @@ def causal_flops(lengths: Sequence[int], heads: int, d_qk: int, d_v: int) -> int
     return 2 * pairs * heads * (d_qk + d_v)
 
 
+def stochastic_length(lengths: Sequence[int], keep_len: int, prob: float,
+                      generator: torch.Generator) -> List[int]:
+    """Stochastic Length ("HSTU Hierarchical Sequential Transduction Units",
+    §6 Why it works: long user histories are randomly shortened during
+    training).  The page gives no formula; the reading taken here: every
+    history longer than ``keep_len`` events is, with probability ``prob``,
+    cut to its latest ``keep_len`` events (a contiguous suffix, so order and
+    timestamps stay increasing); shorter histories are kept whole.  One
+    uniform draw per sequence, in sequence order, from ``generator``."""
+    if keep_len < 0 or not (0.0 <= prob <= 1.0):
+        raise ValueError("keep_len must be >= 0 and prob in [0, 1]")
+    draws = torch.rand(len(lengths), generator=generator, dtype=torch.float64).tolist()
+    return [keep_len if (n > keep_len and r < prob) else int(n)
+            for n, r in zip(lengths, draws)]
+
+
+def stochastic_length_rows(offsets: Sequence[int], new_lengths: Sequence[int]):
+    """Packed-token rows that a shortening keeps: for sequence b, its last
+    new_lengths[b] tokens.  Returns (new int32 offsets [B+1], int64 rows),
+    so that a packed tensor x becomes x[rows]."""
+    offs = [int(o) for o in offsets]
+    if len(offs) != len(new_lengths) + 1:
+        raise ValueError("offsets must have one entry more than new_lengths")
+    rows, new_offs = [], [0]
+    for b, m in enumerate(new_lengths):
+        s, e = offs[b], offs[b + 1]
+        if not (0 <= m <= e - s):
+            raise ValueError("sequence %d: kept length %d outside [0, %d]" % (b, m, e - s))
+        rows.extend(range(e - m, e))
+        new_offs.append(new_offs[-1] + m)
+    return (torch.tensor(new_offs, dtype=torch.int32),
+            torch.tensor(rows, dtype=torch.int64))
+
+
 def make_inputs(spec: Spec, seed: int = 0) -> Inputs:
     """Draw one problem for ``spec`` from a CPU generator seeded with ``seed``."""
     g = torch.Generator(device="cpu").manual_seed(seed)
@@ -140,6 +185,9 @@ def make_inputs(spec: Spec, seed: int = 0) -> Inputs:
         lengths = torch.randint(lo, hi + 1, (spec.batch,), generator=g).tolist()
     else:
         lengths = [spec.seq_len] * spec.batch
+    if spec.stochastic_length is not None:
+        keep_len, prob = spec.stochastic_length
+        lengths = stochastic_length(lengths, int(keep_len), float(prob), g)
     offs = [0]
     for n in lengths:
         offs.append(offs[-1] + n)

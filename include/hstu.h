@@ -157,9 +157,10 @@ HSTU_API hstu_status_t hstu_selftest_wait_timeout(void *workspace, uint64_t budg
  * Same arguments, results and synchronous errors as hstu_attn_bwd, minus the
  * workspace: the scratch lives in a fixed 16 MiB array in device global memory
  * that the library reserves on every device it is loaded on and keeps until
- * the process exits.  Problems whose backward workspace
- * (hstu_attn_workspace_size(p, 1)) is larger return HSTU_ERR_WORKSPACE before
- * anything is enqueued.  The function calls no allocation routine.  The first
+ * the process exits.  The argument checks of hstu_attn_bwd run first and
+ * return the same codes; then problems whose backward workspace
+ * (hstu_attn_workspace_size(p, 1)) is larger than the array return
+ * HSTU_ERR_WORKSPACE.  A rejected call enqueues nothing.  The function calls no allocation routine.  The first
  * call on a device looks up the array's device address (with that device
  * current) and caches it.  All calls share the one array: calls that may
  * overlap on the GPU (different streams, no ordering between them) race on it

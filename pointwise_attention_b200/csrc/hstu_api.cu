@@ -3,6 +3,7 @@
 // maps, and kernel dispatch.  No exception crosses the boundary.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -16,6 +17,13 @@
 using namespace hstu;
 
 namespace {
+
+// NVTX range around one library call (visible in Nsight timelines; a no-op
+// unless a profiler injects its NVTX handler).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;
@@ -132,10 +140,14 @@ hstu_status_t check_problem(const hstu_problem_t* p) {
 }
 
 bool bf16_supported(const hstu_problem_t* p) {
-  // The forward numbers its (sequence, query tile) work slots in 32 bits.
-  const int64_t slots = 2 * static_cast<int64_t>(p->batch) * ((p->max_seq_len + 127) / 128);
+  // The forward numbers its (sequence, query tile) work slots in 32 bits, and
+  // the backward launches one CTA per (head, sequence, tile): both counts
+  // must stay below 2^31.
+  const int64_t tiles = (p->max_seq_len + 127) / 128;
+  const int64_t slots = 2 * static_cast<int64_t>(p->batch) * tiles;
+  const int64_t ctas = static_cast<int64_t>(p->num_heads) * p->batch * tiles;
   return p->dtype == HSTU_BF16 && p->d_qk == 128 && p->d_v == 128 && p->num_heads <= 8 &&
-         slots <= 0x7FFFFF00LL;
+         slots <= 0x7FFFFF00LL && ctas <= 0x7FFFFFFFLL;
 }
 
 bool f32_supported(const hstu_problem_t* p) {
@@ -219,6 +231,7 @@ hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* 
                             const void* u, void* y, float* o_save, float* ln_mean,
                             float* ln_rstd, void* workspace, size_t workspace_bytes,
                             void* stream) {
+  NvtxRange range("hstu_attn_fwd");
   hstu_status_t st = check_problem(p);
   if (st != HSTU_OK) return st;
   if (p->total_tokens > 0) {
@@ -266,11 +279,16 @@ hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* 
   return err == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
-hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void* q, const void* k,
-                            const void* v, const void* u, const float* o_save,
-                            const float* ln_mean, const float* ln_rstd, void* dq, void* dk,
-                            void* dv, void* du, float* d_rab_pos, float* d_rab_time,
-                            void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+// Every check hstu_attn_bwd makes before it enqueues anything, except the
+// workspace's (shared with the workspace-free entry point).
+hstu_status_t hstu::check_bwd_args(const hstu_problem_t* p, const void* dy, const void* q,
+                                   const void* k, const void* v, const void* u,
+                                   const float* o_save, const float* ln_mean,
+                                   const float* ln_rstd, const void* dq, const void* dk,
+                                   const void* dv, const void* du, const float* d_rab_pos,
+                                   const float* d_rab_time) {
   hstu_status_t st = check_problem(p);
   if (st != HSTU_OK) return st;
   if (p->total_tokens > 0) {
@@ -284,6 +302,20 @@ hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void*
   if (d_rab_pos && !p->rab_pos) return HSTU_ERR_INVALID_ARG;
   if (d_rab_time && !p->rab_time) return HSTU_ERR_INVALID_ARG;
   if (!bf16_supported(p) && !f32_supported(p)) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+extern "C" {
+
+hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void* q, const void* k,
+                            const void* v, const void* u, const float* o_save,
+                            const float* ln_mean, const float* ln_rstd, void* dq, void* dk,
+                            void* dv, void* du, float* d_rab_pos, float* d_rab_time,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange range("hstu_attn_bwd");
+  hstu_status_t st = check_bwd_args(p, dy, q, k, v, u, o_save, ln_mean, ln_rstd, dq, dk, dv, du,
+                                    d_rab_pos, d_rab_time);
+  if (st != HSTU_OK) return st;
   st = check_ws(p, 1, workspace, workspace_bytes);
   if (st != HSTU_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "hstu.h"
+
 namespace hstu {
 
 // Bits of the device status word (first 4 bytes of the workspace).
@@ -84,6 +86,13 @@ struct BwdArgs {
   float eps;
   BucketTable bt;
 };
+
+// The synchronous argument checks of hstu_attn_bwd (all but the workspace's).
+hstu_status_t check_bwd_args(const hstu_problem_t* p, const void* dy, const void* q,
+                             const void* k, const void* v, const void* u, const float* o_save,
+                             const float* ln_mean, const float* ln_rstd, const void* dq,
+                             const void* dk, const void* dv, const void* du,
+                             const float* d_rab_pos, const float* d_rab_time);
 
 // Kernel launchers (return cudaSuccess or the launch error).
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,

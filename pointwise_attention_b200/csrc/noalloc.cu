@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "hstu.h"
+#include "internal.h"
 
 namespace {
 
@@ -49,11 +50,16 @@ extern "C" HSTU_API hstu_status_t hstu_attn_bwd_noalloc(
     const hstu_problem_t* p, const void* dy, const void* q, const void* k, const void* v,
     const void* u, const float* o_save, const float* ln_mean, const float* ln_rstd, void* dq,
     void* dk, void* dv, void* du, float* d_rab_pos, float* d_rab_time, void* stream) {
+  // The same argument checks as hstu_attn_bwd first, so that a rejected call
+  // returns the same status and leaves nothing queued on the stream.
+  hstu_status_t st = hstu::check_bwd_args(p, dy, q, k, v, u, o_save, ln_mean, ln_rstd, dq, dk,
+                                          dv, du, d_rab_pos, d_rab_time);
+  if (st != HSTU_OK) return st;
   const size_t need = hstu_attn_workspace_size(p, 1);
   if (need == 0) return HSTU_ERR_INVALID_ARG;            // the problem itself is invalid
   if (need > kNoAllocScratchBytes) return HSTU_ERR_WORKSPACE;
   void* scratch = nullptr;
-  hstu_status_t st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != HSTU_OK) return st;
   // The array keeps the previous call's contents; the device status word at
   // its start must begin at zero.  Everything else the backward clears itself.

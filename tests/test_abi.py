@@ -183,3 +183,36 @@ def test_check_and_selftest_reject_missing_workspace(lib):
 def test_empty_problem_is_a_no_op(lib):
     p, _ = problem(lib, batch=0, total_tokens=0, max_seq_len=0, offsets=None)
     assert call_fwd(lib, p) == 0
+
+
+def test_bwd_rejects_grids_beyond_32_bits(lib):
+    """The backward launches one CTA per (head, sequence, 128-row tile); a
+    count of 2^31 or more is refused before anything is enqueued."""
+    so = lib.load_library()
+    vp = ctypes.c_void_p
+    args = [vp(FAKE)] * 12
+    # 8 heads x 2^20 sequences x 256 tiles = 2^31 CTAs
+    p, _ = problem(lib, batch=1 << 20, total_tokens=1 << 20, max_seq_len=256 * 128,
+                   num_heads=8)
+    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), 1 << 40, None) == 2
+    # one tile fewer per sequence fits
+    p, _ = problem(lib, batch=1 << 20, total_tokens=1 << 20, max_seq_len=255 * 128,
+                   num_heads=8)
+    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), 0, None) == 5
+
+
+def test_noalloc_rejects_like_bwd_without_enqueueing(lib):
+    """The workspace-free backward runs the backward's own argument checks
+    first: same codes, nothing queued (these calls never reach the device)."""
+    so = lib.load_library()
+    vp = ctypes.c_void_p
+    args = [vp(FAKE)] * 12
+    # unsupported and larger than the built-in scratch: UNSUPPORTED, as hstu_attn_bwd says
+    p, _ = problem(lib, d_qk=64, d_v=64, total_tokens=1 << 20, max_seq_len=4096)
+    assert so.hstu_attn_bwd_noalloc(ctypes.byref(p), *args, None, None, None) == 2
+    a2 = list(args)
+    a2[8] = None                                    # dq missing
+    p, _ = problem(lib)
+    assert so.hstu_attn_bwd_noalloc(ctypes.byref(p), *a2, None, None, None) == 1
+    p, _ = problem(lib, ln_eps=0.0)
+    assert so.hstu_attn_bwd_noalloc(ctypes.byref(p), *args, None, None, None) == 1

@@ -64,10 +64,8 @@ def test_train_shapes_with_time_bias():
 
 
 def test_train_full_size():
-    """Full training workload on the GPU; gradients of two whole sequences are
-    compared with the oracle run on those sequences alone (sequences are
-    independent), and d(rab_pos), a sum over all sequences, with the oracle
-    on the full problem."""
+    """Full training workload on the GPU: every element of dQ, dK, dV, dU and
+    d(rab_pos) compared with the oracle's gradients of the full problem."""
     inp = hi.make_inputs(hi.WORKLOADS["train"], seed=0)
     y, saved, dev = run_fwd(inp)
     g = run_bwd(inp, dev, saved)
@@ -75,3 +73,11 @@ def test_train_full_size():
     for name in ("dq", "dk", "dv", "du"):
         assert_close(np64(g[name]), ref_full[name], "bf16", name)
     assert_close(np64(g["d_rab_pos"]), ref_full["d_rab_pos"], "bf16", "d_rab_pos")
+
+
+def test_train_sl_reduced_batch():
+    """Training on histories shortened by Stochastic Length (lengths from the
+    train_sl generator: jagged, some cut to 2048), with both biases."""
+    inp = hi.make_inputs(hi.workload("train_sl", batch=5), seed=2)
+    assert len(set(inp.lengths)) > 1
+    check_bwd(inp, "bf16")
