@@ -1,7 +1,7 @@
 // fwd_sm100.cu -- bf16 forward of HSTU causal pointwise aggregated attention
-// on sm_100a: TMA-staged Q/K/V tiles, tcgen05 MMAs with TMEM accumulators,
-// a register epilogue for bias + SiLU + causal mask between the two MMAs,
-// and the LayerNorm-over-heads + SiLU(U) gate fused into the store.
+// on sm_100a: TMA-staged Q/K/V tiles, tcgen05 MMAs with TMEM accumulators, a
+// register epilogue for bias + SiLU + causal mask between the two MMAs, and
+// the LayerNorm-over-heads + SiLU(U) gate in the same kernel.
 //
 // Operation: "HSTU (Generative Recommender)" model card, Exported PyTorch,
 // HSTUBlock.forward (silu(q k^T)/t, tril, attn @ v, gate by silu(u));
@@ -9,46 +9,47 @@
 // Units", §1 and §3; post-pooling normalisation then U gate: the HSTU
 // reproduction note's flowchart.
 //
-// Work decomposition.  A work item is one (sequence b, query tile m): 128
-// query rows against key tiles n = 0..m (tiles above the diagonal are skipped;
-// only the diagonal tile is masked), for all H heads.  The H CTAs of a
-// thread-block cluster take one head each, so the LayerNorm over the
-// concatenated heads exchanges per-row statistics through distributed shared
-// memory.  The kernel is persistent: the grid holds as many clusters as can
-// be resident, and each cluster loops over items that its leader CTA (rank 0)
-// claims from a work counter in global memory (the first one, slot c for
-// cluster c, without a claim).  Items are numbered from the most expensive
-// (largest m) down, so the claims form a longest-first list schedule; slots
-// whose tile lies past the end of its sequence are skipped in runs of up to
-// 32 per claim.  The leader claims the next item once its loads
-// for the current item are issued and hands it to every CTA of the cluster
-// through an 8-entry ring in shared memory.  While the epilogue normalises
-// item j, the TMA and MMA warps already load and multiply item j+1.
+// Work decomposition.  A work item is one (sequence b, query tile m, head h):
+// 128 query rows of one head against key tiles n = 0..m (tiles above the
+// diagonal are skipped; only the diagonal tile is masked).  The kernel is
+// persistent, one CTA per SM, and each CTA claims items from a counter in the
+// workspace (its first item, slot c for CTA c, without a claim).  Slots are
+// numbered heaviest first (largest m), the heads of one (b, m) next to each
+// other, in groups of sequences whose K and V fit in L2 together.
 //
-// Roles (640 threads): warp 0 issues TMA (and, in the leader, claims items);
-// warp 1 allocates TMEM and issues the S = Q K^T MMAs; warp 18 issues the
-// O += P V MMAs; warps 2..17 form the epilogue: warp w owns TMEM lane quarter
-// w%4 (rows 32*(w%4) ..) and the 32 columns (w-2)/4 of every tile.  Each warp
-// stages the position-bias diagonals and key timestamps of its own 32x32
-// block in a private buffer, fetched from global memory one tile ahead.  A
-// tcgen05.mma instruction costs its issuing thread about 110 cycles whatever
-// its N up to 128, about as long as the tensor core needs for 128x128x16, so
-// the two GEMMs of a tile are issued by two threads in parallel.
+// LayerNorm over heads.  The normalisation of a row needs all H heads of the
+// row, which different CTAs compute at different times.  When a CTA finishes
+// its head of a (b, m) block it stores O (bf16, less its per-row head mean,
+// into the rows of Y that will later hold the result; fp32 into o_save when
+// the caller keeps O) and the per-row statistics of its 128 values (mean, sum
+// of squared deviations) in the workspace, then counts itself done on the
+// block's counter.  The CTA that completes the count normalises and gates the
+// whole 128 x (H*128) block: no CTA ever waits for another.
 //
-// TMEM (512 columns): three S/P buffers [0,128) [128,256) [256,384) and O
-// [384,512).  S(x) = Q K^T lands in buffer x % 3 in fp32; the epilogue writes
-// P' = SiLU(S+bias) over it as packed bf16 pairs (each warp only over columns
-// it has already read: its 32 keys take 16 columns), and P' is the A operand
-// (from TMEM) of O' += P' V; O = O' / N in the epilogue.  S(x+3) reuses the
-// buffer once P(x).V has completed; with three buffers S(x+1) and S(x+2) are
-// computed while the epilogue is on tile x.
+// Roles (608 threads): warp 0 claims items and issues TMA; warp 1 allocates
+// TMEM and issues S = Q K^T; warp 2 issues O += P V (a tcgen05.mma of
+// 128x128x16 occupies its issuing thread about as long as the tensor core
+// needs for it, so the two GEMMs of a tile get one issuer each); warps 3..18
+// are the epilogue: warp w owns TMEM lane quarter w%4 (rows 32*(w%4) ..) and
+// the 32 columns (w-3)/4 of every tile, so all sixteen share each tile and
+// its latency stays short against the three-buffer S -> P -> P.V cycle.  Each
+// warp stages the position-bias diagonals and key timestamps of its own 32x32
+// block in a private buffer, fetched from global memory one tile ahead.
 //
-// Every tcgen05.ld/st is warp-collective (.sync.aligned): they are issued by
-// all 32 lanes with warp-uniform control flow; only global accesses are
-// predicated per row.
+// TMEM (512 columns): S/P buffers [0,128) [128,256) [256,384) and O
+// [384,512).  P' = SiLU(S + bias) is written over S as packed bf16 pairs
+// (keys 32c..32c+31 of column group c into columns 32c..32c+15, which that
+// group's warps have already read) and is the A operand of O' += P' V;
+// O = O' / N in the epilogue.  The bias add and SiLU
+// run on bf16 pairs: hx = S/2 + bias/2, P' = hx (1 + tanh hx) with one
+// tanh.approx.bf16x2 per two elements.
+//
+// Every tcgen05.ld/st is warp-collective (.sync.aligned) and issued with
+// warp-uniform control flow; only global accesses are predicated per row.
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -57,44 +58,41 @@
 namespace hstu {
 namespace {
 
-constexpr int kThreads = 640;
-constexpr int kEpiThreads = 512;
-constexpr int kColGroups = 4;               // epilogue warpgroups, 32 columns each
 constexpr int kRows = 128;                  // query rows per tile
 constexpr int kCols = 128;                  // keys per tile
 constexpr int kHalf = 16384;                // 128 rows x 64 bf16 (one 128B-swizzle slab)
 constexpr int kTile = 2 * kHalf;            // 128 x 128 bf16
-constexpr int kKStages = 3;                 // K tiles in flight (S = Q K^T needs them first)
-constexpr int kVStages = 2;                 // V tiles in flight (P.V comes a tile later)
-constexpr int kRing = 8;                    // claimed items handed to the cluster, in flight
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kSBufs = 3;                   // S/P buffers in TMEM
+constexpr int kRing = 8;                    // claimed items in flight inside the CTA
 constexpr int kMaxHeads = 8;
+constexpr int kWarpS = 1, kWarpPV = 2, kWarpEpi = 3;
+constexpr int kEpiWarps = 16;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = (kWarpEpi + kEpiWarps) * 32;   // 608
 
 // shared-memory map (byte offsets from a 1024-aligned base)
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTile;                    // kKStages tiles
-constexpr int kOffV = kOffK + kKStages * kTile;         // kVStages tiles
+constexpr int kOffK = kOffQ + kTile;
+constexpr int kOffV = kOffK + kKStages * kTile;
 // Per epilogue warp: the half position bias of the 63 diagonals its 32x32
 // block touches, as 64 overlapping bf16 pairs (entry k holds diagonals k and
-// k-1, the two an element pair needs), and 32 int64 key timestamps.
-constexpr int kWarpStage = 64 * 4 + 32 * 8;             // bytes per warp
+// k-1, the two an element pair needs); its 32 key timestamps (64-bit and low
+// 32 bits).
+constexpr int kWarpStage = 64 * 4 + 32 * 8 + 32 * 4;
 constexpr int kOffWarp = kOffV + kVStages * kTile;
-// LayerNorm partials of the four column groups, [4][128] (sum, M2) pairs.  They
-// alias the staging buffers, which are idle between an item's last tile and
-// the next item's first.
-constexpr int kOffLoc = kOffWarp;
-constexpr int kOffThr = kOffWarp + 16 * kWarpStage;     // kThrLen int64 thresholds
-constexpr int kOffFirst = kOffThr + kThrLen * 8;        // 64 int8 first bucket per octave
-constexpr int kOffRabT = kOffFirst + 64;                // 128 fp32 half time-bias row
-// Cluster exchange slots of the per-head row statistics: [2 item parities]
-// [kMaxHeads][128 rows] (sum, M2) pairs.
-constexpr int kOffRed = kOffRabT + 128 * 4;
-constexpr int kRedBytes = 2 * kMaxHeads * 128 * 8;
-constexpr int kOffRing = kOffRed + kRedBytes;           // kRing (m, b) pairs
-constexpr int kOffBar = kOffRing + kRing * 8;           // mbarriers (8 B each)
-constexpr int kNumBars = 43;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;        // tmem base, abort flag
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;        // + alignment slack
-static_assert(16 * kWarpStage >= kColGroups * 128 * 8, "LayerNorm partials must fit the staging");
+constexpr int kOffLoc = kOffWarp + kEpiWarps * kWarpStage;   // [4][128] (sum, M2) of O
+constexpr int kOffRabT = kOffLoc + 4 * 128 * 8;              // 128 fp32 half time bias (item's head)
+constexpr int kOffOct = kOffRabT + 128 * 4;
+constexpr int kOffThr32 = kOffOct + 32 * 16;
+constexpr int kOffThr = kOffThr32 + kMaxBuckets * 4;
+constexpr int kOffFirst = kOffThr + kThrLen * 8;
+constexpr int kOffRing = kOffFirst + 64;                     // kRing int4 {m, b, h, -}
+constexpr int kOffBar = kOffRing + kRing * 16;
+constexpr int kNumBars = 40;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;             // tmem base, abort flag, broadcast
+constexpr int kSmemBytes = kOffMisc + 64 + 1024;             // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 // barrier indices
@@ -104,21 +102,21 @@ constexpr int B_KFULL = 2;    // +K stage
 constexpr int B_KEMPTY = 5;   // +K stage
 constexpr int B_VFULL = 8;    // +V stage
 constexpr int B_VEMPTY = 10;  // +V stage
-constexpr int kSBufs = 3;     // S/P buffers in TMEM
 constexpr int B_SFULL = 12;   // +buffer: S(x) computed
-constexpr int B_PFULL = 15;   // +buffer: P(x) written over S(x)
+constexpr int B_PFULL = 15;   // +buffer: P(x) written over S(x) (one arrival per epilogue warp)
 constexpr int B_PVDONE = 18;  // +buffer: P(x).V completed, the buffer may be rewritten
-constexpr int B_OFULL = 21;
-constexpr int B_DONE = 22;    // every MMA of both issuers has completed
-constexpr int B_RED = 23;     // +item parity: LayerNorm statistics of all heads arrived
-constexpr int B_RFULL = 25;   // +ring slot: item written
-constexpr int B_REMPTY = 33;  // +ring slot (leader only): every CTA has read the item
-constexpr int B_ULOAD = 41;   // the item's U tile has landed in the LayerNorm buffer
-constexpr int B_LNFREE = 42;  // the LayerNorm is done with its buffer (a V stage)
-static_assert(B_LNFREE < kNumBars, "barrier count");
+constexpr int B_OFULL = 21;   // every P.V of the item completed
+constexpr int B_OFREE = 22;   // O read out of TMEM (one arrival per epilogue warp)
+constexpr int B_DONE = 23;    // every MMA of both issuers has completed
+constexpr int B_RFULL = 24;   // +ring slot: item written
+constexpr int B_REMPTY = 32;  // +ring slot: every role has read the item
+static_assert(B_REMPTY + kRing == kNumBars, "barrier count");
+constexpr uint32_t kRingReaders = 2 + kEpiWarps;   // both issuers + each epilogue warp
 constexpr int kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 384;
-constexpr int kWarpPV = 18;   // warp of the P.V issuer
+constexpr uint32_t kColO = 384;
+// named barriers of the epilogue warps (0 is __syncthreads)
+constexpr int NB_EXIT = 1;    // OR-reduced decisions to stop
+constexpr int NB_SYNC = 2;
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);   // Q (K-major) x K (K-major)
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);   // P (TMEM) x V (MN-major)
@@ -127,147 +125,61 @@ __device__ __forceinline__ void set_status(int* status, int bit) {
   if (status) atomicOr(status, bit);
 }
 
-struct EpiCtx {
-  const uint32_t* wpk;        // warp's half position bias pairs: element pair (lane, 2i, 2i+1)
-                              // -> wpk[lane - 2i] = (diag of col 2i, diag of col 2i+1)
-  const long long* kts;       // warp's 32 key timestamps
-  const long long* thr;       // bucket thresholds
-  const signed char* first;   // first bucket per octave
-  const float* rabt;          // half time bias per bucket
-  long long my_ts;            // this row's timestamp
-  bool chunk_sorted;          // the warp's key timestamps are non-decreasing
-  float inv_n;                // 1 / N_b
-  int r;                      // row in the tile
-  int lane;
-};
-
-// Time bias of a 32-column chunk for this row.  With the tile's key timestamps
-// sorted and the row not before the chunk's last key, |t_i - t_j| falls along
-// the chunk, so the bucket lies between the buckets k0 >= k1 of its two ends;
-// when they differ by at most one, the columns before `split` (bisection) take
-// k0 and the rest k1 ("simple").  Otherwise every element takes the full search.
-struct ChunkTime {
-  float hi, lo;     // half time bias of buckets k0 and k1
-  int split;        // columns [0, split) take `hi`
-  bool simple;
-};
-
-__device__ __forceinline__ ChunkTime chunk_time(const EpiCtx& e) {
-  ChunkTime ct;
-  ct.hi = ct.lo = 0.f;
-  ct.split = 0;
-  const long long d0 = e.my_ts - e.kts[0];
-  const long long d1 = e.my_ts - e.kts[31];
-  ct.simple = e.chunk_sorted && d1 >= 0;
-  if (ct.simple) {
-    const int k0 = time_bucket(d0, e.thr, e.first);
-    const int k1 = time_bucket(d1, e.thr, e.first);
-    ct.simple = (k0 - k1) <= 1;
-    ct.hi = e.rabt[k0];
-    ct.lo = e.rabt[k1];
-    if (k0 != k1) {
-      // columns c with t_i - t_c >= thr[k0]  <=>  t_c <= t_i - thr[k0]
-      const long long lim = e.my_ts - e.thr[k0];
-      int lo = 0, hi = 32;   // first column with kts > lim
-#pragma unroll 1
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (e.kts[mid] <= lim) lo = mid + 1; else hi = mid;
-      }
-      ct.split = lo;
+// Passes a bounded wait's result through; when it failed, records the
+// timeout bit and, for the first failure of the launch, where it happened in
+// status words 2..5 (wait site, CTA, item, tile) for diagnosis.
+__device__ __forceinline__ bool waited(bool r, int* status, int site, int j, int x) {
+  if (!r && status) {
+    atomicOr(status, kStatusTimeout);
+    if (atomicCAS(status + 2, 0, site) == 0) {
+      status[3] = static_cast<int>(blockIdx.x);
+      status[4] = j;
+      status[5] = x;
     }
   }
-  return ct;
+  return r;
 }
 
-// P' = N * SiLU(S + bias) / N for two adjacent columns, packed as bf16x2:
-//   hx = (S + bias)/2,  P' = hx (1 + tanh(hx)) = SiLU(S + bias).
-// hx is rounded to bf16, tanh and the fused multiply-add run on bf16 pairs
-// (one MUFU operation per two elements); the 1/N factor is applied to O in
-// fp32 after the A.V accumulation instead of to every element of P.
-__device__ __forceinline__ uint32_t p_pair(float hx0, float hx1) {
-  __nv_bfloat162 h2 = __floats2bfloat162_rn(hx0, hx1);   // .x (low half) = hx0
-  const uint32_t hv = *reinterpret_cast<uint32_t*>(&h2);
-  uint32_t tv, pv;
-  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(tv) : "r"(hv));
-  asm("fma.rn.bf16x2 %0, %1, %2, %1;" : "=r"(pv) : "r"(hv), "r"(tv));
-  return pv;
+// ------------------------------------------------------------- bf16x2 helpers
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x (low half) = lo
+  return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// MODE 0: position bias only (or none); 1: plus a per-row time bias constant
-// (`lo`); 2: plus the per-row two-value split; 3: per-element bucket search.
-template <bool POS, int MODE, bool DIAG>
-__device__ __forceinline__ void chunk_to_p(const uint32_t (&sraw)[32], int c0, const EpiCtx& e,
-                                           const ChunkTime& ct, uint32_t (&packed)[16]) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float hx[2], hbp[2] = {0.f, 0.f};
-    if (POS) {
-      const uint32_t w = e.wpk[e.lane - 2 * i];
-      hbp[0] = __uint_as_float(w << 16);
-      hbp[1] = __uint_as_float(w & 0xFFFF0000u);
-    }
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int cl = 2 * i + hh;
-      float hb = hbp[hh];
-      if (MODE == 1) hb += ct.lo;
-      if (MODE == 2) hb += (cl < ct.split) ? ct.hi : ct.lo;
-      if (MODE == 3) hb += e.rabt[time_bucket(e.my_ts - e.kts[cl], e.thr, e.first)];
-      hx[hh] = fmaf(__uint_as_float(sraw[cl]), 0.5f, hb);
-    }
-    uint32_t pv = p_pair(hx[0], hx[1]);
-    if (DIAG) {   // causal mask: column c > row r is exactly zero
-      const int c = c0 + 2 * i;
-      const uint32_t keep = (c > e.r ? 0u : 0x0000FFFFu) | (c + 1 > e.r ? 0u : 0xFFFF0000u);
-      pv &= keep;
-    }
-    packed[i] = pv;
-  }
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
-// Chunk k (32 columns) of this thread's 64 columns -> 16 packed P words.
-template <bool POS, bool TIME, bool DIAG>
-__device__ __forceinline__ void chunk_p(const uint32_t (&sv)[32], int c0, const EpiCtx& e,
-                                        uint32_t (&packed)[16]) {
-  if (!TIME) {
-    chunk_to_p<POS, 0, DIAG>(sv, c0, e, ChunkTime{}, packed);
-  } else {
-    const ChunkTime ct = chunk_time(e);
-    // Warp-uniform choice of the element loop.
-    if (!__all_sync(0xffffffffu, ct.simple)) {
-      chunk_to_p<POS, 3, DIAG>(sv, c0, e, ct, packed);
-    } else if (__any_sync(0xffffffffu, ct.split != 0)) {
-      chunk_to_p<POS, 2, DIAG>(sv, c0, e, ct, packed);
-    } else {
-      chunk_to_p<POS, 1, DIAG>(sv, c0, e, ct, packed);
-    }
-  }
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
-// This thread's 32 columns (col0 .. col0+31) of the S tile -> P in TMEM,
-// packed into columns col0 .. col0+15 of the same buffer (already read).
-// `wpk` holds the warp's 64 staged diagonal pairs, `kts` its 32 key timestamps.
-template <bool POS, bool TIME, bool DIAG>
-__device__ __forceinline__ void chunk_to_tmem(uint32_t s_addr, int col0, EpiCtx& e,
-                                              const uint32_t* wpk, const long long* kts,
-                                              bool sorted) {
-  uint32_t sv[32];
-  uint32_t packed[16];
-  tmem_ld32_nowait(s_addr + col0, sv);
-  tmem_wait_ld_dep(sv);
-  // element (lane, cl) uses diagonal index lane - cl + 31
-  e.wpk = wpk + 31;
-  e.kts = kts;
-  e.chunk_sorted = sorted;
-  chunk_p<POS, TIME, DIAG>(sv, col0, e, packed);
-  tmem_st16(s_addr + col0, packed);
+__device__ __forceinline__ uint32_t tanh2(uint32_t x) {
+  uint32_t t;
+  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(x));
+  return t;
 }
+
+constexpr uint32_t kHalfPair = 0x3F003F00u;   // (0.5, 0.5) in bf16
+
+// SiLU of a pair of half arguments hx = x/2: x/2 (1 + tanh(x/2)) = SiLU(x).
+__device__ __forceinline__ uint32_t silu_pair(uint32_t hx) { return hfma2(hx, tanh2(hx), hx); }
 
 // SiLU of the gate input through tanh: x/2 (1 + tanh(x/2)).
 __device__ __forceinline__ float silu_gate(float x) {
   const float hx = 0.5f * x;
   return fmaf(hx, tanh_approx(hx), hx);
+}
+
+// bucket(|dt|) for 0 <= |dt| < 2^31 from the packed per-octave thresholds.
+__device__ __forceinline__ int bucket32(uint32_t a, const uint4* oct) {
+  a = a < 1u ? 1u : a;
+  const uint4 o = oct[31 - __clz(static_cast<int>(a))];
+  return static_cast<int>(o.x) + (a >= o.y) + (a >= o.z) + (a >= o.w);
 }
 
 // Start and length of sequence b; inconsistent offsets give length -1.
@@ -280,26 +192,32 @@ __device__ __forceinline__ int2 load_seq(const FwdArgs& a, int b, bool pos) {
 }
 
 // Work slots: sequences are taken in groups of G whose keys and values fit in
-// L2 together; inside a group, slot r is the item (m = M-1 - r/G, b = group
-// * G + r mod G), so the most expensive query tiles of the group come first
-// (a longest-first list schedule), and the K/V tiles every query tile of a
-// sequence reads stay in L2 while the group is worked on.
-__device__ __forceinline__ int2 slot_item(unsigned k, unsigned G, int M) {
-  const unsigned per = G * static_cast<unsigned>(M);
+// L2 together; inside a group, slot r is the item (m = M-1 - r/(G H),
+// b = group * G + (r / H) mod G, h = r mod H): the most expensive query tiles
+// of the group come first (a longest-first list schedule) and the heads of
+// one (b, m) block are claimed together.
+struct Item {
+  int m, b, h;
+};
+
+__device__ __forceinline__ Item slot_item(unsigned k, unsigned G, int M, int H) {
+  const unsigned GH = G * static_cast<unsigned>(H);
+  const unsigned per = GH * static_cast<unsigned>(M);
   const unsigned grp = k / per, r = k % per;
-  return make_int2(M - 1 - static_cast<int>(r / G), static_cast<int>(grp * G + r % G));
+  const unsigned rest = r % GH;
+  return Item{M - 1 - static_cast<int>(r / GH), static_cast<int>(grp * G + rest / H),
+              static_cast<int>(rest % static_cast<unsigned>(H))};
 }
 
-// Claims this cluster's next item (warp-collective; leader CTA's warp 0).  Cluster c takes slot c as its first
-// item without touching the counter (the first `base` slots, one per
-// cluster); every later claim takes slot base + the counter's old value from
-// an atomic add.  A slot whose tile lies past its sequence end holds no work:
-// the warp then tests the 31 slots after it and raises the counter past the
-// empty ones among them (atomicMax; every skipped slot was seen empty, and no
-// slot is handed out twice), then claims again.  Returns (-1, -1) once the
-// slots are exhausted.
+// Claims the CTA's next item (warp-collective).  The CTA's first item is slot
+// `first` (its block index) without touching the counter; every later claim
+// takes slot base + the counter's old value from an atomic add.  A slot whose
+// tile lies past its sequence end holds no work: the warp then tests the 31
+// slots after it and raises the counter past the empty ones among them
+// (atomicMax; every skipped slot was seen empty, and no slot is handed out
+// twice), then claims again.  Returns m = -1 once the slots are exhausted.
 template <bool POS>
-__device__ int2 claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots, unsigned base,
+__device__ Item claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots, unsigned base,
                            int first, int lane) {
   const unsigned G = static_cast<unsigned>(a.group);
   const int M = a.max_tiles;
@@ -310,23 +228,23 @@ __device__ int2 claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots,
       if (lane == 0) k = atomicAdd(counter, 1u) + base;
       k = __shfl_sync(0xffffffffu, k, 0);
     }
-    if (k >= nslots) return make_int2(-1, -1);
+    if (k >= nslots) return Item{-1, -1, -1};
     const unsigned slot = k + static_cast<unsigned>(lane);
     bool valid = false;
     if (slot < nslots && (!fixed || lane == 0)) {
-      const int2 it = slot_item(slot, G, M);
-      if (it.y < a.B) {   // the last group may be partial
-        const int2 sq = load_seq(a, it.y, POS);
+      const Item it = slot_item(slot, G, M, a.H);
+      if (it.b < a.B) {   // the last group may be partial
+        const int2 sq = load_seq(a, it.b, POS);
         if (sq.y < 0) {
-          if (it.x == 0) set_status(a.status, kStatusBadOffsets);
+          if (it.m == 0 && it.h == 0) set_status(a.status, kStatusBadOffsets);
         } else {
-          valid = kRows * it.x < sq.y;
+          valid = kRows * it.m < sq.y;
         }
       }
     }
     const unsigned vb = __ballot_sync(0xffffffffu, valid);
-    if (vb & 1u) return slot_item(k, G, M);
-    if (fixed) {          // the cluster's own first slot is empty: claim from the counter
+    if (vb & 1u) return slot_item(k, G, M, a.H);
+    if (fixed) {          // the CTA's own first slot is empty: claim from the counter
       fixed = false;
       continue;
     }
@@ -336,13 +254,68 @@ __device__ int2 claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots,
   }
 }
 
+// Time bias of one 32-key chunk for one row, as a plan the element loop uses.
+// With the chunk's keys ascending and all at or before the row (and |dt| <
+// 2^31), dt falls along the chunk and the bucket lies between the buckets k0
+// >= k1 of its two ends: one value (CONST) or two with a split column (SPLIT,
+// found by bisection).  Otherwise every element takes its own bucket (GEN32
+// with 32-bit differences, GEN64 for time spans of 2^31 or more).
+enum { T_CONST = 0, T_SPLIT = 1, T_GEN32 = 2, T_GEN64 = 3 };
+
+struct EpiShared {
+  const uint4* oct;
+  const unsigned* thr32;
+  const long long* thr;
+  const signed char* first;
+  const float* rabt;         // half time bias per bucket
+};
+
+// P' pairs of one 32-column chunk: sv = S (fp32), wpk = the warp's staged
+// position-bias pairs, indexed (lane - 2i + 31) for columns 2i, 2i+1 (halved
+// bf16), result packed[16].  TM selects the time plan.
+template <bool POS, bool TIME, int TM>
+__device__ __forceinline__ void chunk_pairs(const uint32_t (&sv)[32], const uint32_t* wpk,
+                                            uint32_t tconst, uint32_t thh, uint32_t tll,
+                                            uint32_t thl, int split, uint32_t my32,
+                                            long long my64, const uint32_t* kts32,
+                                            const long long* kts64, const EpiShared& es,
+                                            uint32_t (&packed)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t s2 = pack_bf16x2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
+    uint32_t hx = hfma2(s2, kHalfPair, POS ? wpk[-2 * i] : 0u);
+    if (TIME) {
+      uint32_t tb;
+      if (TM == T_CONST) {
+        tb = tconst;
+      } else if (TM == T_SPLIT) {
+        tb = (2 * i + 1 < split) ? thh : ((2 * i < split) ? thl : tll);
+      } else {
+        float tv[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          int k;
+          if (TM == T_GEN32) {
+            const int d = static_cast<int>(my32 - kts32[2 * i + hh]);
+            k = bucket32(static_cast<uint32_t>(d < 0 ? -d : d), es.oct);
+          } else {
+            k = time_bucket(my64 - kts64[2 * i + hh], es.thr, es.first);
+          }
+          tv[hh] = es.rabt[k];
+        }
+        tb = pack_bf16x2(tv[0], tv[1]);
+      }
+      hx = hadd2(hx, tb);
+    }
+    packed[i] = silu_pair(hx);
+  }
+}
+
 template <bool POS, bool TIME>
 __global__ void __launch_bounds__(kThreads, 1)
     hstu_fwd_bf16_sm100(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
-                        const __grid_constant__ CUtensorMap tm_u,
-                        const __grid_constant__ CUtensorMap tm_y,
                         const __grid_constant__ FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -351,63 +324,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int H = a.H;
-  const int h = static_cast<int>(cluster_ctarank());   // head = rank in the cluster
-  const bool leader = (h == 0);
 
   auto bar = [&](int i) { return sbase + kOffBar + 8u * i; };
-  auto ring_addr = [&](int slot) { return sbase + kOffRing + 8u * slot; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-
-  long long* s_thr = reinterpret_cast<long long*>(smem + kOffThr);
-  signed char* s_first = reinterpret_cast<signed char*>(smem + kOffFirst);
-  float* s_rabt = reinterpret_cast<float*>(smem + kOffRabT);
+  int4* ring = reinterpret_cast<int4*>(smem + kOffRing);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
-      if (i >= B_PFULL && i < B_PFULL + kSBufs) count = kEpiThreads;
+      if ((i >= B_PFULL && i < B_PFULL + kSBufs) || i == B_OFREE) count = kEpiWarps;
       if (i == B_DONE) count = 2;                                        // both issuers
-      if (i >= B_REMPTY && i < B_REMPTY + kRing) count = static_cast<uint32_t>(H);
+      if (i >= B_REMPTY && i < B_REMPTY + kRing) count = kRingReaders;
       mbar_init(bar(i), count);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kWarpS) {
     tmem_alloc(sbase + kOffMisc, kTmemCols);
     tmem_relinquish();
   }
-  if (TIME && warp >= 2 && warp < kWarpPV) {
-    const int et = threadIdx.x - 64;
+  if (TIME && warp >= kWarpEpi) {
+    const int et = threadIdx.x - kWarpEpi * 32;
+    long long* s_thr = reinterpret_cast<long long*>(smem + kOffThr);
     for (int i = et; i < kThrLen; i += kEpiThreads) s_thr[i] = a.bt.thr[i];
-    if (et < 64) s_first[et] = a.bt.first_k[et];
-    if (et < a.nb) s_rabt[et] = 0.5f * __ldg(a.rab_time + static_cast<size_t>(h) * a.nb + et);
+    if (et < kMaxBuckets) reinterpret_cast<unsigned*>(smem + kOffThr32)[et] = a.bt.thr32[et];
+    if (et < 32) reinterpret_cast<uint4*>(smem + kOffOct)[et] = a.bt.oct[et];
+    if (et < 64) reinterpret_cast<signed char*>(smem + kOffFirst)[et] = a.bt.first_k[et];
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_u);
-    tma_prefetch_desc(&tm_y);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // Every CTA of the cluster has initialised its barriers before any remote access.
-  cluster_arrive();
-  cluster_wait();
   const uint32_t tmem = misc[0];
 
-  // Item j of this cluster sits in ring slot j % kRing; every role reads it in order.
   auto wait_item = [&](int j) -> bool {
-    return mbar_wait<true>(bar(B_RFULL + j % kRing), (j / kRing) & 1, abort_flag);
+    return waited(mbar_wait(bar(B_RFULL + j % kRing), (j / kRing) & 1, abort_flag), a.status,
+                  warp < kWarpEpi ? 10 + warp : 20, j, -1);
   };
-  auto read_item = [&](int j) -> int2 {
-    int2 v;
-    asm volatile("ld.shared.v2.s32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(ring_addr(j % kRing))
-                 : "memory");
-    return v;
+  auto read_item = [&](int j) -> Item {
+    const int4 v = ring[j % kRing];
+    return Item{v.x, v.y, v.z};
   };
 
   if (warp == 0) {
@@ -415,51 +377,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned* counter = reinterpret_cast<unsigned*>(a.status) + kSchedCounterWord;
     unsigned* done = reinterpret_cast<unsigned*>(a.status) + kSchedDoneWord;
     const unsigned nslots = static_cast<unsigned>((a.B + a.group - 1) / a.group) *
-                            static_cast<unsigned>(a.group) * static_cast<unsigned>(a.max_tiles);
-    // Leader: claim item j and hand it to every CTA of the cluster (warp-collective).
-    auto fetch = [&](int j) -> int2 {
+                            static_cast<unsigned>(a.group) * static_cast<unsigned>(a.max_tiles) *
+                            static_cast<unsigned>(H);
+    // Claim item j and publish it in the ring (warp-collective).
+    auto fetch = [&](int j) -> Item {
       bool okf = true;
-      int2 it = make_int2(-1, -1);
-      if (leader) {
-        // The slot's previous item (j - kRing) must have been read by every CTA.
-        if (lane == 0 && j >= kRing)
-          okf = mbar_wait<true>(bar(B_REMPTY + j % kRing), ((j / kRing) - 1) & 1, abort_flag);
-        okf = __shfl_sync(0xffffffffu, okf, 0);
-        if (okf) {
-          const unsigned clusters = gridDim.x / static_cast<unsigned>(H);
-          it = claim_item<POS>(a, counter, nslots, clusters,
-                               j == 0 ? static_cast<int>(blockIdx.x / static_cast<unsigned>(H)) : -1,
-                               lane);
-          if (lane == 0) {
-            for (int pr = 0; pr < H; ++pr) {
-              st_cluster_v2_s32(mapa_shared(ring_addr(j % kRing), pr), it.x, it.y);
-              mbar_arrive_cluster(mapa_shared(bar(B_RFULL + j % kRing), pr));
-            }
-          }
-        }
-      } else {
-        if (lane == 0) {
-          okf = wait_item(j);
-          if (okf) it = read_item(j);
-        }
-        okf = __shfl_sync(0xffffffffu, okf, 0);
-        it.x = __shfl_sync(0xffffffffu, it.x, 0);
-        it.y = __shfl_sync(0xffffffffu, it.y, 0);
+      if (lane == 0 && j >= kRing)
+        okf = waited(mbar_wait(bar(B_REMPTY + j % kRing), ((j / kRing) - 1) & 1, abort_flag),
+                     a.status, 1, j, -1);
+      okf = __shfl_sync(0xffffffffu, okf, 0);
+      if (!okf) return Item{-2, -2, -2};
+      const Item it = claim_item<POS>(a, counter, nslots, gridDim.x,
+                                      j == 0 ? static_cast<int>(blockIdx.x) : -1, lane);
+      if (lane == 0) {
+        ring[j % kRing] = make_int4(it.m, it.b, it.h, 0);
+        mbar_arrive(bar(B_RFULL + j % kRing));
       }
       __syncwarp();
-      return okf ? it : make_int2(-2, -2);
+      return it;
     };
 
     int k_last[kKStages] = {-1, -1, -1}, v_last[kVStages] = {-1, -1};
     int q_last = -1;
     bool ok = true;
     int j = 0, g = 0;
-    int2 it = fetch(0);
-    while (it.x >= 0) {
+    Item it = fetch(0);
+    while (it.m >= 0) {
       if (lane == 0) {
-        const int m = it.x, nt = m + 1;
-        const int s = __ldg(a.offsets + it.y);
-        if (j > 0) ok = mbar_wait(bar(B_QEMPTY), (j - 1) & 1, abort_flag);
+        const int m = it.m, nt = m + 1, h = it.h;
+        const int s = __ldg(a.offsets + it.b);
+        if (j > 0) ok = waited(mbar_wait(bar(B_QEMPTY), (j - 1) & 1, abort_flag), a.status, 2, j, g);
         if (ok) {
           const int row0 = s + kRows * m;
           mbar_arrive_expect_tx(bar(B_QFULL), kTile);
@@ -471,7 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // stage frees only when P(x-2).V completes.  x is the running tile index.
         auto load_k = [&](int x, int n) -> bool {
           const int st = x % kKStages, use = x / kKStages;
-          if (use > 0 && !mbar_wait(bar(B_KEMPTY + st), (use - 1) & 1, abort_flag)) return false;
+          if (use > 0 && !waited(mbar_wait(bar(B_KEMPTY + st), (use - 1) & 1, abort_flag), a.status,
+                                 3, j, x))
+            return false;
           const int krow = s + kCols * n;
           mbar_arrive_expect_tx(bar(B_KFULL + st), kTile);
           tma_load_3d(sbase + kOffK + st * kTile, &tm_k, bar(B_KFULL + st), 0, h, krow);
@@ -481,7 +430,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto load_v = [&](int x, int n) -> bool {
           const int st = x % kVStages, use = x / kVStages;
-          if (use > 0 && !mbar_wait(bar(B_VEMPTY + st), (use - 1) & 1, abort_flag)) return false;
+          if (use > 0 && !waited(mbar_wait(bar(B_VEMPTY + st), (use - 1) & 1, abort_flag), a.status,
+                                 4, j, x))
+            return false;
           const int krow = s + kCols * n;
           mbar_arrive_expect_tx(bar(B_VFULL + st), kTile);
           tma_load_3d(sbase + kOffV + st * kTile, &tm_v, bar(B_VFULL + st), 0, h, krow);
@@ -492,19 +443,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = load_k(g, 0);
         for (int n = 0; n < nt && ok; ++n) {
           if (n + 1 < nt) ok = load_k(g + n + 1, n + 1);
-          // The previous item's LayerNorm borrows the V stage of this item's
-          // first tile: wait until its U load and Y store are done with it.
-          if (ok && n == 0 && j > 0) ok = mbar_wait(bar(B_LNFREE), (j - 1) & 1, abort_flag);
           if (ok) ok = load_v(g + n, n);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      g += it.x + 1;
+      g += it.m + 1;
       ++j;
       it = fetch(j);
     }
-    if (it.x == -2) ok = false;
+    if (it.m == -2) ok = false;
+    if (!ok && lane == 0) {
+      // Let the other roles leave: publish an end marker where they wait next.
+      ring[j % kRing] = make_int4(-2, -2, -2, 0);
+      mbar_arrive(bar(B_RFULL + j % kRing));
+    }
     if (lane == 0) {
       if (!ok) {
         set_status(a.status, kStatusTimeout);
@@ -516,17 +469,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int st = 0; st < kVStages; ++st)
           if (v_last[st] >= 0) mbar_wait(bar(B_VFULL + st), v_last[st] & 1, nullptr);
       }
-      if (leader) {
-        // The last cluster to finish returns the work counter to zero for the next launch.
-        __threadfence();
-        const unsigned clusters = gridDim.x / static_cast<unsigned>(H);
-        if (atomicAdd(done, 1u) == clusters - 1) {
-          atomicExch(counter, 0u);
-          atomicExch(done, 0u);
-        }
+      // The last CTA to finish returns the work counter to zero for the next launch.
+      __threadfence();
+      if (atomicAdd(done, 1u) == gridDim.x - 1) {
+        atomicExch(counter, 0u);
+        atomicExch(done, 0u);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpS) {
     // ------------------------------------------------------------ S issuer
     if (lane == 0) {
       bool ok = true;
@@ -534,19 +484,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (;;) {
         ok = wait_item(j);
         if (!ok) break;
-        const int2 it = read_item(j);
-        if (it.x < 0) break;
-        const int nt = it.x + 1;
-        ok = mbar_wait(bar(B_QFULL), j & 1, abort_flag);
+        const Item it = read_item(j);
+        mbar_arrive(bar(B_REMPTY + j % kRing));
+        if (it.m < 0) break;
+        const int nt = it.m + 1;
+        ok = waited(mbar_wait(bar(B_QFULL), j & 1, abort_flag), a.status, 5, j, g);
         for (int n = 0; n < nt && ok; ++n) {
           const int x = g + n, st = x % kKStages, buf = x % kSBufs;
           // The buffer's previous tile x-3 has been consumed by its P.V.
           if (x >= kSBufs)
-            ok = mbar_wait(bar(B_PVDONE + buf), ((x - kSBufs) / kSBufs) & 1, abort_flag);
-          if (ok) ok = mbar_wait(bar(B_KFULL + st), (x / kKStages) & 1, abort_flag);
+            ok = waited(mbar_wait(bar(B_PVDONE + buf), ((x - kSBufs) / kSBufs) & 1, abort_flag),
+                        a.status, 6, j, x);
+          if (ok)
+            ok = waited(mbar_wait(bar(B_KFULL + st), (x / kKStages) & 1, abort_flag), a.status, 7, j,
+                        x);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t d = tmem + kColS0 + 128u * buf;
+          const uint32_t d = tmem + 128u * buf;
           const uint32_t qa = sbase + kOffQ, ka = sbase + kOffK + st * kTile;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
@@ -576,22 +530,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (;;) {
         ok = wait_item(j);
         if (!ok) break;
-        const int2 it = read_item(j);
-        if (it.x < 0) break;
-        const int nt = it.x + 1;
+        const Item it = read_item(j);
+        mbar_arrive(bar(B_REMPTY + j % kRing));
+        if (it.m < 0) break;
+        const int nt = it.m + 1;
+        // The previous item's O has been read out of TMEM.
+        if (j > 0) ok = waited(mbar_wait(bar(B_OFREE), (j - 1) & 1, abort_flag), a.status, 8, j, g);
         for (int n = 0; n < nt && ok; ++n) {
           const int x = g + n, st = x % kVStages, buf = x % kSBufs;
-          ok = mbar_wait(bar(B_PFULL + buf), (x / kSBufs) & 1, abort_flag);
-          if (ok) ok = mbar_wait(bar(B_VFULL + st), (x / kVStages) & 1, abort_flag);
+          ok = waited(mbar_wait(bar(B_PFULL + buf), (x / kSBufs) & 1, abort_flag), a.status, 9, j, x);
+          if (ok)
+            ok = waited(mbar_wait(bar(B_VFULL + st), (x / kVStages) & 1, abort_flag), a.status, 30,
+                        j, x);
           if (!ok) break;
           tc_fence_after();
           const uint32_t va = sbase + kOffV + st * kTile;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            // 16 keys per step: rows 16ks.. of the V tile; the two 64-column
-            // halves of d_v are 16 KB apart (leading byte offset).
-            // P keys 16ks..16ks+15: column group ks/2 holds its 32 keys in 16 columns.
-            mma_ts(tmem + kColO, tmem + kColS0 + 128u * buf + 32u * (ks >> 1) + 8u * (ks & 1),
+            // Keys 16ks..16ks+15: column group ks/2 holds its 32 keys in its
+            // first 16 columns; rows 16ks.. of the V tile, whose two
+            // 64-column halves of d_v are 16 KB apart (leading byte offset).
+            mma_ts(tmem + kColO, tmem + 128u * buf + 32u * (ks >> 1) + 8u * (ks & 1),
                    sw128_desc(va + ks * 2048, kHalf, 1024), kIdescPV, (n > 0 || ks > 0));
           }
           mma_commit(bar(B_VEMPTY + st));
@@ -608,27 +567,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(bar(B_DONE));
     }
-  } else if (warp < kWarpPV) {
+  } else {
     // ------------------------------------------------------------ epilogue
+    const int ew = warp - kWarpEpi;               // 0..15
     const int q4 = warp & 3;                      // TMEM lane quarter
-    const int cq = (warp - 2) >> 2;               // 32-column group of the S/P and O tiles
+    const int cq = ew >> 2;                       // 32-column group of the S/P and O tiles
     const int r = q4 * 32 + lane;                 // row within the tile
-    const int et = threadIdx.x - 64;              // 0..511 among epilogue threads
+    const int et = threadIdx.x - kWarpEpi * 32;   // 0..511 among epilogue threads
     const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
     const int Lw = 2 * a.L - 1;
     const int D = H * 128;
-    uint8_t* wstage = smem + kOffWarp + (warp - 2) * kWarpStage;
+    uint8_t* wstage = smem + kOffWarp + ew * kWarpStage;
     uint32_t* wpk = reinterpret_cast<uint32_t*>(wstage);
     long long* wts = reinterpret_cast<long long*>(wstage + 64 * 4);
+    uint32_t* wts32 = reinterpret_cast<uint32_t*>(wstage + 64 * 4 + 32 * 8);
     float2* loc = reinterpret_cast<float2*>(smem + kOffLoc);   // [4][128]
-    float2* red = reinterpret_cast<float2*>(smem + kOffRed);   // [2][kMaxHeads][128]
-    const uint32_t rempty_leader = mapa_shared(bar(B_REMPTY), 0);
-    EpiCtx ec;
-    ec.thr = s_thr;
-    ec.first = s_first;
-    ec.rabt = s_rabt;
-    ec.r = r;
-    ec.lane = lane;
+    float* s_rabt = reinterpret_cast<float*>(smem + kOffRabT);
+    volatile unsigned* bcast = reinterpret_cast<volatile unsigned*>(misc + 2);
+    EpiShared es;
+    es.oct = reinterpret_cast<const uint4*>(smem + kOffOct);
+    es.thr32 = reinterpret_cast<const unsigned*>(smem + kOffThr32);
+    es.thr = reinterpret_cast<const long long*>(smem + kOffThr);
+    es.first = reinterpret_cast<const signed char*>(smem + kOffFirst);
+    es.rabt = s_rabt;
     bool ok = true;
     int j = 0, g = 0;
 
@@ -636,34 +597,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     // at the same point: the decisions to stop are OR-reduced over all of them.
     for (;;) {
       const bool got = __all_sync(0xffffffffu, wait_item(j));
-      const int2 it = got ? read_item(j) : make_int2(-2, -2);
-      if (named_bar_or(2, kEpiThreads, !ok || it.x < 0)) {
-        if (it.x == -2) ok = false;
+      const Item it = got ? read_item(j) : Item{-2, -2, -2};
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_REMPTY + j % kRing));
+      // The previous item's last use of the time-bias row precedes the
+      // barriers at its end: the row of this item's head replaces it here.
+      if (TIME && got && it.m >= 0 && et < a.nb)
+        s_rabt[et] = 0.5f * __ldg(a.rab_time + static_cast<size_t>(it.h) * a.nb + et);
+      if (named_bar_or(NB_EXIT, kEpiThreads, !ok || it.m < 0)) {
+        if (it.m == -2) ok = false;
         break;
       }
-      const int m = it.x, nt = m + 1;
-      const int s = __ldg(a.offsets + it.y);
-      const int n_b = __ldg(a.offsets + it.y + 1) - s;
+      const int m = it.m, nt = m + 1, b = it.b, h = it.h;
+      const int s = __ldg(a.offsets + b);
+      const int n_b = __ldg(a.offsets + b + 1) - s;
       const int i_loc = kRows * m + r;            // local row index in the sequence
       const bool row_ok = i_loc < n_b;
       const int t_row = s + (row_ok ? i_loc : 0);
       const float nrm = a.norm_len > 0 ? static_cast<float>(a.norm_len) : static_cast<float>(n_b);
       // Rows past the sequence end (never stored) take the last token's
-      // timestamp: every key is then at or before them, the chunk plans stay
-      // on the cheap path, and no warp drops to the per-element search.
-      ec.my_ts = TIME ? a.timestamps[row_ok ? t_row : s + n_b - 1] : 0;
-      ec.inv_n = 1.0f / nrm;
-      // The gate input of this row is read at the end of the item: ask L2 for it now.
+      // timestamp: every key is then at or before them and the plans stay cheap.
+      long long my64 = 0;
+      if (TIME) my64 = a.timestamps[row_ok ? t_row : s + n_b - 1];
+      const uint32_t my32 = static_cast<uint32_t>(my64);
+      // The gate input of this row is read at the end of the block: ask L2 for it now.
       if (row_ok)
-        prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(a.u) +
-                    static_cast<size_t>(t_row) * (H * 128) + h * 128 + 32 * cq);
+        prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(a.u) + static_cast<size_t>(t_row) * D +
+                    h * 128 + 32 * cq);
 
       // Staging of this warp's 32 x 32 block of tile n: half position bias of
       // the 63 diagonals d = r - c in [32 q4 - 32 cq - 31, 32 q4 - 32 cq + 31]
       // (table index 128 (m - n) + d + L - 1), entry k as the bf16 pair
       // (diagonal k, diagonal k-1), and the timestamps of its 32 keys (keys
       // past the sequence end repeat its last timestamp, which keeps them
-      // non-decreasing; those keys are masked anyway).
+      // ascending; those keys are masked anyway), with their minimum, maximum
+      // and whether they ascend.
       const int dbase = 32 * q4 - 32 * cq - 31;
       float pre_w0 = 0.f, pre_w1 = 0.f;
       long long pre_t = 0;
@@ -679,8 +647,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           pre_t = a.timestamps[s + (jj < n_b ? jj : n_b - 1)];
         }
       };
-      bool sorted = true;
-      auto stage = [&]() {   // previous users of the buffer (this warp) are done
+      long long kmin = 0, kmax = 0;
+      bool asc = true;
+      auto stage = [&]() {   // this warp's previous reads of its buffer are done
         if (POS) {
           const float v0 = 0.5f * pre_w0, v1 = 0.5f * pre_w1;
           float p0 = __shfl_up_sync(0xffffffffu, v0, 1);
@@ -690,15 +659,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             p0 = 0.f;
             p1 = e0;
           }
-          __nv_bfloat162 b0 = __floats2bfloat162_rn(v0, p0);   // .x (low) = diagonal k
-          __nv_bfloat162 b1 = __floats2bfloat162_rn(v1, p1);
-          wpk[lane] = *reinterpret_cast<uint32_t*>(&b0);
-          wpk[32 + lane] = *reinterpret_cast<uint32_t*>(&b1);
+          wpk[lane] = pack_bf16x2(v0, p0);        // low half: diagonal k
+          wpk[32 + lane] = pack_bf16x2(v1, p1);
         }
         if (TIME) {
           wts[lane] = pre_t;
+          wts32[lane] = static_cast<uint32_t>(pre_t);
+          long long mn = pre_t, mx = pre_t;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const long long a2 = __shfl_xor_sync(0xffffffffu, mn, o);
+            const long long b2 = __shfl_xor_sync(0xffffffffu, mx, o);
+            mn = a2 < mn ? a2 : mn;
+            mx = b2 > mx ? b2 : mx;
+          }
+          kmin = mn;
+          kmax = mx;
           const long long nx = __shfl_down_sync(0xffffffffu, pre_t, 1);
-          sorted = !__any_sync(0xffffffffu, lane < 31 && nx < pre_t);
+          asc = !__any_sync(0xffffffffu, lane < 31 && nx < pre_t);
         }
         __syncwarp();
       };
@@ -708,76 +686,112 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = 0; n < nt; ++n) {
         const int x = g + n, buf = x % kSBufs;
         if (n + 1 < nt) prefetch(n + 1);          // global loads overlap this tile
-        if (ok) ok = mbar_wait(bar(B_SFULL + buf), (x / kSBufs) & 1, abort_flag);
-        // The TMEM loads/stores below are warp-collective: keep the decision warp-uniform.
+        if (ok)
+          ok = waited(mbar_wait(bar(B_SFULL + buf), (x / kSBufs) & 1, abort_flag), a.status, 40,
+                      j, x);
+        // The TMEM accesses below are warp-collective: keep the decision warp-uniform.
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;                           // on to the collective exit below
         tc_fence_after();
-        const uint32_t s_addr = tmem + lane_addr + kColS0 + 128u * buf;
-        if (n == m)
-          chunk_to_tmem<POS, TIME, true>(s_addr, 32 * cq, ec, wpk, wts, sorted);
-        else
-          chunk_to_tmem<POS, TIME, false>(s_addr, 32 * cq, ec, wpk, wts, sorted);
+        const uint32_t s_addr = tmem + lane_addr + 128u * buf;
+        uint32_t packed[16];
+        const bool diag = (n == m);
+        if (diag && cq > q4) {                    // entirely above the diagonal
+#pragma unroll
+          for (int i = 0; i < 16; ++i) packed[i] = 0u;
+        } else {
+          uint32_t sv[32];
+          tmem_ld32_nowait(s_addr + 32u * cq, sv);
+          tmem_wait_ld_dep(sv);
+          // element (lane, c) uses diagonal index lane - c + 31
+          const uint32_t* wp = wpk + 31 + lane;
+          if (!TIME) {
+            chunk_pairs<POS, false, T_CONST>(sv, wp, 0u, 0u, 0u, 0u, 0, 0u, 0ll, nullptr,
+                                             nullptr, es, packed);
+          } else {
+            // plan of this row's 32 keys
+            const long long dmax = my64 - kmin, dmin = my64 - kmax;
+            const bool fast = dmax < 0x7FFFFFFFll && dmax > -0x7FFFFFFFll &&
+                              dmin < 0x7FFFFFFFll && dmin > -0x7FFFFFFFll;
+            const bool mono = fast && asc && dmin >= 0;
+            int k0 = 0, k1 = 0;
+            if (mono) {
+              k0 = bucket32(static_cast<uint32_t>(dmax), es.oct);
+              k1 = bucket32(static_cast<uint32_t>(dmin), es.oct);
+            }
+            if (__all_sync(0xffffffffu, mono && k0 == k1)) {
+              const float tv = es.rabt[k0];
+              chunk_pairs<POS, true, T_CONST>(sv, wp, pack_bf16x2(tv, tv), 0u, 0u, 0u, 0, my32,
+                                              my64, wts32, wts, es, packed);
+            } else if (__all_sync(0xffffffffu, mono && k0 - k1 <= 1)) {
+              // first column whose bucket is k1: dt < thr[k0]
+              int split = 32;
+              if (k0 != k1) {
+                const uint32_t th = es.thr32[k0];
+                int lo = 0, hi = 32;
+#pragma unroll 1
+                while (lo < hi) {
+                  const int mid = (lo + hi) >> 1;
+                  if (my32 - wts32[mid] >= th) lo = mid + 1; else hi = mid;
+                }
+                split = lo;
+              }
+              const float hv = es.rabt[k0], lv = es.rabt[k1];
+              chunk_pairs<POS, true, T_SPLIT>(sv, wp, 0u, pack_bf16x2(hv, hv),
+                                              pack_bf16x2(lv, lv), pack_bf16x2(hv, lv), split,
+                                              my32, my64, wts32, wts, es, packed);
+            } else if (__all_sync(0xffffffffu, fast)) {
+              chunk_pairs<POS, true, T_GEN32>(sv, wp, 0u, 0u, 0u, 0u, 0, my32, my64, wts32, wts,
+                                              es, packed);
+            } else {
+              chunk_pairs<POS, true, T_GEN64>(sv, wp, 0u, 0u, 0u, 0u, 0, my32, my64, wts32, wts,
+                                              es, packed);
+            }
+          }
+          if (diag && cq == q4) {                 // causal mask: column 32 cq + c > row r
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint32_t keep = (2 * i > lane ? 0u : 0x0000FFFFu) |
+                                    (2 * i + 1 > lane ? 0u : 0xFFFF0000u);
+              packed[i] &= keep;
+            }
+          }
+        }
+        tmem_st16(s_addr + 32u * cq, packed);   // over this warp's own, already read S columns
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL + buf));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PFULL + buf));
         if (n + 1 < nt) stage();
       }
 
-      // -------------------------------------------- LayerNorm over heads + gate
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), j & 1, abort_flag));
-      if (ok) tc_fence_after();
-      // The row's 32 values of this head and column quarter stay in registers.
+      // -------------------------------------- O of the item: statistics and stash
+      if (named_bar_or(NB_EXIT, kEpiThreads, !ok)) {
+        ok = false;
+        break;
+      }
+      ok = waited(mbar_wait(bar(B_OFULL), j & 1, abort_flag), a.status, 50, j, g + nt - 1);
+      ok = __all_sync(0xffffffffu, ok);
       float ov[32];
       {
         uint32_t o0[32];
         if (ok) {
+          tc_fence_after();
           tmem_ld32_nowait(tmem + lane_addr + kColO + 32u * cq, o0);
           tmem_wait_ld_dep(o0);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o0[i] = 0u;
         }
-        // O accumulated SiLU(.) terms: apply 1/N here, in fp32.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_OFREE));   // the next item's P.V may overwrite O
+        const float inv_n = 1.0f / nrm;             // O accumulated SiLU(.) terms
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(o0[i]) * ec.inv_n;
+        for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(o0[i]) * inv_n;
       }
-      const size_t rowD = static_cast<size_t>(t_row) * D + static_cast<size_t>(h) * 128 + 32 * cq;
-      // U and Y of the item travel by TMA through the V stage of the next
-      // item's first tile (every P.V of this item has completed; the producer
-      // waits for B_LNFREE before loading it again).  In that 128B-swizzled
-      // tile, 16-byte chunk c of row r sits at r * 128 + 16 (c ^ (r % 8)) of
-      // its 64-column half: a warp's 32 rows hit every bank once per 8 rows.
-      const uint32_t lnbuf = sbase + kOffV + ((g + nt) % kVStages) * kTile;
-      if (et == 0) {
-        const int row0 = s + kRows * m;
-        mbar_arrive_expect_tx(bar(B_ULOAD), kTile);
-        tma_load_3d(lnbuf, &tm_u, bar(B_ULOAD), 0, h, row0);
-        tma_load_3d(lnbuf + kHalf, &tm_u, bar(B_ULOAD), 64, h, row0);
-      }
-      const uint32_t myrow = lnbuf + (cq >> 1) * kHalf + r * 128;
-      auto chunk_addr = [&](int i) {   // i-th 16-byte chunk of this thread's 32 columns
-        return myrow + 16u * static_cast<uint32_t>((4 * (cq & 1) + i) ^ (r & 7));
-      };
-      if (ok && row_ok && a.o_save) {
-        float* od = a.o_save + rowD;
-        if (a.vec32) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t w[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) w[q] = __float_as_uint(ov[8 * i + q]);
-            st_global_v8(od + 8 * i, w);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(od)[i] =
-                make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
-        }
-      }
-      // Row statistics of the 32 values: sum and sum of squared deviations.
       {
+        // sum and sum of squared deviations of this thread's 32 values
         float sum = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) sum += ov[i];
@@ -790,101 +804,123 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         loc[cq * 128 + r] = make_float2(sum, m2);
       }
-      tc_fence_before();
-      if (named_bar_or(1, kEpiThreads, !ok)) {
-        ok = false;
-        break;
-      }
-      // Every role of this CTA has read item j: release its ring slot.
-      if (et == 0) mbar_arrive_cluster(rempty_leader + 8u * (j % kRing));
-      const int pj = j & 1;
-      if (cq == 0) {
-        // Combine the four 32-column groups (equal counts) into this head's
-        // (sum, M2) and send it to every CTA of the cluster.
-        const float2 p0 = loc[r], p1 = loc[128 + r], p2 = loc[256 + r], p3 = loc[384 + r];
-        const float hs = (p0.x + p1.x) + (p2.x + p3.x);
-        const float mh = hs * (1.0f / 128.0f);
-        const float e0 = p0.x * (1.0f / 32.0f) - mh, e1 = p1.x * (1.0f / 32.0f) - mh;
-        const float e2 = p2.x * (1.0f / 32.0f) - mh, e3 = p3.x * (1.0f / 32.0f) - mh;
-        const float hm2 = (p0.y + p1.y) + (p2.y + p3.y) +
-                          32.0f * ((e0 * e0 + e1 * e1) + (e2 * e2 + e3 * e3));
-        const uint32_t slot = smem_u32(red + (pj * kMaxHeads + h) * 128 + r);
-        for (int pr = 0; pr < H; ++pr)
-          st_async_v2_f32(mapa_shared(slot, pr), hs, hm2, mapa_shared(bar(B_RED + pj), pr));
-      }
-      if (et == 0) mbar_arrive_expect_tx(bar(B_RED + pj), static_cast<uint32_t>(H * 128 * 8));
-      // Gate values while the statistics travel.
-      if (!mbar_wait(bar(B_ULOAD), j & 1, abort_flag)) set_status(a.status, kStatusTimeout);
-      float gate[32];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 ui = ld_shared_v4(chunk_addr(i));
-        const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&ui);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 uf = __bfloat1622float2(u2[q]);
-          gate[8 * i + 2 * q] = silu_gate(uf.x);
-          gate[8 * i + 2 * q + 1] = silu_gate(uf.y);
-        }
-      }
-      if (!mbar_wait<true>(bar(B_RED + pj), (j >> 1) & 1, nullptr)) set_status(a.status, kStatusTimeout);
-      // Chan's combination of the H per-head (sum, M2) pairs of 128 values each.
-      const float2* rr = red + pj * kMaxHeads * 128 + r;
-      float tot = 0.f;
-      for (int k = 0; k < H; ++k) tot += rr[k * 128].x;
-      const float mean = tot / static_cast<float>(D);
-      float m2 = 0.f;
-      for (int k = 0; k < H; ++k) {
-        const float2 pk = rr[k * 128];
-        const float dk = pk.x * (1.0f / 128.0f) - mean;
-        m2 += pk.y + 128.0f * dk * dk;
-      }
-      const float var = m2 / static_cast<float>(D);
-      const float rstd = 1.0f / sqrtf(var + a.eps);
-      {
-        uint32_t yw[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          __nv_bfloat162 pr = __floats2bfloat162_rn((ov[2 * q] - mean) * rstd * gate[2 * q],
-                                                    (ov[2 * q + 1] - mean) * rstd * gate[2 * q + 1]);
-          yw[q] = *reinterpret_cast<uint32_t*>(&pr);
-        }
-        // A tile whose 128 rows all belong to the sequence leaves by one TMA
-        // store; the last, partial tile of a sequence stores its rows directly.
-        const bool full = kRows * m + kRows <= n_b;
-        if (full) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            st_shared_v4(chunk_addr(i), make_uint4(yw[4 * i], yw[4 * i + 1], yw[4 * i + 2],
-                                                   yw[4 * i + 3]));
-          fence_proxy_async_smem();
-        } else if (row_ok) {
-          __nv_bfloat16* yd = reinterpret_cast<__nv_bfloat16*>(a.y) + rowD;
+      named_bar_sync(NB_SYNC, kEpiThreads);
+      // The head's (mean, M2) of the row from its four 32-column groups.
+      const float2 p0 = loc[r], p1 = loc[128 + r], p2 = loc[256 + r], p3 = loc[384 + r];
+      const float mean_h = ((p0.x + p1.x) + (p2.x + p3.x)) * (1.0f / 128.0f);
+      const float e0 = p0.x * (1.0f / 32.0f) - mean_h, e1 = p1.x * (1.0f / 32.0f) - mean_h;
+      const float e2 = p2.x * (1.0f / 32.0f) - mean_h, e3 = p3.x * (1.0f / 32.0f) - mean_h;
+      const float m2_h = (p0.y + p1.y) + (p2.y + p3.y) +
+                         32.0f * ((e0 * e0 + e1 * e1) + (e2 * e2 + e3 * e3));
+      const size_t rowD = static_cast<size_t>(t_row) * D + static_cast<size_t>(h) * 128 + 32 * cq;
+      if (ok && row_ok) {
+        if (a.o_save) {
+          float* od = a.o_save + rowD;
           if (a.vec32) {
-            st_global_v8(yd, reinterpret_cast<const uint32_t(&)[8]>(yw[0]));
-            st_global_v8(yd + 16, reinterpret_cast<const uint32_t(&)[8]>(yw[8]));
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              st_global_v8(od + 8 * v, reinterpret_cast<const uint32_t(&)[8]>(ov[8 * v]));
           } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              reinterpret_cast<uint4*>(yd)[i] =
-                  make_uint4(yw[4 * i], yw[4 * i + 1], yw[4 * i + 2], yw[4 * i + 3]);
+            for (int v = 0; v < 8; ++v)
+              reinterpret_cast<float4*>(od)[v] =
+                  make_float4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
+          }
+        } else {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(ov[2 * i] - mean_h, ov[2 * i + 1] - mean_h);
+          __nv_bfloat16* yd = reinterpret_cast<__nv_bfloat16*>(a.y) + rowD;
+          if (a.vec32) {
+            st_global_v8(yd, reinterpret_cast<const uint32_t(&)[8]>(w[0]));
+            st_global_v8(yd + 16, reinterpret_cast<const uint32_t(&)[8]>(w[8]));
+          } else {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              reinterpret_cast<uint4*>(yd)[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2],
+                                                           w[4 * v + 3]);
           }
         }
-        if (row_ok && h == 0 && cq == 0 && a.ln_mean) {
-          a.ln_mean[t_row] = mean;
-          a.ln_rstd[t_row] = rstd;
-        }
-        // Every thread is done with the buffer (its U read, its Y written).
-        named_bar_sync(3, kEpiThreads);
-        if (et == 0) {
-          if (full) {
-            tma_store_3d(&tm_y, lnbuf, 0, h, s + kRows * m);
-            tma_store_3d(&tm_y, lnbuf + kHalf, 64, h, s + kRows * m);
-            bulk_commit_group();
-            bulk_wait_group_read0();
+        if (cq == 0)
+          a.stats[static_cast<size_t>(t_row) * H + h] =
+              make_float4(mean_h, m2_h, a.o_save ? 0.f : mean_h, 0.f);
+      }
+      // ---- count this head done on the (b, m) block; the last one normalises it.
+      // Release: each thread fences its stash and statistics stores before
+      // the barrier, then one thread counts; acquire: that thread fences
+      // after the count, and every thread again after the barrier, before
+      // reading the other heads' data.
+      __threadfence();
+      named_bar_sync(NB_SYNC, kEpiThreads);      // also: every loc read is done
+      if (et == 0) {
+        __threadfence();
+        const unsigned old = atomicAdd(a.item_cnt + static_cast<size_t>(b) * a.max_tiles + m, 1u);
+        __threadfence();
+        *bcast = old;
+      }
+      named_bar_sync(NB_SYNC, kEpiThreads);
+      if (ok && *bcast == static_cast<unsigned>(H - 1)) {
+        __threadfence();
+        // ---------------------------------- LayerNorm over heads + gate, rows of the block
+        const int nrows = min(kRows, n_b - kRows * m);
+        const bool fp32_stash = a.o_save != nullptr;
+        const float invD = 1.0f / static_cast<float>(D);
+        for (int rr = ew; rr < nrows; rr += kEpiWarps) {
+          const int t = s + kRows * m + rr;
+          float4 st = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (lane < H) st = ld_global_cg_f4(a.stats + static_cast<size_t>(t) * H + lane);
+          float tot = lane < H ? st.x : 0.f;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+          const float mean = tot / static_cast<float>(H);
+          const float dh = st.x - mean;
+          float m2 = lane < H ? st.y + 128.0f * dh * dh : 0.f;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+          const float rstd = 1.0f / sqrtf(m2 * invD + a.eps);
+          // value = stash + shift_h, with shift_h = mean_h - mean (bf16 stash) or -mean
+          const float shift = st.z - mean;
+          const size_t rowt = static_cast<size_t>(t) * D;
+          for (int c0 = 0; c0 < D; c0 += 256) {     // warp-uniform; lanes past D idle
+            const int c = c0 + 8 * lane;
+            const float sh = __shfl_sync(0xffffffffu, shift, (c >> 7) & 7);
+            if (c >= D) continue;
+            float o8[8];
+            if (fp32_stash) {
+              const float4 x0 = ld_global_cg_f4(a.o_save + rowt + c);
+              const float4 x1 = ld_global_cg_f4(a.o_save + rowt + c + 4);
+              o8[0] = x0.x; o8[1] = x0.y; o8[2] = x0.z; o8[3] = x0.w;
+              o8[4] = x1.x; o8[5] = x1.y; o8[6] = x1.z; o8[7] = x1.w;
+            } else {
+              const uint4 w4 =
+                  ld_global_cg_u4(reinterpret_cast<const __nv_bfloat16*>(a.y) + rowt + c);
+              const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[i]));
+                o8[2 * i] = f.x;
+                o8[2 * i + 1] = f.y;
+              }
+            }
+            const uint4 uw = __ldg(reinterpret_cast<const uint4*>(
+                reinterpret_cast<const __nv_bfloat16*>(a.u) + rowt + c));
+            const uint32_t uv[4] = {uw.x, uw.y, uw.z, uw.w};
+            uint32_t yv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 uf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv[i]));
+              yv[i] = pack_bf16x2((o8[2 * i] + sh) * rstd * silu_gate(uf.x),
+                                  (o8[2 * i + 1] + sh) * rstd * silu_gate(uf.y));
+            }
+            *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.y) + rowt + c) =
+                make_uint4(yv[0], yv[1], yv[2], yv[3]);
           }
-          mbar_arrive(bar(B_LNFREE));
+          if (lane == 0 && a.ln_mean) {
+            a.ln_mean[t] = mean;
+            a.ln_rstd[t] = rstd;
+          }
         }
+        if (et == 0) a.item_cnt[static_cast<size_t>(b) * a.max_tiles + m] = 0u;
       }
       g += nt;
       ++j;
@@ -893,84 +929,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       set_status(a.status, kStatusTimeout);
       *abort_flag = 1;
     }
-    if (et == 0) bulk_wait_group0();   // the last Y stores have landed
     tc_fence_before();
   }
 
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpS) {
     tc_fence_after();
     // Every MMA has completed once B_DONE fired; wait for it before freeing TMEM.
     if (lane == 0) mbar_wait(bar(B_DONE), 0, nullptr);
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
   }
-  // No CTA leaves while another may still write into its shared memory.
-  cluster_arrive();
-  cluster_wait();
 }
+
+// Per-device launch state: the shared-memory opt-in is a per-device function
+// attribute and the resident CTA count a per-device property; both are taken
+// once per device (not inside a stream capture of a later call).  Host
+// threads may launch concurrently: the values are atomics, and two threads
+// that both find them unset just compute and store the same values.
+struct DeviceState {
+  std::atomic<int> configured[4];
+  std::atomic<int> resident[4];
+};
+DeviceState g_state[64];
 
 template <bool POS, bool TIME>
 cudaError_t launch_variant(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                           const CUtensorMap& tv, const CUtensorMap& tu, const CUtensorMap& ty,
-                           cudaStream_t stream) {
-  // The shared-memory opt-in is a per-device function attribute, and the
-  // number of co-resident clusters a per-device, per-cluster-size property:
-  // both are taken once per device (not inside a stream capture of a later call).
-  static bool configured[64] = {};
-  static int max_clusters[64][kMaxHeads + 1] = {};
+                           const CUtensorMap& tv, cudaStream_t stream) {
+  constexpr int var = (POS ? 1 : 0) + (TIME ? 2 : 0);
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
+  DeviceState& ds = g_state[dev];
+  if (!ds.configured[var].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(hstu_fwd_bf16_sm100<POS, TIME>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
-    configured[dev] = true;
+    ds.configured[var].store(1, std::memory_order_release);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(a.H);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int& resident = max_clusters[dev][a.H];
+  int resident = ds.resident[var].load(std::memory_order_acquire);
   if (resident == 0) {
-    cfg.gridDim = dim3(static_cast<unsigned>(a.H), 1, 1);
-    int n = 0;
-    err = cudaOccupancyMaxActiveClusters(&n, hstu_fwd_bf16_sm100<POS, TIME>, &cfg);
+    int per_sm = 0, sms = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hstu_fwd_bf16_sm100<POS, TIME>,
+                                                        kThreads, kSmemBytes);
     if (err != cudaSuccess) return err;
-    resident = n > 0 ? n : 1;
+    err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    resident = std::max(1, per_sm) * std::max(1, sms);
+    ds.resident[var].store(resident, std::memory_order_release);
   }
   const long long nslots = static_cast<long long>((a.B + a.group - 1) / a.group) * a.group *
-                           a.max_tiles;
-  const long long clusters = std::min<long long>(resident, nslots);
-  cfg.gridDim = dim3(static_cast<unsigned>(clusters * a.H), 1, 1);
-  return cudaLaunchKernelEx(&cfg, hstu_fwd_bf16_sm100<POS, TIME>, tq, tk, tv, tu, ty, a);
+                           a.max_tiles * a.H;
+  const long long grid = std::min<long long>(resident, nslots);
+  hstu_fwd_bf16_sm100<POS, TIME><<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
+      tq, tk, tv, a);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                                  const CUtensorMap& tv, const CUtensorMap& tu,
-                                  const CUtensorMap& ty, cudaStream_t stream) {
+                                  const CUtensorMap& tv, cudaStream_t stream) {
   if (a.B == 0 || a.max_tiles == 0) return cudaSuccess;
   if (a.H < 1 || a.H > kMaxHeads) return cudaErrorInvalidValue;
-  // Work slots are numbered in 32 bits (plus one claim window of 32).
+  // Work slots are numbered in 32 bits (plus one claim window of 32 and the grid).
   if (a.group < 1 || a.group > a.B) return cudaErrorInvalidValue;
-  if ((static_cast<long long>(a.B) + a.group) * a.max_tiles > 0x7FFFFF00LL)
+  if ((static_cast<long long>(a.B) + a.group) * a.max_tiles * a.H > 0x7FFFFF00LL)
     return cudaErrorInvalidValue;
   const bool pos = a.rab_pos != nullptr, tim = a.rab_time != nullptr;
-  if (pos && tim) return launch_variant<true, true>(a, tq, tk, tv, tu, ty, stream);
-  if (pos) return launch_variant<true, false>(a, tq, tk, tv, tu, ty, stream);
-  if (tim) return launch_variant<false, true>(a, tq, tk, tv, tu, ty, stream);
-  return launch_variant<false, false>(a, tq, tk, tv, tu, ty, stream);
+  if (pos && tim) return launch_variant<true, true>(a, tq, tk, tv, stream);
+  if (pos) return launch_variant<true, false>(a, tq, tk, tv, stream);
+  if (tim) return launch_variant<false, true>(a, tq, tk, tv, stream);
+  return launch_variant<false, false>(a, tq, tk, tv, stream);
 }
 
 }  // namespace hstu

@@ -73,6 +73,13 @@ void fill_bucket_table(BucketTable* bt, int nb) {
     while (k + 1 < nb && bt->thr[k + 1] <= p) ++k;
     bt->first_k[e] = static_cast<signed char>(k);
   }
+  for (int k = 0; k < kMaxBuckets; ++k)
+    bt->thr32[k] = (bt->thr[k] <= 0xFFFFFFFFll) ? static_cast<unsigned>(bt->thr[k]) : 0xFFFFFFFFu;
+  for (int e = 0; e < 32; ++e) {
+    const int k = bt->first_k[e];
+    auto t = [&](int i) { return k + i < kMaxBuckets ? bt->thr32[k + i] : 0xFFFFFFFFu; };
+    bt->oct[e] = make_uint4(static_cast<unsigned>(k), t(1), t(2), t(3));
+  }
 }
 
 // ---------------------------------------------------------- TMA tensor maps
@@ -140,14 +147,13 @@ hstu_status_t check_problem(const hstu_problem_t* p) {
 }
 
 bool bf16_supported(const hstu_problem_t* p) {
-  // The forward numbers its (sequence, query tile) work slots in 32 bits, and
-  // the backward launches one CTA per (head, sequence, tile): both counts
-  // must stay below 2^31.
+  // The forward numbers its (sequence, query tile, head) work slots in 32
+  // bits (with room for one scheduling group more and a claim window), and
+  // the backward launches one CTA per (head, sequence, tile).
   const int64_t tiles = (p->max_seq_len + 127) / 128;
-  const int64_t slots = 2 * static_cast<int64_t>(p->batch) * tiles;
-  const int64_t ctas = static_cast<int64_t>(p->num_heads) * p->batch * tiles;
+  const int64_t slots = 2 * static_cast<int64_t>(p->batch) * tiles * p->num_heads;
   return p->dtype == HSTU_BF16 && p->d_qk == 128 && p->d_v == 128 && p->num_heads <= 8 &&
-         slots <= 0x7FFFFF00LL && ctas <= 0x7FFFFFFFLL;
+         slots <= 0x7FFFFF00LL;
 }
 
 bool f32_supported(const hstu_problem_t* p) {
@@ -155,18 +161,28 @@ bool f32_supported(const hstu_problem_t* p) {
          p->num_heads * p->d_v <= 1024;
 }
 
-// Workspace layout: [status 256 B][dO: T*H*dv in the input dtype] (backward)
+// Workspace layout:
+//   forward (bf16): [status 256 B][per (sequence, query tile) head counters:
+//                    B * ceil(max_seq_len/128) u32][per (token, head) row
+//                    statistics: T * H float4]
+//   backward:       [status 256 B][dO: T*H*dv in the input dtype]
 struct WsLayout {
-  size_t dO_off, total;
+  size_t cnt_off, stats_off, dO_off, total;
 };
 
 WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
   WsLayout l{};
   size_t off = kStatusBytes;
+  const size_t T = static_cast<size_t>(p->total_tokens);
   if (is_bwd) {
-    const size_t T = static_cast<size_t>(p->total_tokens);
     l.dO_off = off;
     off += align_up(T * p->num_heads * p->d_v * (p->dtype == HSTU_BF16 ? 2 : 4));
+  } else if (p->dtype == HSTU_BF16) {
+    const size_t tiles = static_cast<size_t>((p->max_seq_len + 127) / 128);
+    l.cnt_off = off;
+    off += align_up(static_cast<size_t>(p->batch) * tiles * 4);
+    l.stats_off = off;
+    off += align_up(T * p->num_heads * 16);
   }
   l.total = off;
   return l;
@@ -262,17 +278,19 @@ hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* 
   }
   auto al32 = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 31u) == 0; };
   a.vec32 = al32(u) && al32(y) && (!o_save || al32(o_save));
+  const WsLayout l = ws_layout(p, 0);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.item_cnt = reinterpret_cast<unsigned*>(ws + l.cnt_off);
+  a.stats = reinterpret_cast<float4*>(ws + l.stats_off);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (p->dtype == HSTU_BF16) {
-    CUtensorMap tq, tk, tv, tu, ty;   // U and Y [T, H*128] seen as [T, H, 128]
+    CUtensorMap tq, tk, tv;
     if (!make_map_3d(&tq, q, p->total_tokens, p->num_heads, 128) ||
         !make_map_3d(&tk, k, p->total_tokens, p->num_heads, 128) ||
-        !make_map_3d(&tv, v, p->total_tokens, p->num_heads, 128) ||
-        !make_map_3d(&tu, u, p->total_tokens, p->num_heads, 128) ||
-        !make_map_3d(&ty, y, p->total_tokens, p->num_heads, 128))
+        !make_map_3d(&tv, v, p->total_tokens, p->num_heads, 128))
       return HSTU_ERR_CUDA;
-    err = launch_fwd_bf16_sm100(a, tq, tk, tv, tu, ty, s);
+    err = launch_fwd_bf16_sm100(a, tq, tk, tv, s);
   } else {
     err = launch_fwd_f32_simt(a, s);
   }

@@ -13,9 +13,9 @@ constexpr int kStatusBadOffsets = 1;   // offsets contradict T / max_seq_len / L
 constexpr int kStatusTimeout = 2;      // a bounded wait ran out
 
 // The 256-byte head of the workspace: word 0 is the status word; words 16 and
-// 17 are the bf16 forward's work counter and finished-cluster counter.  The
-// forward leaves both counters at zero when it ends (the last cluster to
-// finish resets them), so a zero-filled workspace stays valid across calls.
+// 17 are the bf16 forward's work counter and finished-CTA counter.  The
+// forward leaves both counters (and its per-item head counters) at zero when
+// it ends, so a zero-filled workspace stays valid across calls.
 constexpr int kSchedCounterWord = 16;
 constexpr int kSchedDoneWord = 17;
 
@@ -27,6 +27,12 @@ constexpr int kThrLen = kMaxBuckets + 4;
 struct BucketTable {
   long long thr[kThrLen];
   signed char first_k[64];   // bucket(2^e), e = 0..62
+  // 32-bit form for |dt| < 2^31: thr32[k] = thr[k] (0xFFFFFFFF where thr[k]
+  // >= 2^32 or k >= NB), and per octave e = 0..31 the packed
+  // {bucket(2^e), thr32[k+1], thr32[k+2], thr32[k+3]} (at most three
+  // thresholds lie in one octave, as ln 2 / 0.301 < 3).
+  unsigned thr32[kMaxBuckets];
+  uint4 oct[32];
 };
 
 // Arguments common to the forward kernels (bf16 tcgen05 and fp32 SIMT).
@@ -53,6 +59,11 @@ struct FwdArgs {
   float eps;
   int vec32;         // u, y and o_save (if given) are 32-byte aligned
   int group;         // bf16 forward: sequences per scheduling group (>= 1)
+  // bf16 forward, workspace: per (sequence, query tile) count of heads done
+  // [B * max_tiles], and per (token, head) row statistics of O
+  // {mean, M2, shift, 0} [T * H] for the LayerNorm over heads.
+  unsigned* item_cnt;
+  float4* stats;
   BucketTable bt;
 };
 
@@ -96,8 +107,7 @@ hstu_status_t check_bwd_args(const hstu_problem_t* p, const void* dy, const void
 
 // Kernel launchers (return cudaSuccess or the launch error).
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                                  const CUtensorMap& tv, const CUtensorMap& tu,
-                                  const CUtensorMap& ty, cudaStream_t stream);
+                                  const CUtensorMap& tv, cudaStream_t stream);
 cudaError_t launch_fwd_f32_simt(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_f32_simt(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_bf16_simt(const BwdArgs& a, cudaStream_t stream);

@@ -186,8 +186,10 @@ def test_empty_problem_is_a_no_op(lib):
 
 
 def test_bwd_rejects_grids_beyond_32_bits(lib):
-    """The backward launches one CTA per (head, sequence, 128-row tile); a
-    count of 2^31 or more is refused before anything is enqueued."""
+    """The backward launches one CTA per (head, sequence, 128-row tile) and the
+    forward numbers (sequence, tile, head) slots in 32 bits with room for twice
+    their count: problems past that bound are refused before anything is
+    enqueued."""
     so = lib.load_library()
     vp = ctypes.c_void_p
     args = [vp(FAKE)] * 12
@@ -195,8 +197,13 @@ def test_bwd_rejects_grids_beyond_32_bits(lib):
     p, _ = problem(lib, batch=1 << 20, total_tokens=1 << 20, max_seq_len=256 * 128,
                    num_heads=8)
     assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), 1 << 40, None) == 2
-    # one tile fewer per sequence fits
-    p, _ = problem(lib, batch=1 << 20, total_tokens=1 << 20, max_seq_len=255 * 128,
+    assert call_fwd(lib, p) == 2
+    # 8 x 2^20 x 128 = 2^30 slots: twice that passes the 2^31 - 256 bound no more
+    p, _ = problem(lib, batch=1 << 20, total_tokens=1 << 20, max_seq_len=128 * 128,
+                   num_heads=8)
+    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), 0, None) == 2
+    # 127 tiles per sequence fit: the call gets as far as the workspace check
+    p, _ = problem(lib, batch=1 << 20, total_tokens=1 << 20, max_seq_len=127 * 128,
                    num_heads=8)
     assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), 0, None) == 5
 

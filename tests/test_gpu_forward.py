@@ -159,13 +159,18 @@ def test_degenerate_shapes():
 
 
 def test_work_counters_return_to_zero_and_calls_repeat():
-    """The bf16 forward hands (sequence, query tile) items to its clusters from
-    a counter in the workspace head; the last cluster to finish zeroes it, so
-    back-to-back calls on one workspace (and a workspace first used with many
-    empty slots: long and short sequences mixed) all see every item."""
+    """The bf16 forward hands (sequence, query tile, head) items to its CTAs
+    from a counter in the workspace head, and counts the heads done per
+    (sequence, query tile) block; the last CTA to finish zeroes the first, the
+    CTA that normalises a block zeroes its count.  So back-to-back calls on
+    one workspace (first used with many empty slots: long and short sequences
+    mixed) all see every item, and the counters are zero after every call."""
     inp = hi.make_inputs(spec((1500, 3, 700, 1, 0, 1200), H=4, time=True), seed=31)
     dev = to_dev(inp)
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    p = pa.make_problem(dev["q"], dev["v"], dev["offsets"], inp.max_seq_len, dev["timestamps"],
+                        dev["rab_pos"], dev["rab_time"], inp.norm_len)
+    ws = pa.new_workspace(p, False, "cuda")
+    n_cnt = len(inp.lengths) * ((inp.max_seq_len + 127) // 128)
     ref = oracle.fwd(inp)
     for call in range(3):
         y, _ = pa.hstu_attn_fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["offsets"],
@@ -175,6 +180,7 @@ def test_work_counters_return_to_zero_and_calls_repeat():
         torch.cuda.synchronize()
         words = ws.view(torch.int32).cpu().numpy()
         assert words[16] == 0 and words[17] == 0, words[:20]
+        assert not words[64:64 + n_cnt].any(), words[64:64 + n_cnt]
         assert pa.hstu_attn_check(ws) == 0
         assert_close(np64(y), ref["y"], "bf16", "y (call %d)" % call)
 
@@ -223,7 +229,8 @@ def test_bad_device_offsets_reported():
     by the kernel: the sequence is skipped and the status word says so."""
     inp = hi.make_inputs(spec((300, 100), H=2), seed=7)
     dev = to_dev(inp)
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    p = pa.make_problem(dev["q"], dev["v"], dev["offsets"], 200)
+    ws = pa.new_workspace(p, False, "cuda")
     pa.hstu_attn_fwd(dev["q"], dev["k"], dev["v"], dev["u"], dev["offsets"], 200,
                      rab_pos=None, workspace=ws)
     assert pa.hstu_attn_check(ws) == 1

@@ -63,5 +63,6 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     p.offsets = 0x7F0000000000          # placeholder, rejected before any use
     assert pa.hstu_attn_workspace_size(p, True) > 16 << 20
     fake = ctypes.c_void_p(0x7F0000000000)
-    rc = lib.hstu_attn_bwd_noalloc(ctypes.byref(p), *([fake] * 14), None)
+    # valid arguments (no bias tables, so no bias gradients) except the size
+    rc = lib.hstu_attn_bwd_noalloc(ctypes.byref(p), *([fake] * 12), None, None, None)
     assert rc == 5        # HSTU_ERR_WORKSPACE
