@@ -11,7 +11,7 @@ and the named workloads below.  Every draw comes from one CPU
 ``torch.Generator`` seeded per workload, in a fixed order:
 
     lengths [-> Stochastic Length draws] -> Q -> K -> V -> U -> timestamps
-    -> rab_pos -> rab_time -> dY
+    -> rab_pos -> rab_time -> dY [-> LayerNorm weight -> LayerNorm bias]
 
 Floating values are drawn in fp32 with ``randn`` and rounded (round to nearest
 even) to bf16 for the bf16 workloads; the same rounded host tensors feed the
@@ -57,6 +57,9 @@ class Spec:
     # Stochastic Length: (keep_len, prob).  Each drawn length above keep_len
     # is cut to keep_len with probability prob (see stochastic_length).
     stochastic_length: Optional[tuple] = None
+    # LayerNorm affine over the D = H*d_v features: weight 1 + N(0, 0.1^2) and
+    # bias N(0, 0.1^2), drawn last; False: no tables (unit affine).
+    ln_affine: bool = False
 
 
 def _spec_table() -> Dict[str, Spec]:
@@ -114,6 +117,8 @@ class Inputs:
     dy: Optional[torch.Tensor]          # [T, H*d_v]
     norm_len: int                   # >0: divide by it; 0: by each sequence's length
     rab_pos_len: int                # L (0 if no position table)
+    ln_weight: Optional[torch.Tensor] = None   # fp32 [H*d_v] or None (unit affine)
+    ln_bias: Optional[torch.Tensor] = None     # fp32 [H*d_v] or None
 
     @property
     def lengths(self) -> List[int]:
@@ -228,9 +233,15 @@ def make_inputs(spec: Spec, seed: int = 0) -> Inputs:
         rab_time = torch.randn((H, NUM_TIME_BUCKETS), generator=g,
                                dtype=torch.float32) * spec.rab_std
     dy = draw((T, H * spec.d_v), 1.0) if spec.grad else None
+    ln_weight = ln_bias = None
+    if spec.ln_affine:
+        D = H * spec.d_v
+        ln_weight = 1.0 + 0.1 * torch.randn(D, generator=g, dtype=torch.float32)
+        ln_bias = 0.1 * torch.randn(D, generator=g, dtype=torch.float32)
 
     if spec.norm == "own":
         norm_len = 0
     else:
         norm_len = spec.norm_len if spec.norm_len > 0 else (spec.seq_len or max(lengths or [1]))
-    return Inputs(spec, offsets, q, k, v, u, ts, rab_pos, rab_time, dy, norm_len, L)
+    return Inputs(spec, offsets, q, k, v, u, ts, rab_pos, rab_time, dy, norm_len, L,
+                  ln_weight, ln_bias)

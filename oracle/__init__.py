@@ -59,6 +59,8 @@ class _Problem(ctypes.Structure):
         ("num_time_buckets", ctypes.c_int32),
         ("norm_len", ctypes.c_int32),
         ("ln_eps", ctypes.c_double),
+        ("ln_weight", ctypes.c_void_p),
+        ("ln_bias", ctypes.c_void_p),
     ]
 
 
@@ -72,7 +74,7 @@ def _bind(path: str):
     lib.hstu_ref_fwd.restype = ctypes.c_int
     lib.hstu_ref_fwd_rows.argtypes = [P] + [vp] * 5 + [i64] + [vp] * 4 + [i32]
     lib.hstu_ref_fwd_rows.restype = ctypes.c_int
-    lib.hstu_ref_bwd.argtypes = [P] + [vp] * 11 + [i32]
+    lib.hstu_ref_bwd.argtypes = [P] + [vp] * 13 + [i32]
     lib.hstu_ref_bwd.restype = ctypes.c_int
     return lib
 
@@ -115,7 +117,7 @@ class _Args:
     """Keeps the fp64 copies alive while the C call runs."""
 
     def __init__(self, offsets, q, k, v, u, timestamps=None, rab_pos=None, rab_time=None,
-                 norm_len=0, rab_pos_len=0, ln_eps=LN_EPS):
+                 norm_len=0, rab_pos_len=0, ln_eps=LN_EPS, ln_weight=None, ln_bias=None):
         self.offsets = np.ascontiguousarray(np.asarray(offsets), dtype=np.int32)
         self.q, self.k, self.v, self.u = _f64(q), _f64(k), _f64(v), _f64(u)
         T = int(self.offsets[-1])
@@ -128,6 +130,8 @@ class _Args:
             np.asarray(timestamps), dtype=np.int64)
         self.rab_pos = _f64(rab_pos)
         self.rab_time = _f64(rab_time)
+        self.ln_weight = _f64(ln_weight)
+        self.ln_bias = _f64(ln_bias)
         if self.rab_pos is not None and rab_pos_len <= 0:
             rab_pos_len = (self.rab_pos.shape[-1] + 1) // 2
         self.prob = _Problem(
@@ -136,10 +140,13 @@ class _Args:
             rab_pos_len=int(rab_pos_len), rab_time=_ptr(self.rab_time),
             num_time_buckets=(self.rab_time.shape[-1] if self.rab_time is not None
                               else NUM_TIME_BUCKETS),
-            norm_len=int(norm_len), ln_eps=float(ln_eps))
+            norm_len=int(norm_len), ln_eps=float(ln_eps), ln_weight=_ptr(self.ln_weight),
+            ln_bias=_ptr(self.ln_bias))
 
 
 def _args_from_inputs(inp, **kw):
+    kw.setdefault("ln_weight", getattr(inp, "ln_weight", None))
+    kw.setdefault("ln_bias", getattr(inp, "ln_bias", None))
     return _Args(inp.offsets.numpy(), inp.q, inp.k, inp.v, inp.u,
                  None if inp.timestamps is None else inp.timestamps.numpy(),
                  inp.rab_pos, inp.rab_time, inp.norm_len, inp.rab_pos_len, **kw)
@@ -176,19 +183,23 @@ def fwd_rows_raw(a: _Args, rows: Sequence[int], threads: int = 0):
 
 
 def bwd_raw(a: _Args, dy, threads: int = 0):
-    """Backward: returns dict dq, dk [T,H,dqk], dv [T,H,dv], du [T,D], d_rab_pos, d_rab_time."""
+    """Backward: returns dict dq, dk [T,H,dqk], dv [T,H,dv], du [T,D], d_rab_pos,
+    d_rab_time, and d_ln_weight, d_ln_bias [D] (those of the unit affine when
+    the problem has no LayerNorm tables)."""
     lib = _load()
     dyd = _f64(dy)
     dq = np.zeros((a.T, a.H, a.dqk)); dk = np.zeros((a.T, a.H, a.dqk))
     dv = np.zeros((a.T, a.H, a.dv)); du = np.zeros((a.T, a.D))
     drp = None if a.rab_pos is None else np.zeros_like(a.rab_pos)
     drt = None if a.rab_time is None else np.zeros_like(a.rab_time)
+    dlw = np.zeros(a.D); dlb = np.zeros(a.D)
     rc = lib.hstu_ref_bwd(ctypes.byref(a.prob), _ptr(a.q), _ptr(a.k), _ptr(a.v), _ptr(a.u),
                           _ptr(dyd), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(du), _ptr(drp),
-                          _ptr(drt), int(threads))
+                          _ptr(drt), _ptr(dlw), _ptr(dlb), int(threads))
     if rc != 0:
         raise ValueError("hstu_ref_bwd rejected the problem (code %d)" % rc)
-    return dict(dq=dq, dk=dk, dv=dv, du=du, d_rab_pos=drp, d_rab_time=drt)
+    return dict(dq=dq, dk=dk, dv=dv, du=du, d_rab_pos=drp, d_rab_time=drt, d_ln_weight=dlw,
+                d_ln_bias=dlb)
 
 
 def fwd(inp, threads: int = 0):

@@ -13,7 +13,7 @@
  *     S_ij = q_i . k_j + rab_pos[h][(i-j)+L-1] + rab_time[h][bucket(t_i - t_j)]
  *     A_ij = SiLU(S_ij) / N_b,           SiLU(x) = x / (1 + exp(-x))
  *     O_i  = sum_{j<=i} A_ij v_j         (heads concatenated to width D = H*dv)
- *     Y_i  = LayerNorm_D(O_i) * SiLU(U_i)
+ *     Y_i  = (gamma * LayerNorm_D(O_i) + beta) * SiLU(U_i)
  *
  * Sources:
  *  - score without 1/sqrt(d), SiLU instead of softmax, divide by the length,
@@ -30,15 +30,18 @@
  *  - post-pooling normalisation followed by the U gate: the reproduction
  *    note's flowchart; the gate `o * F.silu(u)`: the model card's
  *    HSTUBlock.forward.
- *  - LayerNorm with biased variance, eps 1e-5, unit affine (nn.LayerNorm's
- *    defaults, as the model card's block uses nn.LayerNorm); the time bucket
+ *  - LayerNorm with biased variance, eps 1e-5 and an elementwise affine
+ *    gamma, beta over the D features (the model card's block norms with
+ *    nn.LayerNorm, whose weight and bias start at ones and zeros: NULL
+ *    tables mean exactly that unit affine); the time bucket
  *    min(NB-1, floor(ln(max(1,|dt|))/0.301)); the position index (i-j)+L-1
  *    into a [H, 2L-1] table; normalisation by a fixed N or by each sequence's
  *    own length: readings taken where the pages print no formula (their
  *    equation sections lost the equations in extraction).
  *
  * The backward is the chain rule of the same definition, in fp64:
- *   g = SiLU(U), dU = dY * xhat * SiLU'(U), dxhat = dY * g,
+ *   g = SiLU(U), dU = dY * (gamma xhat + beta) * SiLU'(U),
+ *   dxhat = dY * g * gamma, d_gamma = sum_t dY * g * xhat, d_beta = sum_t dY * g,
  *   dO = rstd * (dxhat - mean_D(dxhat) - xhat * mean_D(dxhat * xhat)),
  *   dV_j = sum_{i>=j} A_ij dO_i,  dA_ij = dO_i . v_j,
  *   dS_ij = dA_ij * SiLU'(S_ij) / N_b,  dQ_i = sum_j dS_ij k_j,
@@ -155,7 +158,11 @@ static void fwd_row(const hstu_ref_problem *p, const double *q, const double *k,
     var /= (double)D;
     double rstd = 1.0 / sqrt(var + p->ln_eps);
     const double *ur = u + t * D;
-    for (int c = 0; c < D; ++c) y_row[c] = (o_row[c] - mu) * rstd * ref_silu(ur[c]);
+    for (int c = 0; c < D; ++c) {
+        double w = p->ln_weight ? p->ln_weight[c] : 1.0;
+        double bb = p->ln_bias ? p->ln_bias[c] : 0.0;
+        y_row[c] = ((o_row[c] - mu) * rstd * w + bb) * ref_silu(ur[c]);
+    }
     *mean_out = mu;
     *rstd_out = rstd;
 }
@@ -227,7 +234,8 @@ int hstu_ref_fwd(const hstu_ref_problem *p, const double *q, const double *k,
 int hstu_ref_bwd(const hstu_ref_problem *p, const double *q, const double *k,
                  const double *v, const double *u, const double *dy,
                  double *dq, double *dk, double *dv, double *du,
-                 double *d_rab_pos, double *d_rab_time, int num_threads) {
+                 double *d_rab_pos, double *d_rab_time, double *d_ln_weight,
+                 double *d_ln_bias, int num_threads) {
     int rc = validate(p);
     if (rc) return rc;
     if (!dy || !dq || !dk || !dv || !du) return -8;
@@ -255,19 +263,38 @@ int hstu_ref_bwd(const hstu_ref_problem *p, const double *q, const double *k,
         double *dur = du + t * D, *dOr = dO + t * D;
         double m1 = 0.0, m2 = 0.0;   /* mean(dxhat), mean(dxhat * xhat) */
         for (int c = 0; c < D; ++c) {
+            double w = p->ln_weight ? p->ln_weight[c] : 1.0;
+            double bb = p->ln_bias ? p->ln_bias[c] : 0.0;
             double xhat = (orow[c] - mean[t]) * rstd[t];
             double g = ref_silu(ur[c]);
-            dur[c] = dyr[c] * xhat * ref_silu_grad(ur[c]);
-            double dxh = dyr[c] * g;
+            dur[c] = dyr[c] * (w * xhat + bb) * ref_silu_grad(ur[c]);
+            double dxh = dyr[c] * g * w;
             m1 += dxh;
             m2 += dxh * xhat;
         }
         m1 /= (double)D;
         m2 /= (double)D;
         for (int c = 0; c < D; ++c) {
+            double w = p->ln_weight ? p->ln_weight[c] : 1.0;
             double xhat = (orow[c] - mean[t]) * rstd[t];
-            double dxh = dyr[c] * ref_silu(ur[c]);
+            double dxh = dyr[c] * ref_silu(ur[c]) * w;
             dOr[c] = rstd[t] * (dxh - m1 - xhat * m2);
+        }
+    }
+    /* LayerNorm affine gradients: sums over every token, in token order. */
+    if (d_ln_weight || d_ln_bias) {
+        for (int c = 0; c < D; ++c) {
+            if (d_ln_weight) d_ln_weight[c] = 0.0;
+            if (d_ln_bias) d_ln_bias[c] = 0.0;
+        }
+        for (int64_t t = 0; t < T; ++t) {
+            const double *orow = o + t * D, *dyr = dy + t * D, *ur = u + t * D;
+            for (int c = 0; c < D; ++c) {
+                double xhat = (orow[c] - mean[t]) * rstd[t];
+                double dyg = dyr[c] * ref_silu(ur[c]);
+                if (d_ln_weight) d_ln_weight[c] += dyg * xhat;
+                if (d_ln_bias) d_ln_bias[c] += dyg;
+            }
         }
     }
 

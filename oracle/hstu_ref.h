@@ -28,6 +28,8 @@ typedef struct {
     int32_t num_time_buckets;   /* 128 in the workloads                            */
     int32_t norm_len;           /* >0: divide by it; 0: divide by each n_b         */
     double ln_eps;              /* LayerNorm epsilon (1e-5)                        */
+    const double *ln_weight;    /* [H*dv] LayerNorm scale, or NULL (all ones)      */
+    const double *ln_bias;      /* [H*dv] LayerNorm shift, or NULL (all zeros)     */
 } hstu_ref_problem;
 
 /* Time bucket of a timestamp difference: min(NB-1, floor(ln(max(1,|dt|))/0.301)). */
@@ -48,12 +50,14 @@ int hstu_ref_fwd_rows(const hstu_ref_problem *p, const double *q, const double *
                       double *rstd, int num_threads);
 
 /* Backward from dy [T,H*dv].  Writes dq, dk [T,H,dqk], dv [T,H,dv],
- * du [T,H*dv]; d_rab_pos [H,2L-1] and d_rab_time [H,NB] are overwritten
- * (not accumulated) when non-NULL.  The forward is recomputed internally. */
+ * du [T,H*dv]; d_rab_pos [H,2L-1], d_rab_time [H,NB], d_ln_weight and
+ * d_ln_bias [H*dv] are overwritten (not accumulated) when non-NULL.  The
+ * forward is recomputed internally. */
 int hstu_ref_bwd(const hstu_ref_problem *p, const double *q, const double *k,
                  const double *v, const double *u, const double *dy,
                  double *dq, double *dk, double *dv, double *du,
-                 double *d_rab_pos, double *d_rab_time, int num_threads);
+                 double *d_rab_pos, double *d_rab_time, double *d_ln_weight,
+                 double *d_ln_bias, int num_threads);
 
 #ifdef __cplusplus
 }

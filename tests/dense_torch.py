@@ -2,8 +2,8 @@
 
 It follows the model card's HSTUBlock.forward ("HSTU (Generative Recommender)",
 Exported PyTorch): per head, ``tril(silu(q @ k^T + bias) / N) @ v`` as whole
-matrices, then ``F.layer_norm`` over the concatenated heads and the
-``* F.silu(u)`` gate.  It is built from library primitives (matmul, tril,
+matrices, then ``F.layer_norm`` over the concatenated heads (with its weight
+and bias when given) and the ``* F.silu(u)`` gate.  It is built from library primitives (matmul, tril,
 layer_norm, autograd) rather than the oracle's scalar loops, so agreement
 between the two checks each against the other.
 """
@@ -26,7 +26,7 @@ def bucket_matrix(ts_seq: torch.Tensor, num_buckets: int) -> torch.Tensor:
 
 
 def dense_forward(offsets, q, k, v, u, ts=None, rab_pos=None, rab_time=None,
-                  norm_len=0, eps=1e-5, return_o=False):
+                  norm_len=0, eps=1e-5, return_o=False, ln_weight=None, ln_bias=None):
     """All inputs fp64 torch tensors (may require grad). Returns Y [T, D] (and O)."""
     T, H, dqk = q.shape
     dv = v.shape[-1]
@@ -54,5 +54,5 @@ def dense_forward(offsets, q, k, v, u, ts=None, rab_pos=None, rab_time=None,
         A = torch.tril(F.silu(S) / Nn)
         outs.append((A @ vb).transpose(0, 1).reshape(n, H * dv))
     O = torch.cat(outs, 0) if outs else torch.zeros(0, H * dv, dtype=q.dtype)
-    Y = F.layer_norm(O, (H * dv,), eps=eps) * F.silu(u)
+    Y = F.layer_norm(O, (H * dv,), weight=ln_weight, bias=ln_bias, eps=eps) * F.silu(u)
     return (Y, O) if return_o else Y

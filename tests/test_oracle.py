@@ -26,12 +26,12 @@ from tests.dense_torch import dense_forward
 
 def small_inputs(lengths=(5, 9, 1, 12), H=3, dqk=6, dv=4, rab_pos=True, rab_time=True,
                  norm="own", norm_len=0, seed=0, qk_std=0.7, rab_std=0.5, grad=True,
-                 ts_sorted=True, L=None):
+                 ts_sorted=True, L=None, ln_affine=False):
     spec = hi.Spec("t", "f32", batch=len(lengths), heads=H, d_qk=dqk, d_v=dv,
                    lengths=tuple(lengths), qk_std=qk_std, vu_std=1.0,
                    rab_pos_len=(L or max(lengths)) if rab_pos else 0, rab_time=rab_time,
                    rab_std=rab_std, norm=norm, norm_len=norm_len, grad=grad,
-                   ts_sorted=ts_sorted)
+                   ts_sorted=ts_sorted, ln_affine=ln_affine)
     inp = hi.make_inputs(spec, seed=seed)
     if rab_time:
         # Spread the timestamps so that many buckets are reached in small cases.
@@ -52,7 +52,7 @@ def torch_args(inp, requires_grad=False):
     d = lambda x: None if x is None else x.to(torch.float64).clone().requires_grad_(requires_grad)
     return dict(offsets=inp.offsets.tolist(), q=d(inp.q), k=d(inp.k), v=d(inp.v), u=d(inp.u),
                 ts=inp.timestamps, rab_pos=d(inp.rab_pos), rab_time=d(inp.rab_time),
-                norm_len=inp.norm_len)
+                norm_len=inp.norm_len, ln_weight=d(inp.ln_weight), ln_bias=d(inp.ln_bias))
 
 
 def rel_err(a, b):
@@ -70,6 +70,7 @@ def rel_err(a, b):
     dict(lengths=(0, 7, 0, 3), H=2),
     dict(lengths=(16,), H=1, dqk=3, dv=5, qk_std=2.0, rab_std=2.0),
     dict(L=20),
+    dict(ln_affine=True),
 ])
 def test_forward_matches_dense_torch(oracle_lib, case):
     inp = small_inputs(**case)
@@ -85,6 +86,7 @@ def test_forward_matches_dense_torch(oracle_lib, case):
     dict(ts_sorted=False),
     dict(lengths=(0, 7, 0, 3), H=2),
     dict(rab_pos=False, rab_time=False, lengths=(13,), H=2, qk_std=1.5),
+    dict(ln_affine=True),
 ])
 def test_backward_matches_autograd(oracle_lib, case):
     inp = small_inputs(**case)
@@ -100,19 +102,24 @@ def test_backward_matches_autograd(oracle_lib, case):
         assert rel_err(got["d_rab_pos"], ta["rab_pos"].grad.numpy()) < 1e-10
     if inp.rab_time is not None:
         assert rel_err(got["d_rab_time"], ta["rab_time"].grad.numpy()) < 1e-10
+    if inp.ln_weight is not None:
+        assert rel_err(got["d_ln_weight"], ta["ln_weight"].grad.numpy()) < 1e-10
+        assert rel_err(got["d_ln_bias"], ta["ln_bias"].grad.numpy()) < 1e-10
 
 
 def test_backward_finite_differences(oracle_lib):
     """<grad, R> from the oracle's backward equals the central difference of
-    sum(Y * dY) along a random direction R, for every differentiable input."""
-    inp = small_inputs(lengths=(6, 4), H=2, dqk=3, dv=3)
+    sum(Y * dY) along a random direction R, for every differentiable input
+    (the LayerNorm weight and bias included)."""
+    inp = small_inputs(lengths=(6, 4), H=2, dqk=3, dv=3, ln_affine=True)
     a = oracle_lib._args_from_inputs(inp)
     dy = inp.dy.to(torch.float64).numpy()
     grads = oracle_lib.bwd_raw(a, dy)
     rng = np.random.default_rng(1)
     h = 1e-6
     fields = [("q", "dq"), ("k", "dk"), ("v", "dv"), ("u", "du"),
-              ("rab_pos", "d_rab_pos"), ("rab_time", "d_rab_time")]
+              ("rab_pos", "d_rab_pos"), ("rab_time", "d_rab_time"),
+              ("ln_weight", "d_ln_weight"), ("ln_bias", "d_ln_bias")]
     for name, gname in fields:
         base = getattr(a, name).copy()
         R = rng.standard_normal(base.shape)
@@ -330,3 +337,25 @@ def test_golden_regression(oracle_lib):
                                atol=1e-14)
     for dt, kb in fx["buckets"]:
         assert oracle_lib.time_bucket(dt) == kb
+
+
+def test_layernorm_affine_closed_forms(oracle_lib):
+    """With the LayerNorm weight at zero every output is bias * SiLU(U),
+    whatever the attention computes; a constant weight c (no bias) scales the
+    unit-affine output by c; and the bias gradient is sum_t dY * SiLU(U),
+    which involves neither the attention nor the normalisation."""
+    inp = small_inputs(lengths=(7, 3), H=2, dqk=4, dv=3, ln_affine=True)
+    D = inp.u.shape[1]
+    u = inp.u.to(torch.float64).numpy()
+    silu_u = u / (1.0 + np.exp(-u))
+    beta = inp.ln_bias.to(torch.float64).numpy()
+    a = oracle_lib._args_from_inputs(inp, ln_weight=np.zeros(D))
+    y0 = oracle_lib.fwd_raw(a)["y"]
+    assert np.abs(y0 - beta[None, :] * silu_u).max() <= 1e-14 * max(1.0, np.abs(y0).max())
+    unit = oracle_lib.fwd_raw(oracle_lib._args_from_inputs(inp, ln_weight=None, ln_bias=None))
+    scaled = oracle_lib.fwd_raw(oracle_lib._args_from_inputs(inp, ln_weight=np.full(D, 2.5),
+                                                             ln_bias=None))
+    assert rel_err(scaled["y"], 2.5 * unit["y"]) < 1e-14
+    g = oracle_lib.bwd(inp)
+    dy = inp.dy.to(torch.float64).numpy()
+    assert rel_err(g["d_ln_bias"], (dy * silu_u).sum(0)) < 1e-12

@@ -49,11 +49,14 @@ MUTANTS = [
      "double rstd = 1.0 / sqrt(var + p->ln_eps);",
      "double rstd = 1.0 / (sqrt(var) + p->ln_eps);", 0),
     ("mean not subtracted",
-     "y_row[c] = (o_row[c] - mu) * rstd * ref_silu(ur[c]);",
-     "y_row[c] = o_row[c] * rstd * ref_silu(ur[c]);", 0),
+     "y_row[c] = ((o_row[c] - mu) * rstd * w + bb) * ref_silu(ur[c]);",
+     "y_row[c] = (o_row[c] * rstd * w + bb) * ref_silu(ur[c]);", 0),
     ("gate without SiLU",
-     "y_row[c] = (o_row[c] - mu) * rstd * ref_silu(ur[c]);",
-     "y_row[c] = (o_row[c] - mu) * rstd * ur[c];", 0),
+     "y_row[c] = ((o_row[c] - mu) * rstd * w + bb) * ref_silu(ur[c]);",
+     "y_row[c] = ((o_row[c] - mu) * rstd * w + bb) * ur[c];", 0),
+    ("LayerNorm bias scaled by the weight",
+     "y_row[c] = ((o_row[c] - mu) * rstd * w + bb) * ref_silu(ur[c]);",
+     "y_row[c] = ((o_row[c] - mu) * rstd + bb) * w * ref_silu(ur[c]);", 0),
     ("decimal log in the bucket",
      "double b = floor(log(a) / 0.301);", "double b = floor(log10(a) / 0.301);", 0),
     ("query and key swapped",
@@ -66,8 +69,15 @@ MUTANTS = [
     ("mean of dxhat dropped",
      "dOr[c] = rstd[t] * (dxh - m1 - xhat * m2);", "dOr[c] = rstd[t] * (dxh - xhat * m2);", 0),
     ("dU without xhat",
-     "dur[c] = dyr[c] * xhat * ref_silu_grad(ur[c]);",
-     "dur[c] = dyr[c] * ref_silu_grad(ur[c]);", 0),
+     "dur[c] = dyr[c] * (w * xhat + bb) * ref_silu_grad(ur[c]);",
+     "dur[c] = dyr[c] * (w + bb) * ref_silu_grad(ur[c]);", 0),
+    ("dxhat without the LayerNorm weight",
+     "double dxh = dyr[c] * g * w;", "double dxh = dyr[c] * g;", 0),
+    ("LayerNorm bias gradient times xhat",
+     "if (d_ln_bias) d_ln_bias[c] += dyg;", "if (d_ln_bias) d_ln_bias[c] += dyg * xhat;", 0),
+    ("LayerNorm weight gradient without xhat",
+     "if (d_ln_weight) d_ln_weight[c] += dyg * xhat;", "if (d_ln_weight) d_ln_weight[c] += dyg;",
+     0),
     ("dS without 1/N",
      "double dS = dA * ref_silu_grad(S) / Nn;", "double dS = dA * ref_silu_grad(S);", 0),
     ("dV from dS instead of A",
@@ -92,11 +102,13 @@ CONSISTENT_MUTANTS = [
        " + ref_bias(p, h, s, i, j);")]),
     ("sigmoid as the SiLU", [("return x / (1.0 + exp(-x));", "return 1.0 / (1.0 + exp(-x));")]),
     ("gate without SiLU",
-     [("y_row[c] = (o_row[c] - mu) * rstd * ref_silu(ur[c]);",
-       "y_row[c] = (o_row[c] - mu) * rstd * ur[c];"),
+     [("y_row[c] = ((o_row[c] - mu) * rstd * w + bb) * ref_silu(ur[c]);",
+       "y_row[c] = ((o_row[c] - mu) * rstd * w + bb) * ur[c];"),
       ("double g = ref_silu(ur[c]);", "double g = ur[c];"),
-      ("dur[c] = dyr[c] * xhat * ref_silu_grad(ur[c]);", "dur[c] = dyr[c] * xhat;"),
-      ("double dxh = dyr[c] * ref_silu(ur[c]);", "double dxh = dyr[c] * ur[c];")]),
+      ("dur[c] = dyr[c] * (w * xhat + bb) * ref_silu_grad(ur[c]);",
+       "dur[c] = dyr[c] * (w * xhat + bb);"),
+      ("double dxh = dyr[c] * ref_silu(ur[c]) * w;", "double dxh = dyr[c] * ur[c] * w;"),
+      ("double dyg = dyr[c] * ref_silu(ur[c]);", "double dyg = dyr[c] * ur[c];")]),
     ("position index sign",
      [("+ (i - j) + L - 1];", "+ (j - i) + L - 1];"),
       ("if (pp) pp[(i - j) + L - 1] += dS;", "if (pp) pp[(j - i) + L - 1] += dS;")]),
@@ -117,6 +129,7 @@ PINS = [
     T.test_layernorm_rows,
     T.test_time_bucket_thresholds,
     T.test_backward_finite_differences,
+    T.test_layernorm_affine_closed_forms,
 ]
 
 
