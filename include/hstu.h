@@ -13,13 +13,14 @@
  *     S_ij = q_i . k_j + rab_pos[h][(i-j)+L-1] + rab_time[h][bucket(t_i - t_j)]
  *     A_ij = SiLU(S_ij) / N_b        (no softmax; N_b = norm_len or n_b)
  *     O_i  = sum_{j<=i} A_ij v_j     (heads concatenated: width D = H*d_v)
- *     Y_i  = LayerNorm_D(O_i) (unit affine, biased variance, eps) * SiLU(U_i)
+ *     Y_i  = (gamma * LayerNorm_D(O_i) + beta) * SiLU(U_i)   (biased variance, eps)
  *   bucket(dt) = min(NB-1, floor(ln(max(1,|dt|)) / 0.301)).
  *
  * Layouts (row-major, token-major, packed over the B sequences):
  *   q, k  [T, H, d_qk]    v [T, H, d_v]    u, y, dy [T, H*d_v]
  *   offsets int32 [B+1] (offsets[0] = 0, non-decreasing, offsets[B] = T)
- *   timestamps int64 [T]; rab_pos fp32 [H, 2L-1]; rab_time fp32 [H, NB]
+ *   timestamps int64 [T]; rab_pos fp32 [H, 2L-1]; rab_time fp32 [H, NB];
+ *   ln_weight, ln_bias fp32 [H*d_v] (gamma, beta; NULL = ones, zeros)
  *
  * Ownership: the caller owns every buffer.  Device pointers must point to
  * memory of the current CUDA device; the library allocates nothing, and all
@@ -77,6 +78,8 @@ typedef struct {
   int32_t num_time_buckets;   /* NB in [1, 128] when rab_time is given            */
   int32_t norm_len;           /* > 0: divide by it; 0: divide by each n_b         */
   float ln_eps;               /* LayerNorm epsilon, > 0 (1e-5)                    */
+  const float *ln_weight;     /* device [H*d_v] LayerNorm weight, or NULL (ones)  */
+  const float *ln_bias;       /* device [H*d_v] LayerNorm bias, or NULL (zeros)   */
 } hstu_problem_t;
 
 /*
@@ -107,16 +110,18 @@ HSTU_API hstu_status_t hstu_attn_fwd(const hstu_problem_t *p, const void *q, con
  * Backward of hstu_attn_fwd.  dy [T, H*d_v] (dtype) is the upstream gradient;
  * o_save, ln_mean, ln_rstd are the forward's saved fp32 outputs (required).
  * Writes dq, dk [T,H,d_qk], dv [T,H,d_v], du [T,H*d_v] (dtype); d_rab_pos
- * [H,2L-1] and d_rab_time [H,NB] (fp32) are overwritten, not accumulated,
- * when non-NULL (entries with i-j < 0 are zero).  Supported shapes are those
- * of hstu_attn_fwd.
+ * [H,2L-1], d_rab_time [H,NB], d_ln_weight and d_ln_bias [H*d_v] (fp32) are
+ * overwritten, not accumulated, when non-NULL (entries with i-j < 0 are
+ * zero); each needs its table in the problem.  The bias and LayerNorm
+ * gradients are sums over all tokens taken with fp32 atomics, so their last
+ * bits may differ between runs.  Supported shapes are those of hstu_attn_fwd.
  */
 HSTU_API hstu_status_t hstu_attn_bwd(const hstu_problem_t *p, const void *dy, const void *q,
                             const void *k, const void *v, const void *u,
                             const float *o_save, const float *ln_mean, const float *ln_rstd,
                             void *dq, void *dk, void *dv, void *du, float *d_rab_pos,
-                            float *d_rab_time, void *workspace, size_t workspace_bytes,
-                            void *stream);
+                            float *d_rab_time, float *d_ln_weight, float *d_ln_bias,
+                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Waits for `stream`, reads the device status word of `workspace`, resets it
@@ -174,7 +179,8 @@ HSTU_API hstu_status_t hstu_attn_bwd_noalloc(const hstu_problem_t *p, const void
                                              const void *u, const float *o_save,
                                              const float *ln_mean, const float *ln_rstd,
                                              void *dq, void *dk, void *dv, void *du,
-                                             float *d_rab_pos, float *d_rab_time, void *stream);
+                                             float *d_rab_pos, float *d_rab_time,
+                                             float *d_ln_weight, float *d_ln_bias, void *stream);
 
 #ifdef __cplusplus
 }

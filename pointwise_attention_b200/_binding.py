@@ -50,6 +50,8 @@ class hstu_problem_t(ctypes.Structure):
         ("num_time_buckets", ctypes.c_int32),
         ("norm_len", ctypes.c_int32),
         ("ln_eps", ctypes.c_float),
+        ("ln_weight", ctypes.c_void_p),
+        ("ln_bias", ctypes.c_void_p),
     ]
 
 
@@ -71,7 +73,7 @@ def load_library():
     lib.hstu_attn_workspace_size.restype = sz
     lib.hstu_attn_fwd.argtypes = [P] + [vp] * 5 + [vp] * 3 + [vp, sz, vp]
     lib.hstu_attn_fwd.restype = ctypes.c_int
-    lib.hstu_attn_bwd.argtypes = [P] + [vp] * 5 + [vp] * 3 + [vp] * 4 + [vp] * 2 + [vp, sz, vp]
+    lib.hstu_attn_bwd.argtypes = [P] + [vp] * 5 + [vp] * 3 + [vp] * 4 + [vp] * 4 + [vp, sz, vp]
     lib.hstu_attn_bwd.restype = ctypes.c_int
     lib.hstu_attn_check.argtypes = [vp, vp]
     lib.hstu_attn_check.restype = ctypes.c_int
@@ -81,7 +83,7 @@ def load_library():
     lib.hstu_time_bucket_thresholds.restype = ctypes.c_int32
     lib.hstu_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
     lib.hstu_selftest_wait_timeout.restype = ctypes.c_int
-    lib.hstu_attn_bwd_noalloc.argtypes = [P] + [vp] * 5 + [vp] * 3 + [vp] * 4 + [vp] * 2 + [vp]
+    lib.hstu_attn_bwd_noalloc.argtypes = [P] + [vp] * 5 + [vp] * 3 + [vp] * 4 + [vp] * 4 + [vp]
     lib.hstu_attn_bwd_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -114,8 +116,9 @@ def _stream_ptr(stream):
 
 
 def make_problem(q, v, offsets, max_seq_len, timestamps=None, rab_pos=None, rab_time=None,
-                 norm_len=0, eps=1e-5, offsets_host=None):
-    """hstu_problem_t for tensors q [T,H,dqk], v [T,H,dv] and int32 offsets [B+1]."""
+                 norm_len=0, eps=1e-5, offsets_host=None, ln_weight=None, ln_bias=None):
+    """hstu_problem_t for tensors q [T,H,dqk], v [T,H,dv] and int32 offsets [B+1];
+    ln_weight, ln_bias: fp32 [H*dv] LayerNorm affine, or None (ones, zeros)."""
     if q.dtype == torch.bfloat16:
         dt = HSTU_BF16
     elif q.dtype == torch.float32:
@@ -140,6 +143,8 @@ def make_problem(q, v, offsets, max_seq_len, timestamps=None, rab_pos=None, rab_
     p.num_time_buckets = 0 if rab_time is None else rab_time.shape[-1]
     p.norm_len = int(norm_len)
     p.ln_eps = float(eps)
+    p.ln_weight = None if ln_weight is None else ln_weight.data_ptr()
+    p.ln_bias = None if ln_bias is None else ln_bias.data_ptr()
     return p
 
 
@@ -155,8 +160,9 @@ def new_workspace(problem: hstu_problem_t, is_bwd: bool, device) -> torch.Tensor
 
 
 def hstu_attn_fwd(q, k, v, u, offsets, max_seq_len, *, timestamps=None, rab_pos=None,
-                  rab_time=None, norm_len=0, eps=1e-5, save_for_backward=False,
-                  offsets_host=None, y=None, saved=None, workspace=None, stream=None):
+                  rab_time=None, norm_len=0, eps=1e-5, ln_weight=None, ln_bias=None,
+                  save_for_backward=False, offsets_host=None, y=None, saved=None,
+                  workspace=None, stream=None):
     """Forward.  Returns (y, saved) with saved = (o_save, ln_mean, ln_rstd) or None."""
     lib = load_library()
     for name, t in (("q", q), ("k", k), ("v", v), ("u", u)):
@@ -165,10 +171,12 @@ def hstu_attn_fwd(q, k, v, u, offsets, max_seq_len, *, timestamps=None, rab_pos=
     _dev(timestamps, "timestamps", torch.int64)
     _dev(rab_pos, "rab_pos", torch.float32)
     _dev(rab_time, "rab_time", torch.float32)
+    _dev(ln_weight, "ln_weight", torch.float32)
+    _dev(ln_bias, "ln_bias", torch.float32)
     T, H, _ = q.shape
     D = H * v.shape[-1]
     p = make_problem(q, v, offsets, max_seq_len, timestamps, rab_pos, rab_time, norm_len, eps,
-                     offsets_host)
+                     offsets_host, ln_weight, ln_bias)
     if y is None:
         y = torch.empty((T, D), dtype=q.dtype, device=q.device)
     _dev(y, "y", q.dtype)
@@ -190,9 +198,11 @@ def hstu_attn_fwd(q, k, v, u, offsets, max_seq_len, *, timestamps=None, rab_pos=
 
 
 def hstu_attn_bwd(dy, q, k, v, u, offsets, max_seq_len, saved, *, timestamps=None,
-                  rab_pos=None, rab_time=None, norm_len=0, eps=1e-5, offsets_host=None,
-                  need_rab_grads=True, grads=None, workspace=None, stream=None):
-    """Backward.  Returns dict dq, dk, dv, du, d_rab_pos, d_rab_time."""
+                  rab_pos=None, rab_time=None, norm_len=0, eps=1e-5, ln_weight=None,
+                  ln_bias=None, offsets_host=None, need_rab_grads=True, grads=None,
+                  workspace=None, stream=None):
+    """Backward.  Returns dict dq, dk, dv, du, d_rab_pos, d_rab_time, d_ln_weight,
+    d_ln_bias (the table gradients None where the table is absent)."""
     lib = load_library()
     for name, t in (("dy", dy), ("q", q), ("k", k), ("v", v), ("u", u)):
         _dev(t, name, q.dtype)
@@ -200,21 +210,30 @@ def hstu_attn_bwd(dy, q, k, v, u, offsets, max_seq_len, saved, *, timestamps=Non
     o_save, mean, rstd = saved
     for name, t in (("o_save", o_save), ("ln_mean", mean), ("ln_rstd", rstd)):
         _dev(t, name, torch.float32)
+    _dev(ln_weight, "ln_weight", torch.float32)
+    _dev(ln_bias, "ln_bias", torch.float32)
     p = make_problem(q, v, offsets, max_seq_len, timestamps, rab_pos, rab_time, norm_len, eps,
-                     offsets_host)
+                     offsets_host, ln_weight, ln_bias)
     if grads is None:
         grads = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
                      du=torch.empty_like(u),
                      d_rab_pos=(torch.empty_like(rab_pos)
                                 if (rab_pos is not None and need_rab_grads) else None),
                      d_rab_time=(torch.empty_like(rab_time)
-                                 if (rab_time is not None and need_rab_grads) else None))
+                                 if (rab_time is not None and need_rab_grads) else None),
+                     d_ln_weight=(torch.empty_like(ln_weight)
+                                  if (ln_weight is not None and need_rab_grads) else None),
+                     d_ln_bias=(torch.empty_like(ln_bias)
+                                if (ln_bias is not None and need_rab_grads) else None))
+    grads.setdefault("d_ln_weight", None)
+    grads.setdefault("d_ln_bias", None)
     if workspace is None:
         workspace = new_workspace(p, True, q.device)
     rc = lib.hstu_attn_bwd(ctypes.byref(p), _ptr(dy), _ptr(q), _ptr(k), _ptr(v), _ptr(u),
                            _ptr(o_save), _ptr(mean), _ptr(rstd), _ptr(grads["dq"]),
                            _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["du"]),
                            _ptr(grads["d_rab_pos"]), _ptr(grads["d_rab_time"]),
+                           _ptr(grads["d_ln_weight"]), _ptr(grads["d_ln_bias"]),
                            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     if rc != HSTU_OK:
         raise HSTUError(rc, "hstu_attn_bwd")

@@ -905,12 +905,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint4 uw = __ldg(reinterpret_cast<const uint4*>(
                 reinterpret_cast<const __nv_bfloat16*>(a.u) + rowt + c));
             const uint32_t uv[4] = {uw.x, uw.y, uw.z, uw.w};
+            // LayerNorm weight and bias of these 8 columns (ones and zeros without tables)
+            float gw[8], gb[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              gw[i] = 1.f;
+              gb[i] = 0.f;
+            }
+            if (a.ln_weight) {
+              const float4 w0 = __ldg(reinterpret_cast<const float4*>(a.ln_weight + c));
+              const float4 w1 = __ldg(reinterpret_cast<const float4*>(a.ln_weight + c + 4));
+              gw[0] = w0.x; gw[1] = w0.y; gw[2] = w0.z; gw[3] = w0.w;
+              gw[4] = w1.x; gw[5] = w1.y; gw[6] = w1.z; gw[7] = w1.w;
+            }
+            if (a.ln_bias) {
+              const float4 b0 = __ldg(reinterpret_cast<const float4*>(a.ln_bias + c));
+              const float4 b1 = __ldg(reinterpret_cast<const float4*>(a.ln_bias + c + 4));
+              gb[0] = b0.x; gb[1] = b0.y; gb[2] = b0.z; gb[3] = b0.w;
+              gb[4] = b1.x; gb[5] = b1.y; gb[6] = b1.z; gb[7] = b1.w;
+            }
             uint32_t yv[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float2 uf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv[i]));
-              yv[i] = pack_bf16x2((o8[2 * i] + sh) * rstd * silu_gate(uf.x),
-                                  (o8[2 * i + 1] + sh) * rstd * silu_gate(uf.y));
+              yv[i] = pack_bf16x2(
+                  fmaf((o8[2 * i] + sh) * rstd, gw[2 * i], gb[2 * i]) * silu_gate(uf.x),
+                  fmaf((o8[2 * i + 1] + sh) * rstd, gw[2 * i + 1], gb[2 * i + 1]) * silu_gate(uf.y));
             }
             *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.y) + rowt + c) =
                 make_uint4(yv[0], yv[1], yv[2], yv[3]);

@@ -211,6 +211,8 @@ void fill_common(const hstu_problem_t* p, int* status, FwdArgs* a) {
   a->nb = p->rab_time ? p->num_time_buckets : 0;
   a->norm_len = p->norm_len;
   a->eps = p->ln_eps;
+  a->ln_weight = p->ln_weight;
+  a->ln_bias = p->ln_bias;
   fill_bucket_table(&a->bt, p->rab_time ? p->num_time_buckets : 1);
 }
 
@@ -306,7 +308,8 @@ hstu_status_t hstu::check_bwd_args(const hstu_problem_t* p, const void* dy, cons
                                    const float* o_save, const float* ln_mean,
                                    const float* ln_rstd, const void* dq, const void* dk,
                                    const void* dv, const void* du, const float* d_rab_pos,
-                                   const float* d_rab_time) {
+                                   const float* d_rab_time, const float* d_ln_weight,
+                                   const float* d_ln_bias) {
   hstu_status_t st = check_problem(p);
   if (st != HSTU_OK) return st;
   if (p->total_tokens > 0) {
@@ -319,6 +322,8 @@ hstu_status_t hstu::check_bwd_args(const hstu_problem_t* p, const void* dy, cons
   }
   if (d_rab_pos && !p->rab_pos) return HSTU_ERR_INVALID_ARG;
   if (d_rab_time && !p->rab_time) return HSTU_ERR_INVALID_ARG;
+  if (d_ln_weight && !p->ln_weight) return HSTU_ERR_INVALID_ARG;
+  if (d_ln_bias && !p->ln_bias) return HSTU_ERR_INVALID_ARG;
   if (!bf16_supported(p) && !f32_supported(p)) return HSTU_ERR_UNSUPPORTED;
   return HSTU_OK;
 }
@@ -329,10 +334,11 @@ hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void*
                             const void* v, const void* u, const float* o_save,
                             const float* ln_mean, const float* ln_rstd, void* dq, void* dk,
                             void* dv, void* du, float* d_rab_pos, float* d_rab_time,
-                            void* workspace, size_t workspace_bytes, void* stream) {
+                            float* d_ln_weight, float* d_ln_bias, void* workspace,
+                            size_t workspace_bytes, void* stream) {
   NvtxRange range("hstu_attn_bwd");
   hstu_status_t st = check_bwd_args(p, dy, q, k, v, u, o_save, ln_mean, ln_rstd, dq, dk, dv, du,
-                                    d_rab_pos, d_rab_time);
+                                    d_rab_pos, d_rab_time, d_ln_weight, d_ln_bias);
   if (st != HSTU_OK) return st;
   st = check_ws(p, 1, workspace, workspace_bytes);
   if (st != HSTU_OK) return st;
@@ -346,6 +352,9 @@ hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void*
       cudaMemsetAsync(d_rab_time, 0, sizeof(float) * p->num_heads * p->num_time_buckets, s) !=
           cudaSuccess)
     return HSTU_ERR_CUDA;
+  const size_t Dbytes = sizeof(float) * p->num_heads * p->d_v;
+  if (d_ln_weight && cudaMemsetAsync(d_ln_weight, 0, Dbytes, s) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (d_ln_bias && cudaMemsetAsync(d_ln_bias, 0, Dbytes, s) != cudaSuccess) return HSTU_ERR_CUDA;
   if (p->total_tokens == 0 || p->batch == 0) return HSTU_OK;
 
   const WsLayout l = ws_layout(p, 1);
@@ -361,6 +370,8 @@ hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void*
   a.o_save = o_save; a.ln_mean = ln_mean; a.ln_rstd = ln_rstd;
   a.dq = dq; a.dk = dk; a.dv = dv; a.du = du;
   a.d_rab_pos = d_rab_pos; a.d_rab_time = d_rab_time;
+  a.ln_weight = p->ln_weight; a.ln_bias = p->ln_bias;
+  a.d_ln_weight = d_ln_weight; a.d_ln_bias = d_ln_bias;
   a.dO = ws + l.dO_off;
   a.status = common.status;
   a.B = common.B; a.T = common.T; a.H = common.H; a.d_qk = common.d_qk; a.d_v = common.d_v;

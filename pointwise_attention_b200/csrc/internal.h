@@ -57,6 +57,8 @@ struct FwdArgs {
   int nb;            // number of time buckets (0 if no time table)
   int norm_len;
   float eps;
+  const float* ln_weight;   // [H*d_v] or nullptr (ones)
+  const float* ln_bias;     // [H*d_v] or nullptr (zeros)
   int vec32;         // u, y and o_save (if given) are 32-byte aligned
   int group;         // bf16 forward: sequences per scheduling group (>= 1)
   // bf16 forward, workspace: per (sequence, query tile) count of heads done
@@ -86,6 +88,10 @@ struct BwdArgs {
   void* du;
   float* d_rab_pos;
   float* d_rab_time;
+  const float* ln_weight;   // [H*d_v] or nullptr (ones)
+  const float* ln_bias;     // [H*d_v] or nullptr (zeros)
+  float* d_ln_weight;       // [H*d_v] or nullptr; zeroed by the caller of the kernels
+  float* d_ln_bias;
   void* dO;          // workspace: dO in the compute dtype [T, H*d_v]
   int* status;
   int B, T, H, d_qk, d_v;
@@ -103,7 +109,8 @@ hstu_status_t check_bwd_args(const hstu_problem_t* p, const void* dy, const void
                              const void* k, const void* v, const void* u, const float* o_save,
                              const float* ln_mean, const float* ln_rstd, const void* dq,
                              const void* dk, const void* dv, const void* du,
-                             const float* d_rab_pos, const float* d_rab_time);
+                             const float* d_rab_pos, const float* d_rab_time,
+                             const float* d_ln_weight, const float* d_ln_bias);
 
 // Kernel launchers (return cudaSuccess or the launch error).
 cudaError_t launch_fwd_bf16_sm100(const FwdArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,

@@ -49,11 +49,12 @@ hstu_status_t scratch_address(void** out) {
 extern "C" HSTU_API hstu_status_t hstu_attn_bwd_noalloc(
     const hstu_problem_t* p, const void* dy, const void* q, const void* k, const void* v,
     const void* u, const float* o_save, const float* ln_mean, const float* ln_rstd, void* dq,
-    void* dk, void* dv, void* du, float* d_rab_pos, float* d_rab_time, void* stream) {
+    void* dk, void* dv, void* du, float* d_rab_pos, float* d_rab_time, float* d_ln_weight,
+    float* d_ln_bias, void* stream) {
   // The same argument checks as hstu_attn_bwd first, so that a rejected call
   // returns the same status and leaves nothing queued on the stream.
   hstu_status_t st = hstu::check_bwd_args(p, dy, q, k, v, u, o_save, ln_mean, ln_rstd, dq, dk,
-                                          dv, du, d_rab_pos, d_rab_time);
+                                          dv, du, d_rab_pos, d_rab_time, d_ln_weight, d_ln_bias);
   if (st != HSTU_OK) return st;
   const size_t need = hstu_attn_workspace_size(p, 1);
   if (need == 0) return HSTU_ERR_INVALID_ARG;            // the problem itself is invalid
@@ -66,5 +67,5 @@ extern "C" HSTU_API hstu_status_t hstu_attn_bwd_noalloc(
   if (cudaMemsetAsync(scratch, 0, sizeof(int), static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return HSTU_ERR_CUDA;
   return hstu_attn_bwd(p, dy, q, k, v, u, o_save, ln_mean, ln_rstd, dq, dk, dv, du, d_rab_pos,
-                       d_rab_time, scratch, kNoAllocScratchBytes, stream);
+                       d_rab_time, d_ln_weight, d_ln_bias, scratch, kNoAllocScratchBytes, stream);
 }

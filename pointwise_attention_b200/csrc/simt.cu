@@ -12,6 +12,8 @@
 // U gate from the HSTU reproduction note's flowchart).
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "internal.h"
 
 namespace hstu {
@@ -143,7 +145,8 @@ __global__ void __launch_bounds__(kT) fwd_simt(const FwdArgs a) {
   E* y = static_cast<E*>(a.y);
   for (int c = threadIdx.x; c < D; c += kT) {
     const size_t o = static_cast<size_t>(t) * D + c;
-    st(y, o, (o_row[c] - mean) * rstd * silu_f(ld(u, o)));
+    const float w = a.ln_weight ? a.ln_weight[c] : 1.f, bb = a.ln_bias ? a.ln_bias[c] : 0.f;
+    st(y, o, fmaf((o_row[c] - mean) * rstd, w, bb) * silu_f(ld(u, o)));
     if (a.o_save) a.o_save[o] = o_row[c];
   }
   if (threadIdx.x == 0 && a.ln_mean) {
@@ -153,9 +156,11 @@ __global__ void __launch_bounds__(kT) fwd_simt(const FwdArgs a) {
 }
 
 // LayerNorm + gate backward, one block per row: dU (output) and dO (workspace,
-// storage type E):
-//   dU = dY xhat SiLU'(U),  dxhat = dY SiLU(U),
-//   dO = rstd (dxhat - mean(dxhat) - xhat mean(dxhat xhat)).
+// storage type E), with the LayerNorm weight gamma and bias beta (ones and
+// zeros without tables):
+//   dU = dY (gamma xhat + beta) SiLU'(U),  dxhat = dY SiLU(U) gamma,
+//   dO = rstd (dxhat - mean(dxhat) - xhat mean(dxhat xhat)),
+//   d_gamma += dY SiLU(U) xhat,  d_beta += dY SiLU(U)  (fp32 atomics).
 template <typename E>
 __global__ void __launch_bounds__(kT) bwd_pre_simt(const BwdArgs a) {
   __shared__ float red[kT / 32];
@@ -169,10 +174,14 @@ __global__ void __launch_bounds__(kT) bwd_pre_simt(const BwdArgs a) {
   float m1 = 0.f, m2 = 0.f;
   for (int c = threadIdx.x; c < D; c += kT) {
     const size_t o = static_cast<size_t>(t) * D + c;
+    const float w = a.ln_weight ? a.ln_weight[c] : 1.f, bb = a.ln_bias ? a.ln_bias[c] : 0.f;
     const float xhat = (a.o_save[o] - mean) * rstd;
     const float uu = ld(u, o), g = ld(dy, o);
-    const float dxh = g * silu_f(uu);
-    st(du, o, g * xhat * silu_grad_f(uu));
+    const float dyg = g * silu_f(uu);
+    const float dxh = dyg * w;
+    st(du, o, g * fmaf(w, xhat, bb) * silu_grad_f(uu));
+    if (a.d_ln_weight) atomicAdd(a.d_ln_weight + c, dyg * xhat);
+    if (a.d_ln_bias) atomicAdd(a.d_ln_bias + c, dyg);
     m1 += dxh;
     m2 = fmaf(dxh, xhat, m2);
   }
@@ -180,8 +189,9 @@ __global__ void __launch_bounds__(kT) bwd_pre_simt(const BwdArgs a) {
   m2 = block_sum(m2, red) / static_cast<float>(D);
   for (int c = threadIdx.x; c < D; c += kT) {
     const size_t o = static_cast<size_t>(t) * D + c;
+    const float w = a.ln_weight ? a.ln_weight[c] : 1.f;
     const float xhat = (a.o_save[o] - mean) * rstd;
-    const float dxh = ld(dy, o) * silu_f(ld(u, o));
+    const float dxh = ld(dy, o) * silu_f(ld(u, o)) * w;
     st(dO, o, rstd * (dxh - m1 - xhat * m2));
   }
 }
@@ -196,70 +206,117 @@ __global__ void __launch_bounds__(kT) bwd_pre_simt(const BwdArgs a) {
 // reductions and the dO pass.
 constexpr int kRowsPerBlock = 8;
 
-template <int NC>
+// AFFINE: with the LayerNorm weight and bias (either may be absent: ones and
+// zeros), and their gradients when asked for.  The affine form loops over
+// rows (grid-stride) and keeps each lane's d_gamma / d_beta partial sums of
+// its columns in registers, then adds them up per block in shared memory and
+// once per block and column to the outputs (fp32 atomics).
+template <int NC, bool AFFINE>
 __global__ void __launch_bounds__(32 * kRowsPerBlock) bwd_pre_rows_bf16(const BwdArgs a) {
-  const int t = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (t >= a.T) return;
   constexpr int D = NC * 128;
-  const size_t base = static_cast<size_t>(t) * D + 4 * lane;
   const __nv_bfloat16* u = static_cast<const __nv_bfloat16*>(a.u);
   const __nv_bfloat16* dy = static_cast<const __nv_bfloat16*>(a.dy);
   __nv_bfloat16* du = static_cast<__nv_bfloat16*>(a.du);
   __nv_bfloat16* dO = static_cast<__nv_bfloat16*>(a.dO);
-  float4 ov[NC];
-  uint2 uv[NC], gv[NC];
+  float gw[4 * NC], gb[4 * NC], acc_w[4 * NC], acc_b[4 * NC];
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
-    const size_t o = base + 128 * c;
-    ov[c] = __ldcs(reinterpret_cast<const float4*>(a.o_save + o));
-    uv[c] = __ldcs(reinterpret_cast<const uint2*>(u + o));
-    gv[c] = __ldcs(reinterpret_cast<const uint2*>(dy + o));
-  }
-  const float mean = __ldg(a.ln_mean + t), rstd = __ldg(a.ln_rstd + t);
-  float xh[4 * NC], dx[4 * NC];
-  float m1 = 0.f, m2 = 0.f;
-#pragma unroll
-  for (int c = 0; c < NC; ++c) {
-    const float2 u01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv[c].x));
-    const float2 u23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv[c].y));
-    const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv[c].x));
-    const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv[c].y));
-    const float ovs[4] = {ov[c].x, ov[c].y, ov[c].z, ov[c].w};
-    const float us[4] = {u01.x, u01.y, u23.x, u23.y};
-    const float gs[4] = {g01.x, g01.y, g23.x, g23.y};
-    float dus[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float x = (ovs[e] - mean) * rstd;
-      const float d = gs[e] * silu_f(us[e]);
-      dus[e] = gs[e] * x * silu_grad_f(us[e]);
-      xh[4 * c + e] = x;
-      dx[4 * c + e] = d;
-      m1 += d;
-      m2 = fmaf(d, x, m2);
+      const int col = 128 * c + 4 * lane + e;
+      gw[4 * c + e] = (AFFINE && a.ln_weight) ? __ldg(a.ln_weight + col) : 1.f;
+      gb[4 * c + e] = (AFFINE && a.ln_bias) ? __ldg(a.ln_bias + col) : 0.f;
+      acc_w[4 * c + e] = 0.f;
+      acc_b[4 * c + e] = 0.f;
     }
-    __nv_bfloat162 d01 = __floats2bfloat162_rn(dus[0], dus[1]);
-    __nv_bfloat162 d23 = __floats2bfloat162_rn(dus[2], dus[3]);
-    __stcs(reinterpret_cast<uint2*>(du + base + 128 * c),
-           make_uint2(*reinterpret_cast<uint32_t*>(&d01), *reinterpret_cast<uint32_t*>(&d23)));
   }
+  const int stride = AFFINE ? static_cast<int>(gridDim.x) * kRowsPerBlock : 0;
+  for (int t = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5); t < a.T; t += stride) {
+    const size_t base = static_cast<size_t>(t) * D + 4 * lane;
+    float4 ov[NC];
+    uint2 uv[NC], gv[NC];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    m1 += __shfl_xor_sync(0xffffffffu, m1, off);
-    m2 += __shfl_xor_sync(0xffffffffu, m2, off);
+    for (int c = 0; c < NC; ++c) {
+      const size_t o = base + 128 * c;
+      ov[c] = __ldcs(reinterpret_cast<const float4*>(a.o_save + o));
+      uv[c] = __ldcs(reinterpret_cast<const uint2*>(u + o));
+      gv[c] = __ldcs(reinterpret_cast<const uint2*>(dy + o));
+    }
+    const float mean = __ldg(a.ln_mean + t), rstd = __ldg(a.ln_rstd + t);
+    float xh[4 * NC], dx[4 * NC];
+    float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const float2 u01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv[c].x));
+      const float2 u23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uv[c].y));
+      const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv[c].x));
+      const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv[c].y));
+      const float ovs[4] = {ov[c].x, ov[c].y, ov[c].z, ov[c].w};
+      const float us[4] = {u01.x, u01.y, u23.x, u23.y};
+      const float gs[4] = {g01.x, g01.y, g23.x, g23.y};
+      float dus[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = 4 * c + e;
+        const float x = (ovs[e] - mean) * rstd;
+        const float dyg = gs[e] * silu_f(us[e]);
+        const float d = AFFINE ? dyg * gw[k] : dyg;
+        dus[e] = AFFINE ? gs[e] * fmaf(gw[k], x, gb[k]) * silu_grad_f(us[e])
+                        : gs[e] * x * silu_grad_f(us[e]);
+        if (AFFINE) {
+          acc_w[k] = fmaf(dyg, x, acc_w[k]);
+          acc_b[k] += dyg;
+        }
+        xh[k] = x;
+        dx[k] = d;
+        m1 += d;
+        m2 = fmaf(d, x, m2);
+      }
+      __nv_bfloat162 d01 = __floats2bfloat162_rn(dus[0], dus[1]);
+      __nv_bfloat162 d23 = __floats2bfloat162_rn(dus[2], dus[3]);
+      __stcs(reinterpret_cast<uint2*>(du + base + 128 * c),
+             make_uint2(*reinterpret_cast<uint32_t*>(&d01), *reinterpret_cast<uint32_t*>(&d23)));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      m1 += __shfl_xor_sync(0xffffffffu, m1, off);
+      m2 += __shfl_xor_sync(0xffffffffu, m2, off);
+    }
+    m1 /= static_cast<float>(D);
+    m2 /= static_cast<float>(D);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      float r4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) r4[e] = rstd * (dx[4 * c + e] - m1 - xh[4 * c + e] * m2);
+      __nv_bfloat162 d01 = __floats2bfloat162_rn(r4[0], r4[1]);
+      __nv_bfloat162 d23 = __floats2bfloat162_rn(r4[2], r4[3]);
+      *reinterpret_cast<uint2*>(dO + base + 128 * c) =
+          make_uint2(*reinterpret_cast<uint32_t*>(&d01), *reinterpret_cast<uint32_t*>(&d23));
+    }
+    if (!AFFINE) break;
   }
-  m1 /= static_cast<float>(D);
-  m2 /= static_cast<float>(D);
+  if (AFFINE && (a.d_ln_weight || a.d_ln_bias)) {
+    __shared__ float s_w[D], s_b[D];
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+      s_w[i] = 0.f;
+      s_b[i] = 0.f;
+    }
+    __syncthreads();
 #pragma unroll
-  for (int c = 0; c < NC; ++c) {
-    float r4[4];
+    for (int c = 0; c < NC; ++c)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) r4[e] = rstd * (dx[4 * c + e] - m1 - xh[4 * c + e] * m2);
-    __nv_bfloat162 d01 = __floats2bfloat162_rn(r4[0], r4[1]);
-    __nv_bfloat162 d23 = __floats2bfloat162_rn(r4[2], r4[3]);
-    *reinterpret_cast<uint2*>(dO + base + 128 * c) =
-        make_uint2(*reinterpret_cast<uint32_t*>(&d01), *reinterpret_cast<uint32_t*>(&d23));
+      for (int e = 0; e < 4; ++e) {
+        const int col = 128 * c + 4 * lane + e;
+        atomicAdd(&s_w[col], acc_w[4 * c + e]);
+        atomicAdd(&s_b[col], acc_b[4 * c + e]);
+      }
+    __syncthreads();
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+      if (a.d_ln_weight) atomicAdd(a.d_ln_weight + i, s_w[i]);
+      if (a.d_ln_bias) atomicAdd(a.d_ln_bias + i, s_b[i]);
+    }
   }
 }
 
@@ -398,18 +455,36 @@ cudaError_t launch_bwd_bf16_simt(const BwdArgs& a, cudaStream_t stream) {
 cudaError_t launch_bwd_pre_bf16(const BwdArgs& a, cudaStream_t stream) {
   if (a.T == 0) return cudaSuccess;
   if (a.d_v == 128 && a.H >= 1 && a.H <= 8) {
-    const unsigned blocks = static_cast<unsigned>((a.T + kRowsPerBlock - 1) / kRowsPerBlock);
-    const dim3 g(blocks), b(32 * kRowsPerBlock);
-    switch (a.H) {
-      case 1: bwd_pre_rows_bf16<1><<<g, b, 0, stream>>>(a); break;
-      case 2: bwd_pre_rows_bf16<2><<<g, b, 0, stream>>>(a); break;
-      case 3: bwd_pre_rows_bf16<3><<<g, b, 0, stream>>>(a); break;
-      case 4: bwd_pre_rows_bf16<4><<<g, b, 0, stream>>>(a); break;
-      case 5: bwd_pre_rows_bf16<5><<<g, b, 0, stream>>>(a); break;
-      case 6: bwd_pre_rows_bf16<6><<<g, b, 0, stream>>>(a); break;
-      case 7: bwd_pre_rows_bf16<7><<<g, b, 0, stream>>>(a); break;
-      default: bwd_pre_rows_bf16<8><<<g, b, 0, stream>>>(a); break;
+    const bool affine = a.ln_weight || a.ln_bias || a.d_ln_weight || a.d_ln_bias;
+    unsigned blocks = static_cast<unsigned>((a.T + kRowsPerBlock - 1) / kRowsPerBlock);
+    if (affine) {
+      // rows loop per block: a few blocks per SM keep HBM busy, and the
+      // per-block gradient sums stay few
+      int sms = 148, dev = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      blocks = std::min(blocks, static_cast<unsigned>(4 * sms));
     }
+    const dim3 g(blocks), b(32 * kRowsPerBlock);
+#define HSTU_ROWS_CASE(NC)                                                   \
+  case NC:                                                                   \
+    if (affine) bwd_pre_rows_bf16<NC, true><<<g, b, 0, stream>>>(a);        \
+    else bwd_pre_rows_bf16<NC, false><<<g, b, 0, stream>>>(a);              \
+    break;
+    switch (a.H) {
+      HSTU_ROWS_CASE(1)
+      HSTU_ROWS_CASE(2)
+      HSTU_ROWS_CASE(3)
+      HSTU_ROWS_CASE(4)
+      HSTU_ROWS_CASE(5)
+      HSTU_ROWS_CASE(6)
+      HSTU_ROWS_CASE(7)
+      default:
+        if (affine) bwd_pre_rows_bf16<8, true><<<g, b, 0, stream>>>(a);
+        else bwd_pre_rows_bf16<8, false><<<g, b, 0, stream>>>(a);
+        break;
+    }
+#undef HSTU_ROWS_CASE
   } else {
     bwd_pre_simt<__nv_bfloat16><<<a.T, kT, 0, stream>>>(a);
   }

@@ -19,7 +19,7 @@ def to_dev(inp, device="cuda"):
     d = lambda x: None if x is None else x.to(device).contiguous()
     return dict(q=d(inp.q), k=d(inp.k), v=d(inp.v), u=d(inp.u), offsets=d(inp.offsets),
                 timestamps=d(inp.timestamps), rab_pos=d(inp.rab_pos), rab_time=d(inp.rab_time),
-                dy=d(inp.dy))
+                dy=d(inp.dy), ln_weight=d(inp.ln_weight), ln_bias=d(inp.ln_bias))
 
 
 def max_len(inp):
@@ -32,6 +32,7 @@ def run_fwd(inp, save=True, dev=None, workspace=None, check=True):
                                 max_len(inp), timestamps=dev["timestamps"],
                                 rab_pos=dev["rab_pos"], rab_time=dev["rab_time"],
                                 norm_len=inp.norm_len, save_for_backward=save,
+                                ln_weight=dev["ln_weight"], ln_bias=dev["ln_bias"],
                                 offsets_host=inp.offsets, workspace=workspace)
     if check:
         ws = workspace
@@ -45,7 +46,8 @@ def run_bwd(inp, dev, saved):
     g = pa.hstu_attn_bwd(dev["dy"], dev["q"], dev["k"], dev["v"], dev["u"], dev["offsets"],
                          max_len(inp), saved, timestamps=dev["timestamps"],
                          rab_pos=dev["rab_pos"], rab_time=dev["rab_time"],
-                         norm_len=inp.norm_len, offsets_host=inp.offsets)
+                         norm_len=inp.norm_len, ln_weight=dev["ln_weight"],
+                         ln_bias=dev["ln_bias"], offsets_host=inp.offsets)
     torch.cuda.synchronize()
     return g
 

@@ -162,14 +162,16 @@ def test_bwd_workspace_size_and_rejections(lib):
     vp = ctypes.c_void_p
     args = [vp(FAKE)] * 12
     # d_rab_pos requested without a position table
-    rc = so.hstu_attn_bwd(ctypes.byref(p), *args, vp(FAKE), None, vp(FAKE), need, None)
+    rc = so.hstu_attn_bwd(ctypes.byref(p), *args, vp(FAKE), None, None, None, vp(FAKE),
+                          need, None)
     assert rc == 1
     # missing saved statistics
     a2 = list(args)
     a2[6] = None
-    rc = so.hstu_attn_bwd(ctypes.byref(p), *a2, None, None, vp(FAKE), need, None)
+    rc = so.hstu_attn_bwd(ctypes.byref(p), *a2, None, None, None, None, vp(FAKE), need, None)
     assert rc == 1
-    rc = so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), need - 256, None)
+    rc = so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, None, None, vp(FAKE), need - 256,
+                          None)
     assert rc == 5
 
 
@@ -196,16 +198,17 @@ def test_bwd_rejects_grids_beyond_32_bits(lib):
     # 8 heads x 2^20 sequences x 256 tiles = 2^31 CTAs
     p, _ = problem(lib, batch=1 << 20, total_tokens=1 << 20, max_seq_len=256 * 128,
                    num_heads=8)
-    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), 1 << 40, None) == 2
+    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, None, None, vp(FAKE), 1 << 40,
+                            None) == 2
     assert call_fwd(lib, p) == 2
     # 8 x 2^20 x 128 = 2^30 slots: twice that passes the 2^31 - 256 bound no more
     p, _ = problem(lib, batch=1 << 20, total_tokens=1 << 20, max_seq_len=128 * 128,
                    num_heads=8)
-    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), 0, None) == 2
+    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, None, None, vp(FAKE), 0, None) == 2
     # 127 tiles per sequence fit: the call gets as far as the workspace check
     p, _ = problem(lib, batch=1 << 20, total_tokens=1 << 20, max_seq_len=127 * 128,
                    num_heads=8)
-    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), 0, None) == 5
+    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, None, None, vp(FAKE), 0, None) == 5
 
 
 def test_noalloc_rejects_like_bwd_without_enqueueing(lib):
@@ -216,10 +219,23 @@ def test_noalloc_rejects_like_bwd_without_enqueueing(lib):
     args = [vp(FAKE)] * 12
     # unsupported and larger than the built-in scratch: UNSUPPORTED, as hstu_attn_bwd says
     p, _ = problem(lib, d_qk=64, d_v=64, total_tokens=1 << 20, max_seq_len=4096)
-    assert so.hstu_attn_bwd_noalloc(ctypes.byref(p), *args, None, None, None) == 2
+    assert so.hstu_attn_bwd_noalloc(ctypes.byref(p), *args, None, None, None, None, None) == 2
     a2 = list(args)
     a2[8] = None                                    # dq missing
     p, _ = problem(lib)
-    assert so.hstu_attn_bwd_noalloc(ctypes.byref(p), *a2, None, None, None) == 1
+    assert so.hstu_attn_bwd_noalloc(ctypes.byref(p), *a2, None, None, None, None, None) == 1
     p, _ = problem(lib, ln_eps=0.0)
-    assert so.hstu_attn_bwd_noalloc(ctypes.byref(p), *args, None, None, None) == 1
+    assert so.hstu_attn_bwd_noalloc(ctypes.byref(p), *args, None, None, None, None, None) == 1
+
+
+def test_bwd_rejects_layernorm_gradients_without_tables(lib):
+    """d_ln_weight / d_ln_bias need the matching table in the problem."""
+    so = lib.load_library()
+    vp = ctypes.c_void_p
+    args = [vp(FAKE)] * 12
+    p, _ = problem(lib)
+    need = lib.hstu_attn_workspace_size(p, True)
+    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, vp(FAKE), None, vp(FAKE), need,
+                            None) == 1
+    assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, None, vp(FAKE), vp(FAKE), need,
+                            None) == 1

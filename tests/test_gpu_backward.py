@@ -11,11 +11,12 @@ pytestmark = pytest.mark.gpu
 
 
 def spec(lengths, H=4, d=128, dtype="bf16", pos=True, time=False, norm="own", norm_len=0,
-         qk_std=1 / np.sqrt(128), L=None, ts_sorted=True):
+         qk_std=1 / np.sqrt(128), L=None, ts_sorted=True, affine=False):
     return hi.Spec("case", dtype, batch=len(lengths), heads=H, d_qk=d, d_v=d,
                    lengths=tuple(lengths), qk_std=qk_std, vu_std=1.0,
                    rab_pos_len=(L or max(lengths)) if pos else 0, rab_time=time,
-                   norm=norm, norm_len=norm_len, grad=True, ts_sorted=ts_sorted)
+                   norm=norm, norm_len=norm_len, grad=True, ts_sorted=ts_sorted,
+                   ln_affine=affine)
 
 
 def check_bwd(inp, dtype, rows_of=None):
@@ -28,11 +29,15 @@ def check_bwd(inp, dtype, rows_of=None):
         assert_close(np64(g["d_rab_pos"]), ref["d_rab_pos"], dtype, "d_rab_pos")
     if inp.rab_time is not None:
         assert_close(np64(g["d_rab_time"]), ref["d_rab_time"], dtype, "d_rab_time")
+    if inp.ln_weight is not None:
+        assert_close(np64(g["d_ln_weight"]), ref["d_ln_weight"], dtype, "d_ln_weight")
+        assert_close(np64(g["d_ln_bias"]), ref["d_ln_bias"], dtype, "d_ln_bias")
 
 
 @pytest.mark.parametrize("case", [
     dict(lengths=(40, 3), H=2, d=16, dtype="f32", time=True),
     dict(lengths=(130,), H=3, d=64, dtype="f32", norm="fixed", norm_len=200),
+    dict(lengths=(33, 8), H=2, d=32, dtype="f32", time=True, affine=True),
 ])
 def test_fp32_backward(case):
     check_bwd(hi.make_inputs(spec(**case, qk_std=0.5), seed=11), "f32")
@@ -47,6 +52,9 @@ def test_fp32_backward(case):
     # the dQ kernel accumulates d(rab_time) per element
     dict(lengths=(260, 131), H=2, time=True, ts_sorted=False),
     dict(lengths=(200,), H=4, pos=False, time=True, ts_sorted=False),
+    # LayerNorm weight and bias, and their gradients (summed over every token)
+    dict(lengths=(300, 1, 170), H=4, time=True, affine=True),
+    dict(lengths=(257,), H=8, affine=True),
 ])
 def test_bf16_backward_small(case):
     check_bwd(hi.make_inputs(spec(**case), seed=12), "bf16")
@@ -81,3 +89,9 @@ def test_train_sl_reduced_batch():
     inp = hi.make_inputs(hi.workload("train_sl", batch=5), seed=2)
     assert len(set(inp.lengths)) > 1
     check_bwd(inp, "bf16")
+
+
+def test_train_with_layernorm_affine():
+    """Training shapes (2 x 2048 tokens, H=4) with the LayerNorm weight and bias:
+    the affine form of the LayerNorm/gate backward and its table gradients."""
+    check_bwd(hi.make_inputs(hi.workload("train", batch=2, ln_affine=True), seed=4), "bf16")

@@ -17,11 +17,12 @@ pytestmark = pytest.mark.gpu
 
 
 def spec(lengths, H=4, d=128, dtype="bf16", pos=True, time=False, norm="own", norm_len=0,
-         qk_std=1 / np.sqrt(128), rab_std=0.02, L=None, ts_sorted=True):
+         qk_std=1 / np.sqrt(128), rab_std=0.02, L=None, ts_sorted=True, affine=False):
     return hi.Spec("case", dtype, batch=len(lengths), heads=H, d_qk=d, d_v=d,
                    lengths=tuple(lengths), qk_std=qk_std, vu_std=1.0,
                    rab_pos_len=(L or max(max(lengths), 1)) if pos else 0, rab_time=time,
-                   rab_std=rab_std, norm=norm, norm_len=norm_len, ts_sorted=ts_sorted)
+                   rab_std=rab_std, norm=norm, norm_len=norm_len, ts_sorted=ts_sorted,
+                   ln_affine=affine)
 
 
 def check_full(inp, dtype):
@@ -48,8 +49,10 @@ def test_tiny_fp32_workload():
     dict(lengths=(640,), H=3, time=True, L=1000),
     dict(lengths=(260, 131), H=2, time=True, ts_sorted=False),
     dict(lengths=(300, 257), H=4, qk_std=1.0, rab_std=1.0, time=True),   # stress: large logits
-    dict(lengths=(257, 100, 33), H=5, time=True),                          # odd cluster sizes
+    dict(lengths=(257, 100, 33), H=5, time=True),                          # odd head counts
     dict(lengths=(129, 129, 129), H=7),
+    dict(lengths=(300, 70, 129), H=4, time=True, affine=True),             # LayerNorm affine
+    dict(lengths=(200,), H=3, affine=True),
 ])
 def test_bf16_small(case):
     inp = hi.make_inputs(spec(**case), seed=1)
@@ -59,6 +62,7 @@ def test_bf16_small(case):
 @pytest.mark.parametrize("case", [
     dict(lengths=(5, 70, 130), H=2, d=32, dtype="f32", time=True),
     dict(lengths=(64, 1), H=4, d=100, dtype="f32", pos=False, norm="fixed", norm_len=64),
+    dict(lengths=(40, 9), H=2, d=32, dtype="f32", time=True, affine=True),
 ])
 def test_fp32_small(case):
     inp = hi.make_inputs(spec(**case, qk_std=0.5), seed=2)
