@@ -76,6 +76,11 @@ def _bind(path: str):
     lib.hstu_ref_fwd_rows.restype = ctypes.c_int
     lib.hstu_ref_bwd.argtypes = [P] + [vp] * 13 + [i32]
     lib.hstu_ref_bwd.restype = ctypes.c_int
+    lib.hstu_ref_uvqk.argtypes = [i64] + [ctypes.c_int32] * 5 + [vp] * 7
+    lib.hstu_ref_uvqk.restype = ctypes.c_int
+    lib.hstu_ref_out.argtypes = [i64, ctypes.c_int32, ctypes.c_int32] + [vp] * 6 + [
+        ctypes.c_double] + [vp] * 3
+    lib.hstu_ref_out.restype = ctypes.c_int
     return lib
 
 
@@ -214,3 +219,35 @@ def fwd_rows(inp, rows, threads: int = 0):
 def bwd(inp, threads: int = 0):
     """Backward of an ``hstu_inputs.Inputs`` problem (uses ``inp.dy``)."""
     return bwd_raw(_args_from_inputs(inp), inp.dy, threads)
+
+
+def uvqk(x, w, b, H: int, dqk: int, dv: int, act: int = 0):
+    """UVQK projection of x [T, E] by w [H(2dv+2dqk), E] (+ b): dict u, v, q, k
+    ([T, H*dv] twice, [T, H*dqk] twice, fp64)."""
+    lib = _load()
+    xd, wd, bd = _f64(x), _f64(w), _f64(b)
+    T, E = xd.shape
+    Nu, Nq = H * dv, H * dqk
+    out = dict(u=np.zeros((T, Nu)), v=np.zeros((T, Nu)), q=np.zeros((T, Nq)),
+               k=np.zeros((T, Nq)))
+    rc = lib.hstu_ref_uvqk(int(T), int(E), int(H), int(dqk), int(dv), int(act), _ptr(xd),
+                           _ptr(wd), _ptr(bd), _ptr(out["u"]), _ptr(out["v"]), _ptr(out["q"]),
+                           _ptr(out["k"]))
+    if rc != 0:
+        raise ValueError("hstu_ref_uvqk rejected the sizes (code %d)" % rc)
+    return out
+
+
+def out_proj(y, x, w, b=None, gamma=None, beta=None, eps: float = LN_EPS):
+    """Z = LayerNorm_E(x + y w^T + b) (gamma, beta): dict z [T, E], mean, rstd [T]."""
+    lib = _load()
+    yd, xd, wd = _f64(y), _f64(x), _f64(w)
+    bd, gd, btd = _f64(b), _f64(gamma), _f64(beta)
+    T, E = xd.shape
+    Dy = yd.shape[1]
+    z = np.zeros((T, E)); mean = np.zeros(T); rstd = np.zeros(T)
+    rc = lib.hstu_ref_out(int(T), int(E), int(Dy), _ptr(yd), _ptr(xd), _ptr(wd), _ptr(bd),
+                          _ptr(gd), _ptr(btd), float(eps), _ptr(z), _ptr(mean), _ptr(rstd))
+    if rc != 0:
+        raise ValueError("hstu_ref_out rejected the sizes (code %d)" % rc)
+    return dict(z=z, mean=mean, rstd=rstd)

@@ -362,3 +362,69 @@ int hstu_ref_bwd(const hstu_ref_problem *p, const double *q, const double *k,
     free(o); free(mean); free(rstd); free(dO);
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Projections either side of the attention.
+ *
+ * UVQK: the model card's `self.uvqk(x).split([h*dv, h*dv, h*dqk, h*dqk])`
+ * (nn.Linear: x W^T + b), optionally followed by SiLU as in the reproduction
+ * note's key formula SiLU(Norm(X) W_UVQK).  Output: the model card's
+ * `self.norm(x + self.out(...))`, nn.Linear then nn.LayerNorm over E.
+ * Plain loops, fp64, fixed order (c ascending).
+ * ------------------------------------------------------------------------ */
+int hstu_ref_uvqk(int64_t T, int32_t E, int32_t H, int32_t dqk, int32_t dv, int32_t act,
+                  const double *x, const double *w, const double *b,
+                  double *u, double *v, double *q, double *k) {
+    if (T < 0 || E <= 0 || H <= 0 || dqk <= 0 || dv <= 0 || !x || !w) return -1;
+    const int64_t Nu = (int64_t)H * dv, Nq = (int64_t)H * dqk;
+    const int64_t N = 2 * Nu + 2 * Nq;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const double *xr = x + t * E;
+        for (int64_t n = 0; n < N; ++n) {
+            const double *wr = w + n * E;
+            double acc = 0.0;
+            for (int c = 0; c < E; ++c) acc += xr[c] * wr[c];
+            if (b) acc += b[n];
+            if (act) acc = ref_silu(acc);
+            if (n < Nu) u[t * Nu + n] = acc;
+            else if (n < 2 * Nu) v[t * Nu + (n - Nu)] = acc;
+            else if (n < 2 * Nu + Nq) q[t * Nq + (n - 2 * Nu)] = acc;
+            else k[t * Nq + (n - 2 * Nu - Nq)] = acc;
+        }
+    }
+    return 0;
+}
+
+int hstu_ref_out(int64_t T, int32_t E, int32_t Dy, const double *y, const double *x,
+                 const double *w, const double *b, const double *gamma, const double *beta,
+                 double eps, double *z, double *mean, double *rstd) {
+    if (T < 0 || E <= 0 || Dy <= 0 || !y || !x || !w || !z) return -1;
+#pragma omp parallel
+    {
+        double *r = (double *)malloc(sizeof(double) * E);
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            const double *yr = y + t * Dy, *xr = x + t * E;
+            for (int e = 0; e < E; ++e) {
+                const double *wr = w + (int64_t)e * Dy;
+                double acc = 0.0;
+                for (int c = 0; c < Dy; ++c) acc += yr[c] * wr[c];
+                r[e] = xr[e] + acc + (b ? b[e] : 0.0);
+            }
+            double mu = 0.0;
+            for (int e = 0; e < E; ++e) mu += r[e];
+            mu /= (double)E;
+            double var = 0.0;
+            for (int e = 0; e < E; ++e) var += (r[e] - mu) * (r[e] - mu);
+            var /= (double)E;
+            double rs = 1.0 / sqrt(var + eps);
+            for (int e = 0; e < E; ++e)
+                z[t * E + e] = (r[e] - mu) * rs * (gamma ? gamma[e] : 1.0) + (beta ? beta[e] : 0.0);
+            if (mean) mean[t] = mu;
+            if (rstd) rstd[t] = rs;
+        }
+        free(r);
+    }
+    return 0;
+}

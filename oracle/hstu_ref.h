@@ -59,6 +59,25 @@ int hstu_ref_bwd(const hstu_ref_problem *p, const double *q, const double *k,
                  double *d_rab_pos, double *d_rab_time, double *d_ln_weight,
                  double *d_ln_bias, int num_threads);
 
+/* The projections either side of the attention (one HSTU block, "HSTU
+ * (Generative Recommender)" model card, HSTUBlock):
+ *
+ * UVQK: P = X W^T + b over the T rows of X [T, E], W [H(2dv+2dqk), E],
+ * b [H(2dv+2dqk)] or NULL; with act = 1, P = SiLU(P) (the reproduction note's
+ * SiLU(Norm(X) W_UVQK)).  P's columns split, in order, into u [T, H*dv],
+ * v [T, H*dv], q [T, H*dqk], k [T, H*dqk].  Returns 0, or < 0 for bad sizes. */
+int hstu_ref_uvqk(int64_t T, int32_t E, int32_t H, int32_t dqk, int32_t dv, int32_t act,
+                  const double *x, const double *w, const double *b,
+                  double *u, double *v, double *q, double *k);
+
+/* Output: Z = LayerNorm_E(X + Y W_out^T + b_out) with weight gamma and bias
+ * beta (NULL: ones, zeros), biased variance and eps.  Y [T, Dy] (Dy = H*dv),
+ * X [T, E] (the residual), W_out [E, Dy], b_out [E] or NULL.  Writes z [T, E]
+ * and, when non-NULL, the row mean and rstd [T]. */
+int hstu_ref_out(int64_t T, int32_t E, int32_t Dy, const double *y, const double *x,
+                 const double *w, const double *b, const double *gamma, const double *beta,
+                 double eps, double *z, double *mean, double *rstd);
+
 #ifdef __cplusplus
 }
 #endif

@@ -359,3 +359,84 @@ def test_layernorm_affine_closed_forms(oracle_lib):
     g = oracle_lib.bwd(inp)
     dy = inp.dy.to(torch.float64).numpy()
     assert rel_err(g["d_ln_bias"], (dy * silu_u).sum(0)) < 1e-12
+
+
+# ---------------------------------------------------------------- projections
+def _proj_case(T=9, E=16, H=2, dqk=4, dv=3, seed=3):
+    rng = np.random.default_rng(seed)
+    N = H * (2 * dv + 2 * dqk)
+    return dict(x=rng.standard_normal((T, E)), w=rng.standard_normal((N, E)) / 4,
+                b=rng.standard_normal(N), H=H, dqk=dqk, dv=dv)
+
+
+@pytest.mark.parametrize("act", [0, 1])
+def test_uvqk_matches_torch(oracle_lib, act):
+    """The model card's uvqk(x).split([h dv, h dv, h dqk, h dqk]) (nn.Linear:
+    x W^T + b), with the reproduction note's SiLU when act = 1."""
+    c = _proj_case()
+    got = oracle_lib.uvqk(c["x"], c["w"], c["b"], c["H"], c["dqk"], c["dv"], act)
+    P = torch.from_numpy(c["x"]) @ torch.from_numpy(c["w"]).T + torch.from_numpy(c["b"])
+    if act:
+        P = torch.nn.functional.silu(P)
+    Nu, Nq = c["H"] * c["dv"], c["H"] * c["dqk"]
+    parts = torch.split(P, [Nu, Nu, Nq, Nq], dim=-1)
+    for name, ref in zip("uvqk", parts):
+        assert rel_err(got[name], ref.numpy()) < 1e-12, name
+
+
+def test_uvqk_closed_forms(oracle_lib):
+    """Weight rows that are unit vectors copy input columns into the outputs,
+    in the split order u, v, q, k; zero weights leave SiLU(bias) on every row."""
+    c = _proj_case(T=4, E=32, H=2, dqk=4, dv=3)
+    H, dqk, dv = c["H"], c["dqk"], c["dv"]
+    N = H * (2 * dv + 2 * dqk)
+    w = np.zeros((N, 32))
+    for n in range(N):
+        w[n, n] = 1.0
+    got = oracle_lib.uvqk(c["x"], w, None, H, dqk, dv, 0)
+    Nu, Nq = H * dv, H * dqk
+    assert np.array_equal(got["u"], c["x"][:, :Nu])
+    assert np.array_equal(got["v"], c["x"][:, Nu:2 * Nu])
+    assert np.array_equal(got["q"], c["x"][:, 2 * Nu:2 * Nu + Nq])
+    assert np.array_equal(got["k"], c["x"][:, 2 * Nu + Nq:N])
+    b = c["b"]
+    got = oracle_lib.uvqk(c["x"], np.zeros((N, 32)), b, H, dqk, dv, 1)
+    silu_b = b / (1.0 + np.exp(-b))
+    assert np.allclose(got["q"], np.broadcast_to(silu_b[2 * Nu:2 * Nu + Nq], got["q"].shape),
+                       rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("affine", [False, True])
+def test_out_proj_matches_torch(oracle_lib, affine):
+    """The model card's norm(x + out(o * silu(u))): nn.Linear then nn.LayerNorm
+    over E (here the gated, normalised attention output is y)."""
+    rng = np.random.default_rng(5)
+    T, E, Dy = 7, 24, 12
+    y, x = rng.standard_normal((T, Dy)), rng.standard_normal((T, E))
+    w, b = rng.standard_normal((E, Dy)) / 3, rng.standard_normal(E)
+    g = 1 + 0.2 * rng.standard_normal(E) if affine else None
+    be = 0.3 * rng.standard_normal(E) if affine else None
+    got = oracle_lib.out_proj(y, x, w, b, g, be)
+    t = lambda a: None if a is None else torch.from_numpy(a)
+    r = t(x) + t(y) @ t(w).T + t(b)
+    ref = torch.nn.functional.layer_norm(r, (E,), weight=t(g), bias=t(be), eps=1e-5)
+    assert rel_err(got["z"], ref.numpy()) < 1e-12
+    assert rel_err(got["mean"], r.mean(-1).numpy()) < 1e-12
+
+
+def test_out_proj_closed_forms(oracle_lib):
+    """With no projection weight and no input, every row is the normalised
+    bias; the residual alone gives LayerNorm rows of mean 0 and variance
+    var/(var + eps)."""
+    rng = np.random.default_rng(6)
+    T, E, Dy = 5, 16, 8
+    b = rng.standard_normal(E)
+    got = oracle_lib.out_proj(np.zeros((T, Dy)), np.zeros((T, E)), np.zeros((E, Dy)), b)
+    bn = (b - b.mean()) / np.sqrt(b.var() + 1e-5)
+    assert np.abs(got["z"] - bn[None, :]).max() < 1e-13
+    x = rng.standard_normal((T, E)) * 3
+    got = oracle_lib.out_proj(rng.standard_normal((T, Dy)), x, np.zeros((E, Dy)))
+    z = got["z"]
+    var = x.var(axis=1)
+    assert np.abs(z.mean(axis=1)).max() < 1e-13
+    assert np.abs(z.var(axis=1) - var / (var + 1e-5)).max() < 1e-12

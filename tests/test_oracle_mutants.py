@@ -78,6 +78,16 @@ MUTANTS = [
     ("LayerNorm weight gradient without xhat",
      "if (d_ln_weight) d_ln_weight[c] += dyg * xhat;", "if (d_ln_weight) d_ln_weight[c] += dyg;",
      0),
+    # projections either side of the attention
+    ("UVQK split with v before u",
+     "if (n < Nu) u[t * Nu + n] = acc;\n            else if (n < 2 * Nu) v[t * Nu + (n - Nu)] = acc;",
+     "if (n < Nu) v[t * Nu + n] = acc;\n            else if (n < 2 * Nu) u[t * Nu + (n - Nu)] = acc;",
+     0),
+    ("UVQK weight row read in reverse", "for (int c = 0; c < E; ++c) acc += xr[c] * wr[c];",
+     "for (int c = 0; c < E; ++c) acc += xr[c] * wr[E - 1 - c];", 0),
+    ("output residual dropped", "r[e] = xr[e] + acc + (b ? b[e] : 0.0);",
+     "r[e] = acc + (b ? b[e] : 0.0);", 0),
+    ("output bias dropped", "r[e] = xr[e] + acc + (b ? b[e] : 0.0);", "r[e] = xr[e] + acc;", 0),
     ("dS without 1/N",
      "double dS = dA * ref_silu_grad(S) / Nn;", "double dS = dA * ref_silu_grad(S);", 0),
     ("dV from dS instead of A",
@@ -130,6 +140,8 @@ PINS = [
     T.test_time_bucket_thresholds,
     T.test_backward_finite_differences,
     T.test_layernorm_affine_closed_forms,
+    T.test_uvqk_closed_forms,
+    T.test_out_proj_closed_forms,
 ]
 
 
