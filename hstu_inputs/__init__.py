@@ -26,7 +26,7 @@ from typing import Dict, List, Optional, Sequence
 import torch
 
 __all__ = ["Spec", "Inputs", "WORKLOADS", "make_inputs", "workload", "causal_flops",
-           "stochastic_length", "stochastic_length_rows"]
+           "stochastic_length", "stochastic_length_rows", "ProjInputs", "make_proj_inputs"]
 
 NUM_TIME_BUCKETS = 128
 TIME_T0 = 1_700_000_000      # first timestamp of every sequence (seconds)
@@ -245,3 +245,47 @@ def make_inputs(spec: Spec, seed: int = 0) -> Inputs:
         norm_len = spec.norm_len if spec.norm_len > 0 else (spec.seq_len or max(lengths or [1]))
     return Inputs(spec, offsets, q, k, v, u, ts, rab_pos, rab_time, dy, norm_len, L,
                   ln_weight, ln_bias)
+
+
+@dataclasses.dataclass
+class ProjInputs:
+    """Host tensors of the two projections around one HSTU layer's attention.
+
+    x [T, E] layer input (already normalised; bf16), w_uvqk [H(2dv+2dqk), E]
+    and b_uvqk [N]; y [T, H dv] an attention output (bf16), w_out [E, H dv],
+    b_out [E], ln_weight, ln_bias [E] (fp32)."""
+    T: int
+    E: int
+    H: int
+    d_qk: int
+    d_v: int
+    x: torch.Tensor
+    w_uvqk: torch.Tensor
+    b_uvqk: torch.Tensor
+    y: torch.Tensor
+    w_out: torch.Tensor
+    b_out: torch.Tensor
+    ln_weight: torch.Tensor
+    ln_bias: torch.Tensor
+
+
+def make_proj_inputs(T: int, E: int = 512, H: int = 4, d_qk: int = 128, d_v: int = 128,
+                     seed: int = 0) -> ProjInputs:
+    """Seeded projection inputs, drawn in the order x, w_uvqk, b_uvqk, y, w_out,
+    b_out, ln_weight, ln_bias.  Weights are randn / sqrt(fan_in) (the scale of a
+    default-initialised linear layer), biases 0.1 randn, the LayerNorm weight
+    1 + 0.1 randn; matrices are rounded to bf16."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    bf = torch.bfloat16
+    N = 2 * H * d_v + 2 * H * d_qk
+    D = H * d_v
+    x = torch.randn(T, E, generator=g).to(bf)
+    w_uvqk = (torch.randn(N, E, generator=g) / math.sqrt(E)).to(bf)
+    b_uvqk = 0.1 * torch.randn(N, generator=g)
+    y = torch.randn(T, D, generator=g).to(bf)
+    w_out = (torch.randn(E, D, generator=g) / math.sqrt(D)).to(bf)
+    b_out = 0.1 * torch.randn(E, generator=g)
+    ln_weight = 1.0 + 0.1 * torch.randn(E, generator=g)
+    ln_bias = 0.1 * torch.randn(E, generator=g)
+    return ProjInputs(T, E, H, d_qk, d_v, x, w_uvqk, b_uvqk, y, w_out, b_out, ln_weight,
+                      ln_bias)

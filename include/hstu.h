@@ -182,6 +182,50 @@ HSTU_API hstu_status_t hstu_attn_bwd_noalloc(const hstu_problem_t *p, const void
                                              float *d_rab_pos, float *d_rab_time,
                                              float *d_ln_weight, float *d_ln_bias, void *stream);
 
+/*
+ * The projections either side of the attention in an HSTU layer ("HSTU
+ * (Generative Recommender)" model card, Exported PyTorch, HSTUBlock: the
+ * uvqk linear split into u, v, q, k, and norm(x + out(y)); the reproduction
+ * note's key formulas: U, V, Q, K = Split(SiLU(Norm(X) W_UVQK)) and the
+ * residual around the layer).  Both are bf16 GEMMs on the tcgen05 tensor
+ * cores with fp32 accumulation and a fused epilogue; outputs are rounded to
+ * bf16 once.  All matrices are row-major bf16, 16-byte aligned; fp32 vectors
+ * 16-byte aligned.  `workspace` (>= 256 bytes, 256-byte aligned, zero-filled
+ * before first use) holds only the device status word that hstu_attn_check
+ * reads.  Argument checks are synchronous (HSTU_ERR_INVALID_ARG,
+ * HSTU_ERR_UNSUPPORTED, HSTU_ERR_WORKSPACE) and enqueue nothing; T = 0 is a
+ * no-op.
+ */
+
+/*
+ * UVQK projection: P = act(X W^T + bias), X [T, E], W [N, E] (the nn.Linear
+ * weight layout), N = 2*H*d_v + 2*H*d_qk, bias fp32 [N] or NULL, act 0 =
+ * identity, 1 = SiLU.  Columns [0, Hd_v) go to u [T, H*d_v], [Hd_v, 2Hd_v)
+ * to v [T, H, d_v], the next H*d_qk to q [T, H, d_qk] and the last H*d_qk to
+ * k [T, H, d_qk] -- the layouts hstu_attn_fwd reads.  Supported: E a
+ * multiple of 64; H*d_v and H*d_qk multiples of 256; T <= 8388480.
+ */
+HSTU_API hstu_status_t hstu_uvqk_fwd(int32_t T, int32_t E, int32_t H, int32_t d_qk, int32_t d_v,
+                                     int32_t act, const void *x, const void *w, const float *bias,
+                                     void *u, void *v, void *q, void *k, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
+/*
+ * Output projection, residual and LayerNorm over E:
+ *   R = X + Y W^T + bias,  Z = (R - mean(R)) * rstd * ln_weight + ln_bias,
+ *   rstd = 1 / sqrt(biased variance of R + eps).
+ * Y [T, D] (the attention output, D = H*d_v), W [E, D] (nn.Linear layout),
+ * X [T, E] the residual (the layer input), bias, ln_weight, ln_bias fp32 [E]
+ * or NULL (zeros, ones, zeros); z [T, E] bf16 output; mean, rstd fp32 [T]
+ * (both or neither) receive the row statistics of R.  Supported: E in
+ * {256, 512}; D a multiple of 64.
+ */
+HSTU_API hstu_status_t hstu_out_fwd(int32_t T, int32_t E, int32_t D, const void *y, const void *w,
+                                    const void *x, const float *bias, const float *ln_weight,
+                                    const float *ln_bias, float eps, void *z, float *mean,
+                                    float *rstd, void *workspace, size_t workspace_bytes,
+                                    void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,7 @@ HSTU_F32, HSTU_BF16 = 0, 1
 
 EXPORTED = ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_attn_check",
             "hstu_status_string", "hstu_time_bucket_thresholds", "hstu_selftest_wait_timeout",
-            "hstu_attn_bwd_noalloc")
+            "hstu_attn_bwd_noalloc", "hstu_uvqk_fwd", "hstu_out_fwd")
 
 
 class HSTUError(RuntimeError):
@@ -85,6 +85,11 @@ def load_library():
     lib.hstu_selftest_wait_timeout.restype = ctypes.c_int
     lib.hstu_attn_bwd_noalloc.argtypes = [P] + [vp] * 5 + [vp] * 3 + [vp] * 4 + [vp] * 4 + [vp]
     lib.hstu_attn_bwd_noalloc.restype = ctypes.c_int
+    i32 = ctypes.c_int32
+    lib.hstu_uvqk_fwd.argtypes = [i32] * 6 + [vp] * 7 + [vp, sz, vp]
+    lib.hstu_uvqk_fwd.restype = ctypes.c_int
+    lib.hstu_out_fwd.argtypes = [i32] * 3 + [vp] * 6 + [ctypes.c_float] + [vp] * 3 + [vp, sz, vp]
+    lib.hstu_out_fwd.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -259,3 +264,66 @@ def hstu_selftest_wait_timeout(workspace, budget_ns: int = 50_000_000, stream=No
     """Runs the bounded-wait self-test kernel; returns the launch status."""
     return int(load_library().hstu_selftest_wait_timeout(_ptr(workspace), int(budget_ns),
                                                          _stream_ptr(stream)))
+
+
+def _status_workspace(device):
+    return torch.zeros(256, dtype=torch.uint8, device=device)
+
+
+def hstu_uvqk_fwd(x, w, num_heads: int, d_qk: int, d_v: int, *, bias=None, act: int = 0,
+                  out=None, workspace=None, stream=None):
+    """UVQK projection act(x w^T + bias) of x [T, E] by w [H(2dv+2dqk), E] (bf16).
+
+    Returns dict u [T, H*dv], v [T, H, dv], q [T, H, dqk], k [T, H, dqk] (bf16)."""
+    lib = load_library()
+    _dev(x, "x", torch.bfloat16)
+    _dev(w, "w", torch.bfloat16)
+    _dev(bias, "bias", torch.float32)
+    T, E = x.shape
+    H = int(num_heads)
+    if out is None:
+        out = dict(u=torch.empty((T, H * d_v), dtype=x.dtype, device=x.device),
+                   v=torch.empty((T, H, d_v), dtype=x.dtype, device=x.device),
+                   q=torch.empty((T, H, d_qk), dtype=x.dtype, device=x.device),
+                   k=torch.empty((T, H, d_qk), dtype=x.dtype, device=x.device))
+    for n in ("u", "v", "q", "k"):
+        _dev(out[n], n, x.dtype)
+    if workspace is None:
+        workspace = _status_workspace(x.device)
+    rc = lib.hstu_uvqk_fwd(int(T), int(E), H, int(d_qk), int(d_v), int(act), _ptr(x), _ptr(w),
+                           _ptr(bias), _ptr(out["u"]), _ptr(out["v"]), _ptr(out["q"]),
+                           _ptr(out["k"]), _ptr(workspace), workspace.numel(),
+                           _stream_ptr(stream))
+    if rc != HSTU_OK:
+        raise HSTUError(rc, "hstu_uvqk_fwd")
+    return out
+
+
+def hstu_out_fwd(y, w, x, *, bias=None, ln_weight=None, ln_bias=None, eps: float = 1e-5,
+                 save_stats: bool = False, z=None, workspace=None, stream=None):
+    """Z = LayerNorm(x + y w^T + bias) * ln_weight + ln_bias for y [T, D], w [E, D],
+    x [T, E] (bf16).  Returns (z, (mean, rstd) or None)."""
+    lib = load_library()
+    _dev(y, "y", torch.bfloat16)
+    _dev(w, "w", torch.bfloat16)
+    _dev(x, "x", torch.bfloat16)
+    for n, t in (("bias", bias), ("ln_weight", ln_weight), ("ln_bias", ln_bias)):
+        _dev(t, n, torch.float32)
+    T, D = y.shape
+    E = x.shape[1]
+    if z is None:
+        z = torch.empty((T, E), dtype=x.dtype, device=x.device)
+    _dev(z, "z", x.dtype)
+    stats = None
+    if save_stats:
+        stats = (torch.empty(T, dtype=torch.float32, device=x.device),
+                 torch.empty(T, dtype=torch.float32, device=x.device))
+    if workspace is None:
+        workspace = _status_workspace(x.device)
+    mean, rstd = stats if stats is not None else (None, None)
+    rc = lib.hstu_out_fwd(int(T), int(E), int(D), _ptr(y), _ptr(w), _ptr(x), _ptr(bias),
+                          _ptr(ln_weight), _ptr(ln_bias), float(eps), _ptr(z), _ptr(mean),
+                          _ptr(rstd), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    if rc != HSTU_OK:
+        raise HSTUError(rc, "hstu_out_fwd")
+    return z, stats

@@ -117,6 +117,22 @@ bool make_map_3d(CUtensorMap* map, const void* base, int T, int H, int box_rows)
   return r == CUDA_SUCCESS;
 }
 
+// [rows, cols] bf16 row-major as a 2-D tensor (col, row); box = 64 x box_rows,
+// 128-byte swizzle: one box is box_rows rows x 128 bytes of a K-major tile.
+// Rows past `rows` read as zeros.
+bool make_map_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------- validation
 hstu_status_t check_problem(const hstu_problem_t* p) {
   if (!p) return HSTU_ERR_INVALID_ARG;
@@ -408,6 +424,85 @@ hstu_status_t hstu_attn_check(void* workspace, void* stream) {
   if (word & kStatusTimeout) return HSTU_ERR_TIMEOUT;
   if (word & kStatusBadOffsets) return HSTU_ERR_INVALID_ARG;
   return HSTU_OK;
+}
+
+// ---------------------------------------------------------- projections
+static bool al32(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 31u) == 0; }
+
+static hstu_status_t check_status_ws(void* ws, size_t bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 || bytes < kStatusBytes)
+    return HSTU_ERR_WORKSPACE;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_uvqk_fwd(int32_t T, int32_t E, int32_t H, int32_t d_qk, int32_t d_v,
+                            int32_t act, const void* x, const void* w, const float* bias, void* u,
+                            void* v, void* q, void* k, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  NvtxRange range("hstu_uvqk_fwd");
+  if (T < 0 || E < 1 || H < 1 || d_qk < 1 || d_v < 1 || (act != 0 && act != 1))
+    return HSTU_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, w, u, v, q, k};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  if (bias && !aligned16(bias)) return HSTU_ERR_INVALID_ARG;
+  const int64_t Nu = static_cast<int64_t>(H) * d_v, Nq = static_cast<int64_t>(H) * d_qk;
+  if (E % 64 != 0 || Nu % 256 != 0 || Nq % 256 != 0 || 2 * (Nu + Nq) > 65535 * 256 ||
+      (static_cast<int64_t>(T) + 127) / 128 > 65535)
+    return HSTU_ERR_UNSUPPORTED;
+  hstu_status_t st = check_status_ws(workspace, workspace_bytes);
+  if (st != HSTU_OK) return st;
+  if (T == 0) return HSTU_OK;
+  ProjArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.bias = bias;
+  a.out0 = u; a.out1 = v; a.out2 = q; a.out3 = k;
+  a.status = static_cast<int*>(workspace);
+  a.T = T; a.K = E; a.E = E;
+  a.Nu = static_cast<int>(Nu); a.Nq = static_cast<int>(Nq);
+  a.act = act;
+  a.vec32 = al32(u) && al32(v) && al32(q) && al32(k);
+  CUtensorMap tx, tw;
+  if (!make_map_2d(&tx, x, T, E, 128) || !make_map_2d(&tw, w, 2 * (Nu + Nq), E, 256))
+    return HSTU_ERR_CUDA;
+  const cudaError_t err = launch_uvqk_sm100(a, tx, tw, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_out_fwd(int32_t T, int32_t E, int32_t D, const void* y, const void* w,
+                           const void* x, const float* bias, const float* ln_weight,
+                           const float* ln_bias, float eps, void* z, float* mean, float* rstd,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange range("hstu_out_fwd");
+  if (T < 0 || E < 1 || D < 1 || !(eps > 0.0f) || !std::isfinite(eps)) return HSTU_ERR_INVALID_ARG;
+  const void* ptrs[] = {y, w, x, z};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  const void* opt[] = {bias, ln_weight, ln_bias};
+  for (const void* p : opt)
+    if (p && !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  if ((mean == nullptr) != (rstd == nullptr)) return HSTU_ERR_INVALID_ARG;
+  if ((E != 256 && E != 512) || D % 64 != 0) return HSTU_ERR_UNSUPPORTED;
+  hstu_status_t st = check_status_ws(workspace, workspace_bytes);
+  if (st != HSTU_OK) return st;
+  if (T == 0) return HSTU_OK;
+  ProjArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.bias = bias;
+  a.ln_weight = ln_weight;
+  a.ln_bias = ln_bias;
+  a.res = x;
+  a.out0 = z;
+  a.mean = mean;
+  a.rstd = rstd;
+  a.status = static_cast<int*>(workspace);
+  a.T = T; a.K = D; a.E = E;
+  a.eps = eps;
+  a.vec32 = al32(z);
+  CUtensorMap ty, tw;
+  if (!make_map_2d(&ty, y, T, D, 128) || !make_map_2d(&tw, w, E, D, 256)) return HSTU_ERR_CUDA;
+  const cudaError_t err = launch_out_sm100(a, ty, tw, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
 }  // extern "C"

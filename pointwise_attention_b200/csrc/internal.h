@@ -104,6 +104,26 @@ struct BwdArgs {
   BucketTable bt;
 };
 
+// Arguments of the projection GEMMs (UVQK and output + residual + LayerNorm).
+// A [rows, K] bf16 and B [N, K] bf16 are read through TMA maps; K % 64 == 0.
+struct ProjArgs {
+  const float* bias;        // [N] or nullptr
+  const float* ln_weight;   // output projection: [E] or nullptr (ones)
+  const float* ln_bias;     // output projection: [E] or nullptr (zeros)
+  const void* res;          // output projection: residual X [T, E] bf16
+  void* out0;               // UVQK: u [T, Nu]; output projection: z [T, E]
+  void* out1;               // UVQK: v [T, Nu]
+  void* out2;               // UVQK: q [T, Nq]
+  void* out3;               // UVQK: k [T, Nq]
+  float* mean;              // output projection: [T] or nullptr (with rstd)
+  float* rstd;
+  int* status;
+  int T, K, E, Nu, Nq;
+  int act;                  // UVQK: 1 = SiLU after the bias
+  int vec32;                // every output pointer is 32-byte aligned
+  float eps;
+};
+
 // The synchronous argument checks of hstu_attn_bwd (all but the workspace's).
 hstu_status_t check_bwd_args(const hstu_problem_t* p, const void* dy, const void* q,
                              const void* k, const void* v, const void* u, const float* o_save,
@@ -119,6 +139,10 @@ cudaError_t launch_fwd_f32_simt(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_f32_simt(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_bf16_simt(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_pre_bf16(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_uvqk_sm100(const ProjArgs& a, const CUtensorMap& tx, const CUtensorMap& tw,
+                              cudaStream_t stream);
+cudaError_t launch_out_sm100(const ProjArgs& a, const CUtensorMap& ty, const CUtensorMap& tw,
+                             cudaStream_t stream);
 cudaError_t launch_bwd_attn_bf16_sm100(const BwdArgs& a, const CUtensorMap* maps,
                                        cudaStream_t stream);
 

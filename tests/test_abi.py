@@ -239,3 +239,49 @@ def test_bwd_rejects_layernorm_gradients_without_tables(lib):
                             None) == 1
     assert so.hstu_attn_bwd(ctypes.byref(p), *args, None, None, None, vp(FAKE), vp(FAKE), need,
                             None) == 1
+
+
+def call_uvqk(lib, T=300, E=512, H=4, dqk=128, dv=128, act=0, x=FAKE, bias=None, u=FAKE,
+              ws=FAKE, ws_bytes=256):
+    so = lib.load_library()
+    vp = ctypes.c_void_p
+    return so.hstu_uvqk_fwd(T, E, H, dqk, dv, act, vp(x) if x else None, vp(FAKE),
+                            vp(bias) if bias else None, vp(u) if u else None, vp(FAKE),
+                            vp(FAKE), vp(FAKE), vp(ws) if ws else None, ws_bytes, None)
+
+
+def call_out(lib, T=300, E=512, D=512, eps=1e-5, y=FAKE, ln_weight=None, mean=None, rstd=None,
+             z=FAKE, ws=FAKE, ws_bytes=256):
+    so = lib.load_library()
+    vp = ctypes.c_void_p
+    opt = lambda a: vp(a) if a else None
+    return so.hstu_out_fwd(T, E, D, opt(y), vp(FAKE), vp(FAKE), None, opt(ln_weight), None,
+                           eps, opt(z), opt(mean), opt(rstd), opt(ws), ws_bytes, None)
+
+
+def test_uvqk_rejections(lib):
+    assert call_uvqk(lib, T=-1) == 1
+    assert call_uvqk(lib, act=2) == 1
+    assert call_uvqk(lib, x=None) == 1
+    assert call_uvqk(lib, u=FAKE + 8) == 1                  # not 16-byte aligned
+    assert call_uvqk(lib, bias=FAKE + 4) == 1
+    assert call_uvqk(lib, E=96) == 2                        # E not a multiple of 64
+    assert call_uvqk(lib, H=1, dv=128) == 2                 # H*dv not a multiple of 256
+    assert call_uvqk(lib, T=65536 * 128) == 2               # row tiles beyond the grid's y limit
+    assert call_uvqk(lib, ws=None) == 5
+    assert call_uvqk(lib, ws_bytes=255) == 5
+    assert call_uvqk(lib, ws=FAKE + 16) == 5
+    assert call_uvqk(lib, T=0) == 0                         # empty: nothing to do
+
+
+def test_out_rejections(lib):
+    assert call_out(lib, eps=0.0) == 1
+    assert call_out(lib, eps=float("inf")) == 1
+    assert call_out(lib, y=None) == 1
+    assert call_out(lib, z=FAKE + 2) == 1
+    assert call_out(lib, ln_weight=FAKE + 4) == 1
+    assert call_out(lib, mean=FAKE) == 1                    # mean and rstd together or neither
+    assert call_out(lib, E=384) == 2
+    assert call_out(lib, D=100) == 2
+    assert call_out(lib, ws=None) == 5
+    assert call_out(lib, T=0) == 0
