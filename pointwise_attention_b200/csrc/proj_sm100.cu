@@ -15,8 +15,11 @@
 // Warp 0 issues TMA loads of 128 x 64 (A) and NT x 64 (B) bf16 boxes with
 // the 128-byte swizzle, warp 1 allocates TMEM and issues one 128 x 256 x 16
 // MMA per 256 columns and 16-element K step (N = 256 keeps one issuing
-// thread at the tensor core's rate), warps 2..5 are the epilogue, one
-// accumulator row (TMEM lane) per thread.  Every wait is bounded.
+// thread at the tensor core's rate), warps 2.. are the epilogue: S warps
+// per TMEM lane quarter, one accumulator row (TMEM lane) per thread and NT/S
+// columns per warp (S = 2 for UVQK, two CTAs per SM; S = 4 for the output
+// projection, whose tile fills TMEM and runs one CTA per SM).  Every wait is
+// bounded.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -31,20 +34,26 @@ namespace {
 
 constexpr int kBM = 128;                   // rows per tile
 constexpr int kBK = 64;                    // K elements per stage (one 128-byte swizzle row)
-constexpr int kThreads = 192;
 constexpr int kABytes = kBM * kBK * 2;     // 16 KB
 
 enum { EPI_UVQK = 0, EPI_OUT = 1 };
 
-template <int NT>
+// NT columns per tile; the epilogue has S warps per TMEM lane quarter, each
+// taking NT / S consecutive columns of its 32 rows.
+template <int EPI, int NT>
 struct Cfg {
+  static constexpr int S = EPI == EPI_UVQK ? 2 : 4;
+  static constexpr int kThreads = 64 + 128 * S;
+  static constexpr int kMinBlocks = EPI == EPI_UVQK ? 2 : 1;
+  static constexpr int kCols = NT / S;   // per epilogue thread
   static constexpr int kBBytes = NT * kBK * 2;
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kStages = 2;   // 96 KB at NT = 256 (two CTAs per SM), 160 KB at 512
   static constexpr int kOffBar = kStages * kStage;
   static constexpr int kNumBars = 2 * kStages + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmem = kOffMisc + 16 + 1024;
+  static constexpr int kOffStats = kOffMisc + 16;           // float2 [S][128] row partials
+  static constexpr int kSmem = kOffStats + S * kBM * 8 + 1024;
 };
 
 __device__ __forceinline__ bool wait_or_flag(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -74,25 +83,24 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
   }
 }
 
-__device__ __forceinline__ void load_row32(const __nv_bfloat16* src, float (&f)[32]) {
+// 8 consecutive fp32 values (16-byte aligned), or `fill` when p is null.
+__device__ __forceinline__ void ldg_f8(const float* p, float fill, float (&v)[8]) {
+  if (p) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src) + i);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws[j]));
-      f[8 * i + 2 * j] = p.x;
-      f[8 * i + 2 * j + 1] = p.y;
-    }
+    for (int i = 0; i < 8; ++i) v[i] = fill;
   }
 }
 
 template <int EPI, int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<EPI, NT>::kThreads, Cfg<EPI, NT>::kMinBlocks)
     proj_gemm_sm100(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ ProjArgs a) {
-  using C = Cfg<NT>;
+  using C = Cfg<EPI, NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -176,16 +184,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q4 = warp & 3;                         // TMEM lane quarter
-    const int r = 32 * q4 + lane;
+    const int q4 = warp & 3;                         // TMEM lane quarter of this warp
+    const int cs = (warp - 2) >> 2;                  // column slice 0..S-1
+    const int r = 32 * q4 + lane;                    // tile row = TMEM lane
     const int t = m0 + r;
     const bool row_ok = t < a.T;
-    const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
+    const int c0 = cs * C::kCols;                    // first tile column of the slice
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q4) << 16) + c0;
     bool ok = wait_or_flag(bar(B_TFULL), 0, abort_flag, a.status) && !*abort_flag;
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      tc_fence_after();
-      if (EPI == EPI_UVQK) {
+    if (ok) tc_fence_after();
+    if (EPI == EPI_UVQK) {
+      if (ok) {
         // the output tensor and column this tile starts at
         const int Nu = a.Nu, Nq = a.Nq;
         __nv_bfloat16* dst;
@@ -194,64 +204,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         else if (n0 < 2 * Nu) { dst = static_cast<__nv_bfloat16*>(a.out1); col = n0 - Nu; ld = Nu; }
         else if (n0 < 2 * Nu + Nq) { dst = static_cast<__nv_bfloat16*>(a.out2); col = n0 - 2 * Nu; ld = Nq; }
         else { dst = static_cast<__nv_bfloat16*>(a.out3); col = n0 - 2 * Nu - Nq; ld = Nq; }
-        __nv_bfloat16* drow = dst + static_cast<size_t>(t) * ld + col;
+        __nv_bfloat16* drow = dst + static_cast<size_t>(t) * ld + col + c0;
+        const float* brow = a.bias ? a.bias + n0 + c0 : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < NT / 32; ++c) {
+        for (int c = 0; c < C::kCols / 32; ++c) {
           uint32_t v[32];
-          tmem_ld32_nowait(tmem + lane_addr + 32u * c, v);
+          tmem_ld32_nowait(taddr + 32u * c, v);
           tmem_wait_ld_dep(v);
-          float f[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
-          if (a.bias) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.bias + n0 + 32 * c) + i);
-              f[4 * i] += b4.x; f[4 * i + 1] += b4.y; f[4 * i + 2] += b4.z; f[4 * i + 3] += b4.w;
-            }
-          }
-          if (a.act) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float hx = 0.5f * f[i];
-              f[i] = fmaf(hx, tanh_approx(hx), hx);   // SiLU(x) = x/2 (1 + tanh(x/2))
-            }
-          }
           uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = pack2(f[2 * i], f[2 * i + 1]);
-          if (row_ok) store_row32(drow + 32 * c, w, a.vec32);
-        }
-      } else {
-        // Z = LayerNorm(X + Y W^T + b): pass 1 row statistics, pass 2 normalise.
-        const int E = NT;
-        const __nv_bfloat16* xrow = static_cast<const __nv_bfloat16*>(a.res) +
-                                    static_cast<size_t>(row_ok ? t : 0) * E;
-        auto chunk = [&](int c, float (&f)[32]) {
-          uint32_t v[32];
-          tmem_ld32_nowait(tmem + lane_addr + 32u * c, v);
-          tmem_wait_ld_dep(v);
-          float xr[32];
-          if (row_ok) load_row32(xrow + 32 * c, xr);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]) + (row_ok ? xr[i] : 0.f);
-          if (a.bias) {
+          for (int g = 0; g < 4; ++g) {
+            float f[8], b[8];
+            ldg_f8(brow ? brow + 32 * c + 8 * g : nullptr, 0.f, b);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.bias + 32 * c) + i);
-              f[4 * i] += b4.x; f[4 * i + 1] += b4.y; f[4 * i + 2] += b4.z; f[4 * i + 3] += b4.w;
+              f[i] = __uint_as_float(v[8 * g + i]) + b[i];
+              if (a.act) {
+                const float hx = 0.5f * f[i];
+                f[i] = fmaf(hx, tanh_approx(hx), hx);   // SiLU(x) = x/2 (1 + tanh(x/2))
+              }
             }
-          }
-        };
-        float cnt = 0.f, mean = 0.f, m2 = 0.f;       // Chan's merge of 32-value chunks
-#pragma unroll 1
-        for (int c = 0; c < E / 32; ++c) {
-          float f[32];
-          chunk(c, f);
-          float s = 0.f;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) s += f[i];
-          const float mc = s * (1.0f / 32.0f);
+            for (int i = 0; i < 4; ++i) w[4 * g + i] = pack2(f[2 * i], f[2 * i + 1]);
+          }
+          if (row_ok) store_row32(drow + 32 * c, w, a.vec32);
+        }
+      }
+    } else {
+      // Z = LayerNorm(X + Y W^T + b): each thread reduces its slice of the row
+      // (Chan's merge of 32-column chunks), the S slices of a row merge through
+      // shared memory, then each thread normalises its slice.
+      const __nv_bfloat16* xrow = static_cast<const __nv_bfloat16*>(a.res) +
+                                  static_cast<size_t>(row_ok ? t : 0) * NT + c0;
+      // R = acc + x + b for 8 columns starting at slice column j
+      auto resid8 = [&](const uint32_t* v, int j, float (&f)[8]) {
+        float b[8];
+        ldg_f8(a.bias ? a.bias + c0 + j : nullptr, 0.f, b);
+        uint4 xw = make_uint4(0u, 0u, 0u, 0u);
+        if (row_ok) xw = __ldg(reinterpret_cast<const uint4*>(xrow + j));
+        const uint32_t xs[4] = {xw.x, xw.y, xw.z, xw.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[i]));
+          f[2 * i] = __uint_as_float(v[2 * i]) + x2.x + b[2 * i];
+          f[2 * i + 1] = __uint_as_float(v[2 * i + 1]) + x2.y + b[2 * i + 1];
+        }
+      };
+      float cnt = 0.f, mean = 0.f, m2 = 0.f;
+      if (ok) {
+#pragma unroll 1
+        for (int c = 0; c < C::kCols / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32_nowait(taddr + 32u * c, v);
+          tmem_wait_ld_dep(v);
+          float f[32];
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            resid8(v + 8 * g, 32 * c + 8 * g, reinterpret_cast<float(&)[8]>(f[8 * g]));
+          float sum = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sum += f[i];
+          const float mc = sum * (1.0f / 32.0f);
           float mc2 = 0.f;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -263,41 +276,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           m2 += mc2 + dl * dl * (cnt * 32.f / n1);
           cnt = n1;
         }
-        const float rstd = 1.0f / sqrtf(m2 / static_cast<float>(E) + a.eps);
-        __nv_bfloat16* zrow = static_cast<__nv_bfloat16*>(a.out0) + static_cast<size_t>(t) * E;
+      }
+      float2* part = reinterpret_cast<float2*>(smem + C::kOffStats);
+      part[cs * kBM + r] = make_float2(mean, m2);
+      named_bar_sync(1, 128 * C::S);
+      float mu = 0.f, M2 = 0.f;
+#pragma unroll
+      for (int i = 0; i < C::S; ++i) mu += part[i * kBM + r].x;
+      mu *= 1.0f / C::S;
+#pragma unroll
+      for (int i = 0; i < C::S; ++i) {
+        const float2 pi = part[i * kBM + r];
+        const float d = pi.x - mu;
+        M2 += pi.y + static_cast<float>(C::kCols) * d * d;
+      }
+      const float rstd = 1.0f / sqrtf(M2 / static_cast<float>(NT) + a.eps);
+      if (ok) {
+        __nv_bfloat16* zrow = static_cast<__nv_bfloat16*>(a.out0) + static_cast<size_t>(t) * NT + c0;
 #pragma unroll 1
-        for (int c = 0; c < E / 32; ++c) {
-          float f[32];
-          chunk(c, f);
-          float g[32], bb[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            g[i] = 1.f;
-            bb[i] = 0.f;
-          }
-          if (a.ln_weight) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 w4 = __ldg(reinterpret_cast<const float4*>(a.ln_weight + 32 * c) + i);
-              g[4 * i] = w4.x; g[4 * i + 1] = w4.y; g[4 * i + 2] = w4.z; g[4 * i + 3] = w4.w;
-            }
-          }
-          if (a.ln_bias) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.ln_bias + 32 * c) + i);
-              bb[4 * i] = b4.x; bb[4 * i + 1] = b4.y; bb[4 * i + 2] = b4.z; bb[4 * i + 3] = b4.w;
-            }
-          }
+        for (int c = 0; c < C::kCols / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32_nowait(taddr + 32u * c, v);
+          tmem_wait_ld_dep(v);
           uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            w[i] = pack2(fmaf((f[2 * i] - mean) * rstd, g[2 * i], bb[2 * i]),
-                         fmaf((f[2 * i + 1] - mean) * rstd, g[2 * i + 1], bb[2 * i + 1]));
+          for (int g = 0; g < 4; ++g) {
+            const int j = 32 * c + 8 * g;
+            float f[8], gw[8], gb[8];
+            resid8(v + 8 * g, j, f);
+            ldg_f8(a.ln_weight ? a.ln_weight + c0 + j : nullptr, 1.f, gw);
+            ldg_f8(a.ln_bias ? a.ln_bias + c0 + j : nullptr, 0.f, gb);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              w[4 * g + i] = pack2(fmaf((f[2 * i] - mu) * rstd, gw[2 * i], gb[2 * i]),
+                                   fmaf((f[2 * i + 1] - mu) * rstd, gw[2 * i + 1], gb[2 * i + 1]));
+          }
           if (row_ok) store_row32(zrow + 32 * c, w, a.vec32);
         }
-        if (row_ok && a.mean) {
-          a.mean[t] = mean;
+        if (row_ok && cs == 0 && a.mean) {
+          a.mean[t] = mu;
           a.rstd[t] = rstd;
         }
       }
@@ -314,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int EPI, int NT>
 cudaError_t launch(const ProjArgs& a, const CUtensorMap& ta, const CUtensorMap& tb, dim3 grid,
                    cudaStream_t stream) {
-  using C = Cfg<NT>;
+  using C = Cfg<EPI, NT>;
   static std::atomic<bool> configured[64];   // per device: shared-memory opt-in done
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -325,7 +342,7 @@ cudaError_t launch(const ProjArgs& a, const CUtensorMap& ta, const CUtensorMap& 
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) configured[dev].store(true, std::memory_order_release);
   }
-  proj_gemm_sm100<EPI, NT><<<grid, kThreads, C::kSmem, stream>>>(ta, tb, a);
+  proj_gemm_sm100<EPI, NT><<<grid, C::kThreads, C::kSmem, stream>>>(ta, tb, a);
   return cudaGetLastError();
 }
 
