@@ -544,6 +544,70 @@ def timed_e2e(wl, steps: int, device):
     return e0.elapsed_time(e1) / 1e3, h2d, d2h
 
 
+def measure_proj(T: int, steps: int, device, world: int):
+    """The projections around the attention at the model card's block shape
+    (embed 512, 4 heads, d = 128): UVQK (+ bias, SiLU) and the output
+    projection + residual + LayerNorm, each timed alone (CUDA graph of R
+    calls, events on the launching stream)."""
+    import pointwise_attention_b200 as pa
+    peaks, peak_kind = load_peaks()
+    E, H, d = 512, 4, 128
+    N, D = 4 * H * d, H * d
+    # enough copies that one graph's operands exceed the 126 MB L2
+    per_set = T * (E + N + D + E) * 2
+    R = max(2, -(-256 * 2 ** 20 // per_set))
+    sets = []
+    for r in range(R):
+        p = hi.make_proj_inputs(T, E, H, d, d, seed=100 + r)
+        dd = {k: getattr(p, k).to(device) for k in ("x", "w_uvqk", "b_uvqk", "y", "w_out",
+                                                    "b_out", "ln_weight", "ln_bias")}
+        dd["out"] = pa.hstu_uvqk_fwd(dd["x"], dd["w_uvqk"], H, d, d, bias=dd["b_uvqk"], act=1)
+        dd["z"], _ = pa.hstu_out_fwd(dd["y"], dd["w_out"], dd["x"], bias=dd["b_out"],
+                                     ln_weight=dd["ln_weight"], ln_bias=dd["ln_bias"])
+        dd["ws"] = torch.zeros(256, dtype=torch.uint8, device=device)
+        sets.append(dd)
+
+    def uvqk(i, stream=None):
+        dd = sets[i % R]
+        pa.hstu_uvqk_fwd(dd["x"], dd["w_uvqk"], H, d, d, bias=dd["b_uvqk"], act=1,
+                         out=dd["out"], workspace=dd["ws"], stream=stream)
+
+    def out(i, stream=None):
+        dd = sets[i % R]
+        pa.hstu_out_fwd(dd["y"], dd["w_out"], dd["x"], bias=dd["b_out"],
+                        ln_weight=dd["ln_weight"], ln_bias=dd["ln_bias"], z=dd["z"],
+                        workspace=dd["ws"], stream=stream)
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    result = {"workload": "proj_E512_H4_d128_T%d" % T, "steps_timed": steps}
+    for name, fn, flops, nbytes, kern in (
+            ("uvqk", uvqk, 2.0 * T * E * N, T * (E + N) * 2 + N * E * 2, "proj_gemm_sm100<0,256>"),
+            ("out", out, 2.0 * T * D * E, T * (D + 2 * E) * 2 + E * D * 2,
+             "proj_gemm_sm100<1,512>")):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        t, _ = time_graphs(steps, R, fn, stream, world)
+        t = reduce_max(t, world, device) / steps
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+        t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+        if t_tc >= t_hbm:
+            roof = {"bound": "tensor", "achieved": flops / t / 1e12, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s"}
+        roof.update(frac=roof["achieved"] / roof["peak"], kernel=kern, peak_source=peak_kind,
+                    algorithmic_flops=flops, algorithmic_bytes=nbytes, us_per_launch=t * 1e6,
+                    tflops=flops / t / 1e12, traffic=None)
+        for s_ in sets:
+            if pa.hstu_attn_check(s_["ws"]) != 0:
+                raise RuntimeError("device status after the projection timing")
+        result[name] = roof
+    return result
+
+
 def summary_of(spec, res, world):
     roof = dict(res["roofline"])
     return {"workload": spec.name, "value": res["value"], "unit": "TFLOP/s",
@@ -574,6 +638,10 @@ def run_gpu(args, spec):
 
     also = {}
     for name in [x for x in args.also.split(",") if x and x != spec.name]:
+        if name == "proj":
+            also[name] = measure_proj(131072, args.also_steps, device, world)
+            torch.cuda.empty_cache()
+            continue
         sp = hi.WORKLOADS[name]
         steps = args.also_steps
         r2, wl2 = measure(sp, rank_seed(args.seed, rank), steps, 3, device, world, local,
@@ -625,8 +693,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--also", default="long,train",
-                    help="comma-separated workloads timed after the main one ('' for none)")
+    ap.add_argument("--also", default="long,train,proj",
+                    help="comma-separated workloads timed after the main one, 'proj' for the "
+                         "projection GEMMs ('' for none)")
     ap.add_argument("--also-steps", type=int, default=50)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--cpu-budget-single", type=float, default=6.0)

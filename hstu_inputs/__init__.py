@@ -26,7 +26,8 @@ from typing import Dict, List, Optional, Sequence
 import torch
 
 __all__ = ["Spec", "Inputs", "WORKLOADS", "make_inputs", "workload", "causal_flops",
-           "stochastic_length", "stochastic_length_rows", "ProjInputs", "make_proj_inputs"]
+           "stochastic_length", "stochastic_length_rows", "ProjInputs", "make_proj_inputs",
+           "CandInputs", "make_cand_inputs", "CAND_WORKLOADS"]
 
 NUM_TIME_BUCKETS = 128
 TIME_T0 = 1_700_000_000      # first timestamp of every sequence (seconds)
@@ -289,3 +290,82 @@ def make_proj_inputs(T: int, E: int = 512, H: int = 4, d_qk: int = 128, d_v: int
     ln_bias = 0.1 * torch.randn(E, generator=g)
     return ProjInputs(T, E, H, d_qk, d_v, x, w_uvqk, b_uvqk, y, w_out, b_out, ln_weight,
                       ln_bias)
+
+
+@dataclasses.dataclass
+class CandInputs:
+    """Candidate scoring against cached histories (M-FALCON).
+
+    ``hist`` holds the users' histories as an ordinary problem (its k, v and
+    timestamps are the cached keys, values and event times; its q and u are
+    drawn but unused).  Candidates of user b are rows cand_offsets[b] ..
+    cand_offsets[b+1]-1 of qc, kc [C, H, d_qk], vc [C, H, d_v], uc [C, H*d_v],
+    with request timestamps cand_ts [C] (None without a time table)."""
+    hist: Inputs
+    cand_offsets: torch.Tensor      # int32 [B+1]
+    qc: torch.Tensor
+    kc: torch.Tensor
+    vc: torch.Tensor
+    uc: torch.Tensor
+    cand_ts: Optional[torch.Tensor]
+
+    @property
+    def counts(self) -> List[int]:
+        o = self.cand_offsets.tolist()
+        return [o[i + 1] - o[i] for i in range(len(o) - 1)]
+
+    @property
+    def total_cands(self) -> int:
+        return int(self.cand_offsets[-1])
+
+
+def make_cand_inputs(spec: Spec, cands, seed: int = 0) -> CandInputs:
+    """History from ``make_inputs(spec, seed)``; then, from a second generator
+    seeded with seed + 7919, per user a candidate count (``cands`` an int, or
+    an inclusive (lo, hi) range drawn uniformly), qc, kc, vc, uc with the
+    spec's distributions, and request times: each candidate of user b at
+    (last history time) + max(1, round(Exp(mean 300 s))), the history's
+    first time when it is empty."""
+    hist = make_inputs(spec, seed)
+    g = torch.Generator(device="cpu").manual_seed(seed + 7919)
+    B, H = spec.batch, spec.heads
+    if isinstance(cands, int):
+        counts = [cands] * B
+    else:
+        lo, hi = cands
+        counts = torch.randint(lo, hi + 1, (B,), generator=g).tolist()
+    offs = [0]
+    for c in counts:
+        offs.append(offs[-1] + c)
+    C = offs[-1]
+    dt = _torch_dtype(spec.dtype)
+
+    def draw(shape, std):
+        return (torch.randn(shape, generator=g, dtype=torch.float32) * std).to(dt)
+
+    qc = draw((C, H, spec.d_qk), spec.qk_std)
+    kc = draw((C, H, spec.d_qk), spec.qk_std)
+    vc = draw((C, H, spec.d_v), spec.vu_std)
+    uc = draw((C, H * spec.d_v), spec.vu_std)
+    cand_ts = None
+    if spec.rab_time:
+        parts = []
+        ho = hist.offsets.tolist()
+        for b, c in enumerate(counts):
+            last = int(hist.timestamps[ho[b + 1] - 1]) if ho[b + 1] > ho[b] else TIME_T0
+            gaps = torch.empty(c, dtype=torch.float64).exponential_(1.0 / TIME_GAP_MEAN,
+                                                                    generator=g)
+            parts.append(last + torch.clamp(torch.round(gaps), min=1.0).to(torch.int64))
+        cand_ts = torch.cat(parts) if parts else torch.empty(0, dtype=torch.int64)
+    return CandInputs(hist, torch.tensor(offs, dtype=torch.int32), qc, kc, vc, uc, cand_ts)
+
+
+# Candidate-scoring workloads: (history spec, candidates per user).
+#   mfalcon: 32 users with histories of U{256..4096} events (as the jagged
+#   workload: 8 heads, position and time bias, own-length normaliser), 512
+#   candidates each; the position table reaches relative position 4096.
+CAND_WORKLOADS = {
+    "mfalcon": (Spec("mfalcon", "bf16", batch=32, heads=8, d_qk=128, d_v=128,
+                     len_range=(256, 4096), qk_std=1.0 / math.sqrt(128.0), rab_pos_len=4097,
+                     rab_time=True, norm="own"), 512),
+}

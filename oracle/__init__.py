@@ -81,6 +81,8 @@ def _bind(path: str):
     lib.hstu_ref_out.argtypes = [i64, ctypes.c_int32, ctypes.c_int32] + [vp] * 6 + [
         ctypes.c_double] + [vp] * 3
     lib.hstu_ref_out.restype = ctypes.c_int
+    lib.hstu_ref_mfalcon.argtypes = [P] + [vp] * 12 + [i32]
+    lib.hstu_ref_mfalcon.restype = ctypes.c_int
     return lib
 
 
@@ -251,3 +253,26 @@ def out_proj(y, x, w, b=None, gamma=None, beta=None, eps: float = LN_EPS):
     if rc != 0:
         raise ValueError("hstu_ref_out rejected the sizes (code %d)" % rc)
     return dict(z=z, mean=mean, rstd=rstd)
+
+
+def mfalcon(ci, threads: int = 0):
+    """Candidate scoring (M-FALCON reading: each candidate is the token after
+    its user's history, attending to the history and itself only) of an
+    ``hstu_inputs.CandInputs``: dict y, o [C, D], mean, rstd [C] (fp64)."""
+    lib = _load()
+    h = ci.hist
+    a = _Args(h.offsets.numpy(), h.k, h.k, h.v, h.u,
+              None if h.timestamps is None else h.timestamps.numpy(), h.rab_pos, h.rab_time,
+              h.norm_len, h.rab_pos_len, ln_weight=h.ln_weight, ln_bias=h.ln_bias)
+    co = np.ascontiguousarray(ci.cand_offsets.numpy(), dtype=np.int32)
+    cts = None if ci.cand_ts is None else np.ascontiguousarray(ci.cand_ts.numpy(),
+                                                                dtype=np.int64)
+    qc, kc, vc, uc = _f64(ci.qc), _f64(ci.kc), _f64(ci.vc), _f64(ci.uc)
+    C = int(co[-1])
+    y = np.zeros((C, a.D)); o = np.zeros((C, a.D)); mean = np.zeros(C); rstd = np.zeros(C)
+    rc = lib.hstu_ref_mfalcon(ctypes.byref(a.prob), _ptr(a.k), _ptr(a.v), _ptr(co), _ptr(cts),
+                              _ptr(qc), _ptr(kc), _ptr(vc), _ptr(uc), _ptr(y), _ptr(o),
+                              _ptr(mean), _ptr(rstd), int(threads))
+    if rc != 0:
+        raise ValueError("hstu_ref_mfalcon rejected the problem (code %d)" % rc)
+    return dict(y=y, o=o, mean=mean, rstd=rstd)

@@ -428,3 +428,85 @@ int hstu_ref_out(int64_t T, int32_t E, int32_t Dy, const double *y, const double
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Candidate scoring against a cached history ("HSTU Hierarchical Sequential
+ * Transduction Units", §6 Why it works: M-FALCON, micro-batched candidate
+ * scoring with key/value reuse).  The pages give no formula.  Reading taken:
+ * candidate c of user b is the token that follows the user's n_b history
+ * tokens, on its own: it attends to every history token j < n_b and to itself,
+ * never to another candidate.  Its local row index is n_b, its time is its
+ * own timestamp, and its normaliser is norm_len (> 0) or n_b + 1, the length
+ * of (history, c).  Micro-batching and the reuse of the history's keys and
+ * values change the cost, not the result, so neither appears here.
+ * ------------------------------------------------------------------------ */
+int hstu_ref_mfalcon(const hstu_ref_problem *p, const double *k_hist, const double *v_hist,
+                     const int32_t *cand_offsets, const int64_t *cand_ts, const double *qc,
+                     const double *kc, const double *vc, const double *uc, double *y,
+                     double *o, double *mean, double *rstd, int num_threads) {
+    int rc = validate(p);
+    if (rc != 0) return rc;
+    if (!cand_offsets || cand_offsets[0] != 0) return -7;
+    if (p->rab_time && !cand_ts) return -8;
+    for (int b = 0; b < p->batch; ++b) {
+        if (cand_offsets[b + 1] < cand_offsets[b]) return -9;
+        /* the candidate's position index n_b must be in the table */
+        if (p->rab_pos && p->offsets[b + 1] - p->offsets[b] + 1 > p->rab_pos_len) return -4;
+    }
+    const int H = p->num_heads, dqk = p->d_qk, dv = p->d_v, D = H * dv;
+    const int64_t C = cand_offsets[p->batch];
+    const int64_t L = p->rab_pos_len, NB = p->num_time_buckets;
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#pragma omp parallel
+    {
+        double *orow = (double *)malloc(sizeof(double) * D);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t c = 0; c < C; ++c) {
+            int b = 0;
+            while (cand_offsets[b + 1] <= c) ++b;
+            const int64_t s = p->offsets[b];
+            const int n = p->offsets[b + 1] - p->offsets[b];
+            const double Nn = p->norm_len > 0 ? (double)p->norm_len : (double)(n + 1);
+            for (int e = 0; e < D; ++e) orow[e] = 0.0;
+            for (int h = 0; h < H; ++h) {
+                const double *q = qc + (c * H + h) * dqk;
+                double *oh = orow + h * dv;
+                /* history tokens j < n, relative position n - j */
+                for (int j = 0; j < n; ++j) {
+                    double S = ref_dot(q, k_hist + ((s + j) * H + h) * dqk, dqk);
+                    if (p->rab_pos) S += p->rab_pos[h * (2 * L - 1) + (n - j) + L - 1];
+                    if (p->rab_time)
+                        S += p->rab_time[h * NB + hstu_ref_time_bucket(cand_ts[c] - p->timestamps[s + j],
+                                                                       p->num_time_buckets)];
+                    const double A = ref_silu(S) / Nn;
+                    const double *vj = v_hist + ((s + j) * H + h) * dv;
+                    for (int e = 0; e < dv; ++e) oh[e] += A * vj[e];
+                }
+                /* the candidate itself: relative position 0, time difference 0 */
+                double S = ref_dot(q, kc + (c * H + h) * dqk, dqk);
+                if (p->rab_pos) S += p->rab_pos[h * (2 * L - 1) + L - 1];
+                if (p->rab_time) S += p->rab_time[h * NB + hstu_ref_time_bucket(0, p->num_time_buckets)];
+                const double A = ref_silu(S) / Nn;
+                const double *vs = vc + (c * H + h) * dv;
+                for (int e = 0; e < dv; ++e) oh[e] += A * vs[e];
+            }
+            double mu = 0.0;
+            for (int e = 0; e < D; ++e) mu += orow[e];
+            mu /= (double)D;
+            double var = 0.0;
+            for (int e = 0; e < D; ++e) var += (orow[e] - mu) * (orow[e] - mu);
+            var /= (double)D;
+            const double rs = 1.0 / sqrt(var + p->ln_eps);
+            for (int e = 0; e < D; ++e) {
+                const double w = p->ln_weight ? p->ln_weight[e] : 1.0;
+                const double bb = p->ln_bias ? p->ln_bias[e] : 0.0;
+                y[c * D + e] = ((orow[e] - mu) * rs * w + bb) * ref_silu(uc[c * D + e]);
+                if (o) o[c * D + e] = orow[e];
+            }
+            if (mean) mean[c] = mu;
+            if (rstd) rstd[c] = rs;
+        }
+        free(orow);
+    }
+    return 0;
+}

@@ -78,6 +78,18 @@ int hstu_ref_out(int64_t T, int32_t E, int32_t Dy, const double *y, const double
                  const double *w, const double *b, const double *gamma, const double *beta,
                  double eps, double *z, double *mean, double *rstd);
 
+/* Candidate scoring against a cached history (M-FALCON).  p describes the
+ * history: offsets [B+1] over T_h history tokens, timestamps [T_h].  k_hist
+ * [T_h,H,dqk], v_hist [T_h,H,dv]; cand_offsets [B+1] over C candidates with
+ * timestamps cand_ts [C] (or NULL without a time table); qc, kc [C,H,dqk],
+ * vc [C,H,dv], uc [C,H*dv].  Candidate c of user b attends to the user's
+ * history and to itself only, as row n_b of (history, c).  Writes y
+ * [C,H*dv]; o [C,H*dv], mean, rstd [C] when non-NULL. */
+int hstu_ref_mfalcon(const hstu_ref_problem *p, const double *k_hist, const double *v_hist,
+                     const int32_t *cand_offsets, const int64_t *cand_ts, const double *qc,
+                     const double *kc, const double *vc, const double *uc, double *y,
+                     double *o, double *mean, double *rstd, int num_threads);
+
 #ifdef __cplusplus
 }
 #endif

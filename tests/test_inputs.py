@@ -87,3 +87,22 @@ def test_train_sl_workload_lengths():
     o = inp.offsets.numpy()
     for b in range(spec.batch):
         assert np.all(np.diff(t[o[b]:o[b + 1]]) > 0)
+
+
+def test_candidate_inputs_follow_their_history():
+    sp = hi.workload("jagged", batch=5, len_range=(0, 40), heads=2, rab_pos_len=41)
+    a = hi.make_cand_inputs(sp, (0, 6), seed=3)
+    b = hi.make_cand_inputs(sp, (0, 6), seed=3)
+    assert a.counts == b.counts and torch.equal(a.qc, b.qc) and torch.equal(a.cand_ts, b.cand_ts)
+    assert a.qc.shape == (a.total_cands, 2, 128) and a.uc.shape == (a.total_cands, 256)
+    ho, co = a.hist.offsets.tolist(), a.cand_offsets.tolist()
+    for u in range(5):
+        last = int(a.hist.timestamps[ho[u + 1] - 1]) if ho[u + 1] > ho[u] else None
+        for c in range(co[u], co[u + 1]):
+            if last is not None:
+                assert int(a.cand_ts[c]) > last       # requests come after the history
+    # the history part is exactly the ordinary problem of the same seed
+    h = hi.make_inputs(sp, seed=3)
+    assert torch.equal(h.k, a.hist.k) and torch.equal(h.timestamps, a.hist.timestamps)
+    spec, n = hi.CAND_WORKLOADS["mfalcon"]
+    assert spec.rab_pos_len >= spec.len_range[1] + 1 and n == 512

@@ -440,3 +440,100 @@ def test_out_proj_closed_forms(oracle_lib):
     var = x.var(axis=1)
     assert np.abs(z.mean(axis=1)).max() < 1e-13
     assert np.abs(z.var(axis=1) - var / (var + 1e-5)).max() < 1e-12
+
+
+# ---------------------------------------------------------------- M-FALCON
+def cand_case(lengths=(5, 0, 12), counts=(3, 2, 4), H=3, dqk=6, dv=4, rab_pos=True,
+              rab_time=True, norm="own", norm_len=0, seed=0, ln_affine=False):
+    """Histories from small_inputs (position table long enough for relative
+    position n_b) and per-user candidates with request times after the history."""
+    hist = small_inputs(lengths=lengths, H=H, dqk=dqk, dv=dv, rab_pos=rab_pos,
+                        rab_time=rab_time, norm=norm, norm_len=norm_len, seed=seed,
+                        L=max(lengths) + 1, ln_affine=ln_affine, grad=False)
+    g = torch.Generator().manual_seed(seed + 50)
+    C = sum(counts)
+    offs = [0]
+    for c in counts:
+        offs.append(offs[-1] + c)
+    qc = torch.randn(C, H, dqk, generator=g) * 0.7
+    kc = torch.randn(C, H, dqk, generator=g) * 0.7
+    vc = torch.randn(C, H, dv, generator=g)
+    uc = torch.randn(C, H * dv, generator=g)
+    cts = None
+    if rab_time:
+        ho = hist.offsets.tolist()
+        cts = []
+        for b, c in enumerate(counts):
+            last = int(hist.timestamps[ho[b + 1] - 1]) if ho[b + 1] > ho[b] else 1_700_000_000
+            cts.append(last + torch.randint(0, 5000, (c,), generator=g).to(torch.int64))
+        cts = torch.cat(cts)
+    return hi.CandInputs(hist, torch.tensor(offs, dtype=torch.int32), qc, kc, vc, uc, cts)
+
+
+def history_plus(ci, c):
+    """The problem (history of c's user, then c) as one sequence."""
+    h = ci.hist
+    b = int(np.searchsorted(ci.cand_offsets.numpy(), c, side="right")) - 1
+    s, e = int(h.offsets[b]), int(h.offsets[b + 1])
+    cat = lambda a, x: torch.cat([a[s:e], x[c:c + 1]])
+    ts = None if h.timestamps is None else cat(h.timestamps, ci.cand_ts)
+    return hi.Inputs(h.spec, torch.tensor([0, e - s + 1], dtype=torch.int32),
+                     cat(h.q, ci.qc), cat(h.k, ci.kc), cat(h.v, ci.vc), cat(h.u, ci.uc), ts,
+                     h.rab_pos, h.rab_time, None, h.norm_len, h.rab_pos_len, h.ln_weight,
+                     h.ln_bias)
+
+
+@pytest.mark.parametrize("case", [
+    dict(), dict(norm="fixed", norm_len=9), dict(rab_time=False), dict(rab_pos=False),
+    dict(ln_affine=True), dict(lengths=(1, 7), counts=(5, 0), H=1),
+])
+def test_mfalcon_is_the_token_after_the_history(oracle_lib, case):
+    """Each candidate's output equals the last row of the causal forward on
+    (its user's history, the candidate): position n_b, its own time, the
+    normaliser of that sequence (the reading of M-FALCON scoring)."""
+    ci = cand_case(**case)
+    got = oracle_lib.mfalcon(ci)
+    for c in range(ci.total_cands):
+        ref = oracle_lib.fwd(history_plus(ci, c))
+        assert rel_err(got["o"][c], ref["o"][-1]) < 1e-12
+        assert rel_err(got["y"][c], ref["y"][-1]) < 1e-12
+        assert abs(got["rstd"][c] - ref["rstd"][-1]) <= 1e-12 * ref["rstd"][-1]
+
+
+def test_mfalcon_empty_history_closed_form(oracle_lib):
+    """With no history a candidate attends to itself only:
+    O = SiLU(q.k + rab_pos[L-1] + rab_time[bucket 0]) / N * v, N = 1 (own length)."""
+    ci = cand_case(lengths=(0, 4), counts=(3, 1))
+    got = oracle_lib.mfalcon(ci)
+    h = ci.hist
+    L = h.rab_pos_len
+    for c in range(3):
+        for hh in range(3):
+            x = float(ci.qc[c, hh].double() @ ci.kc[c, hh].double())
+            x += float(h.rab_pos[hh, L - 1]) + float(h.rab_time[hh, 0])
+            silu = x / (1.0 + math.exp(-x))
+            want = silu * ci.vc[c, hh].double().numpy()
+            np.testing.assert_allclose(got["o"][c, hh * 4:(hh + 1) * 4], want, rtol=1e-13,
+                                       atol=1e-15)
+
+
+def test_mfalcon_candidates_do_not_see_each_other(oracle_lib):
+    """Changing one candidate leaves every other candidate's output bitwise
+    unchanged, and reordering a user's candidates reorders the outputs."""
+    ci = cand_case()
+    base = oracle_lib.mfalcon(ci)
+    ci2 = cand_case()
+    for t in (ci2.qc, ci2.kc, ci2.vc, ci2.uc):
+        t[1] += 3.0
+    if ci2.cand_ts is not None:
+        ci2.cand_ts[1] += 10 ** 6
+    pert = oracle_lib.mfalcon(ci2)
+    keep = [c for c in range(ci.total_cands) if c != 1]
+    assert np.array_equal(base["y"][keep], pert["y"][keep])
+    assert not np.array_equal(base["y"][1], pert["y"][1])
+    perm = torch.tensor([2, 0, 1, 3, 4, 8, 6, 5, 7])
+    ci3 = cand_case()
+    ci3.qc, ci3.kc, ci3.vc, ci3.uc = (t[perm] for t in (ci3.qc, ci3.kc, ci3.vc, ci3.uc))
+    ci3.cand_ts = ci3.cand_ts[perm]
+    got = oracle_lib.mfalcon(ci3)
+    assert np.array_equal(got["y"], base["y"][perm.numpy()])

@@ -98,6 +98,20 @@ MUTANTS = [
      "if (pp) pp[(i - j) + L - 1] += dS;", "if (pp) pp[(j - i) + L - 1] += dS;", 0),
     ("time gradient one bucket low",
      "tp[bk] += dS;", "tp[bk > 0 ? bk - 1 : 0] += dS;", 0),
+    # candidate scoring against a cached history
+    ("candidate position one step short",
+     "S += p->rab_pos[h * (2 * L - 1) + (n - j) + L - 1];",
+     "S += p->rab_pos[h * (2 * L - 1) + (n - 1 - j) + L - 1];", 0),
+    ("candidate normaliser without the candidate",
+     "const double Nn = p->norm_len > 0 ? (double)p->norm_len : (double)(n + 1);",
+     "const double Nn = p->norm_len > 0 ? (double)p->norm_len : (double)(n > 0 ? n : 1);", 0),
+    ("candidate self term dropped",
+     "for (int e = 0; e < dv; ++e) oh[e] += A * vs[e];", "(void)vs;", 0),
+    ("candidate time measured from the first event",
+     "cand_ts[c] - p->timestamps[s + j]", "cand_ts[c] - p->timestamps[s]", 0),
+    ("candidate self term at relative position 1",
+     "if (p->rab_pos) S += p->rab_pos[h * (2 * L - 1) + L - 1];",
+     "if (p->rab_pos) S += p->rab_pos[h * (2 * L - 1) + L];", 0),
 ]
 
 # The same mistake in the forward and the backward: (name, [(text, replacement)]),
@@ -142,7 +156,17 @@ PINS = [
     T.test_layernorm_affine_closed_forms,
     T.test_uvqk_closed_forms,
     T.test_out_proj_closed_forms,
+    T.test_mfalcon_empty_history_closed_form,
+    T.test_mfalcon_candidates_do_not_see_each_other,
 ]
+
+
+def _mfalcon_history_pin(o):
+    for case in ({}, {"norm": "fixed", "norm_len": 9}, {"rab_pos": False}):
+        T.test_mfalcon_is_the_token_after_the_history(o, case)
+
+
+PINS.append(_mfalcon_history_pin)
 
 
 def _plant(text, old, new, occurrence):
