@@ -226,6 +226,40 @@ HSTU_API hstu_status_t hstu_out_fwd(int32_t T, int32_t E, int32_t D, const void 
                                     float *rstd, void *workspace, size_t workspace_bytes,
                                     void *stream);
 
+/*
+ * Candidate scoring against cached histories (M-FALCON: "HSTU Hierarchical
+ * Sequential Transduction Units", §6 Why it works, micro-batched candidate
+ * scoring with key/value reuse; the pages print no formula).  Reading taken:
+ * candidate c of user b is the token that follows the user's n_b history
+ * tokens, on its own -- it attends to every history token j < n_b (relative
+ * position n_b - j, time bucket of t_c - t_j) and to itself (relative
+ * position 0, time difference 0), never to another candidate; the
+ * normaliser is norm_len (> 0) or n_b + 1.  Y_c is thus the last row of
+ * hstu_attn_fwd over the sequence (history of b, c).  Each history key and
+ * value tile is read once per micro-batch of 128 candidates and head.
+ *
+ * p describes the histories: batch, total_tokens (history tokens T_h),
+ * max_seq_len (>= every n_b), offsets, timestamps (history), the bias tables
+ * (rab_pos_len >= max_seq_len + 1, as a candidate sits at position n_b),
+ * norm_len, ln_eps, ln_weight/ln_bias.  k_hist, v_hist [T_h, H, 128]: the
+ * cached keys and values.  cand_offsets device int32 [B+1] over total_cands
+ * candidates (at most max_cands per user); cand_timestamps device int64
+ * [total_cands] (required with rab_time).  q, k, v [C, H, 128], u [C, H*128]:
+ * the candidates' projections; y [C, H*128] output.  Supported: bf16,
+ * d_qk = d_v = 128, 1 <= H <= 16.  workspace: hstu_cand_workspace_size bytes,
+ * 256-byte aligned, zero-filled before its first use (its per-micro-batch
+ * counters return to zero after each call); candidate offsets found
+ * inconsistent on the device are reported by hstu_attn_check.
+ */
+HSTU_API size_t hstu_cand_workspace_size(const hstu_problem_t *p, int32_t total_cands,
+                                         int32_t max_cands);
+HSTU_API hstu_status_t hstu_cand_fwd(const hstu_problem_t *p, const void *k_hist,
+                                     const void *v_hist, const int32_t *cand_offsets,
+                                     int32_t total_cands, int32_t max_cands,
+                                     const int64_t *cand_timestamps, const void *q, const void *k,
+                                     const void *v, const void *u, void *y, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,8 @@ HSTU_F32, HSTU_BF16 = 0, 1
 
 EXPORTED = ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_attn_check",
             "hstu_status_string", "hstu_time_bucket_thresholds", "hstu_selftest_wait_timeout",
-            "hstu_attn_bwd_noalloc", "hstu_uvqk_fwd", "hstu_out_fwd")
+            "hstu_attn_bwd_noalloc", "hstu_uvqk_fwd", "hstu_out_fwd", "hstu_cand_workspace_size",
+            "hstu_cand_fwd")
 
 
 class HSTUError(RuntimeError):
@@ -90,6 +91,10 @@ def load_library():
     lib.hstu_uvqk_fwd.restype = ctypes.c_int
     lib.hstu_out_fwd.argtypes = [i32] * 3 + [vp] * 6 + [ctypes.c_float] + [vp] * 3 + [vp, sz, vp]
     lib.hstu_out_fwd.restype = ctypes.c_int
+    lib.hstu_cand_workspace_size.argtypes = [P, i32, i32]
+    lib.hstu_cand_workspace_size.restype = sz
+    lib.hstu_cand_fwd.argtypes = [P, vp, vp, vp, i32, i32] + [vp] * 6 + [vp, sz, vp]
+    lib.hstu_cand_fwd.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -327,3 +332,42 @@ def hstu_out_fwd(y, w, x, *, bias=None, ln_weight=None, ln_bias=None, eps: float
     if rc != HSTU_OK:
         raise HSTUError(rc, "hstu_out_fwd")
     return z, stats
+
+
+def hstu_cand_fwd(k_hist, v_hist, offsets, max_seq_len, q, k, v, u, cand_offsets,
+                  max_cands: int, *, timestamps=None, cand_timestamps=None, rab_pos=None,
+                  rab_time=None, norm_len=0, eps=1e-5, ln_weight=None, ln_bias=None,
+                  offsets_host=None, y=None, workspace=None, stream=None):
+    """Candidate scoring against cached histories (M-FALCON): every candidate
+    of user b attends to b's history (k_hist, v_hist [T_h, H, 128], offsets)
+    and to itself.  q, k, v [C, H, 128], u [C, H*128] (bf16); cand_offsets
+    int32 [B+1].  Returns y [C, H*128]."""
+    lib = load_library()
+    for name, t in (("k_hist", k_hist), ("v_hist", v_hist), ("q", q), ("k", k), ("v", v),
+                    ("u", u)):
+        _dev(t, name, torch.bfloat16)
+    _dev(offsets, "offsets", torch.int32)
+    _dev(cand_offsets, "cand_offsets", torch.int32)
+    _dev(timestamps, "timestamps", torch.int64)
+    _dev(cand_timestamps, "cand_timestamps", torch.int64)
+    for name, t in (("rab_pos", rab_pos), ("rab_time", rab_time), ("ln_weight", ln_weight),
+                    ("ln_bias", ln_bias)):
+        _dev(t, name, torch.float32)
+    p = make_problem(k_hist, v_hist, offsets, max_seq_len, timestamps, rab_pos, rab_time,
+                     norm_len, eps, offsets_host, ln_weight, ln_bias)
+    C, H, _ = q.shape
+    if y is None:
+        y = torch.empty((C, H * v.shape[-1]), dtype=q.dtype, device=q.device)
+    _dev(y, "y", q.dtype)
+    if workspace is None:
+        n = int(lib.hstu_cand_workspace_size(ctypes.byref(p), int(C), int(max_cands)))
+        if n == 0:
+            raise HSTUError(HSTU_ERR_INVALID_ARG, "hstu_cand_workspace_size")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=q.device)
+    rc = lib.hstu_cand_fwd(ctypes.byref(p), _ptr(k_hist), _ptr(v_hist), _ptr(cand_offsets),
+                           int(C), int(max_cands), _ptr(cand_timestamps), _ptr(q), _ptr(k),
+                           _ptr(v), _ptr(u), _ptr(y), _ptr(workspace), workspace.numel(),
+                           _stream_ptr(stream))
+    if rc != HSTU_OK:
+        raise HSTUError(rc, "hstu_cand_fwd")
+    return y

@@ -505,4 +505,84 @@ hstu_status_t hstu_out_fwd(int32_t T, int32_t E, int32_t D, const void* y, const
   return err == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
+// ---------------------------------------------------------- candidate scoring
+static size_t cand_tiles(int32_t max_cands) { return (static_cast<size_t>(max_cands) + 127) / 128; }
+
+size_t hstu_cand_workspace_size(const hstu_problem_t* p, int32_t total_cands, int32_t max_cands) {
+  if (check_problem(p) != HSTU_OK || total_cands < 0 || max_cands < 0) return 0;
+  return kStatusBytes + align_up(static_cast<size_t>(p->batch) * cand_tiles(max_cands) * 4) +
+         align_up(static_cast<size_t>(total_cands) * p->num_heads * p->d_v * 4);
+}
+
+hstu_status_t hstu_cand_fwd(const hstu_problem_t* p, const void* k_hist, const void* v_hist,
+                            const int32_t* cand_offsets, int32_t total_cands, int32_t max_cands,
+                            const int64_t* cand_timestamps, const void* q, const void* k,
+                            const void* v, const void* u, void* y, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  NvtxRange range("hstu_cand_fwd");
+  hstu_status_t st = check_problem(p);
+  if (st != HSTU_OK) return st;
+  if (total_cands < 0 || max_cands < 0 || (total_cands > 0 && max_cands < 1))
+    return HSTU_ERR_INVALID_ARG;
+  if (p->batch > 0 && !cand_offsets) return HSTU_ERR_INVALID_ARG;
+  if (p->rab_pos && p->rab_pos_len < p->max_seq_len + 1) return HSTU_ERR_INVALID_ARG;
+  if (p->rab_time && total_cands > 0 && !cand_timestamps) return HSTU_ERR_INVALID_ARG;
+  if (total_cands > 0) {
+    const void* ptrs[] = {q, k, v, u, y};
+    for (const void* x : ptrs)
+      if (!x || !aligned16(x)) return HSTU_ERR_INVALID_ARG;
+  }
+  if (p->total_tokens > 0 && (!k_hist || !v_hist || !aligned16(k_hist) || !aligned16(v_hist)))
+    return HSTU_ERR_INVALID_ARG;
+  if (p->dtype != HSTU_BF16 || p->d_qk != 128 || p->d_v != 128 || p->num_heads > 16)
+    return HSTU_ERR_UNSUPPORTED;
+  if (static_cast<uint64_t>(p->batch) * cand_tiles(max_cands) > 0x7FFFFFFFull)
+    return HSTU_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
+      workspace_bytes < hstu_cand_workspace_size(p, total_cands, max_cands))
+    return HSTU_ERR_WORKSPACE;
+  if (p->batch == 0 || total_cands == 0) return HSTU_OK;
+
+  FwdArgs common;
+  std::memset(&common, 0, sizeof(common));
+  fill_common(p, static_cast<int*>(workspace), &common);
+  CandArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.offsets = p->offsets;
+  a.cand_offsets = cand_offsets;
+  a.timestamps = p->timestamps;
+  a.cand_ts = cand_timestamps;
+  a.rab_pos = p->rab_pos;
+  a.rab_time = p->rab_time;
+  a.q = q; a.k = k; a.v = v; a.u = u; a.y = y;
+  a.ln_weight = p->ln_weight;
+  a.ln_bias = p->ln_bias;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t cnt_bytes = align_up(static_cast<size_t>(p->batch) * cand_tiles(max_cands) * 4);
+  a.cnt = reinterpret_cast<unsigned*>(ws + kStatusBytes);
+  a.o_ws = reinterpret_cast<float*>(ws + kStatusBytes + cnt_bytes);
+  a.status = static_cast<int*>(workspace);
+  a.B = p->batch;
+  a.T = p->total_tokens;
+  a.C = total_cands;
+  a.H = p->num_heads;
+  a.max_tiles = static_cast<int>(cand_tiles(max_cands));
+  a.max_seq_len = p->max_seq_len;
+  a.L = common.L;
+  a.nb = common.nb;
+  a.norm_len = p->norm_len;
+  a.eps = p->ln_eps;
+  a.bt = common.bt;
+  CUtensorMap tq, tk, tv;
+  // With no history at all the key and value maps are never read; they are
+  // encoded over the candidates so that they stay valid.
+  const bool hist = p->total_tokens > 0;
+  if (!make_map_3d(&tq, q, total_cands, p->num_heads, 128) ||
+      !make_map_3d(&tk, hist ? k_hist : k, hist ? p->total_tokens : total_cands, p->num_heads, 128) ||
+      !make_map_3d(&tv, hist ? v_hist : v, hist ? p->total_tokens : total_cands, p->num_heads, 128))
+    return HSTU_ERR_CUDA;
+  const cudaError_t err = launch_cand_sm100(a, tq, tk, tv, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -124,6 +124,32 @@ struct ProjArgs {
   float eps;
 };
 
+// Arguments of the candidate-scoring kernel (scoring against cached histories).
+struct CandArgs {
+  const int32_t* offsets;        // history [B+1]
+  const int32_t* cand_offsets;   // candidates [B+1]
+  const int64_t* timestamps;     // history [T] (with a time table)
+  const int64_t* cand_ts;        // candidates [C] (with a time table)
+  const float* rab_pos;          // [H, 2L-1] or nullptr
+  const float* rab_time;         // [H, nb] or nullptr
+  const void* q;                 // candidates [C, H, 128] bf16 (also read through TMA)
+  const void* k;                 // candidates [C, H, 128]
+  const void* v;                 // candidates [C, H, 128]
+  const void* u;                 // candidates [C, H*128]
+  void* y;                       // candidates [C, H*128]
+  const float* ln_weight;        // [H*128] or nullptr
+  const float* ln_bias;
+  float* o_ws;                   // workspace: O / N per candidate [C, H*128] fp32
+  unsigned* cnt;                 // workspace: head CTAs done per (user, micro-batch)
+  int* status;
+  int B, T, C, H;
+  int max_tiles;                 // micro-batches per user in the grid
+  int max_seq_len;
+  int L, nb, norm_len;
+  float eps;
+  BucketTable bt;
+};
+
 // The synchronous argument checks of hstu_attn_bwd (all but the workspace's).
 hstu_status_t check_bwd_args(const hstu_problem_t* p, const void* dy, const void* q,
                              const void* k, const void* v, const void* u, const float* o_save,
@@ -139,6 +165,8 @@ cudaError_t launch_fwd_f32_simt(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_f32_simt(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_bf16_simt(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_pre_bf16(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_cand_sm100(const CandArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, cudaStream_t stream);
 cudaError_t launch_uvqk_sm100(const ProjArgs& a, const CUtensorMap& tx, const CUtensorMap& tw,
                               cudaStream_t stream);
 cudaError_t launch_out_sm100(const ProjArgs& a, const CUtensorMap& ty, const CUtensorMap& tw,

@@ -285,3 +285,37 @@ def test_out_rejections(lib):
     assert call_out(lib, D=100) == 2
     assert call_out(lib, ws=None) == 5
     assert call_out(lib, T=0) == 0
+
+
+def call_cand(lib, p, C=300, maxc=200, cand_off=FAKE, cts=FAKE, q=FAKE, kh=FAKE, ws=FAKE,
+              ws_bytes=1 << 24):
+    so = lib.load_library()
+    vp = ctypes.c_void_p
+    opt = lambda a: vp(a) if a else None
+    return so.hstu_cand_fwd(ctypes.byref(p), opt(kh), vp(FAKE), opt(cand_off), C, maxc, opt(cts),
+                            opt(q), vp(FAKE), vp(FAKE), vp(FAKE), vp(FAKE), opt(ws), ws_bytes,
+                            None)
+
+
+def test_cand_rejections(lib):
+    p, _ = problem(lib, rab_pos=FAKE, rab_pos_len=201)
+    so = lib.load_library()
+    need = so.hstu_cand_workspace_size(ctypes.byref(p), 300, 200)
+    # status + 2 users x 2 micro-batch counters + O staging (300 x 512 fp32)
+    assert need >= 256 + 300 * 4 * 128 * 4
+    assert call_cand(lib, p, C=-1) == 1
+    assert call_cand(lib, p, maxc=0) == 1                     # candidates but no per-user bound
+    assert call_cand(lib, p, cand_off=None) == 1
+    assert call_cand(lib, p, q=FAKE + 8) == 1
+    assert call_cand(lib, p, kh=None) == 1
+    p2, _ = problem(lib, rab_pos=FAKE, rab_pos_len=200)     # position n_b = 200 not in the table
+    assert call_cand(lib, p2) == 1
+    p3, _ = problem(lib, rab_time=FAKE, timestamps=FAKE, num_time_buckets=128)
+    assert call_cand(lib, p3, cts=None) == 1                  # time table without request times
+    p4, _ = problem(lib, d_qk=64, d_v=64)
+    assert call_cand(lib, p4) == 2
+    p5, _ = problem(lib, dtype=0)
+    assert call_cand(lib, p5) == 2
+    assert call_cand(lib, p, ws=None) == 5
+    assert call_cand(lib, p, ws_bytes=need - 1) == 5
+    assert call_cand(lib, p, C=0) == 0                        # nothing to score
