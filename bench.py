@@ -243,29 +243,35 @@ def bench_config(spec, inp, world: int) -> dict:
 
 
 # ----------------------------------------------------------------- oracle arm
-def _row_sample(inp, stride: int):
-    rows, fl = [], 0
+def _row_sample(inp, nrows: int, seed: int = 0):
+    """nrows token rows drawn uniformly (seeded, without replacement) over the
+    whole packed token axis, and their forward FLOPs.  Row i of a sequence
+    costs i + 1 columns, so a uniform sample keeps the workload's mix of short
+    and long rows and its FLOP rate stands for the whole."""
+    import numpy as np
+    T = inp.total_tokens
+    nrows = max(1, min(int(nrows), T))
+    g = torch.Generator().manual_seed(seed)
+    rows = torch.randperm(T, generator=g)[:nrows].sort().values.numpy().astype(np.int64)
+    offs = inp.offsets.numpy()
+    seq = np.searchsorted(offs, rows, side="right") - 1
+    local = rows - offs[seq]
     H, dqk, dv = inp.q.shape[1], inp.q.shape[2], inp.v.shape[2]
-    for b, n in enumerate(inp.lengths):
-        s = int(inp.offsets[b])
-        for i in range(0, n, stride):
-            rows.append(s + i)
-            fl += 2 * (i + 1) * H * (dqk + dv)      # row i of a sequence: i+1 columns
+    fl = int(2 * (local + 1).sum() * H * (dqk + dv))
     return rows, fl
 
 
 def oracle_step_sample(inp, budget_s: float, threads: int):
     """Times the oracle forward on `threads` host threads: the whole workload
-    if it fits in the budget, else every stride-th row (stride from a small
-    probe); returns (flops, seconds, description, extrapolated)."""
-    import numpy as np
+    if it fits in the budget, else a uniform random sample of its rows sized
+    from a small probe; returns (flops, seconds, description, extrapolated)."""
     import oracle
     oracle.build()
     flops_full = hi.causal_flops(inp.lengths, inp.q.shape[1], inp.q.shape[2], inp.v.shape[2])
-    probe_stride = max(1, int(math.ceil(flops_full / (2e9 if threads > 1 else 2e8))))
-    rows, fl = _row_sample(inp, probe_stride)
+    per_row = flops_full / max(inp.total_tokens, 1)
+    rows, fl = _row_sample(inp, math.ceil((2e9 if threads > 1 else 2e8) / per_row), seed=1)
     t0 = time.perf_counter()
-    oracle.fwd_rows(inp, np.array(rows, dtype=np.int64), threads=threads)
+    oracle.fwd_rows(inp, rows, threads=threads)
     rate = fl / max(time.perf_counter() - t0, 1e-9)
     if flops_full / rate <= budget_s:
         reps, total = 0, 0.0
@@ -275,12 +281,12 @@ def oracle_step_sample(inp, budget_s: float, threads: int):
             total += time.perf_counter() - t0
             reps += 1
         return flops_full * reps, total, "full workload forward x%d" % reps, False
-    stride = max(1, int(math.ceil(flops_full / rate / budget_s)))
-    rows, fl = _row_sample(inp, stride)
+    rows, fl = _row_sample(inp, math.ceil(rate * budget_s / per_row), seed=2)
     t0 = time.perf_counter()
-    oracle.fwd_rows(inp, np.array(rows, dtype=np.int64), threads=threads)
-    return fl, time.perf_counter() - t0, "every %d-th row of the workload (%d rows)" % (
-        stride, len(rows)), True
+    oracle.fwd_rows(inp, rows, threads=threads)
+    return fl, time.perf_counter() - t0, (
+        "%d token rows drawn uniformly from the workload's %d (forward, every head)"
+        % (len(rows), inp.total_tokens)), True
 
 
 def cpu_baseline(inp, budget_all: float, budget_single: float) -> dict:
@@ -608,6 +614,52 @@ def measure_proj(T: int, steps: int, device, world: int):
     return result
 
 
+def measure_cand(name: str, steps: int, device, world: int, seed: int):
+    """Candidate scoring against cached histories (M-FALCON reading) on the
+    named candidate workload, one call per step from a CUDA graph (the
+    histories' keys and values, over 300 MB, exceed the L2)."""
+    import ctypes
+    import pointwise_attention_b200 as pa
+    peaks, peak_kind = load_peaks()
+    sp, ncand = hi.CAND_WORKLOADS[name]
+    ci = hi.make_cand_inputs(sp, ncand, seed=seed)
+    h = ci.hist
+    d = lambda t: None if t is None else t.to(device)
+    args = [d(h.k), d(h.v), d(h.offsets), max(h.lengths), d(ci.qc), d(ci.kc), d(ci.vc),
+            d(ci.uc), d(ci.cand_offsets), max(ci.counts)]
+    kw = dict(timestamps=d(h.timestamps), cand_timestamps=d(ci.cand_ts), rab_pos=d(h.rab_pos),
+              rab_time=d(h.rab_time), norm_len=h.norm_len)
+    p = pa.make_problem(args[0], args[1], args[2], args[3], kw["timestamps"], kw["rab_pos"],
+                        kw["rab_time"], h.norm_len)
+    n = pa.load_library().hstu_cand_workspace_size(ctypes.byref(p), ci.total_cands,
+                                                    max(ci.counts))
+    ws = torch.zeros(n, dtype=torch.uint8, device=device)
+    y = pa.hstu_cand_fwd(*args, workspace=ws, **kw)
+
+    def fn(i, stream=None):
+        pa.hstu_cand_fwd(*args, y=y, workspace=ws, stream=stream, **kw)
+
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    t, _ = time_graphs(steps, 1, fn, stream, world)
+    t = reduce_max(t, world, device) / steps
+    if pa.hstu_attn_check(ws) != 0:
+        raise RuntimeError("device status after the candidate-scoring timing")
+    # each candidate: n_b history keys and itself, H heads, d_qk + d_v
+    flops = 2.0 * sum(c * (nb + 1) for c, nb in zip(ci.counts, h.lengths)) * sp.heads * (
+        sp.d_qk + sp.d_v)
+    roof = {"bound": "tensor", "achieved": flops / t / 1e12, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "kernel": "hstu_cand_sm100", "peak_source": peak_kind + " burst",
+            "algorithmic_flops": flops, "us_per_launch": t * 1e6, "traffic": None}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    return {"workload": name, "users": sp.batch, "candidates_per_user": ncand,
+            "history_tokens": h.total_tokens, "value": roof["achieved"], "unit": "TFLOP/s",
+            "ms_per_step": t * 1e3, "steps_timed": steps, "roofline": roof}
+
+
 def summary_of(spec, res, world):
     roof = dict(res["roofline"])
     return {"workload": spec.name, "value": res["value"], "unit": "TFLOP/s",
@@ -640,6 +692,11 @@ def run_gpu(args, spec):
     for name in [x for x in args.also.split(",") if x and x != spec.name]:
         if name == "proj":
             also[name] = measure_proj(131072, args.also_steps, device, world)
+            torch.cuda.empty_cache()
+            continue
+        if name in hi.CAND_WORKLOADS:
+            also[name] = measure_cand(name, args.also_steps, device, world,
+                                      rank_seed(args.seed, rank))
             torch.cuda.empty_cache()
             continue
         sp = hi.WORKLOADS[name]
@@ -693,7 +750,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--also", default="long,train,proj",
+    ap.add_argument("--also", default="long,train,proj,mfalcon",
                     help="comma-separated workloads timed after the main one, 'proj' for the "
                          "projection GEMMs ('' for none)")
     ap.add_argument("--also-steps", type=int, default=50)
