@@ -273,22 +273,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32_nowait(saddr, sv);
       tmem_wait_ld_dep(sv);
       const int nvalid = nb - (128 * n + 32 * cs);   // columns of this chunk that are history keys
+      // Time bias plan of the chunk: |t_c - t_j| is monotone in t_j, so when
+      // the bucket of this row's smallest and largest |dt| over the chunk's
+      // keys agree (the usual case: the history is in time order and buckets
+      // widen logarithmically) one bias serves all 32 columns.
+      float tconst = 0.f;
+      bool cst = true;
+      if (TIME && nvalid > 0) {
+        long long kmn = jv ? kts : 0x7FFFFFFFFFFFFFFFll, kmx = jv ? kts : -0x7FFFFFFFFFFFFFFFll;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+          kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+        }
+        const long long dlo = my_ts - kmx, dhi = my_ts - kmn;
+        cst = false;
+        if (dlo >= 0 || dhi <= 0) {
+          const int k0 = time_bucket(dlo, s_thr, s_first), k1 = time_bucket(dhi, s_thr, s_first);
+          cst = k0 == k1;
+          tconst = s_rabt[k0];
+        }
+      }
       uint32_t packed[16];
+      if (!TIME || __all_sync(0xffffffffu, cst)) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float p2[2];
+        for (int i = 0; i < 16; ++i) {
+          float p2[2];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = 2 * i + e;
-          float x = __uint_as_float(sv[c]);
-          if (POS) x += __shfl_sync(0xffffffffu, pb, c);
-          if (TIME) {
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * i + e;
+            float x = __uint_as_float(sv[c]) + tconst;
+            if (POS) x += __shfl_sync(0xffffffffu, pb, c);
+            p2[e] = c < nvalid ? silu_t(x) : 0.f;   // keys past the history: exactly 0
+          }
+          packed[i] = pack2(p2[0], p2[1]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float p2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * i + e;
+            float x = __uint_as_float(sv[c]);
+            if (POS) x += __shfl_sync(0xffffffffu, pb, c);
             const long long kt = __shfl_sync(0xffffffffu, kts, c);
             x += s_rabt[time_bucket(my_ts - kt, s_thr, s_first)];
+            p2[e] = c < nvalid ? silu_t(x) : 0.f;
           }
-          p2[e] = c < nvalid ? silu_t(x) : 0.f;   // keys past the history: exactly 0
+          packed[i] = pack2(p2[0], p2[1]);
         }
-        packed[i] = pack2(p2[0], p2[1]);
       }
       tmem_st16(saddr, packed);   // over this warp's own S columns, already read
       tmem_wait_st();

@@ -396,12 +396,13 @@ hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void*
   a.bt = common.bt;
   cudaError_t err;
   if (p->dtype == HSTU_BF16) {
-    CUtensorMap maps[4];
-    if (!make_map_3d(&maps[0], q, p->total_tokens, p->num_heads, 128) ||
-        !make_map_3d(&maps[1], k, p->total_tokens, p->num_heads, 128) ||
-        !make_map_3d(&maps[2], v, p->total_tokens, p->num_heads, 128) ||
-        !make_map_3d(&maps[3], a.dO, p->total_tokens, p->num_heads, 128))
-      return HSTU_ERR_CUDA;
+    // q, k, v, dO with 128-row boxes (resident tiles), then 64-row boxes
+    // (the sub-tile rings)
+    CUtensorMap maps[8];
+    const void* src[4] = {q, k, v, a.dO};
+    for (int i = 0; i < 8; ++i)
+      if (!make_map_3d(&maps[i], src[i & 3], p->total_tokens, p->num_heads, i < 4 ? 128 : 64))
+        return HSTU_ERR_CUDA;
     err = launch_bwd_pre_bf16(a, s);                       // dU and dO (LayerNorm + gate)
     if (err == cudaSuccess) err = launch_bwd_attn_bf16_sm100(a, maps, s);   // dQ, dK, dV, d_rab
   } else {
