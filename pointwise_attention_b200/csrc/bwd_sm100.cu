@@ -135,13 +135,18 @@ __device__ __forceinline__ void run_add(int k, float v, int& run_k, float& run_s
 // P'^T and dS'^T of one 32-column chunk of the dK/dV kernel (rows = keys,
 // columns = queries); the bias gradients come from the dQ kernel.  MASK:
 // the diagonal tile or the sequence's last query tile.
-template <bool POS, bool TIME, bool MASK>
+// TP: 0 no time bias, 1 the chunk's bucket plan, 2 a bucket per element.
+template <bool POS, int TP, bool MASK>
 __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
                                           const Stage* stg, int lane, int r, int c0, bool diag,
-                                          int qlim, const ChunkT& ct, bool generic,
-                                          long long my_ts, const long long* thr,
-                                          const signed char* first, const float* rabt,
-                                          uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+                                          int qlim, const ChunkT& ct, long long my_ts,
+                                          const long long* thr, const signed char* first,
+                                          const float* rabt, uint32_t (&pk)[16],
+                                          uint32_t (&dk)[16]) {
+  float tb[4];
+  if (TP == 1)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tb[j] = rabt[min(ct.k0 + j, kMaxBuckets - 1)];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float p2[2], d2[2];
@@ -150,13 +155,9 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32
       const int cl = 2 * i + hh;
       const int c = c0 + cl;
       float hb = POS ? stg->w[cl - lane + 31] : 0.f;
-      if (TIME) {
-        const int kb = generic ? time_bucket(stg->ts[cl] - my_ts, thr, first)
-                               : ct.k0 + static_cast<int>(cl >= ct.split[0]) +
-                                     static_cast<int>(cl >= ct.split[1]) +
-                                     static_cast<int>(cl >= ct.split[2]);
-        hb += rabt[kb];
-      }
+      if (TP == 1)
+        hb += cl < ct.split[0] ? tb[0] : cl < ct.split[1] ? tb[1] : cl < ct.split[2] ? tb[2] : tb[3];
+      if (TP == 2) hb += rabt[time_bucket(stg->ts[cl] - my_ts, thr, first)];
       const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
       const float t = tanh_approx(hx);
       float p = fmaf(hx, t, hx);
@@ -217,14 +218,18 @@ __device__ __forceinline__ ChunkDn chunk_time_dn(long long my_ts, const long lon
 // keys), and its bias-gradient sums.  MASK: the diagonal tile, keys past the
 // sequence end, or query rows past it (those rows belong to no query of the
 // sequence and must not reach the bias gradients).
-template <bool POS, bool TIME, bool MASK>
+template <bool POS, int TP, bool MASK>
 __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
                                          const Stage* stg, int lane, int r, int c0, bool diag,
-                                         int klim, bool row_ok, const ChunkDn& ct, bool generic,
+                                         int klim, bool row_ok, const ChunkDn& ct,
                                          long long my_ts, const long long* thr,
                                          const signed char* first, const float* rabt, float* win,
                                          int wbase, float* s_dt, uint32_t (&dk)[16], int& run_k,
                                          float& run_s) {
+  float tb[4];
+  if (TP == 1)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tb[j] = rabt[max(ct.khi - j, 0)];
   // Diagonal sums (row - column = const) of the warp's 32 x 32 block: at
   // column cl lane L reads lane (L + cl) mod 32, so every element with
   // row - cl = L, or L - 32, passes through lane L.
@@ -240,16 +245,12 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
       const int c = c0 + cl;
       float hb = POS ? stg->w[lane - cl + 31] : 0.f;
       int kb = 0;
-      bool ge0 = false, ge1 = false, ge2 = false;
-      if (TIME) {
-        if (generic) {
-          kb = time_bucket(my_ts - stg->ts[cl], thr, first);
-        } else {
-          ge0 = cl >= ct.split[0];
-          ge1 = cl >= ct.split[1];
-          ge2 = cl >= ct.split[2];
-          kb = ct.khi - static_cast<int>(ge0) - static_cast<int>(ge1) - static_cast<int>(ge2);
-        }
+      const bool ge0 = TP == 1 && cl >= ct.split[0];
+      const bool ge1 = TP == 1 && cl >= ct.split[1];
+      const bool ge2 = TP == 1 && cl >= ct.split[2];
+      if (TP == 1) hb += ge2 ? tb[3] : ge1 ? tb[2] : ge0 ? tb[1] : tb[0];
+      if (TP == 2) {
+        kb = time_bucket(my_ts - stg->ts[cl], thr, first);
         hb += rabt[kb];
       }
       const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
@@ -262,20 +263,17 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
         const float v = __shfl_sync(0xffffffffu, ds, (lane + cl) & 31);
         if (lane + cl < 32) dpos += v; else dneg += v;
       }
-      if (TIME) {
-        if (!generic) {
-          t_all += ds;
-          if (ge0) t_ge0 += ds;
-          if (ge1) t_ge1 += ds;
-          if (ge2) t_ge2 += ds;
-        } else if (!masked) {
-          run_add(kb, ds, run_k, run_s, s_dt);
-        }
+      if (TP == 1) {
+        t_all += ds;
+        if (ge0) t_ge0 += ds;
+        if (ge1) t_ge1 += ds;
+        if (ge2) t_ge2 += ds;
       }
+      if (TP == 2 && !masked) run_add(kb, ds, run_k, run_s, s_dt);
     }
     dk[i] = pack_bf16(d2[0], d2[1]);
   }
-  if (TIME && !generic) {
+  if (TP == 1) {
     // The warp's 32 rows (consecutive queries) reach neighbouring buckets:
     // sum each bucket over the warp and let one lane add it to the histogram.
     const float tv[4] = {t_all - t_ge0, t_ge0 - t_ge1, t_ge1 - t_ge2, t_ge2};
@@ -595,12 +593,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           ct = chunk_time(my_ts, stg->ts, sorted, s_thr, s_first);
           generic = !__all_sync(0xffffffffu, ct.simple);
         }
-        if (diag || qlim < 128)
-          dkv_chunk<POS, TIME, true>(sv, dav, stg, lane, r, c0, diag, qlim, ct, generic, my_ts,
-                                     s_thr, s_first, s_rabt, pk, dk);
-        else
-          dkv_chunk<POS, TIME, false>(sv, dav, stg, lane, r, c0, diag, qlim, ct, generic, my_ts,
-                                      s_thr, s_first, s_rabt, pk, dk);
+        const bool msk = diag || qlim < 128;
+#define HSTU_DKV(TP_, M_)                                                                    \
+  dkv_chunk<POS, TP_, M_>(sv, dav, stg, lane, r, c0, diag, qlim, ct, my_ts, s_thr, s_first, \
+                          s_rabt, pk, dk)
+        if (!TIME) {
+          if (msk) HSTU_DKV(0, true); else HSTU_DKV(0, false);
+        } else if (generic) {
+          HSTU_DKV(2, true);
+        } else {
+          if (msk) HSTU_DKV(1, true); else HSTU_DKV(1, false);
+        }
+#undef HSTU_DKV
       }
       // The group's warps have read their S^T / dA^T columns before P'^T and
       // dS'^T overwrite them.
@@ -907,14 +911,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // window index r - c + 127 of the block's diagonals
         const int wbase = 32 * q4 - c0 + 127;
-        if (diag || klim < 128 || !__all_sync(0xffffffffu, row_ok))
-          dq_chunk<POS, TIME, true>(sv, dav, stg, lane, r, c0, diag, klim, row_ok, ct, generic,
-                                    my_ts, s_thr, s_first, s_rabt, win, wbase, s_dt, dk, run_k,
-                                    run_s);
-        else
-          dq_chunk<POS, TIME, false>(sv, dav, stg, lane, r, c0, diag, klim, row_ok, ct, generic,
-                                     my_ts, s_thr, s_first, s_rabt, win, wbase, s_dt, dk, run_k,
-                                     run_s);
+        const bool msk = diag || klim < 128 || !__all_sync(0xffffffffu, row_ok);
+#define HSTU_DQ(TP_, M_)                                                                    \
+  dq_chunk<POS, TP_, M_>(sv, dav, stg, lane, r, c0, diag, klim, row_ok, ct, my_ts, s_thr,  \
+                         s_first, s_rabt, win, wbase, s_dt, dk, run_k, run_s)
+        if (!TIME) {
+          if (msk) HSTU_DQ(0, true); else HSTU_DQ(0, false);
+        } else if (generic) {
+          HSTU_DQ(2, true);
+        } else {
+          if (msk) HSTU_DQ(1, true); else HSTU_DQ(1, false);
+        }
+#undef HSTU_DQ
       }
       // The group's warps have read their dA columns before dS' overwrites them.
       named_bar_sync(1 + g, kGroup);
