@@ -741,6 +741,29 @@ def run_gpu(args, spec):
     return 0
 
 
+def run_once(args, spec):
+    """One call of the forward or the backward, run twice on one input set:
+    the launch a profiler captures (ncu -s 1 -c 1), with nothing around it."""
+    import pointwise_attention_b200 as pa
+    torch.cuda.set_device(0)
+    inp = hi.make_inputs(spec, seed=args.seed)
+    d = lambda t: None if t is None else t.to("cuda").contiguous()
+    q, k, v, u, offs = d(inp.q), d(inp.k), d(inp.v), d(inp.u), d(inp.offsets)
+    kw = dict(timestamps=d(inp.timestamps), rab_pos=d(inp.rab_pos), rab_time=d(inp.rab_time),
+              norm_len=inp.norm_len)
+    bwd = args.once == "bwd"
+    y, saved = pa.hstu_attn_fwd(q, k, v, u, offs, inp.max_seq_len, save_for_backward=bwd, **kw)
+    for _ in range(2):
+        if bwd:
+            pa.hstu_attn_bwd(d(inp.dy), q, k, v, u, offs, inp.max_seq_len, saved, **kw)
+        else:
+            pa.hstu_attn_fwd(q, k, v, u, offs, inp.max_seq_len, y=y, **kw)
+    torch.cuda.synchronize()
+    print(json.dumps({"once": args.once, "workload": spec.name, "batch": spec.batch,
+                      "tokens": inp.total_tokens}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -758,10 +781,20 @@ def main(argv=None):
     ap.add_argument("--cpu-budget-single", type=float, default=6.0)
     ap.add_argument("--ref-step-budget", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (profiling a smaller case)")
+    ap.add_argument("--once", choices=["fwd", "bwd"], default=None,
+                    help="run one forward or backward call twice and exit (for ncu captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     spec = hi.WORKLOADS[args.workload]
+    if args.batch > 0:
+        if not args.once:
+            ap.error("--batch only sizes the --once profiling runs")
+        spec = hi.workload(args.workload, batch=args.batch)
+    if args.once:
+        return run_once(args, spec)
     if args.impl == "reference":
         return run_reference(args, spec)
     return run_gpu(args, spec)
