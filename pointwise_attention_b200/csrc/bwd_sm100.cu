@@ -74,7 +74,46 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 struct Stage {
   float w[64];
   long long ts[32];
+  // bf16 pairs of neighbouring diagonals for the packed path: (w[k], w[k+1])
+  // in the dK/dV kernel, (w[k], w[k-1]) in the dQ kernel
+  uint32_t wpk[64];
 };
+
+// ------------------------------------------------------------- bf16x2 arithmetic
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t tanh2(uint32_t x) {
+  uint32_t t;
+  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(x));
+  return t;
+}
+
+constexpr uint32_t kHalf2 = 0x3F003F00u;    // (0.5, 0.5) in bf16
+constexpr uint32_t kOne2 = 0x3F803F80u;     // (1, 1)
+constexpr uint32_t kNegOne2 = 0xBF80BF80u;  // (-1, -1)
+
+// Packed P' and dS' of an element pair from hx = S/2 + bias/2 (bf16 pairs):
+// t = tanh(hx), P' = hx (1 + t), SiLU'(x) = (1 + t)/2 (1 + hx (1 - t)).
+__device__ __forceinline__ uint32_t dsilu_pair(uint32_t hx, uint32_t t, uint32_t da) {
+  const uint32_t sg = hfma2(t, kHalf2, kHalf2);
+  const uint32_t q = hfma2(hx, hfma2(t, kNegOne2, kOne2), kOne2);
+  return hmul2(da, hmul2(sg, q));
+}
+
+__device__ __forceinline__ uint32_t pack_u32_pair(uint32_t lo, uint32_t hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
 
 // Time bias of one 32-column chunk of the dK/dV kernel for a key row: the columns are later
 // queries, so with the chunk's timestamps sorted and dt = t_query - t_key >= 0
@@ -143,6 +182,28 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32
                                           const long long* thr, const signed char* first,
                                           const float* rabt, uint32_t (&pk)[16],
                                           uint32_t (&dk)[16]) {
+  if (TP == 0) {
+    // bf16x2 arithmetic: P' and dS' are bf16 operands of the next MMAs anyway
+    const uint32_t* wp = stg->wpk + 31 - lane;   // pair i: diagonals 2i - lane + 31 (+1)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t hx = hfma2(pack_u32_pair(sv[2 * i], sv[2 * i + 1]), kHalf2,
+                                POS ? wp[2 * i] : 0u);
+      const uint32_t t = tanh2(hx);
+      uint32_t p = hfma2(hx, t, hx);
+      uint32_t d = dsilu_pair(hx, t, pack_u32_pair(dav[2 * i], dav[2 * i + 1]));
+      if (MASK) {
+        const int c = c0 + 2 * i;
+        const uint32_t keep = (((diag && c < r) || c >= qlim) ? 0u : 0x0000FFFFu) |
+                              (((diag && c + 1 < r) || c + 1 >= qlim) ? 0u : 0xFFFF0000u);
+        p &= keep;
+        d &= keep;
+      }
+      pk[i] = p;
+      dk[i] = d;
+    }
+    return;
+  }
   float tb[4];
   if (TP == 1)
 #pragma unroll
@@ -226,6 +287,37 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
                                          const signed char* first, const float* rabt, float* win,
                                          int wbase, float* s_dt, uint32_t (&dk)[16], int& run_k,
                                          float& run_s) {
+  if (TP == 0) {
+    // bf16x2 arithmetic for dS'; the diagonal sums take its fp32 widening
+    const uint32_t* wp = stg->wpk + lane + 31;   // pair i: diagonals lane - 2i + 31 (-1)
+    float dpos = 0.f, dneg = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t hx = hfma2(pack_u32_pair(sv[2 * i], sv[2 * i + 1]), kHalf2,
+                                POS ? wp[-2 * i] : 0u);
+      uint32_t d = dsilu_pair(hx, tanh2(hx), pack_u32_pair(dav[2 * i], dav[2 * i + 1]));
+      if (MASK) {
+        const int c = c0 + 2 * i;
+        const uint32_t keep =
+            (((diag && c > r) || c >= klim || !row_ok) ? 0u : 0x0000FFFFu) |
+            (((diag && c + 1 > r) || c + 1 >= klim || !row_ok) ? 0u : 0xFFFF0000u);
+        d &= keep;
+      }
+      dk[i] = d;
+      if (POS) {
+        const float v0 = __shfl_sync(0xffffffffu, __uint_as_float(d << 16), (lane + 2 * i) & 31);
+        if (lane + 2 * i < 32) dpos += v0; else dneg += v0;
+        const float v1 =
+            __shfl_sync(0xffffffffu, __uint_as_float(d & 0xFFFF0000u), (lane + 2 * i + 1) & 31);
+        if (lane + 2 * i + 1 < 32) dpos += v1; else dneg += v1;
+      }
+    }
+    if (POS) {
+      atomicAdd(&win[wbase + lane], dpos);
+      if (lane > 0) atomicAdd(&win[wbase + lane - 32], dneg);
+    }
+    return;
+  }
   float tb[4];
   if (TP == 1)
 #pragma unroll
@@ -556,8 +648,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool sorted = true;
     auto stage = [&]() {
       if (POS) {
-        stg->w[lane] = 0.5f * pw0;
-        stg->w[32 + lane] = 0.5f * pw1;
+        const float w0 = 0.5f * pw0, w1 = 0.5f * pw1;
+        stg->w[lane] = w0;
+        stg->w[32 + lane] = w1;
+        // pairs (w[k], w[k+1]): k = lane and k = 32 + lane
+        const float n0 = __shfl_down_sync(0xffffffffu, w0, 1);
+        const float n1 = __shfl_down_sync(0xffffffffu, w1, 1);
+        const float w32 = __shfl_sync(0xffffffffu, w1, 0);
+        stg->wpk[lane] = pack_bf16(w0, lane < 31 ? n0 : w32);
+        stg->wpk[32 + lane] = pack_bf16(w1, lane < 31 ? n1 : 0.f);
       }
       if (TIME) {
         stg->ts[lane] = pt;
@@ -867,8 +966,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool sorted = true;
     auto stage = [&]() {
       if (POS) {
-        stg->w[lane] = 0.5f * pw0;
-        stg->w[32 + lane] = 0.5f * pw1;
+        const float w0 = 0.5f * pw0, w1 = 0.5f * pw1;
+        stg->w[lane] = w0;
+        stg->w[32 + lane] = w1;
+        // pairs (w[k], w[k-1]): k = lane and k = 32 + lane
+        const float p0 = __shfl_up_sync(0xffffffffu, w0, 1);
+        const float p1 = __shfl_up_sync(0xffffffffu, w1, 1);
+        const float w31 = __shfl_sync(0xffffffffu, w0, 31);
+        stg->wpk[lane] = pack_bf16(w0, lane > 0 ? p0 : 0.f);
+        stg->wpk[32 + lane] = pack_bf16(w1, lane > 0 ? p1 : w31);
       }
       if (TIME) {
         stg->ts[lane] = pt;
