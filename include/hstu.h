@@ -56,7 +56,8 @@ typedef enum {
   HSTU_ERR_UNSUPPORTED = 2,  /* valid problem outside the implemented shapes     */
   HSTU_ERR_CUDA = 3,         /* a CUDA call or launch failed                     */
   HSTU_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out               */
-  HSTU_ERR_WORKSPACE = 5     /* workspace NULL or smaller than required          */
+  HSTU_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than required          */
+  HSTU_ERR_BOUNDS = 6        /* an index check of a HSTU_DEBUG_BOUNDS build failed */
 } hstu_status_t;
 
 typedef enum { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype_t;
@@ -126,7 +127,10 @@ HSTU_API hstu_status_t hstu_attn_bwd(const hstu_problem_t *p, const void *dy, co
 /*
  * Waits for `stream`, reads the device status word of `workspace`, resets it
  * to zero and returns it (HSTU_OK, HSTU_ERR_INVALID_ARG for offsets found
- * inconsistent on the device, HSTU_ERR_TIMEOUT for an expired wait), or
+ * inconsistent on the device, HSTU_ERR_TIMEOUT for an expired wait,
+ * HSTU_ERR_BOUNDS when a library built with -DHSTU_DEBUG_BOUNDS found an
+ * index outside its buffer: it recorded the first failing check site in
+ * word 6 and its index in word 7 and used index 0 instead), or
  * HSTU_ERR_CUDA when the stream itself reports an error.
  */
 HSTU_API hstu_status_t hstu_attn_check(void *workspace, void *stream);

@@ -15,10 +15,13 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libhstu.so")
+# HSTU_DEBUG_BOUNDS=1 in the environment selects the build with device-side
+# index checks (python -m pointwise_attention_b200.build --debug-bounds).
+LIB_PATH = os.path.join(_HERE, "libhstu_debug.so" if os.environ.get("HSTU_DEBUG_BOUNDS") == "1"
+                        else "libhstu.so")
 
 HSTU_OK, HSTU_ERR_INVALID_ARG, HSTU_ERR_UNSUPPORTED = 0, 1, 2
-HSTU_ERR_CUDA, HSTU_ERR_TIMEOUT, HSTU_ERR_WORKSPACE = 3, 4, 5
+HSTU_ERR_CUDA, HSTU_ERR_TIMEOUT, HSTU_ERR_WORKSPACE, HSTU_ERR_BOUNDS = 3, 4, 5, 6
 HSTU_F32, HSTU_BF16 = 0, 1
 
 EXPORTED = ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd", "hstu_attn_check",

@@ -37,6 +37,7 @@
 #include <algorithm>
 #include <atomic>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 #include "tile_math.cuh"
@@ -522,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
-      const int krow = s + 128 * n;
+      const int krow = checked(a.status, s + 128 * n, a.T, BS_BWD_TMA_K);
       mbar_arrive_expect_tx(bar(B_KVFULL), 2 * kTile);
       tma_load_3d(sbase + kOffT0, &tm_k, bar(B_KVFULL), 0, h, krow);
       tma_load_3d(sbase + kOffT0 + kHalf, &tm_k, bar(B_KVFULL), 64, h, krow);
@@ -532,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int x = 0; x < nx && ok; ++x) {
         const int slot = x % kRing, use = x / kRing;
-        const int qrow = s + 128 * (n + (x >> 1)) + 64 * (x & 1);
+        const int qrow = checked(a.status, s + 128 * (n + (x >> 1)) + 64 * (x & 1), a.T, BS_BWD_TMA_Q);
         if (use > 0) ok = mbar_wait(bar(B_QEMPTY + slot), (use - 1) & 1, abort_flag);
         if (!ok) break;
         const uint32_t qd = sbase + kOffR0 + slot * kSubTile;
@@ -625,7 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int Lw = 2 * a.L - 1;
     // Key rows past the sequence end take the last token's timestamp, which
     // keeps their chunk plans on the cheap path (their elements are masked).
-    const long long my_ts = TIME ? a.timestamps[row_ok ? t_row : s + n_b - 1] : 0;
+    const long long my_ts =
+        TIME ? a.timestamps[checked(a.status, row_ok ? t_row : s + n_b - 1, a.T, BS_BWD_TS)] : 0;
     Stage* stg = reinterpret_cast<Stage*>(smem + kOffStage) + ew;
     float pw0 = 0.f, pw1 = 0.f;
     long long pt = 0;
@@ -642,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (TIME) {
         const int i = 128 * n + cbase + lane;
-        pt = a.timestamps[s + (i < n_b ? i : n_b - 1)];
+        pt = a.timestamps[checked(a.status, s + (i < n_b ? i : n_b - 1), a.T, BS_BWD_TS)];
       }
     };
     bool sorted = true;
@@ -731,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_wait_ld_dep(vv);
     tmem_wait_ld_dep(kv);
     if (ok && row_ok) {
-      const size_t off = (static_cast<size_t>(t_row) * a.H + h) * 128 + 32 * cq;
+      const size_t off = (static_cast<size_t>(checked(a.status, t_row, a.T, BS_BWD_ROW)) * a.H + h) * 128 + 32 * cq;
       uint4* dvp = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dv) + off);
       uint4* dkp = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.dk) + off);
 #pragma unroll
@@ -847,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
-      const int qrow = s + 128 * m;
+      const int qrow = checked(a.status, s + 128 * m, a.T, BS_BWD_TMA_Q);
       mbar_arrive_expect_tx(bar(B_QDOFULL), 2 * kTile);
       tma_load_3d(sbase + kOffT0, &tm_q, bar(B_QDOFULL), 0, h, qrow);
       tma_load_3d(sbase + kOffT0 + kHalf, &tm_q, bar(B_QDOFULL), 64, h, qrow);
@@ -857,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int x = 0; x < nx && ok; ++x) {
         const int slot = x % kRing, use = x / kRing;
-        const int krow = s + 64 * x;
+        const int krow = checked(a.status, s + 64 * x, a.T, BS_BWD_TMA_K);
         if (use > 0) ok = mbar_wait(bar(B_KEMPTY + slot), (use - 1) & 1, abort_flag);
         if (!ok) break;
         const uint32_t kd = sbase + kOffR0 + slot * kSubTile;
@@ -943,7 +945,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int Lw = 2 * a.L - 1;
     // Query rows past the sequence end (never stored) take the last token's
     // timestamp, which keeps their chunk plans on the cheap path.
-    const long long my_ts = TIME ? a.timestamps[row_ok ? t_row : s + n_b - 1] : 0;
+    const long long my_ts =
+        TIME ? a.timestamps[checked(a.status, row_ok ? t_row : s + n_b - 1, a.T, BS_BWD_TS)] : 0;
     Stage* stg = reinterpret_cast<Stage*>(smem + kOffStage) + ew;
     float pw0 = 0.f, pw1 = 0.f;
     long long pt = 0;
@@ -960,7 +963,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (TIME) {
         const int j = kbase + lane;
-        pt = a.timestamps[s + (j < n_b ? j : n_b - 1)];
+        pt = a.timestamps[checked(a.status, s + (j < n_b ? j : n_b - 1), a.T, BS_BWD_TS)];
       }
     };
     bool sorted = true;

@@ -26,6 +26,7 @@
 
 #include <atomic>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 #include "tile_math.cuh"
@@ -162,26 +163,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && nt > 0) {
       int klast[kStages] = {-1, -1}, vlast[kStages] = {-1, -1};
       bool ok = true;
+      const int qrow = checked(a.status, c0 + 128 * mt, a.C, BS_CAND_TMA);
       mbar_arrive_expect_tx(bar(B_QFULL), kTile);
-      tma_load_3d(sbase + kOffQ, &tm_q, bar(B_QFULL), 0, h, c0 + 128 * mt);
-      tma_load_3d(sbase + kOffQ + kHalf, &tm_q, bar(B_QFULL), 64, h, c0 + 128 * mt);
+      tma_load_3d(sbase + kOffQ, &tm_q, bar(B_QFULL), 0, h, qrow);
+      tma_load_3d(sbase + kOffQ + kHalf, &tm_q, bar(B_QFULL), 64, h, qrow);
       for (int n = 0; n < nt && ok; ++n) {
         const int st = n % kStages, use = n / kStages;
         if (use > 0)
           ok = checked(mbar_wait(bar(B_KEMPTY + st), (use - 1) & 1, abort_flag), a.status);
         if (!ok) break;
+        const int krow = checked(a.status, s + 128 * n, a.T, BS_CAND_TMA);
         mbar_arrive_expect_tx(bar(B_KFULL + st), kTile);
-        tma_load_3d(sbase + kOffK + st * kTile, &tm_k, bar(B_KFULL + st), 0, h, s + 128 * n);
-        tma_load_3d(sbase + kOffK + st * kTile + kHalf, &tm_k, bar(B_KFULL + st), 64, h,
-                    s + 128 * n);
+        tma_load_3d(sbase + kOffK + st * kTile, &tm_k, bar(B_KFULL + st), 0, h, krow);
+        tma_load_3d(sbase + kOffK + st * kTile + kHalf, &tm_k, bar(B_KFULL + st), 64, h, krow);
         klast[st] = use;
         if (use > 0)
           ok = checked(mbar_wait(bar(B_VEMPTY + st), (use - 1) & 1, abort_flag), a.status);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(B_VFULL + st), kTile);
-        tma_load_3d(sbase + kOffV + st * kTile, &tm_v, bar(B_VFULL + st), 0, h, s + 128 * n);
-        tma_load_3d(sbase + kOffV + st * kTile + kHalf, &tm_v, bar(B_VFULL + st), 64, h,
-                    s + 128 * n);
+        tma_load_3d(sbase + kOffV + st * kTile, &tm_v, bar(B_VFULL + st), 0, h, krow);
+        tma_load_3d(sbase + kOffV + st * kTile + kHalf, &tm_v, bar(B_VFULL + st), 64, h, krow);
         vlast[st] = use;
       }
       if (!ok) {
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_ok = i_loc < cb;
     const int cand = c0 + (row_ok ? i_loc : 0);
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
-    const long long my_ts = TIME ? __ldg(a.cand_ts + cand) : 0ll;
+    const long long my_ts = TIME ? __ldg(a.cand_ts + checked(a.status, cand, a.C, BS_CAND_ROW)) : 0ll;
     // rpos[d] = this head's position bias at relative position d >= 0
     const float* rpos = POS ? a.rab_pos + static_cast<size_t>(h) * (2 * a.L - 1) + (a.L - 1) : nullptr;
     bool ok = true;
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j = 128 * n + 32 * cs + lane;
       const bool jv = j < nb;
       const float pb = (POS && jv) ? __ldg(rpos + (nb - j)) : 0.f;
-      const long long kts = (TIME && jv) ? __ldg(a.timestamps + s + j) : 0ll;
+      const long long kts = (TIME && jv) ? __ldg(a.timestamps + checked(a.status, s + j, a.T, BS_CAND_TS)) : 0ll;
       if (ok) ok = checked(mbar_wait(bar(B_SFULL + st), (n / kStages) & 1, abort_flag), a.status);
       ok = __all_sync(0xffffffffu, ok);   // the TMEM accesses below are warp-collective
       if (!ok) break;
@@ -389,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __threadfence();
     named_bar_sync(1, kEpiThreads);
     if (ew == 0 && lane == 0) {
-      unsigned* cnt = a.cnt + static_cast<size_t>(b) * a.max_tiles + mt;
+      unsigned* cnt = a.cnt + checked(a.status, static_cast<size_t>(b) * a.max_tiles + mt,
+                                      static_cast<long long>(a.B) * a.max_tiles, BS_CAND_CNT);
       const unsigned old = atomicAdd(cnt, 1u);
       const bool last = old == static_cast<unsigned>(a.H - 1);
       if (last) *cnt = 0u;   // re-armed: every head of this micro-batch has counted

@@ -51,6 +51,7 @@
 #include <algorithm>
 #include <atomic>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 #include "tile_math.cuh"
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = __ldg(a.offsets + it.b);
         if (j > 0) ok = waited(mbar_wait(bar(B_QEMPTY), (j - 1) & 1, abort_flag), a.status, 2, j, g);
         if (ok) {
-          const int row0 = s + kRows * m;
+          const int row0 = checked(a.status, s + kRows * m, a.T, BS_FWD_TMA_Q);
           mbar_arrive_expect_tx(bar(B_QFULL), kTile);
           tma_load_3d(sbase + kOffQ, &tm_q, bar(B_QFULL), 0, h, row0);
           tma_load_3d(sbase + kOffQ + kHalf, &tm_q, bar(B_QFULL), 64, h, row0);
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (use > 0 && !waited(mbar_wait(bar(B_KEMPTY + st), (use - 1) & 1, abort_flag), a.status,
                                  3, j, x))
             return false;
-          const int krow = s + kCols * n;
+          const int krow = checked(a.status, s + kCols * n, a.T, BS_FWD_TMA_KV);
           mbar_arrive_expect_tx(bar(B_KFULL + st), kTile);
           tma_load_3d(sbase + kOffK + st * kTile, &tm_k, bar(B_KFULL + st), 0, h, krow);
           tma_load_3d(sbase + kOffK + st * kTile + kHalf, &tm_k, bar(B_KFULL + st), 64, h, krow);
@@ -433,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (use > 0 && !waited(mbar_wait(bar(B_VEMPTY + st), (use - 1) & 1, abort_flag), a.status,
                                  4, j, x))
             return false;
-          const int krow = s + kCols * n;
+          const int krow = checked(a.status, s + kCols * n, a.T, BS_FWD_TMA_KV);
           mbar_arrive_expect_tx(bar(B_VFULL + st), kTile);
           tma_load_3d(sbase + kOffV + st * kTile, &tm_v, bar(B_VFULL + st), 0, h, krow);
           tma_load_3d(sbase + kOffV + st * kTile + kHalf, &tm_v, bar(B_VFULL + st), 64, h, krow);
@@ -618,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Rows past the sequence end (never stored) take the last token's
       // timestamp: every key is then at or before them and the plans stay cheap.
       long long my64 = 0;
-      if (TIME) my64 = a.timestamps[row_ok ? t_row : s + n_b - 1];
+      if (TIME) my64 = a.timestamps[checked(a.status, row_ok ? t_row : s + n_b - 1, a.T, BS_FWD_TS)];
       const uint32_t my32 = static_cast<uint32_t>(my64);
       // The gate input of this row is read at the end of the block: ask L2 for it now.
       if (row_ok)
@@ -644,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (TIME) {
           const int jj = kCols * n + 32 * cq + lane;
-          pre_t = a.timestamps[s + (jj < n_b ? jj : n_b - 1)];
+          pre_t = a.timestamps[checked(a.status, s + (jj < n_b ? jj : n_b - 1), a.T, BS_FWD_TS)];
         }
       };
       long long kmin = 0, kmax = 0;
@@ -866,7 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool fp32_stash = a.o_save != nullptr;
         const float invD = 1.0f / static_cast<float>(D);
         for (int rr = ew; rr < nrows; rr += kEpiWarps) {
-          const int t = s + kRows * m + rr;
+          const int t = checked(a.status, s + kRows * m + rr, a.T, BS_FWD_ROW);
           float4 st = make_float4(0.f, 0.f, 0.f, 0.f);
           if (lane < H) st = ld_global_cg_f4(a.stats + static_cast<size_t>(t) * H + lane);
           float tot = lane < H ? st.x : 0.f;

@@ -249,6 +249,7 @@ const char* hstu_status_string(hstu_status_t s) {
     case HSTU_ERR_CUDA: return "HSTU_ERR_CUDA: a CUDA call or launch failed";
     case HSTU_ERR_TIMEOUT: return "HSTU_ERR_TIMEOUT: a bounded device wait ran out";
     case HSTU_ERR_WORKSPACE: return "HSTU_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case HSTU_ERR_BOUNDS: return "HSTU_ERR_BOUNDS: a debug-build index check failed";
   }
   return "HSTU: unknown status";
 }
@@ -424,6 +425,7 @@ hstu_status_t hstu_attn_check(void* workspace, void* stream) {
   }
   if (word & kStatusTimeout) return HSTU_ERR_TIMEOUT;
   if (word & kStatusBadOffsets) return HSTU_ERR_INVALID_ARG;
+  if (word & kStatusBounds) return HSTU_ERR_BOUNDS;
   return HSTU_OK;
 }
 

@@ -11,6 +11,7 @@ namespace hstu {
 // Bits of the device status word (first 4 bytes of the workspace).
 constexpr int kStatusBadOffsets = 1;   // offsets contradict T / max_seq_len / L
 constexpr int kStatusTimeout = 2;      // a bounded wait ran out
+constexpr int kStatusBounds = 4;       // an index check of the HSTU_DEBUG_BOUNDS build failed
 
 // The 256-byte head of the workspace: word 0 is the status word; words 16 and
 // 17 are the bf16 forward's work counter and finished-CTA counter.  The

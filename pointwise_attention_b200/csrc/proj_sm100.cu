@@ -25,6 +25,7 @@
 #include <algorithm>
 #include <atomic>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 #include "tile_math.cuh"
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(Cfg<EPI, NT>::kThreads, Cfg<EPI, NT>::kMinBloc
         if (!ok) break;
         const uint32_t dst = sbase + st * C::kStage;
         mbar_arrive_expect_tx(bar(B_FULL + st), C::kStage);
-        tma_load_2d(dst, &tm_a, bar(B_FULL + st), kb * kBK, m0);
+        tma_load_2d(dst, &tm_a, bar(B_FULL + st), kb * kBK, checked(a.status, m0, a.T, BS_PROJ_TMA));
 #pragma unroll
         for (int nb = 0; nb < NT / 256; ++nb)
           tma_load_2d(dst + kABytes + nb * 256 * 128, &tm_b, bar(B_FULL + st), kb * kBK,

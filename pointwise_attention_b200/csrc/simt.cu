@@ -14,6 +14,7 @@
 
 #include <algorithm>
 
+#include "bounds.cuh"
 #include "internal.h"
 
 namespace hstu {
@@ -368,7 +369,8 @@ __global__ void __launch_bounds__(kT) bwd_dq_simt(const BwdArgs a) {
         atomicAdd(a.d_rab_pos + static_cast<size_t>(h) * (2 * a.L - 1) + (i - j) + a.L - 1, dsv);
       if (a.d_rab_time)
         atomicAdd(a.d_rab_time + h * a.nb +
-                      bucket_of(a.timestamps[s + i] - a.timestamps[s + j], a.bt, a.nb),
+                      bucket_of(a.timestamps[checked(a.status, s + i, a.T, BS_SIMT_TS)] -
+                                    a.timestamps[checked(a.status, s + j, a.T, BS_SIMT_TS)], a.bt, a.nb),
                   dsv);
     }
     ds_s[threadIdx.x] = dsv;

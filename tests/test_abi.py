@@ -51,7 +51,7 @@ def test_thresholds_match_oracle_golden(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert lib.status_string(code).startswith("HSTU_")
     assert "unknown" in lib.status_string(99)
 

@@ -24,15 +24,20 @@ DEV = "cuda:0"
 
 
 def run(ci, max_cands=None, workspace=None):
+    import ctypes
     h = ci.hist
     d = lambda t: None if t is None else t.to(DEV)
+    mc = max_cands if max_cands is not None else max(ci.counts + [0])
+    if workspace is None:
+        p = pa.make_problem(d(h.k), d(h.v), d(h.offsets), max(h.lengths + [0]))
+        n = pa.load_library().hstu_cand_workspace_size(ctypes.byref(p), ci.total_cands, mc)
+        workspace = torch.zeros(max(n, 256), dtype=torch.uint8, device=DEV)
     y = pa.hstu_cand_fwd(d(h.k), d(h.v), d(h.offsets), max(h.lengths + [0]), d(ci.qc),
-                         d(ci.kc), d(ci.vc), d(ci.uc), d(ci.cand_offsets),
-                         max_cands if max_cands is not None else max(ci.counts + [0]),
+                         d(ci.kc), d(ci.vc), d(ci.uc), d(ci.cand_offsets), mc,
                          timestamps=d(h.timestamps), cand_timestamps=d(ci.cand_ts),
                          rab_pos=d(h.rab_pos), rab_time=d(h.rab_time), norm_len=h.norm_len,
                          ln_weight=d(h.ln_weight), ln_bias=d(h.ln_bias), workspace=workspace)
-    torch.cuda.synchronize()
+    assert pa.hstu_attn_check(workspace) == 0
     return y
 
 

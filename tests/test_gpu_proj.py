@@ -38,9 +38,10 @@ def close(got, ref, name, atol=1e-2, rtol=8e-3):
 
 
 def run_uvqk(p, act, bias=True):
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
     out = pa.hstu_uvqk_fwd(p.x.to(DEV), p.w_uvqk.to(DEV), p.H, p.d_qk, p.d_v,
-                           bias=p.b_uvqk.to(DEV) if bias else None, act=act)
-    torch.cuda.synchronize()
+                           bias=p.b_uvqk.to(DEV) if bias else None, act=act, workspace=ws)
+    assert pa.hstu_attn_check(ws) == 0
     return out
 
 
@@ -91,12 +92,13 @@ def test_uvqk_large_sampled_rows():
 
 
 def run_out(p, bias=True, affine=True, stats=True):
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
     z, st = pa.hstu_out_fwd(p.y.to(DEV), p.w_out.to(DEV), p.x.to(DEV),
                             bias=p.b_out.to(DEV) if bias else None,
                             ln_weight=p.ln_weight.to(DEV) if affine else None,
                             ln_bias=p.ln_bias.to(DEV) if affine else None,
-                            save_stats=stats)
-    torch.cuda.synchronize()
+                            save_stats=stats, workspace=ws)
+    assert pa.hstu_attn_check(ws) == 0
     return z, st
 
 
