@@ -666,18 +666,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (TIME) {
           wts[lane] = pre_t;
           wts32[lane] = static_cast<uint32_t>(pre_t);
-          long long mn = pre_t, mx = pre_t;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const long long a2 = __shfl_xor_sync(0xffffffffu, mn, o);
-            const long long b2 = __shfl_xor_sync(0xffffffffu, mx, o);
-            mn = a2 < mn ? a2 : mn;
-            mx = b2 > mx ? b2 : mx;
-          }
-          kmin = mn;
-          kmax = mx;
           const long long nx = __shfl_down_sync(0xffffffffu, pre_t, 1);
           asc = !__any_sync(0xffffffffu, lane < 31 && nx < pre_t);
+          // ascending keys (the usual case): the ends are the extremes
+          if (asc) {
+            kmin = __shfl_sync(0xffffffffu, pre_t, 0);
+            kmax = __shfl_sync(0xffffffffu, pre_t, 31);
+          } else {
+            long long mn = pre_t, mx = pre_t;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              const long long a2 = __shfl_xor_sync(0xffffffffu, mn, o);
+              const long long b2 = __shfl_xor_sync(0xffffffffu, mx, o);
+              mn = a2 < mn ? a2 : mn;
+              mx = b2 > mx ? b2 : mx;
+            }
+            kmin = mn;
+            kmax = mx;
+          }
         }
         __syncwarp();
       };
@@ -728,14 +734,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               // first column whose bucket is k1: dt < thr[k0]
               int split = 32;
               if (k0 != k1) {
+                // leading columns with dt >= thr[k0] (dt falls along the
+                // chunk): a fixed five-step bisection, then the last column
                 const uint32_t th = es.thr32[k0];
-                int lo = 0, hi = 32;
-#pragma unroll 1
-                while (lo < hi) {
-                  const int mid = (lo + hi) >> 1;
-                  if (my32 - wts32[mid] >= th) lo = mid + 1; else hi = mid;
-                }
-                split = lo;
+                int pos = 0;
+#pragma unroll
+                for (int step = 16; step > 0; step >>= 1)
+                  if (my32 - wts32[pos + step - 1] >= th) pos += step;
+                split = pos + static_cast<int>(my32 - wts32[pos] >= th);
               }
               const float hv = es.rabt[k0], lv = es.rabt[k1];
               chunk_pairs<POS, true, T_SPLIT>(sv, wp, 0u, pack_bf16x2(hv, hv),
