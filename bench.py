@@ -51,6 +51,7 @@ KERNEL_SOURCES = {
     "hstu_fwd_bf16_sm100": ["pointwise_attention_b200/csrc/fwd_sm100.cu",
                             "pointwise_attention_b200/csrc/ptx.cuh",
                             "pointwise_attention_b200/csrc/tile_math.cuh",
+                            "pointwise_attention_b200/csrc/bounds.cuh",
                             "pointwise_attention_b200/csrc/internal.h"],
 }
 BWD_FLOP_FACTOR = 2.5      # S recomputed, dA, dV, dQ, dK: five GEMM-equivalents
