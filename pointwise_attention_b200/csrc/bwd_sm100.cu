@@ -65,48 +65,51 @@ __device__ __forceinline__ float silu_grad_h(float hx, float t) {
   return sg * fmaf(hx, 1.0f - t, 1.0f);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
 // Per-warp staging of one 32 x 32 block: 63 position-bias diagonals (fp32,
-// halved) and the 32 column timestamps.
+// halved) and the 32 column timestamps (also their low 32 bits, whose
+// differences are exact while |dt| < 2^31).
 struct Stage {
   float w[64];
   long long ts[32];
+  uint32_t ts32[32];
+  long long cmin, cmax;   // the columns' time range
+  int asc;                // the columns' timestamps ascend
   // bf16 pairs of neighbouring diagonals for the packed path: (w[k], w[k+1])
   // in the dK/dV kernel, (w[k], w[k-1]) in the dQ kernel
   uint32_t wpk[64];
 };
 
-// ------------------------------------------------------------- bf16x2 arithmetic
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
+// Stage the block's 32 column timestamps (lane c holds column c's), whether
+// they ascend, and their range.
+__device__ __forceinline__ void stage_time(Stage* stg, int lane, long long pt) {
+  stg->ts[lane] = pt;
+  stg->ts32[lane] = static_cast<uint32_t>(pt);
+  const long long nxt = __shfl_down_sync(0xffffffffu, pt, 1);
+  const bool asc = !__any_sync(0xffffffffu, lane < 31 && nxt < pt);
+  long long lo = pt, hi = pt;
+  if (!asc) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const long long x = __shfl_xor_sync(0xffffffffu, lo, o);
+      const long long y = __shfl_xor_sync(0xffffffffu, hi, o);
+      lo = x < lo ? x : lo;
+      hi = y > hi ? y : hi;
+    }
+  }
+  if (lane == 0) {
+    stg->cmin = lo;                  // ascending: lane 0 holds the minimum
+    stg->asc = asc;
+  }
+  if (lane == 31) stg->cmax = hi;    // and lane 31 the maximum
 }
 
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t tanh2(uint32_t x) {
-  uint32_t t;
-  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(x));
-  return t;
-}
-
-constexpr uint32_t kHalf2 = 0x3F003F00u;    // (0.5, 0.5) in bf16
 constexpr uint32_t kOne2 = 0x3F803F80u;     // (1, 1)
 constexpr uint32_t kNegOne2 = 0xBF80BF80u;  // (-1, -1)
 
 // Packed P' and dS' of an element pair from hx = S/2 + bias/2 (bf16 pairs):
 // t = tanh(hx), P' = hx (1 + t), SiLU'(x) = (1 + t)/2 (1 + hx (1 - t)).
 __device__ __forceinline__ uint32_t dsilu_pair(uint32_t hx, uint32_t t, uint32_t da) {
-  const uint32_t sg = hfma2(t, kHalf2, kHalf2);
+  const uint32_t sg = hfma2(t, kHalfPair, kHalfPair);
   const uint32_t q = hfma2(hx, hfma2(t, kNegOne2, kOne2), kOne2);
   return hmul2(da, hmul2(sg, q));
 }
@@ -116,51 +119,141 @@ __device__ __forceinline__ uint32_t pack_u32_pair(uint32_t lo, uint32_t hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Time bias of one 32-column chunk of the dK/dV kernel for a key row: the columns are later
-// queries, so with the chunk's timestamps sorted and dt = t_query - t_key >= 0
-// at its first column, |dt| grows along the chunk and its bucket climbs from
-// k0 by at most 3 when the chunk spans few octaves; split[i] is the first
-// column of bucket k0 + i + 1 (32 when none), found by bisection on the
-// integer thresholds.  Otherwise (unsorted timestamps, the diagonal tile,
-// many buckets) each element takes its own bucket.
-struct ChunkT {
-  int k0;
-  int split[3];
-  bool simple;
+// Time-bias plan of one warp's 32 x 32 block, chosen warp-uniformly.  When the
+// block's column timestamps ascend, every |dt| is below 2^31 and dt keeps one
+// sign, each row's bucket moves monotonically along its 32 columns: TB_CONST
+// when no row's bucket changes inside the block, TB_SPLIT when each changes at
+// most once, at a per-row split column found by bisection.  Both add the time
+// bias as one more bf16 pair on the packed path.  Otherwise every element
+// looks its bucket up: TB_GEN32 on 32-bit differences, TB_GEN64 when the span
+// reaches 2^31.  TB_NONE: no time table.
+enum { TB_NONE = 0, TB_CONST = 1, TB_SPLIT = 2, TB_GEN32 = 3, TB_GEN64 = 4 };
+
+// The time-bucket tables in shared memory, at fixed offsets from its base.
+struct TimeTables {
+  const uint8_t* base;
+  __device__ __forceinline__ const long long* thr() const;
+  __device__ __forceinline__ const signed char* first() const;
+  __device__ __forceinline__ const float* rabt() const;    // half time bias per bucket
+  __device__ __forceinline__ const uint4* oct() const;
+  __device__ __forceinline__ const unsigned* thr32() const;
 };
 
-__device__ __forceinline__ ChunkT chunk_time(long long my_ts, const long long* kts, bool sorted,
-                                             const long long* thr, const signed char* first) {
-  ChunkT c;
-  c.k0 = 0;
-  c.split[0] = c.split[1] = c.split[2] = 32;
-  const long long d0 = kts[0] - my_ts, d1 = kts[31] - my_ts;
-  c.simple = sorted && d0 >= 0;
-  if (c.simple) {
-    const int k0 = time_bucket(d0, thr, first);
-    const int k1 = time_bucket(d1, thr, first);
-    c.simple = k1 - k0 <= 3;
-    c.k0 = k0;
+struct TimePlan {
+  int k_a, k_b;     // buckets of the columns before / from the split
+  int split;        // first column of bucket k_b (32: none)
+  uint32_t t_a, t_b, t_ab;   // half biases as pairs: (a, a), (b, b), (a, b)
+};
+
+// Columns c = 0..31 of the block with ts32[c] - my32 < th (dt rising along
+// ascending columns, dt >= 0): a fixed five-step bisection, then the last
+// column.
+__device__ __forceinline__ int count_below_up(const uint32_t* ts32, uint32_t my32, uint32_t th) {
+  int pos = 0;
 #pragma unroll
-    for (int i = 0; i < 3; ++i) {
-      if (c.simple && k0 + i + 1 <= k1) {
-        const long long th = thr[k0 + i + 1];
-        int lo = 0, hi = 32;
-#pragma unroll 1
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (kts[mid] - my_ts < th) lo = mid + 1; else hi = mid;
-        }
-        c.split[i] = lo;
-      }
-    }
-  }
-  return c;
+  for (int step = 16; step > 0; step >>= 1)
+    if (ts32[pos + step - 1] - my32 < th) pos += step;
+  return pos + static_cast<int>(ts32[pos] - my32 < th);
 }
 
-// Running sum of one key row's dS' per time bucket: with sorted timestamps a
-// row's buckets only climb along its query columns, so a (bucket, sum) pair
-// in registers goes to the shared histogram once per bucket change.
+// Columns with my32 - ts32[c] >= th (dt falling along ascending columns).
+__device__ __forceinline__ int count_at_least_dn(const uint32_t* ts32, uint32_t my32, uint32_t th) {
+  int pos = 0;
+#pragma unroll
+  for (int step = 16; step > 0; step >>= 1)
+    if (my32 - ts32[pos + step - 1] >= th) pos += step;
+  return pos + static_cast<int>(my32 - ts32[pos] >= th);
+}
+
+__device__ __forceinline__ void plan_pairs(TimePlan& p, const TimeTables& tt) {
+  const float va = tt.rabt()[p.k_a], vb = tt.rabt()[p.k_b];
+  p.t_a = pack_bf16x2(va, va);
+  p.t_b = pack_bf16x2(vb, vb);
+  p.t_ab = pack_bf16x2(va, vb);
+}
+
+// Plan of the dK/dV kernel (rows = keys at my_ts, columns = later queries
+// with timestamps in [cmin, cmax]): dt = t_query - t_key rises along the
+// columns, so the bucket climbs from k_a at the first column to k_b.
+__device__ __forceinline__ int plan_up(TimePlan& p, long long my_ts, const Stage* stg,
+                                       const TimeTables& tt) {
+  const bool asc = stg->asc;
+  const long long dlo = stg->cmin - my_ts, dhi = stg->cmax - my_ts;
+  const bool fast = dhi < 0x7FFFFFFFll && dlo > -0x7FFFFFFFll;
+  const bool mono = fast && asc && dlo >= 0;
+  p.k_a = p.k_b = 0;
+  p.split = 32;
+  if (mono) {
+    p.k_a = bucket32(static_cast<uint32_t>(dlo), tt.oct());
+    p.k_b = bucket32(static_cast<uint32_t>(dhi), tt.oct());
+  }
+  if (__all_sync(0xffffffffu, mono)) {
+    const int spread = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(p.k_b - p.k_a));
+    if (spread == 0) {
+      plan_pairs(p, tt);
+      return TB_CONST;
+    }
+    if (spread == 1) {
+      const uint32_t my32 = static_cast<uint32_t>(my_ts);
+      p.split = count_below_up(stg->ts32, my32, tt.thr32()[p.k_b]);
+      plan_pairs(p, tt);
+      return TB_SPLIT;
+    }
+  }
+  return __all_sync(0xffffffffu, fast) ? TB_GEN32 : TB_GEN64;
+}
+
+// Plan of the dQ kernel (rows = queries at my_ts, columns = earlier keys):
+// dt = t_query - t_key falls along the columns, from bucket k_a to k_b.
+__device__ __forceinline__ int plan_dn(TimePlan& p, long long my_ts, const Stage* stg,
+                                       const TimeTables& tt) {
+  const bool asc = stg->asc;
+  const long long dhi = my_ts - stg->cmin, dlo = my_ts - stg->cmax;
+  const bool fast = dhi < 0x7FFFFFFFll && dlo > -0x7FFFFFFFll;
+  const bool mono = fast && asc && dlo >= 0;
+  p.k_a = p.k_b = 0;
+  p.split = 32;
+  if (mono) {
+    p.k_a = bucket32(static_cast<uint32_t>(dhi), tt.oct());
+    p.k_b = bucket32(static_cast<uint32_t>(dlo), tt.oct());
+  }
+  if (__all_sync(0xffffffffu, mono)) {
+    const int spread = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(p.k_a - p.k_b));
+    if (spread == 0) {
+      plan_pairs(p, tt);
+      return TB_CONST;
+    }
+    if (spread == 1) {
+      const uint32_t my32 = static_cast<uint32_t>(my_ts);
+      p.split = count_at_least_dn(stg->ts32, my32, tt.thr32()[p.k_a]);
+      plan_pairs(p, tt);
+      return TB_SPLIT;
+    }
+  }
+  return __all_sync(0xffffffffu, fast) ? TB_GEN32 : TB_GEN64;
+}
+
+// Half time bias pair of columns 2i, 2i+1 under a TB_CONST / TB_SPLIT plan.
+template <int TB>
+__device__ __forceinline__ uint32_t plan_pair(const TimePlan& p, int i) {
+  if (TB == TB_CONST) return p.t_a;
+  return (2 * i + 1 < p.split) ? p.t_a : ((2 * i < p.split) ? p.t_ab : p.t_b);
+}
+
+// Bucket of one element on the per-element paths.
+template <int TB>
+__device__ __forceinline__ int elem_bucket(const Stage* stg, int cl, long long my_ts, uint32_t my32,
+                                           const TimeTables& tt) {
+  if (TB == TB_GEN32) {
+    const int d = static_cast<int>(stg->ts32[cl] - my32);
+    return bucket32(static_cast<uint32_t>(d < 0 ? -d : d), tt.oct());
+  }
+  return time_bucket(stg->ts[cl] - my_ts, tt.thr(), tt.first());
+}
+
+// Running sum of one row's dS' per time bucket on the per-element path: a
+// (bucket, sum) pair in registers goes to the shared histogram when the
+// bucket changes (sorted timestamps change it rarely along a row).
 __device__ __forceinline__ void run_add(int k, float v, int& run_k, float& run_s, float* s_dt) {
   if (v == 0.f) return;
   if (k == run_k) {
@@ -175,21 +268,20 @@ __device__ __forceinline__ void run_add(int k, float v, int& run_k, float& run_s
 // P'^T and dS'^T of one 32-column chunk of the dK/dV kernel (rows = keys,
 // columns = queries); the bias gradients come from the dQ kernel.  MASK:
 // the diagonal tile or the sequence's last query tile.
-// TP: 0 no time bias, 1 the chunk's bucket plan, 2 a bucket per element.
-template <bool POS, int TP, bool MASK>
+template <bool POS, int TB, bool MASK>
 __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
                                           const Stage* stg, int lane, int r, int c0, bool diag,
-                                          int qlim, const ChunkT& ct, long long my_ts,
-                                          const long long* thr, const signed char* first,
-                                          const float* rabt, uint32_t (&pk)[16],
+                                          int qlim, const TimePlan& tp, long long my_ts,
+                                          const TimeTables& tt, uint32_t (&pk)[16],
                                           uint32_t (&dk)[16]) {
-  if (TP == 0) {
+  if (TB <= TB_SPLIT) {
     // bf16x2 arithmetic: P' and dS' are bf16 operands of the next MMAs anyway
     const uint32_t* wp = stg->wpk + 31 - lane;   // pair i: diagonals 2i - lane + 31 (+1)
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const uint32_t hx = hfma2(pack_u32_pair(sv[2 * i], sv[2 * i + 1]), kHalf2,
-                                POS ? wp[2 * i] : 0u);
+      uint32_t hx = hfma2(pack_u32_pair(sv[2 * i], sv[2 * i + 1]), kHalfPair,
+                          POS ? wp[2 * i] : 0u);
+      if (TB != TB_NONE) hx = hadd2(hx, plan_pair<TB>(tp, i));
       const uint32_t t = tanh2(hx);
       uint32_t p = hfma2(hx, t, hx);
       uint32_t d = dsilu_pair(hx, t, pack_u32_pair(dav[2 * i], dav[2 * i + 1]));
@@ -205,10 +297,7 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32
     }
     return;
   }
-  float tb[4];
-  if (TP == 1)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) tb[j] = rabt[min(ct.k0 + j, kMaxBuckets - 1)];
+  const uint32_t my32 = static_cast<uint32_t>(my_ts);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float p2[2], d2[2];
@@ -217,9 +306,7 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32
       const int cl = 2 * i + hh;
       const int c = c0 + cl;
       float hb = POS ? stg->w[cl - lane + 31] : 0.f;
-      if (TP == 1)
-        hb += cl < ct.split[0] ? tb[0] : cl < ct.split[1] ? tb[1] : cl < ct.split[2] ? tb[2] : tb[3];
-      if (TP == 2) hb += rabt[time_bucket(stg->ts[cl] - my_ts, thr, first)];
+      hb += tt.rabt()[elem_bucket<TB>(stg, cl, my_ts, my32, tt)];
       const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
       const float t = tanh_approx(hx);
       float p = fmaf(hx, t, hx);
@@ -231,71 +318,35 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32
       p2[hh] = p;
       d2[hh] = ds;
     }
-    pk[i] = pack_bf16(p2[0], p2[1]);
-    dk[i] = pack_bf16(d2[0], d2[1]);
+    pk[i] = pack_bf16x2(p2[0], p2[1]);
+    dk[i] = pack_bf16x2(d2[0], d2[1]);
   }
-}
-
-// Time bias of one 32-column chunk of the dQ kernel for a query row: the
-// columns are later keys, so with sorted timestamps dt = t_query - t_key
-// falls along the chunk; when it is still >= 0 at the last column the bucket
-// drops from khi by at most 3 (few octaves), split[i] being the first column
-// with bucket below khi - i (32 when none).
-struct ChunkDn {
-  int khi;
-  int split[3];
-  bool simple;
-};
-
-__device__ __forceinline__ ChunkDn chunk_time_dn(long long my_ts, const long long* kts, bool sorted,
-                                                 const long long* thr, const signed char* first) {
-  ChunkDn c;
-  c.khi = 0;
-  c.split[0] = c.split[1] = c.split[2] = 32;
-  const long long d0 = my_ts - kts[0], d1 = my_ts - kts[31];
-  c.simple = sorted && d1 >= 0;
-  if (c.simple) {
-    const int khi = time_bucket(d0, thr, first);
-    const int klo = time_bucket(d1, thr, first);
-    c.simple = khi - klo <= 3;
-    c.khi = khi;
-#pragma unroll
-    for (int i = 0; i < 3; ++i) {
-      if (c.simple && i < khi - klo) {
-        const long long th = thr[khi - i];
-        int lo = 0, hi = 32;
-#pragma unroll 1
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (my_ts - kts[mid] >= th) lo = mid + 1; else hi = mid;
-        }
-        c.split[i] = lo;
-      }
-    }
-  }
-  return c;
 }
 
 // dS' of one 32-column chunk of the dQ kernel (rows = queries, columns =
 // keys), and its bias-gradient sums.  MASK: the diagonal tile, keys past the
 // sequence end, or query rows past it (those rows belong to no query of the
-// sequence and must not reach the bias gradients).
-template <bool POS, int TP, bool MASK>
+// sequence and must not reach the bias gradients).  The sums take dS' as
+// rounded to bf16 for the dQ MMA on the packed paths.
+template <bool POS, int TB, bool MASK>
 __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
                                          const Stage* stg, int lane, int r, int c0, bool diag,
-                                         int klim, bool row_ok, const ChunkDn& ct,
-                                         long long my_ts, const long long* thr,
-                                         const signed char* first, const float* rabt, float* win,
+                                         int klim, bool row_ok, const TimePlan& tp,
+                                         long long my_ts, const TimeTables& tt, float* win,
                                          int wbase, float* s_dt, uint32_t (&dk)[16], int& run_k,
                                          float& run_s) {
-  if (TP == 0) {
-    // bf16x2 arithmetic for dS'; the diagonal sums take its fp32 widening
+  // Diagonal sums (row - column = const) of the warp's 32 x 32 block: at
+  // column cl lane L reads lane (L + cl) mod 32, so every element with
+  // row - cl = L, or L - 32, passes through lane L.
+  float dpos = 0.f, dneg = 0.f;
+  if (TB <= TB_SPLIT) {
     const uint32_t* wp = stg->wpk + lane + 31;   // pair i: diagonals lane - 2i + 31 (-1)
-    float dpos = 0.f, dneg = 0.f;
+    float t_all = 0.f, t_b = 0.f;                // dS' of the row, and of columns >= split
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const uint32_t hx = hfma2(pack_u32_pair(sv[2 * i], sv[2 * i + 1]), kHalf2,
-                                POS ? wp[-2 * i] : 0u);
+      uint32_t hx = hfma2(pack_u32_pair(sv[2 * i], sv[2 * i + 1]), kHalfPair,
+                          POS ? wp[-2 * i] : 0u);
+      if (TB != TB_NONE) hx = hadd2(hx, plan_pair<TB>(tp, i));
       uint32_t d = dsilu_pair(hx, tanh2(hx), pack_u32_pair(dav[2 * i], dav[2 * i + 1]));
       if (MASK) {
         const int c = c0 + 2 * i;
@@ -305,80 +356,58 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
         d &= keep;
       }
       dk[i] = d;
+      const float v0 = __uint_as_float(d << 16), v1 = __uint_as_float(d & 0xFFFF0000u);
       if (POS) {
-        const float v0 = __shfl_sync(0xffffffffu, __uint_as_float(d << 16), (lane + 2 * i) & 31);
-        if (lane + 2 * i < 32) dpos += v0; else dneg += v0;
-        const float v1 =
-            __shfl_sync(0xffffffffu, __uint_as_float(d & 0xFFFF0000u), (lane + 2 * i + 1) & 31);
-        if (lane + 2 * i + 1 < 32) dpos += v1; else dneg += v1;
+        const float w0 = __shfl_sync(0xffffffffu, v0, (lane + 2 * i) & 31);
+        if (lane + 2 * i < 32) dpos += w0; else dneg += w0;
+        const float w1 = __shfl_sync(0xffffffffu, v1, (lane + 2 * i + 1) & 31);
+        if (lane + 2 * i + 1 < 32) dpos += w1; else dneg += w1;
+      }
+      if (TB != TB_NONE) t_all += v0 + v1;
+      if (TB == TB_SPLIT) {
+        if (2 * i >= tp.split) t_b += v0;
+        if (2 * i + 1 >= tp.split) t_b += v1;
       }
     }
-    if (POS) {
-      atomicAdd(&win[wbase + lane], dpos);
-      if (lane > 0) atomicAdd(&win[wbase + lane - 32], dneg);
-    }
-    return;
-  }
-  float tb[4];
-  if (TP == 1)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) tb[j] = rabt[max(ct.khi - j, 0)];
-  // Diagonal sums (row - column = const) of the warp's 32 x 32 block: at
-  // column cl lane L reads lane (L + cl) mod 32, so every element with
-  // row - cl = L, or L - 32, passes through lane L.
-  float dpos = 0.f, dneg = 0.f;
-  // simple time plan: dS' summed over the chunk and over columns past each split
-  float t_all = 0.f, t_ge0 = 0.f, t_ge1 = 0.f, t_ge2 = 0.f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float d2[2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int cl = 2 * i + hh;
-      const int c = c0 + cl;
-      float hb = POS ? stg->w[lane - cl + 31] : 0.f;
-      int kb = 0;
-      const bool ge0 = TP == 1 && cl >= ct.split[0];
-      const bool ge1 = TP == 1 && cl >= ct.split[1];
-      const bool ge2 = TP == 1 && cl >= ct.split[2];
-      if (TP == 1) hb += ge2 ? tb[3] : ge1 ? tb[2] : ge0 ? tb[1] : tb[0];
-      if (TP == 2) {
-        kb = time_bucket(my_ts - stg->ts[cl], thr, first);
-        hb += rabt[kb];
-      }
-      const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
-      const float t = tanh_approx(hx);
-      float ds = __uint_as_float(dav[cl]) * silu_grad_h(hx, t);
-      const bool masked = MASK && ((diag && c > r) || c >= klim || !row_ok);
-      if (masked) ds = 0.f;
-      d2[hh] = ds;
-      if (POS) {
-        const float v = __shfl_sync(0xffffffffu, ds, (lane + cl) & 31);
-        if (lane + cl < 32) dpos += v; else dneg += v;
-      }
-      if (TP == 1) {
-        t_all += ds;
-        if (ge0) t_ge0 += ds;
-        if (ge1) t_ge1 += ds;
-        if (ge2) t_ge2 += ds;
-      }
-      if (TP == 2 && !masked) run_add(kb, ds, run_k, run_s, s_dt);
-    }
-    dk[i] = pack_bf16(d2[0], d2[1]);
-  }
-  if (TP == 1) {
-    // The warp's 32 rows (consecutive queries) reach neighbouring buckets:
-    // sum each bucket over the warp and let one lane add it to the histogram.
-    const float tv[4] = {t_all - t_ge0, t_ge0 - t_ge1, t_ge1 - t_ge2, t_ge2};
-    const int kmin = __reduce_min_sync(0xffffffffu, ct.khi);
-    const int kmax = __reduce_max_sync(0xffffffffu, ct.khi);
+    if (TB != TB_NONE) {
+      // The warp's 32 rows (consecutive queries) reach neighbouring buckets:
+      // sum each bucket over the warp and let one lane add it to the histogram.
+      const float t_a = t_all - t_b;
+      const int kmax = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(tp.k_a));
+      const int kmin = __reduce_min_sync(0xffffffffu, static_cast<unsigned>(tp.k_b));
 #pragma unroll 1
-    for (int j = 0; j <= kmax - kmin + 3; ++j) {
-      const int kb = kmax - j, i = ct.khi - kb;
-      float v = (i == 0) ? tv[0] : (i == 1) ? tv[1] : (i == 2) ? tv[2] : (i == 3) ? tv[3] : 0.f;
+      for (int kb = kmax; kb >= kmin; --kb) {
+        float v = (tp.k_a == kb ? t_a : 0.f) + (tp.k_b == kb && TB == TB_SPLIT ? t_b : 0.f);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && v != 0.f && kb >= 0) atomicAdd(&s_dt[kb], v);
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && v != 0.f) atomicAdd(&s_dt[kb], v);
+      }
+    }
+  } else {
+    const uint32_t my32 = static_cast<uint32_t>(my_ts);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float d2[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int cl = 2 * i + hh;
+        const int c = c0 + cl;
+        float hb = POS ? stg->w[lane - cl + 31] : 0.f;
+        const int kb = elem_bucket<TB>(stg, cl, my_ts, my32, tt);
+        hb += tt.rabt()[kb];
+        const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
+        const float t = tanh_approx(hx);
+        float ds = __uint_as_float(dav[cl]) * silu_grad_h(hx, t);
+        const bool masked = MASK && ((diag && c > r) || c >= klim || !row_ok);
+        if (masked) ds = 0.f;
+        d2[hh] = ds;
+        if (POS) {
+          const float v = __shfl_sync(0xffffffffu, ds, (lane + cl) & 31);
+          if (lane + cl < 32) dpos += v; else dneg += v;
+        }
+        if (!masked) run_add(kb, ds, run_k, run_s, s_dt);
+      }
+      dk[i] = pack_bf16x2(d2[0], d2[1]);
     }
   }
   if (POS) {
@@ -429,7 +458,9 @@ constexpr int kOffDT = kOffWin + 4 * 256 * 4;             // 128 fp32
 constexpr int kOffThr = kOffDT + 128 * 4;
 constexpr int kOffFirst = kOffThr + kThrLen * 8;
 constexpr int kOffRabT = kOffFirst + 64;
-constexpr int kOffBar = kOffRabT + 128 * 4;
+constexpr int kOffOct = kOffRabT + 128 * 4;               // 32 x uint4
+constexpr int kOffThr32 = kOffOct + 32 * 16;
+constexpr int kOffBar = kOffThr32 + kMaxBuckets * 4;
 constexpr int kNumBars = 24;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffMisc + 64 + 1024;
@@ -437,12 +468,39 @@ constexpr int kSmem = kOffMisc + 64 + 1024;
 // accumulators at 256 (dV or dQ) and 384 (dK).
 constexpr uint32_t kColS = 0, kColDA = 128, kColAcc0 = 256, kColAcc1 = 384;
 
+__device__ __forceinline__ const long long* TimeTables::thr() const {
+  return reinterpret_cast<const long long*>(base + kOffThr);
+}
+__device__ __forceinline__ const signed char* TimeTables::first() const {
+  return reinterpret_cast<const signed char*>(base + kOffFirst);
+}
+__device__ __forceinline__ const float* TimeTables::rabt() const {
+  return reinterpret_cast<const float*>(base + kOffRabT);
+}
+__device__ __forceinline__ const uint4* TimeTables::oct() const {
+  return reinterpret_cast<const uint4*>(base + kOffOct);
+}
+__device__ __forceinline__ const unsigned* TimeTables::thr32() const {
+  return reinterpret_cast<const unsigned*>(base + kOffThr32);
+}
+
 // The time-bucket tables of head h in shared memory (epilogue thread et).
-__device__ __forceinline__ void init_tables(const BwdArgs& a, int h, int et, long long* s_thr,
-                                            signed char* s_first, float* s_rabt) {
-  for (int i = et; i < kThrLen; i += kEpi) s_thr[i] = a.bt.thr[i];
-  if (et < 64) s_first[et] = a.bt.first_k[et];
-  if (et < a.nb) s_rabt[et] = 0.5f * __ldg(a.rab_time + static_cast<size_t>(h) * a.nb + et);
+__device__ __forceinline__ TimeTables init_tables(const BwdArgs& a, int h, int et, uint8_t* smem) {
+  TimeTables tt;
+  long long* thr = reinterpret_cast<long long*>(smem + kOffThr);
+  signed char* first = reinterpret_cast<signed char*>(smem + kOffFirst);
+  float* rabt = reinterpret_cast<float*>(smem + kOffRabT);
+  uint4* oct = reinterpret_cast<uint4*>(smem + kOffOct);
+  unsigned* thr32 = reinterpret_cast<unsigned*>(smem + kOffThr32);
+  if (et >= 0) {
+    for (int i = et; i < kThrLen; i += kEpi) thr[i] = a.bt.thr[i];
+    if (et < 64) first[et] = a.bt.first_k[et];
+    if (et < a.nb) rabt[et] = 0.5f * __ldg(a.rab_time + static_cast<size_t>(h) * a.nb + et);
+    if (et < 32) oct[et] = a.bt.oct[et];
+    if (et < kMaxBuckets) thr32[et] = a.bt.thr32[et];
+  }
+  tt.base = smem;
+  return tt;
 }
 
 // ===================================================================== dK, dV
@@ -488,9 +546,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) { return sbase + kOffBar + 8u * i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-  long long* s_thr = reinterpret_cast<long long*>(smem + kOffThr);
-  signed char* s_first = reinterpret_cast<signed char*>(smem + kOffFirst);
-  float* s_rabt = reinterpret_cast<float*>(smem + kOffRabT);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i <= B_OUT; ++i) {
@@ -508,7 +563,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(sbase + kOffMisc, kTmemCols);
     tmem_relinquish();
   }
-  if (TIME && warp >= 2 && warp < kWarpB) init_tables(a, h, threadIdx.x - 64, s_thr, s_first, s_rabt);
+  TimeTables tt{};
+  if (TIME) tt = init_tables(a, h, (warp >= 2 && warp < kWarpB) ? threadIdx.x - 64 : -1, smem);
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -647,7 +703,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         pt = a.timestamps[checked(a.status, s + (i < n_b ? i : n_b - 1), a.T, BS_BWD_TS)];
       }
     };
-    bool sorted = true;
     auto stage = [&]() {
       if (POS) {
         const float w0 = 0.5f * pw0, w1 = 0.5f * pw1;
@@ -657,14 +712,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float n0 = __shfl_down_sync(0xffffffffu, w0, 1);
         const float n1 = __shfl_down_sync(0xffffffffu, w1, 1);
         const float w32 = __shfl_sync(0xffffffffu, w1, 0);
-        stg->wpk[lane] = pack_bf16(w0, lane < 31 ? n0 : w32);
-        stg->wpk[32 + lane] = pack_bf16(w1, lane < 31 ? n1 : 0.f);
+        stg->wpk[lane] = pack_bf16x2(w0, lane < 31 ? n0 : w32);
+        stg->wpk[32 + lane] = pack_bf16x2(w1, lane < 31 ? n1 : 0.f);
       }
-      if (TIME) {
-        stg->ts[lane] = pt;
-        const long long nxt = __shfl_down_sync(0xffffffffu, pt, 1);
-        sorted = !__any_sync(0xffffffffu, lane < 31 && nxt < pt);
-      }
+      if (TIME) stage_time(stg, lane, pt);
       __syncwarp();
     };
     prefetch(g);
@@ -688,24 +739,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld_dep(dav);
         const bool diag = (m == n);
         const int qlim = n_b - 128 * m;           // valid query columns c < qlim
-        ChunkT ct{};
-        bool generic = false;
-        if (TIME) {
-          ct = chunk_time(my_ts, stg->ts, sorted, s_thr, s_first);
-          generic = !__all_sync(0xffffffffu, ct.simple);
-        }
-        const bool msk = diag || qlim < 128;
-#define HSTU_DKV(TP_, M_)                                                                    \
-  dkv_chunk<POS, TP_, M_>(sv, dav, stg, lane, r, c0, diag, qlim, ct, my_ts, s_thr, s_first, \
-                          s_rabt, pk, dk)
-        if (!TIME) {
-          if (msk) HSTU_DKV(0, true); else HSTU_DKV(0, false);
-        } else if (generic) {
-          HSTU_DKV(2, true);
-        } else {
-          if (msk) HSTU_DKV(1, true); else HSTU_DKV(1, false);
-        }
+        {
+          // A block whose queries all precede its keys, or lie past the
+          // end, is all zeros: the masked packed path without a time plan.
+          const bool dead = (diag && c0 + 31 < 32 * q4) || c0 >= qlim;
+          TimePlan tp{};
+          const int tb = (TIME && !dead) ? plan_up(tp, my_ts, stg, tt) : TB_NONE;
+          const bool msk = (diag && c0 < 32 * q4 + 31) || c0 + 31 >= qlim;
+#define HSTU_DKV(TB_, M_)                                                                    \
+  dkv_chunk<POS, TB_, M_>(sv, dav, stg, lane, r, c0, diag, qlim, tp, my_ts, tt, pk, dk)
+          if (tb == TB_NONE) {
+            if (msk) HSTU_DKV(TB_NONE, true); else HSTU_DKV(TB_NONE, false);
+          } else if (tb == TB_CONST) {
+            if (msk) HSTU_DKV(TB_CONST, true); else HSTU_DKV(TB_CONST, false);
+          } else if (tb == TB_SPLIT) {
+            if (msk) HSTU_DKV(TB_SPLIT, true); else HSTU_DKV(TB_SPLIT, false);
+          } else if (tb == TB_GEN32) {
+            HSTU_DKV(TB_GEN32, true);
+          } else {
+            HSTU_DKV(TB_GEN64, true);
+          }
 #undef HSTU_DKV
+        }
       }
       // The group's warps have read their S^T / dA^T columns before P'^T and
       // dS'^T overwrite them.
@@ -739,11 +794,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float* f = reinterpret_cast<const float*>(vv) + 8 * i;
-        dvp[i] = make_uint4(pack_bf16(f[0] * inv_n, f[1] * inv_n), pack_bf16(f[2] * inv_n, f[3] * inv_n),
-                            pack_bf16(f[4] * inv_n, f[5] * inv_n), pack_bf16(f[6] * inv_n, f[7] * inv_n));
+        dvp[i] = make_uint4(pack_bf16x2(f[0] * inv_n, f[1] * inv_n), pack_bf16x2(f[2] * inv_n, f[3] * inv_n),
+                            pack_bf16x2(f[4] * inv_n, f[5] * inv_n), pack_bf16x2(f[6] * inv_n, f[7] * inv_n));
         const float* e = reinterpret_cast<const float*>(kv) + 8 * i;
-        dkp[i] = make_uint4(pack_bf16(e[0] * inv_n, e[1] * inv_n), pack_bf16(e[2] * inv_n, e[3] * inv_n),
-                            pack_bf16(e[4] * inv_n, e[5] * inv_n), pack_bf16(e[6] * inv_n, e[7] * inv_n));
+        dkp[i] = make_uint4(pack_bf16x2(e[0] * inv_n, e[1] * inv_n), pack_bf16x2(e[2] * inv_n, e[3] * inv_n),
+                            pack_bf16x2(e[4] * inv_n, e[5] * inv_n), pack_bf16x2(e[6] * inv_n, e[7] * inv_n));
       }
     }
     tc_fence_before();
@@ -803,9 +858,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) { return sbase + kOffBar + 8u * i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-  long long* s_thr = reinterpret_cast<long long*>(smem + kOffThr);
-  signed char* s_first = reinterpret_cast<signed char*>(smem + kOffFirst);
-  float* s_rabt = reinterpret_cast<float*>(smem + kOffRabT);
   float* s_win = reinterpret_cast<float*>(smem + kOffWin);
   float* s_dt = reinterpret_cast<float*>(smem + kOffDT);
 
@@ -830,11 +882,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_win[et] = 0.f;                        // 4 x 256 windows
       s_win[et + kEpi] = 0.f;
     }
-    if (TIME) {
-      init_tables(a, h, et, s_thr, s_first, s_rabt);
-      if (et < 128) s_dt[et] = 0.f;
-    }
+    if (TIME && et < 128) s_dt[et] = 0.f;
   }
+  TimeTables tt{};
+  if (TIME) tt = init_tables(a, h, (warp >= 2 && warp < kWarpB) ? threadIdx.x - 64 : -1, smem);
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -966,7 +1017,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         pt = a.timestamps[checked(a.status, s + (j < n_b ? j : n_b - 1), a.T, BS_BWD_TS)];
       }
     };
-    bool sorted = true;
     auto stage = [&]() {
       if (POS) {
         const float w0 = 0.5f * pw0, w1 = 0.5f * pw1;
@@ -976,14 +1026,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float p0 = __shfl_up_sync(0xffffffffu, w0, 1);
         const float p1 = __shfl_up_sync(0xffffffffu, w1, 1);
         const float w31 = __shfl_sync(0xffffffffu, w0, 31);
-        stg->wpk[lane] = pack_bf16(w0, lane > 0 ? p0 : 0.f);
-        stg->wpk[32 + lane] = pack_bf16(w1, lane > 0 ? p1 : w31);
+        stg->wpk[lane] = pack_bf16x2(w0, lane > 0 ? p0 : 0.f);
+        stg->wpk[32 + lane] = pack_bf16x2(w1, lane > 0 ? p1 : w31);
       }
-      if (TIME) {
-        stg->ts[lane] = pt;
-        const long long nxt = __shfl_down_sync(0xffffffffu, pt, 1);
-        sorted = !__any_sync(0xffffffffu, lane < 31 && nxt < pt);
-      }
+      if (TIME) stage_time(stg, lane, pt);
       __syncwarp();
     };
     prefetch(g);
@@ -1012,26 +1058,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c0 = 64 * u + 32 * c2;            // key column within tile k
         const bool diag = (k == m);
         const int klim = n_b - 128 * k;             // valid key columns c < klim
-        ChunkDn ct{};
-        bool generic = false;
-        if (TIME) {
-          ct = chunk_time_dn(my_ts, stg->ts, sorted, s_thr, s_first);
-          generic = !__all_sync(0xffffffffu, ct.simple);
-        }
-        // window index r - c + 127 of the block's diagonals
-        const int wbase = 32 * q4 - c0 + 127;
-        const bool msk = diag || klim < 128 || !__all_sync(0xffffffffu, row_ok);
-#define HSTU_DQ(TP_, M_)                                                                    \
-  dq_chunk<POS, TP_, M_>(sv, dav, stg, lane, r, c0, diag, klim, row_ok, ct, my_ts, s_thr,  \
-                         s_first, s_rabt, win, wbase, s_dt, dk, run_k, run_s)
-        if (!TIME) {
-          if (msk) HSTU_DQ(0, true); else HSTU_DQ(0, false);
-        } else if (generic) {
-          HSTU_DQ(2, true);
-        } else {
-          if (msk) HSTU_DQ(1, true); else HSTU_DQ(1, false);
-        }
+        {
+          // A block whose keys all follow its queries, or lie past the end,
+          // or whose rows all do, is all zeros: the masked packed path
+          // without a time plan.
+          const bool dead =
+              (diag && c0 > 32 * q4 + 31) || c0 >= klim || !__any_sync(0xffffffffu, row_ok);
+          TimePlan tp{};
+          const int tb = (TIME && !dead) ? plan_dn(tp, my_ts, stg, tt) : TB_NONE;
+          // window index r - c + 127 of the block's diagonals
+          const int wbase = 32 * q4 - c0 + 127;
+          const bool msk = (diag && c0 + 31 > 32 * q4) || c0 + 31 >= klim ||
+                           !__all_sync(0xffffffffu, row_ok);
+#define HSTU_DQ(TB_, M_)                                                                    \
+  dq_chunk<POS, TB_, M_>(sv, dav, stg, lane, r, c0, diag, klim, row_ok, tp, my_ts, tt, win, \
+                         wbase, s_dt, dk, run_k, run_s)
+          if (tb == TB_NONE) {
+            if (msk) HSTU_DQ(TB_NONE, true); else HSTU_DQ(TB_NONE, false);
+          } else if (tb == TB_CONST) {
+            if (msk) HSTU_DQ(TB_CONST, true); else HSTU_DQ(TB_CONST, false);
+          } else if (tb == TB_SPLIT) {
+            if (msk) HSTU_DQ(TB_SPLIT, true); else HSTU_DQ(TB_SPLIT, false);
+          } else if (tb == TB_GEN32) {
+            HSTU_DQ(TB_GEN32, true);
+          } else {
+            HSTU_DQ(TB_GEN64, true);
+          }
 #undef HSTU_DQ
+        }
       }
       // The group's warps have read their dA columns before dS' overwrites them.
       named_bar_sync(1 + g, kGroup);
@@ -1071,8 +1125,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float* f = reinterpret_cast<const float*>(qv) + 8 * i;
-        dst[i] = make_uint4(pack_bf16(f[0] * inv_n, f[1] * inv_n), pack_bf16(f[2] * inv_n, f[3] * inv_n),
-                            pack_bf16(f[4] * inv_n, f[5] * inv_n), pack_bf16(f[6] * inv_n, f[7] * inv_n));
+        dst[i] = make_uint4(pack_bf16x2(f[0] * inv_n, f[1] * inv_n), pack_bf16x2(f[2] * inv_n, f[3] * inv_n),
+                            pack_bf16x2(f[4] * inv_n, f[5] * inv_n), pack_bf16x2(f[6] * inv_n, f[7] * inv_n));
       }
     }
     if (TIME) {

@@ -141,32 +141,6 @@ __device__ __forceinline__ bool waited(bool r, int* status, int site, int j, int
   return r;
 }
 
-// ------------------------------------------------------------- bf16x2 helpers
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x (low half) = lo
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t tanh2(uint32_t x) {
-  uint32_t t;
-  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(x));
-  return t;
-}
-
-constexpr uint32_t kHalfPair = 0x3F003F00u;   // (0.5, 0.5) in bf16
-
 // SiLU of a pair of half arguments hx = x/2: x/2 (1 + tanh(x/2)) = SiLU(x).
 __device__ __forceinline__ uint32_t silu_pair(uint32_t hx) { return hfma2(hx, tanh2(hx), hx); }
 
@@ -174,13 +148,6 @@ __device__ __forceinline__ uint32_t silu_pair(uint32_t hx) { return hfma2(hx, ta
 __device__ __forceinline__ float silu_gate(float x) {
   const float hx = 0.5f * x;
   return fmaf(hx, tanh_approx(hx), hx);
-}
-
-// bucket(|dt|) for 0 <= |dt| < 2^31 from the packed per-octave thresholds.
-__device__ __forceinline__ int bucket32(uint32_t a, const uint4* oct) {
-  a = a < 1u ? 1u : a;
-  const uint4 o = oct[31 - __clz(static_cast<int>(a))];
-  return static_cast<int>(o.x) + (a >= o.y) + (a >= o.z) + (a >= o.w);
 }
 
 // Start and length of sequence b; inconsistent offsets give length -1.

@@ -1,6 +1,9 @@
 // tile_math.cuh -- per-element helpers shared by the tcgen05 kernels:
-// approximate tanh / SiLU and the integer time-bucket search.
+// approximate tanh / SiLU, bf16x2 arithmetic and the integer time-bucket
+// searches.
 #pragma once
+#include <cuda_bf16.h>
+
 #include <cstdint>
 
 namespace hstu {
@@ -33,5 +36,47 @@ __device__ __forceinline__ int time_bucket(long long dt, const long long* thr,
   k += (aa >= thr[k + 1]);
   return k;
 }
+
+// bucket(|dt|) for 0 <= |dt| < 2^31 from the packed per-octave table oct[e] =
+// {bucket(2^e), thr[k+1], thr[k+2], thr[k+3]} (32-bit thresholds).
+__device__ __forceinline__ int bucket32(uint32_t a, const uint4* oct) {
+  a = a < 1u ? 1u : a;
+  const uint4 o = oct[31 - __clz(static_cast<int>(a))];
+  return static_cast<int>(o.x) + (a >= o.y) + (a >= o.z) + (a >= o.w);
+}
+
+// ------------------------------------------------------------- bf16x2 pairs
+// A pair packs two bf16 values in one 32-bit register, the lower-indexed
+// element in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x (low half) = lo
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t tanh2(uint32_t x) {
+  uint32_t t;
+  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(x));
+  return t;
+}
+
+constexpr uint32_t kHalfPair = 0x3F003F00u;   // (0.5, 0.5) in bf16
 
 }  // namespace hstu
