@@ -146,6 +146,27 @@ def causal_flops(lengths: Sequence[int], heads: int, d_qk: int, d_v: int) -> int
     return 2 * pairs * heads * (d_qk + d_v)
 
 
+def wide_time_span(inp: "Inputs", how: str) -> "Inputs":
+    """Timestamps whose differences reach 2^31 s and beyond, for the kernels'
+    64-bit time paths: "wide" scales every gap of each sequence by 2e7 (gaps of
+    minutes become gaps of decades), "jump" adds 3e9 s to the second half of
+    each sequence.  Sorted order is kept; inp is changed in place and returned."""
+    ts = inp.timestamps.clone()
+    off = inp.offsets.tolist()
+    for b in range(len(off) - 1):
+        s, e = off[b], off[b + 1]
+        if e - s < 2:
+            continue
+        if how == "wide":
+            ts[s:e] = TIME_T0 + (ts[s:e] - ts[s]) * 20_000_000
+        elif how == "jump":
+            ts[s + (e - s) // 2:e] += 3_000_000_000
+        else:
+            raise ValueError(how)
+    inp.timestamps = ts
+    return inp
+
+
 def stochastic_length(lengths: Sequence[int], keep_len: int, prob: float,
                       generator: torch.Generator) -> List[int]:
     """Stochastic Length ("HSTU Hierarchical Sequential Transduction Units",

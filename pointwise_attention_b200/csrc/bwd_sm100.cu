@@ -119,15 +119,31 @@ __device__ __forceinline__ uint32_t pack_u32_pair(uint32_t lo, uint32_t hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Element hh (0: low, 1: high half) of a bf16 pair, widened to fp32.
+__device__ __forceinline__ float bf16_half(uint32_t pair, int hh) {
+  return __uint_as_float(hh ? (pair & 0xFFFF0000u) : (pair << 16));
+}
+
+// S and dA of one 32-column chunk (fp32 from TMEM) as bf16 pairs: every
+// per-element path works from these, so the fp32 registers die here.
+__device__ __forceinline__ void pack_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
+                                           uint32_t (&sp)[16], uint32_t (&dp)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    sp[i] = pack_u32_pair(sv[2 * i], sv[2 * i + 1]);
+    dp[i] = pack_u32_pair(dav[2 * i], dav[2 * i + 1]);
+  }
+}
+
 // Time-bias plan of one warp's 32 x 32 block, chosen warp-uniformly.  When the
 // block's column timestamps ascend, every |dt| is below 2^31 and dt keeps one
-// sign, each row's bucket moves monotonically along its 32 columns: TB_CONST
-// when no row's bucket changes inside the block, TB_SPLIT when each changes at
-// most once, at a per-row split column found by bisection.  Both add the time
-// bias as one more bf16 pair on the packed path.  Otherwise every element
-// looks its bucket up: TB_GEN32 on 32-bit differences, TB_GEN64 when the span
-// reaches 2^31.  TB_NONE: no time table.
-enum { TB_NONE = 0, TB_CONST = 1, TB_SPLIT = 2, TB_GEN32 = 3, TB_GEN64 = 4 };
+// sign, each row's bucket moves monotonically along its 32 columns, by
+// `spread` buckets at most over the warp: TB_CONST (spread 0), TB_SPLIT (1)
+// and TB_MULTI (2 or 3) take per-row split columns found by bisection and
+// add the time bias as one more bf16 pair on the packed path.  Otherwise
+// every element looks its bucket up: TB_GEN32 on 32-bit differences (packed
+// too), TB_GEN64 in fp32 when the span reaches 2^31.  TB_NONE: no time table.
+enum { TB_NONE = 0, TB_CONST = 1, TB_SPLIT = 2, TB_MULTI = 3, TB_GEN32 = 4, TB_GEN64 = 5 };
 
 // The time-bucket tables in shared memory, at fixed offsets from its base.
 struct TimeTables {
@@ -139,10 +155,14 @@ struct TimeTables {
   __device__ __forceinline__ const unsigned* thr32() const;
 };
 
+// Row plan: the bucket of column 0 is k_a; from column s[t] on it is t + 1
+// buckets further (up in the dK/dV kernel, down in the dQ kernel); 32: never.
+// v[t]: the half bias of bucket k_a -+ t as a (v, v) pair; t_ab = (v0, v1).
 struct TimePlan {
-  int k_a, k_b;     // buckets of the columns before / from the split
-  int split;        // first column of bucket k_b (32: none)
-  uint32_t t_a, t_b, t_ab;   // half biases as pairs: (a, a), (b, b), (a, b)
+  int k_a;
+  int s[3];
+  uint32_t v[4];
+  uint32_t t_ab;
 };
 
 // Columns c = 0..31 of the block with ts32[c] - my32 < th (dt rising along
@@ -165,90 +185,127 @@ __device__ __forceinline__ int count_at_least_dn(const uint32_t* ts32, uint32_t 
   return pos + static_cast<int>(my32 - ts32[pos] >= th);
 }
 
-__device__ __forceinline__ void plan_pairs(TimePlan& p, const TimeTables& tt) {
-  const float va = tt.rabt()[p.k_a], vb = tt.rabt()[p.k_b];
-  p.t_a = pack_bf16x2(va, va);
-  p.t_b = pack_bf16x2(vb, vb);
-  p.t_ab = pack_bf16x2(va, vb);
+__device__ __forceinline__ uint32_t bias_pair(const TimeTables& tt, int k) {
+  const float v = tt.rabt()[k];
+  return pack_bf16x2(v, v);
 }
 
-// Plan of the dK/dV kernel (rows = keys at my_ts, columns = later queries
-// with timestamps in [cmin, cmax]): dt = t_query - t_key rises along the
-// columns, so the bucket climbs from k_a at the first column to k_b.
+// Plan of the dK/dV kernel (rows = keys at my_ts, columns = later queries):
+// dt = t_query - t_key rises along the columns, so the bucket climbs.
 __device__ __forceinline__ int plan_up(TimePlan& p, long long my_ts, const Stage* stg,
                                        const TimeTables& tt) {
   const bool asc = stg->asc;
   const long long dlo = stg->cmin - my_ts, dhi = stg->cmax - my_ts;
   const bool fast = dhi < 0x7FFFFFFFll && dlo > -0x7FFFFFFFll;
   const bool mono = fast && asc && dlo >= 0;
-  p.k_a = p.k_b = 0;
-  p.split = 32;
+  int k_b = 0;
+  p.k_a = 0;
   if (mono) {
     p.k_a = bucket32(static_cast<uint32_t>(dlo), tt.oct());
-    p.k_b = bucket32(static_cast<uint32_t>(dhi), tt.oct());
+    k_b = bucket32(static_cast<uint32_t>(dhi), tt.oct());
   }
   if (__all_sync(0xffffffffu, mono)) {
-    const int spread = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(p.k_b - p.k_a));
-    if (spread == 0) {
-      plan_pairs(p, tt);
-      return TB_CONST;
-    }
-    if (spread == 1) {
+    const int spread = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(k_b - p.k_a));
+    if (spread <= 3) {
       const uint32_t my32 = static_cast<uint32_t>(my_ts);
-      p.split = count_below_up(stg->ts32, my32, tt.thr32()[p.k_b]);
-      plan_pairs(p, tt);
-      return TB_SPLIT;
+#pragma unroll
+      for (int t = 0; t < 3; ++t) {
+        const int kt = p.k_a + t + 1;
+        p.s[t] = 32;
+        if (t < spread)
+          p.s[t] = count_below_up(stg->ts32, my32, kt < kMaxBuckets ? tt.thr32()[kt] : 0xFFFFFFFFu);
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        p.v[t] = bias_pair(tt, min(p.k_a + min(t, spread), kMaxBuckets - 1));
+      if (spread == 0) return TB_CONST;
+      if (spread == 1) {
+        p.t_ab = __byte_perm(p.v[0], p.v[1], 0x7610);
+        return TB_SPLIT;
+      }
+      return TB_MULTI;
     }
   }
   return __all_sync(0xffffffffu, fast) ? TB_GEN32 : TB_GEN64;
 }
 
 // Plan of the dQ kernel (rows = queries at my_ts, columns = earlier keys):
-// dt = t_query - t_key falls along the columns, from bucket k_a to k_b.
+// dt = t_query - t_key falls along the columns, so the bucket drops.
 __device__ __forceinline__ int plan_dn(TimePlan& p, long long my_ts, const Stage* stg,
                                        const TimeTables& tt) {
   const bool asc = stg->asc;
   const long long dhi = my_ts - stg->cmin, dlo = my_ts - stg->cmax;
   const bool fast = dhi < 0x7FFFFFFFll && dlo > -0x7FFFFFFFll;
   const bool mono = fast && asc && dlo >= 0;
-  p.k_a = p.k_b = 0;
-  p.split = 32;
+  int k_b = 0;
+  p.k_a = 0;
   if (mono) {
     p.k_a = bucket32(static_cast<uint32_t>(dhi), tt.oct());
-    p.k_b = bucket32(static_cast<uint32_t>(dlo), tt.oct());
+    k_b = bucket32(static_cast<uint32_t>(dlo), tt.oct());
   }
   if (__all_sync(0xffffffffu, mono)) {
-    const int spread = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(p.k_a - p.k_b));
-    if (spread == 0) {
-      plan_pairs(p, tt);
-      return TB_CONST;
-    }
-    if (spread == 1) {
+    const int spread = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(p.k_a - k_b));
+    if (spread <= 3) {
       const uint32_t my32 = static_cast<uint32_t>(my_ts);
-      p.split = count_at_least_dn(stg->ts32, my32, tt.thr32()[p.k_a]);
-      plan_pairs(p, tt);
-      return TB_SPLIT;
+#pragma unroll
+      for (int t = 0; t < 3; ++t) {
+        // columns still in buckets >= k_a - t: dt >= thr[k_a - t]
+        const int kt = p.k_a - t;
+        p.s[t] = 32;
+        if (t < spread && kt > 0) p.s[t] = count_at_least_dn(stg->ts32, my32, tt.thr32()[kt]);
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) p.v[t] = bias_pair(tt, max(p.k_a - min(t, spread), 0));
+      if (spread == 0) return TB_CONST;
+      if (spread == 1) {
+        p.t_ab = __byte_perm(p.v[0], p.v[1], 0x7610);
+        return TB_SPLIT;
+      }
+      return TB_MULTI;
     }
   }
   return __all_sync(0xffffffffu, fast) ? TB_GEN32 : TB_GEN64;
 }
 
-// Half time bias pair of columns 2i, 2i+1 under a TB_CONST / TB_SPLIT plan.
-template <int TB>
-__device__ __forceinline__ uint32_t plan_pair(const TimePlan& p, int i) {
-  if (TB == TB_CONST) return p.t_a;
-  return (2 * i + 1 < p.split) ? p.t_a : ((2 * i < p.split) ? p.t_ab : p.t_b);
+// Index 0..3 of the plan's bias for column c (the buckets passed before it).
+__device__ __forceinline__ uint32_t plan_value(const TimePlan& p, int c) {
+  return c >= p.s[2] ? p.v[3] : c >= p.s[1] ? p.v[2] : c >= p.s[0] ? p.v[1] : p.v[0];
 }
 
-// Bucket of one element on the per-element paths.
+// Half time bias pair of columns 2i, 2i+1 under a TB_CONST / SPLIT / MULTI plan.
 template <int TB>
-__device__ __forceinline__ int elem_bucket(const Stage* stg, int cl, long long my_ts, uint32_t my32,
-                                           const TimeTables& tt) {
-  if (TB == TB_GEN32) {
-    const int d = static_cast<int>(stg->ts32[cl] - my32);
-    return bucket32(static_cast<uint32_t>(d < 0 ? -d : d), tt.oct());
-  }
-  return time_bucket(stg->ts[cl] - my_ts, tt.thr(), tt.first());
+__device__ __forceinline__ uint32_t plan_pair(const TimePlan& p, int i) {
+  if (TB == TB_CONST) return p.v[0];
+  if (TB == TB_SPLIT) return (2 * i + 1 < p.s[0]) ? p.v[0] : ((2 * i < p.s[0]) ? p.t_ab : p.v[1]);
+  return __byte_perm(plan_value(p, 2 * i), plan_value(p, 2 * i + 1), 0x7610);
+}
+
+// Buckets of columns 2i, 2i+1 on the per-element 32-bit path.
+__device__ __forceinline__ int2 gen_buckets(const Stage* stg, int i, uint32_t my32,
+                                            const TimeTables& tt) {
+  const uint2 t2 = *reinterpret_cast<const uint2*>(stg->ts32 + 2 * i);
+  const int d0 = static_cast<int>(t2.x - my32), d1 = static_cast<int>(t2.y - my32);
+  return make_int2(bucket32(static_cast<uint32_t>(d0 < 0 ? -d0 : d0), tt.oct()),
+                   bucket32(static_cast<uint32_t>(d1 < 0 ? -d1 : d1), tt.oct()));
+}
+
+// s_dt[k] += v where flag holds, without a branch.
+__device__ __forceinline__ void red_shared_if(const float* p, float v, bool flag) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q red.shared.add.f32 [%0], %1;\n\t}" ::"r"(
+          smem_u32(p)),
+      "f"(v), "r"(static_cast<unsigned>(flag))
+      : "memory");
+}
+
+// Running (bucket, sum) of one row's dS' on the packed per-element path: the
+// sum goes to the shared histogram when a nonzero element changes the bucket.
+__device__ __forceinline__ void run_add_packed(int k, float v, int& run_k, float& run_s,
+                                               float* s_dt) {
+  const bool chg = v != 0.f && k != run_k;
+  red_shared_if(s_dt + (run_k < 0 ? 0 : run_k), run_s, chg && run_s != 0.f);
+  run_s = chg ? v : run_s + v;
+  run_k = chg ? k : run_k;
 }
 
 // Running sum of one row's dS' per time bucket on the per-element path: a
@@ -269,22 +326,30 @@ __device__ __forceinline__ void run_add(int k, float v, int& run_k, float& run_s
 // columns = queries); the bias gradients come from the dQ kernel.  MASK:
 // the diagonal tile or the sequence's last query tile.
 template <bool POS, int TB, bool MASK>
-__device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
+__device__ __forceinline__ void dkv_chunk(const uint32_t (&sp)[16], const uint32_t (&dp)[16],
                                           const Stage* stg, int lane, int r, int c0, bool diag,
                                           int qlim, const TimePlan& tp, long long my_ts,
                                           const TimeTables& tt, uint32_t (&pk)[16],
                                           uint32_t (&dk)[16]) {
-  if (TB <= TB_SPLIT) {
+  if (TB != TB_GEN64) {
     // bf16x2 arithmetic: P' and dS' are bf16 operands of the next MMAs anyway
     const uint32_t* wp = stg->wpk + 31 - lane;   // pair i: diagonals 2i - lane + 31 (+1)
+    const uint32_t my32 = static_cast<uint32_t>(my_ts);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      uint32_t hx = hfma2(pack_u32_pair(sv[2 * i], sv[2 * i + 1]), kHalfPair,
-                          POS ? wp[2 * i] : 0u);
-      if (TB != TB_NONE) hx = hadd2(hx, plan_pair<TB>(tp, i));
+      // half bias pair (position + time), added before S arrives in the chain
+      uint32_t hb = POS ? wp[2 * i] : 0u;
+      if (TB == TB_GEN32) {
+        const int2 kb = gen_buckets(stg, i, my32, tt);
+        const uint32_t tb = pack_bf16x2(tt.rabt()[kb.x], tt.rabt()[kb.y]);
+        hb = POS ? hadd2(hb, tb) : tb;
+      } else if (TB != TB_NONE) {
+        hb = POS ? hadd2(hb, plan_pair<TB>(tp, i)) : plan_pair<TB>(tp, i);
+      }
+      const uint32_t hx = hfma2(sp[i], kHalfPair, hb);
       const uint32_t t = tanh2(hx);
       uint32_t p = hfma2(hx, t, hx);
-      uint32_t d = dsilu_pair(hx, t, pack_u32_pair(dav[2 * i], dav[2 * i + 1]));
+      uint32_t d = dsilu_pair(hx, t, dp[i]);
       if (MASK) {
         const int c = c0 + 2 * i;
         const uint32_t keep = (((diag && c < r) || c >= qlim) ? 0u : 0x0000FFFFu) |
@@ -297,7 +362,7 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32
     }
     return;
   }
-  const uint32_t my32 = static_cast<uint32_t>(my_ts);
+  // time spans of 2^31 or more: fp32, 64-bit bucket search
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float p2[2], d2[2];
@@ -306,11 +371,11 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32
       const int cl = 2 * i + hh;
       const int c = c0 + cl;
       float hb = POS ? stg->w[cl - lane + 31] : 0.f;
-      hb += tt.rabt()[elem_bucket<TB>(stg, cl, my_ts, my32, tt)];
-      const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
+      hb += tt.rabt()[time_bucket(stg->ts[cl] - my_ts, tt.thr(), tt.first())];
+      const float hx = fmaf(bf16_half(sp[i], hh), 0.5f, hb);
       const float t = tanh_approx(hx);
       float p = fmaf(hx, t, hx);
-      float ds = __uint_as_float(dav[cl]) * silu_grad_h(hx, t);
+      float ds = bf16_half(dp[i], hh) * silu_grad_h(hx, t);
       if (MASK && ((diag && c < r) || c >= qlim)) {
         p = 0.f;
         ds = 0.f;
@@ -326,10 +391,10 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sv)[32], const uint32
 // dS' of one 32-column chunk of the dQ kernel (rows = queries, columns =
 // keys), and its bias-gradient sums.  MASK: the diagonal tile, keys past the
 // sequence end, or query rows past it (those rows belong to no query of the
-// sequence and must not reach the bias gradients).  The sums take dS' as
-// rounded to bf16 for the dQ MMA on the packed paths.
+// sequence and must not reach the bias gradients).  On the packed paths the
+// sums take dS' as rounded to bf16 for the dQ MMA.
 template <bool POS, int TB, bool MASK>
-__device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
+__device__ __forceinline__ void dq_chunk(const uint32_t (&sp)[16], const uint32_t (&dp)[16],
                                          const Stage* stg, int lane, int r, int c0, bool diag,
                                          int klim, bool row_ok, const TimePlan& tp,
                                          long long my_ts, const TimeTables& tt, float* win,
@@ -339,15 +404,25 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
   // column cl lane L reads lane (L + cl) mod 32, so every element with
   // row - cl = L, or L - 32, passes through lane L.
   float dpos = 0.f, dneg = 0.f;
-  if (TB <= TB_SPLIT) {
+  if (TB != TB_GEN64) {
     const uint32_t* wp = stg->wpk + lane + 31;   // pair i: diagonals lane - 2i + 31 (-1)
-    float t_all = 0.f, t_b = 0.f;                // dS' of the row, and of columns >= split
+    const uint32_t my32 = static_cast<uint32_t>(my_ts);
+    // dS' of the row, and of its columns from each split on
+    float t_all = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      uint32_t hx = hfma2(pack_u32_pair(sv[2 * i], sv[2 * i + 1]), kHalfPair,
-                          POS ? wp[-2 * i] : 0u);
-      if (TB != TB_NONE) hx = hadd2(hx, plan_pair<TB>(tp, i));
-      uint32_t d = dsilu_pair(hx, tanh2(hx), pack_u32_pair(dav[2 * i], dav[2 * i + 1]));
+      // half bias pair (position + time), added before S arrives in the chain
+      uint32_t hb = POS ? wp[-2 * i] : 0u;
+      int2 kb = make_int2(0, 0);
+      if (TB == TB_GEN32) {
+        kb = gen_buckets(stg, i, my32, tt);
+        const uint32_t tb = pack_bf16x2(tt.rabt()[kb.x], tt.rabt()[kb.y]);
+        hb = POS ? hadd2(hb, tb) : tb;
+      } else if (TB != TB_NONE) {
+        hb = POS ? hadd2(hb, plan_pair<TB>(tp, i)) : plan_pair<TB>(tp, i);
+      }
+      const uint32_t hx = hfma2(sp[i], kHalfPair, hb);
+      uint32_t d = dsilu_pair(hx, tanh2(hx), dp[i]);
       if (MASK) {
         const int c = c0 + 2 * i;
         const uint32_t keep =
@@ -363,28 +438,44 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
         const float w1 = __shfl_sync(0xffffffffu, v1, (lane + 2 * i + 1) & 31);
         if (lane + 2 * i + 1 < 32) dpos += w1; else dneg += w1;
       }
-      if (TB != TB_NONE) t_all += v0 + v1;
-      if (TB == TB_SPLIT) {
-        if (2 * i >= tp.split) t_b += v0;
-        if (2 * i + 1 >= tp.split) t_b += v1;
+      if (TB == TB_GEN32) {
+        run_add_packed(kb.x, v0, run_k, run_s, s_dt);
+        run_add_packed(kb.y, v1, run_k, run_s, s_dt);
+      } else if (TB != TB_NONE) {
+        t_all += v0 + v1;
+        if (TB >= TB_SPLIT) {
+          if (2 * i >= tp.s[0]) g1 += v0;
+          if (2 * i + 1 >= tp.s[0]) g1 += v1;
+        }
+        if (TB == TB_MULTI) {
+          if (2 * i >= tp.s[1]) g2 += v0;
+          if (2 * i + 1 >= tp.s[1]) g2 += v1;
+          if (2 * i >= tp.s[2]) g3 += v0;
+          if (2 * i + 1 >= tp.s[2]) g3 += v1;
+        }
       }
     }
-    if (TB != TB_NONE) {
+    if (TB == TB_CONST || TB == TB_SPLIT || TB == TB_MULTI) {
       // The warp's 32 rows (consecutive queries) reach neighbouring buckets:
-      // sum each bucket over the warp and let one lane add it to the histogram.
-      const float t_a = t_all - t_b;
+      // sum each bucket over the warp and let one lane add it to the histogram
+      // (per-row running sums instead collide in shared memory: the rows of a
+      // warp change bucket together).
+      const float b0 = t_all - g1, b1 = g1 - g2, b2 = g2 - g3, b3 = g3;
+      const int steps = TB == TB_CONST ? 0 : TB == TB_SPLIT ? 1 : 3;
       const int kmax = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(tp.k_a));
-      const int kmin = __reduce_min_sync(0xffffffffu, static_cast<unsigned>(tp.k_b));
+      int kmin = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<unsigned>(tp.k_a))) - steps;
+      kmin = kmin < 0 ? 0 : kmin;
 #pragma unroll 1
       for (int kb = kmax; kb >= kmin; --kb) {
-        float v = (tp.k_a == kb ? t_a : 0.f) + (tp.k_b == kb && TB == TB_SPLIT ? t_b : 0.f);
+        const int t = tp.k_a - kb;
+        float v = t == 0 ? b0 : t == 1 ? b1 : t == 2 ? b2 : t == 3 ? b3 : 0.f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if (lane == 0 && v != 0.f) atomicAdd(&s_dt[kb], v);
       }
     }
   } else {
-    const uint32_t my32 = static_cast<uint32_t>(my_ts);
+    // time spans of 2^31 or more: fp32, 64-bit bucket search
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       float d2[2];
@@ -393,11 +484,11 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sv)[32], const uint32_
         const int cl = 2 * i + hh;
         const int c = c0 + cl;
         float hb = POS ? stg->w[lane - cl + 31] : 0.f;
-        const int kb = elem_bucket<TB>(stg, cl, my_ts, my32, tt);
+        const int kb = time_bucket(my_ts - stg->ts[cl], tt.thr(), tt.first());
         hb += tt.rabt()[kb];
-        const float hx = fmaf(__uint_as_float(sv[cl]), 0.5f, hb);
+        const float hx = fmaf(bf16_half(sp[i], hh), 0.5f, hb);
         const float t = tanh_approx(hx);
-        float ds = __uint_as_float(dav[cl]) * silu_grad_h(hx, t);
+        float ds = bf16_half(dp[i], hh) * silu_grad_h(hx, t);
         const bool masked = MASK && ((diag && c > r) || c >= klim || !row_ok);
         if (masked) ds = 0.f;
         d2[hh] = ds;
@@ -464,6 +555,9 @@ constexpr int kOffBar = kOffThr32 + kMaxBuckets * 4;
 constexpr int kNumBars = 24;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffMisc + 64 + 1024;
+static_assert(kOffStage % 16 == 0 && sizeof(Stage) % 8 == 0, "staging alignment");
+static_assert(kOffOct % 16 == 0 && kOffThr % 8 == 0 && kOffBar % 8 == 0, "table alignment");
+static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 // TMEM: S (or S^T) of buffer u at 64 u, dA (or dA^T) at 128 + 64 u, the
 // accumulators at 256 (dV or dQ) and 384 (dK).
 constexpr uint32_t kColS = 0, kColDA = 128, kColAcc0 = 256, kColAcc1 = 384;
@@ -737,6 +831,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32_nowait(a_addr + 32u * c2, dav);
         tmem_wait_ld_dep(sv);
         tmem_wait_ld_dep(dav);
+        uint32_t sp[16], dp[16];
+        pack_chunk(sv, dav, sp, dp);
         const bool diag = (m == n);
         const int qlim = n_b - 128 * m;           // valid query columns c < qlim
         {
@@ -747,13 +843,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int tb = (TIME && !dead) ? plan_up(tp, my_ts, stg, tt) : TB_NONE;
           const bool msk = (diag && c0 < 32 * q4 + 31) || c0 + 31 >= qlim;
 #define HSTU_DKV(TB_, M_)                                                                    \
-  dkv_chunk<POS, TB_, M_>(sv, dav, stg, lane, r, c0, diag, qlim, tp, my_ts, tt, pk, dk)
+  dkv_chunk<POS, TB_, M_>(sp, dp, stg, lane, r, c0, diag, qlim, tp, my_ts, tt, pk, dk)
           if (tb == TB_NONE) {
             if (msk) HSTU_DKV(TB_NONE, true); else HSTU_DKV(TB_NONE, false);
           } else if (tb == TB_CONST) {
             if (msk) HSTU_DKV(TB_CONST, true); else HSTU_DKV(TB_CONST, false);
           } else if (tb == TB_SPLIT) {
             if (msk) HSTU_DKV(TB_SPLIT, true); else HSTU_DKV(TB_SPLIT, false);
+          } else if (tb == TB_MULTI) {
+            HSTU_DKV(TB_MULTI, true);
           } else if (tb == TB_GEN32) {
             HSTU_DKV(TB_GEN32, true);
           } else {
@@ -1055,6 +1153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld_dep(dav);
         tc_fence_before();
         mbar_arrive(bar(B_SFREE + u));
+        uint32_t sp[16], dp[16];
+        pack_chunk(sv, dav, sp, dp);
         const int c0 = 64 * u + 32 * c2;            // key column within tile k
         const bool diag = (k == m);
         const int klim = n_b - 128 * k;             // valid key columns c < klim
@@ -1071,7 +1171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool msk = (diag && c0 + 31 > 32 * q4) || c0 + 31 >= klim ||
                            !__all_sync(0xffffffffu, row_ok);
 #define HSTU_DQ(TB_, M_)                                                                    \
-  dq_chunk<POS, TB_, M_>(sv, dav, stg, lane, r, c0, diag, klim, row_ok, tp, my_ts, tt, win, \
+  dq_chunk<POS, TB_, M_>(sp, dp, stg, lane, r, c0, diag, klim, row_ok, tp, my_ts, tt, win, \
                          wbase, s_dt, dk, run_k, run_s)
           if (tb == TB_NONE) {
             if (msk) HSTU_DQ(TB_NONE, true); else HSTU_DQ(TB_NONE, false);
@@ -1079,6 +1179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (msk) HSTU_DQ(TB_CONST, true); else HSTU_DQ(TB_CONST, false);
           } else if (tb == TB_SPLIT) {
             if (msk) HSTU_DQ(TB_SPLIT, true); else HSTU_DQ(TB_SPLIT, false);
+          } else if (tb == TB_MULTI) {
+            HSTU_DQ(TB_MULTI, true);
           } else if (tb == TB_GEN32) {
             HSTU_DQ(TB_GEN32, true);
           } else {

@@ -60,6 +60,14 @@ def test_bf16_backward_small(case):
     check_bwd(hi.make_inputs(spec(**case), seed=12), "bf16")
 
 
+@pytest.mark.parametrize("how", ["wide", "jump"])
+def test_time_span_past_2_31(how):
+    """Time differences of 2^31 s and more: blocks that cross them take the
+    64-bit per-element path, the others the 32-bit plans."""
+    inp = hi.wide_time_span(hi.make_inputs(spec((300, 150), H=2, time=True), seed=13), how)
+    check_bwd(inp, "bf16")
+
+
 def test_train_reduced_batch():
     """The training workload's shapes and distributions with 2 sequences."""
     check_bwd(hi.make_inputs(hi.workload("train", batch=2), seed=0), "bf16")
@@ -81,6 +89,17 @@ def test_train_full_size():
     for name in ("dq", "dk", "dv", "du"):
         assert_close(np64(g[name]), ref_full[name], "bf16", name)
     assert_close(np64(g["d_rab_pos"]), ref_full["d_rab_pos"], "bf16", "d_rab_pos")
+
+
+def test_train_time_full_size():
+    """Full train_time workload (16 x 2048 tokens, H=4, position and time bias):
+    every element of every gradient, d(rab_time) included, against the oracle."""
+    inp = hi.make_inputs(hi.WORKLOADS["train_time"], seed=0)
+    y, saved, dev = run_fwd(inp)
+    g = run_bwd(inp, dev, saved)
+    ref = oracle.bwd(inp)
+    for name in ("dq", "dk", "dv", "du", "d_rab_pos", "d_rab_time"):
+        assert_close(np64(g[name]), ref[name], "bf16", name)
 
 
 def test_train_sl_reduced_batch():

@@ -69,6 +69,13 @@ def test_fp32_small(case):
     check_full(inp, "f32")
 
 
+@pytest.mark.parametrize("how", ["wide", "jump"])
+def test_time_span_past_2_31(how):
+    """Time differences of 2^31 s and more take the 64-bit bucket search."""
+    inp = hi.wide_time_span(hi.make_inputs(spec((300, 150), H=2, time=True), seed=5), how)
+    check_full(inp, "bf16")
+
+
 def test_neurarch_full():
     inp = hi.make_inputs(hi.WORKLOADS["neurarch"], seed=0)
     check_full(inp, "bf16")

@@ -106,3 +106,17 @@ def test_candidate_inputs_follow_their_history():
     assert torch.equal(h.k, a.hist.k) and torch.equal(h.timestamps, a.hist.timestamps)
     spec, n = hi.CAND_WORKLOADS["mfalcon"]
     assert spec.rab_pos_len >= spec.len_range[1] + 1 and n == 512
+
+
+def test_wide_time_span_keeps_order_and_crosses_2_31():
+    sp = hi.Spec("case", "bf16", batch=3, heads=2, d_qk=128, d_v=128, lengths=(300, 1, 150),
+                 rab_time=True)
+    for how in ("wide", "jump"):
+        inp = hi.wide_time_span(hi.make_inputs(sp, seed=2), how)
+        off = inp.offsets.tolist()
+        ts = inp.timestamps
+        for b in range(len(off) - 1):
+            seq = ts[off[b]:off[b + 1]]
+            assert bool((seq[1:] >= seq[:-1]).all())
+            if len(seq) > 1:
+                assert int(seq[-1] - seq[0]) >= 2 ** 31
