@@ -124,15 +124,15 @@ __device__ __forceinline__ float bf16_half(uint32_t pair, int hh) {
   return __uint_as_float(hh ? (pair & 0xFFFF0000u) : (pair << 16));
 }
 
-// S and dA of one 32-column chunk (fp32 from TMEM) as bf16 pairs: every
-// per-element path works from these, so the fp32 registers die here.
-__device__ __forceinline__ void pack_chunk(const uint32_t (&sv)[32], const uint32_t (&dav)[32],
-                                           uint32_t (&sp)[16], uint32_t (&dp)[16]) {
+// 32 fp32 columns of this warp's TMEM lanes, loaded and packed into bf16
+// pairs: every per-element path works from the pairs, so only one block of
+// fp32 registers is ever live.
+__device__ __forceinline__ void load_pairs(uint32_t taddr, uint32_t (&out)[16]) {
+  uint32_t v[32];
+  tmem_ld32_nowait(taddr, v);
+  tmem_wait_ld_dep(v);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    sp[i] = pack_u32_pair(sv[2 * i], sv[2 * i + 1]);
-    dp[i] = pack_u32_pair(dav[2 * i], dav[2 * i + 1]);
-  }
+  for (int i = 0; i < 16; ++i) out[i] = pack_u32_pair(v[2 * i], v[2 * i + 1]);
 }
 
 // Time-bias plan of one warp's 32 x 32 block, chosen warp-uniformly.  When the
@@ -526,14 +526,15 @@ __device__ __forceinline__ void mma_n64(uint32_t d, uint32_t a_smem, uint32_t b_
            ks > 0 ? 1u : 0u);
 }
 
-// D (128 x 128) (+)= A (128 x 64 bf16 pairs in TMEM: the warp pair c2 holds its
-// 32 reduction indices in the first 16 of its 32 columns) * B (64 rows =
-// reduction index, MN-major, 64-column halves kSub apart)
+// D (128 x 128) (+)= A (128 x 64 bf16 pairs in TMEM: the warps of column
+// half c2 hold reduction indices 32 c2 .. 32 c2 + 31 as pairs in the first 16
+// of their own 32 columns, 32 c2 ..) * B (64 rows = reduction index, MN-major,
+// 64-column halves kSub apart)
 __device__ __forceinline__ void mma_tm64(uint32_t d, uint32_t a_tmem, uint32_t b_smem,
                                          bool accumulate) {
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks)
-    mma_ts(d, a_tmem + 16u * (ks >> 1) + 8u * (ks & 1), sw128_desc(b_smem + ks * 2048, kSub, 1024),
+    mma_ts(d, a_tmem + 32u * (ks >> 1) + 8u * (ks & 1), sw128_desc(b_smem + ks * 2048, kSub, 1024),
            kIdescTM, (accumulate || ks > 0) ? 1u : 0u);
 }
 
@@ -826,13 +827,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[16], dk[16];
       if (ok) {
         tc_fence_after();
-        uint32_t sv[32], dav[32];
-        tmem_ld32_nowait(s_addr + 32u * c2, sv);
-        tmem_ld32_nowait(a_addr + 32u * c2, dav);
-        tmem_wait_ld_dep(sv);
-        tmem_wait_ld_dep(dav);
         uint32_t sp[16], dp[16];
-        pack_chunk(sv, dav, sp, dp);
+        load_pairs(s_addr + 32u * c2, sp);
+        load_pairs(a_addr + 32u * c2, dp);
         const bool diag = (m == n);
         const int qlim = n_b - 128 * m;           // valid query columns c < qlim
         {
@@ -860,12 +857,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef HSTU_DKV
         }
       }
-      // The group's warps have read their S^T / dA^T columns before P'^T and
-      // dS'^T overwrite them.
-      named_bar_sync(1 + g, kGroup);
+      // P'^T and dS'^T go over this warp's own, already read S^T / dA^T
+      // columns, so the warps of a group need not wait for one another.
       if (ok) {
-        tmem_st16(s_addr + 16u * c2, pk);
-        tmem_st16(a_addr + 16u * c2, dk);
+        tmem_st16(s_addr + 32u * c2, pk);
+        tmem_st16(a_addr + 32u * c2, dk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_PFULL + u));
@@ -1135,10 +1131,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int run_k = -1;           // this row's running time-bucket sum of dS'
     float run_s = 0.f;
+    // Window w of the group's sub-tile x holds the diagonal sums of
+    // i - j = 128 (m - k) + w - 127 (k = x / 2); thread eg of the group moves
+    // entry eg to d_rab_pos and clears it once every warp has added its part
+    // (the group's sub-tile x + 2 adds to the other window, x + 4 to this one
+    // again only after every warp has passed the start of x + 2).
+    auto flush_window = [&](int x, bool ok_in) -> bool {
+      bool okw = ok_in;
+      if (okw) okw = mbar_wait(bar(B_DSFULL + (x & 1)), (x >> 1) & 1, abort_flag);
+      okw = __all_sync(0xffffffffu, okw);
+      const int k = x >> 1;
+      float* w = s_win + 512 * g + 256 * (k & 1);
+      if (okw && eg < 255) {
+        const float v = w[eg];
+        const int tbl = 128 * (m - k) + eg - 127 + a.L - 1;
+        if (v != 0.f && tbl >= 0 && tbl < Lw)
+          atomicAdd(a.d_rab_pos + static_cast<size_t>(h) * Lw + tbl, v * inv_n);
+        w[eg] = 0.f;
+      }
+      return okw;
+    };
     for (int x = g; x < nx; x += 2) {
       const int u = x & 1, k = x >> 1;              // k = key tile
       float* win = s_win + 512 * g + 256 * (k & 1);
       if (x + 2 < nx) prefetch(x + 2);
+      // Sub-tile x - 2's diagonal sums are complete once its dS' phase is
+      // (every warp adds them before arriving there), and so are the clears
+      // of this sub-tile's window, made at the start of x - 2.
+      if (POS && x >= 2) ok = flush_window(x - 2, ok);
       if (ok) ok = mbar_wait(bar(B_SFULL + u), k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t s_addr = tmem + lane_addr + kColS + 64u * u;
@@ -1146,15 +1166,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t dk[16];
       if (ok) {
         tc_fence_after();
-        uint32_t sv[32], dav[32];
-        tmem_ld32_nowait(s_addr + 32u * c2, sv);
-        tmem_ld32_nowait(a_addr + 32u * c2, dav);
-        tmem_wait_ld_dep(sv);
-        tmem_wait_ld_dep(dav);
-        tc_fence_before();
-        mbar_arrive(bar(B_SFREE + u));
         uint32_t sp[16], dp[16];
-        pack_chunk(sv, dav, sp, dp);
+        load_pairs(s_addr + 32u * c2, sp);
+        tc_fence_before();
+        mbar_arrive(bar(B_SFREE + u));            // S read: its buffer may take S of x + 2
+        load_pairs(a_addr + 32u * c2, dp);
         const int c0 = 64 * u + 32 * c2;            // key column within tile k
         const bool diag = (k == m);
         const int klim = n_b - 128 * k;             // valid key columns c < klim
@@ -1189,26 +1205,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef HSTU_DQ
         }
       }
-      // The group's warps have read their dA columns before dS' overwrites them.
-      named_bar_sync(1 + g, kGroup);
+      // dS' goes over this warp's own, already read dA columns, so the warps
+      // of a group need not wait for one another.
       if (ok) {
-        tmem_st16(a_addr + 16u * c2, dk);
+        tmem_st16(a_addr + 32u * c2, dk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_DSFULL + u));
       }
       if (x + 2 < nx) stage();
-      // The group has added sub-tile x's dS' to its diagonal sums:
-      // window w holds i - j = 128 (m - k) + w - 127.
-      named_bar_sync(1 + g, kGroup);
-      if (POS && eg < 255) {
-        const float v = win[eg];
-        const int tbl = 128 * (m - k) + eg - 127 + a.L - 1;
-        if (v != 0.f && tbl >= 0 && tbl < Lw)
-          atomicAdd(a.d_rab_pos + static_cast<size_t>(h) * Lw + tbl, v * inv_n);
-        win[eg] = 0.f;
-      }
     }
+    // the group's last sub-tile
+    const int x_last = g + 2 * ((nx - 1 - g) >> 1);
+    if (POS && x_last >= 0 && x_last < nx) ok = flush_window(x_last, ok);
     // dQ = (1/N) sum dS' K
     if (ok) ok = mbar_wait(bar(B_OUT), 0, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
