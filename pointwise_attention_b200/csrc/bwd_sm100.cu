@@ -819,9 +819,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = g; x < nx; x += 2) {
       const int u = x & 1, k = x >> 1, m = n + k;
       if (x + 2 < nx) prefetch(x + 2);
+      const int c0 = 64 * u + 32 * c2;              // query column within tile m
+      const bool diag = (m == n);
+      const int qlim = n_b - 128 * m;               // valid query columns c < qlim
+      // A block whose queries all precede its keys, or lie past the end, is
+      // all zeros: the masked packed path without a time plan.  The plan
+      // needs only the staged timestamps: taking it before the wait for S^T
+      // and dA^T hides its chain of shared-memory loads there.
+      const bool dead = (diag && c0 + 31 < 32 * q4) || c0 >= qlim;
+      TimePlan tp{};
+      const int tb = (TIME && !dead) ? plan_up(tp, my_ts, stg, tt) : TB_NONE;
       if (ok) ok = mbar_wait(bar(B_SFULL + u), k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
-      const int c0 = 64 * u + 32 * c2;              // query column within tile m
       const uint32_t s_addr = tmem + lane_addr + kColS + 64u * u;
       const uint32_t a_addr = tmem + lane_addr + kColDA + 64u * u;
       uint32_t pk[16], dk[16];
@@ -830,14 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sp[16], dp[16];
         load_pairs(s_addr + 32u * c2, sp);
         load_pairs(a_addr + 32u * c2, dp);
-        const bool diag = (m == n);
-        const int qlim = n_b - 128 * m;           // valid query columns c < qlim
         {
-          // A block whose queries all precede its keys, or lie past the
-          // end, is all zeros: the masked packed path without a time plan.
-          const bool dead = (diag && c0 + 31 < 32 * q4) || c0 >= qlim;
-          TimePlan tp{};
-          const int tb = (TIME && !dead) ? plan_up(tp, my_ts, stg, tt) : TB_NONE;
           const bool msk = (diag && c0 < 32 * q4 + 31) || c0 + 31 >= qlim;
 #define HSTU_DKV(TB_, M_)                                                                    \
   dkv_chunk<POS, TB_, M_>(sp, dp, stg, lane, r, c0, diag, qlim, tp, my_ts, tt, pk, dk)
@@ -1159,6 +1161,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (every warp adds them before arriving there), and so are the clears
       // of this sub-tile's window, made at the start of x - 2.
       if (POS && x >= 2) ok = flush_window(x - 2, ok);
+      const int c0 = 64 * u + 32 * c2;              // key column within tile k
+      const bool diag = (k == m);
+      const int klim = n_b - 128 * k;               // valid key columns c < klim
+      // A block whose keys all follow its queries, or lie past the end, or
+      // whose rows all do, is all zeros: the masked packed path without a
+      // time plan.  The plan needs only the staged timestamps: taking it
+      // before the wait for S and dA hides its chain of shared-memory loads.
+      const bool dead =
+          (diag && c0 > 32 * q4 + 31) || c0 >= klim || !__any_sync(0xffffffffu, row_ok);
+      TimePlan tp{};
+      const int tb = (TIME && !dead) ? plan_dn(tp, my_ts, stg, tt) : TB_NONE;
       if (ok) ok = mbar_wait(bar(B_SFULL + u), k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t s_addr = tmem + lane_addr + kColS + 64u * u;
@@ -1171,17 +1184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(B_SFREE + u));            // S read: its buffer may take S of x + 2
         load_pairs(a_addr + 32u * c2, dp);
-        const int c0 = 64 * u + 32 * c2;            // key column within tile k
-        const bool diag = (k == m);
-        const int klim = n_b - 128 * k;             // valid key columns c < klim
         {
-          // A block whose keys all follow its queries, or lie past the end,
-          // or whose rows all do, is all zeros: the masked packed path
-          // without a time plan.
-          const bool dead =
-              (diag && c0 > 32 * q4 + 31) || c0 >= klim || !__any_sync(0xffffffffu, row_ok);
-          TimePlan tp{};
-          const int tb = (TIME && !dead) ? plan_dn(tp, my_ts, stg, tt) : TB_NONE;
           // window index r - c + 127 of the block's diagonals
           const int wbase = 32 * q4 - c0 + 127;
           const bool msk = (diag && c0 + 31 > 32 * q4) || c0 + 31 >= klim ||
