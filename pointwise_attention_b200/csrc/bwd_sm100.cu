@@ -135,16 +135,6 @@ __device__ __forceinline__ void load_pairs(uint32_t taddr, uint32_t (&out)[16]) 
   for (int i = 0; i < 16; ++i) out[i] = pack_u32_pair(v[2 * i], v[2 * i + 1]);
 }
 
-// Time-bias plan of one warp's 32 x 32 block, chosen warp-uniformly.  When the
-// block's column timestamps ascend, every |dt| is below 2^31 and dt keeps one
-// sign, each row's bucket moves monotonically along its 32 columns, by
-// `spread` buckets at most over the warp: TB_CONST (spread 0), TB_SPLIT (1)
-// and TB_MULTI (2 or 3) take per-row split columns found by bisection and
-// add the time bias as one more bf16 pair on the packed path.  Otherwise
-// every element looks its bucket up: TB_GEN32 on 32-bit differences (packed
-// too), TB_GEN64 in fp32 when the span reaches 2^31.  TB_NONE: no time table.
-enum { TB_NONE = 0, TB_CONST = 1, TB_SPLIT = 2, TB_MULTI = 3, TB_GEN32 = 4, TB_GEN64 = 5 };
-
 // The time-bucket tables in shared memory, at fixed offsets from its base.
 struct TimeTables {
   const uint8_t* base;
@@ -154,131 +144,6 @@ struct TimeTables {
   __device__ __forceinline__ const uint4* oct() const;
   __device__ __forceinline__ const unsigned* thr32() const;
 };
-
-// Row plan: the bucket of column 0 is k_a; from column s[t] on it is t + 1
-// buckets further (up in the dK/dV kernel, down in the dQ kernel); 32: never.
-// v[t]: the half bias of bucket k_a -+ t as a (v, v) pair; t_ab = (v0, v1).
-struct TimePlan {
-  int k_a;
-  int s[3];
-  uint32_t v[4];
-  uint32_t t_ab;
-};
-
-// Columns c = 0..31 of the block with ts32[c] - my32 < th (dt rising along
-// ascending columns, dt >= 0): a fixed five-step bisection, then the last
-// column.
-__device__ __forceinline__ int count_below_up(const uint32_t* ts32, uint32_t my32, uint32_t th) {
-  int pos = 0;
-#pragma unroll
-  for (int step = 16; step > 0; step >>= 1)
-    if (ts32[pos + step - 1] - my32 < th) pos += step;
-  return pos + static_cast<int>(ts32[pos] - my32 < th);
-}
-
-// Columns with my32 - ts32[c] >= th (dt falling along ascending columns).
-__device__ __forceinline__ int count_at_least_dn(const uint32_t* ts32, uint32_t my32, uint32_t th) {
-  int pos = 0;
-#pragma unroll
-  for (int step = 16; step > 0; step >>= 1)
-    if (my32 - ts32[pos + step - 1] >= th) pos += step;
-  return pos + static_cast<int>(my32 - ts32[pos] >= th);
-}
-
-__device__ __forceinline__ uint32_t bias_pair(const TimeTables& tt, int k) {
-  const float v = tt.rabt()[k];
-  return pack_bf16x2(v, v);
-}
-
-// Plan of the dK/dV kernel (rows = keys at my_ts, columns = later queries):
-// dt = t_query - t_key rises along the columns, so the bucket climbs.
-__device__ __forceinline__ int plan_up(TimePlan& p, long long my_ts, const Stage* stg,
-                                       const TimeTables& tt) {
-  const bool asc = stg->asc;
-  const long long dlo = stg->cmin - my_ts, dhi = stg->cmax - my_ts;
-  const bool fast = dhi < 0x7FFFFFFFll && dlo > -0x7FFFFFFFll;
-  const bool mono = fast && asc && dlo >= 0;
-  int k_b = 0;
-  p.k_a = 0;
-  if (mono) {
-    p.k_a = bucket32(static_cast<uint32_t>(dlo), tt.oct());
-    k_b = bucket32(static_cast<uint32_t>(dhi), tt.oct());
-  }
-  if (__all_sync(0xffffffffu, mono)) {
-    const int spread = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(k_b - p.k_a));
-    if (spread <= 3) {
-      const uint32_t my32 = static_cast<uint32_t>(my_ts);
-#pragma unroll
-      for (int t = 0; t < 3; ++t) {
-        const int kt = p.k_a + t + 1;
-        p.s[t] = 32;
-        if (t < spread)
-          p.s[t] = count_below_up(stg->ts32, my32, kt < kMaxBuckets ? tt.thr32()[kt] : 0xFFFFFFFFu);
-      }
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-        p.v[t] = bias_pair(tt, min(p.k_a + min(t, spread), kMaxBuckets - 1));
-      if (spread == 0) return TB_CONST;
-      if (spread == 1) {
-        p.t_ab = __byte_perm(p.v[0], p.v[1], 0x7610);
-        return TB_SPLIT;
-      }
-      return TB_MULTI;
-    }
-  }
-  return __all_sync(0xffffffffu, fast) ? TB_GEN32 : TB_GEN64;
-}
-
-// Plan of the dQ kernel (rows = queries at my_ts, columns = earlier keys):
-// dt = t_query - t_key falls along the columns, so the bucket drops.
-__device__ __forceinline__ int plan_dn(TimePlan& p, long long my_ts, const Stage* stg,
-                                       const TimeTables& tt) {
-  const bool asc = stg->asc;
-  const long long dhi = my_ts - stg->cmin, dlo = my_ts - stg->cmax;
-  const bool fast = dhi < 0x7FFFFFFFll && dlo > -0x7FFFFFFFll;
-  const bool mono = fast && asc && dlo >= 0;
-  int k_b = 0;
-  p.k_a = 0;
-  if (mono) {
-    p.k_a = bucket32(static_cast<uint32_t>(dhi), tt.oct());
-    k_b = bucket32(static_cast<uint32_t>(dlo), tt.oct());
-  }
-  if (__all_sync(0xffffffffu, mono)) {
-    const int spread = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(p.k_a - k_b));
-    if (spread <= 3) {
-      const uint32_t my32 = static_cast<uint32_t>(my_ts);
-#pragma unroll
-      for (int t = 0; t < 3; ++t) {
-        // columns still in buckets >= k_a - t: dt >= thr[k_a - t]
-        const int kt = p.k_a - t;
-        p.s[t] = 32;
-        if (t < spread && kt > 0) p.s[t] = count_at_least_dn(stg->ts32, my32, tt.thr32()[kt]);
-      }
-#pragma unroll
-      for (int t = 0; t < 4; ++t) p.v[t] = bias_pair(tt, max(p.k_a - min(t, spread), 0));
-      if (spread == 0) return TB_CONST;
-      if (spread == 1) {
-        p.t_ab = __byte_perm(p.v[0], p.v[1], 0x7610);
-        return TB_SPLIT;
-      }
-      return TB_MULTI;
-    }
-  }
-  return __all_sync(0xffffffffu, fast) ? TB_GEN32 : TB_GEN64;
-}
-
-// Index 0..3 of the plan's bias for column c (the buckets passed before it).
-__device__ __forceinline__ uint32_t plan_value(const TimePlan& p, int c) {
-  return c >= p.s[2] ? p.v[3] : c >= p.s[1] ? p.v[2] : c >= p.s[0] ? p.v[1] : p.v[0];
-}
-
-// Half time bias pair of columns 2i, 2i+1 under a TB_CONST / SPLIT / MULTI plan.
-template <int TB>
-__device__ __forceinline__ uint32_t plan_pair(const TimePlan& p, int i) {
-  if (TB == TB_CONST) return p.v[0];
-  if (TB == TB_SPLIT) return (2 * i + 1 < p.s[0]) ? p.v[0] : ((2 * i < p.s[0]) ? p.t_ab : p.v[1]);
-  return __byte_perm(plan_value(p, 2 * i), plan_value(p, 2 * i + 1), 0x7610);
-}
 
 // Buckets of columns 2i, 2i+1 on the per-element 32-bit path.
 __device__ __forceinline__ int2 gen_buckets(const Stage* stg, int i, uint32_t my32,
@@ -828,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // and dA^T hides its chain of shared-memory loads there.
       const bool dead = (diag && c0 + 31 < 32 * q4) || c0 >= qlim;
       TimePlan tp{};
-      const int tb = (TIME && !dead) ? plan_up(tp, my_ts, stg, tt) : TB_NONE;
+      const int tb = (TIME && !dead) ? plan_up(tp, my_ts, stg->cmin, stg->cmax, stg->asc != 0, stg->ts32, tt) : TB_NONE;
       if (ok) ok = mbar_wait(bar(B_SFULL + u), k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t s_addr = tmem + lane_addr + kColS + 64u * u;
@@ -1171,7 +1036,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool dead =
           (diag && c0 > 32 * q4 + 31) || c0 >= klim || !__any_sync(0xffffffffu, row_ok);
       TimePlan tp{};
-      const int tb = (TIME && !dead) ? plan_dn(tp, my_ts, stg, tt) : TB_NONE;
+      const int tb = (TIME && !dead) ? plan_dn(tp, my_ts, stg->cmin, stg->cmax, stg->asc != 0, stg->ts32, tt) : TB_NONE;
       if (ok) ok = mbar_wait(bar(B_SFULL + u), k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t s_addr = tmem + lane_addr + kColS + 64u * u;
