@@ -145,15 +145,6 @@ struct TimeTables {
   __device__ __forceinline__ const unsigned* thr32() const;
 };
 
-// Buckets of columns 2i, 2i+1 on the per-element 32-bit path.
-__device__ __forceinline__ int2 gen_buckets(const Stage* stg, int i, uint32_t my32,
-                                            const TimeTables& tt) {
-  const uint2 t2 = *reinterpret_cast<const uint2*>(stg->ts32 + 2 * i);
-  const int d0 = static_cast<int>(t2.x - my32), d1 = static_cast<int>(t2.y - my32);
-  return make_int2(bucket32(static_cast<uint32_t>(d0 < 0 ? -d0 : d0), tt.oct()),
-                   bucket32(static_cast<uint32_t>(d1 < 0 ? -d1 : d1), tt.oct()));
-}
-
 // s_dt[k] += v where flag holds, without a branch.
 __device__ __forceinline__ void red_shared_if(const float* p, float v, bool flag) {
   asm volatile(
@@ -205,7 +196,7 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sp)[16], const uint32
       // half bias pair (position + time), added before S arrives in the chain
       uint32_t hb = POS ? wp[2 * i] : 0u;
       if (TB == TB_GEN32) {
-        const int2 kb = gen_buckets(stg, i, my32, tt);
+        const int2 kb = gen_bucket_pair(stg->ts32, i, my32, tt);
         const uint32_t tb = pack_bf16x2(tt.rabt()[kb.x], tt.rabt()[kb.y]);
         hb = POS ? hadd2(hb, tb) : tb;
       } else if (TB != TB_NONE) {
@@ -280,7 +271,7 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sp)[16], const uint32_
       uint32_t hb = POS ? wp[-2 * i] : 0u;
       int2 kb = make_int2(0, 0);
       if (TB == TB_GEN32) {
-        kb = gen_buckets(stg, i, my32, tt);
+        kb = gen_bucket_pair(stg->ts32, i, my32, tt);
         const uint32_t tb = pack_bf16x2(tt.rabt()[kb.x], tt.rabt()[kb.y]);
         hb = POS ? hadd2(hb, tb) : tb;
       } else if (TB != TB_NONE) {

@@ -64,7 +64,29 @@ constexpr int kOffThr = kOffMisc + 16;             // long long [kThrLen]
 constexpr int kOffFirst = kOffThr + kThrLen * 8;   // signed char [64]
 constexpr int kOffRabT = kOffFirst + 64;           // float [kMaxBuckets]: this head's time bias
 constexpr int kOffPart = kOffRabT + kMaxBuckets * 4;   // float [4][128] LayerNorm partials
-constexpr int kSmem = kOffPart + 4 * 128 * 4 + 1024;
+constexpr int kOffRabH = kOffPart + 4 * 128 * 4;       // float [kMaxBuckets]: half time bias
+constexpr int kOffOct = kOffRabH + kMaxBuckets * 4;    // uint4 [32]: per-octave thresholds
+constexpr int kOffThr32 = kOffOct + 32 * 16;           // unsigned [kMaxBuckets]
+constexpr int kOffStage = kOffThr32 + kMaxBuckets * 4; // per epilogue warp: Stage
+// Per epilogue warp, the chunk's 32 keys: half position-bias pairs of
+// neighbouring columns and the keys' timestamps (low 32 bits).
+struct Stage {
+  uint32_t ppk[16];
+  uint32_t ts32[32];
+};
+constexpr int kSmem = kOffStage + kEpiWarps * static_cast<int>(sizeof(Stage)) + 1024;
+static_assert(kOffOct % 16 == 0 && kOffStage % 16 == 0, "table alignment");
+static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+
+// The bucket tables of the epilogue in shared memory (half time bias).
+struct CandTab {
+  const uint4* oct_;
+  const unsigned* thr32_;
+  const float* rabh_;
+  __device__ __forceinline__ const uint4* oct() const { return oct_; }
+  __device__ __forceinline__ const unsigned* thr32() const { return thr32_; }
+  __device__ __forceinline__ const float* rabt() const { return rabh_; }
+};
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
@@ -89,6 +111,30 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 }  // namespace
+
+// P pairs of one 32-key chunk on bf16 pairs: half bias (position pair from
+// the staging, time pair from the plan or per element) added to S/2, SiLU as
+// hx (1 + tanh hx), keys at or past nvalid set to exactly 0.
+template <bool POS, int TB>
+__device__ __forceinline__ void cand_pairs(const uint32_t (&sv)[32], const Stage* stg,
+                                           const TimePlan& tp, uint32_t my32, const CandTab& tab,
+                                           int nvalid, uint32_t (&packed)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    uint32_t hb = POS ? stg->ppk[i] : 0u;
+    if (TB == TB_GEN32) {
+      const int2 kb = gen_bucket_pair(stg->ts32, i, my32, tab);
+      const uint32_t t2 = pack_bf16x2(tab.rabt()[kb.x], tab.rabt()[kb.y]);
+      hb = POS ? hadd2(hb, t2) : t2;
+    } else if (TB != TB_NONE) {
+      hb = POS ? hadd2(hb, plan_pair<TB>(tp, i)) : plan_pair<TB>(tp, i);
+    }
+    const uint32_t s2 = pack_bf16x2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
+    const uint32_t hx = hfma2(s2, kHalfPair, hb);
+    const uint32_t keep = (2 * i < nvalid ? 0x0000FFFFu : 0u) | (2 * i + 1 < nvalid ? 0xFFFF0000u : 0u);
+    packed[i] = hfma2(hx, tanh2(hx), hx) & keep;
+  }
+}
 
 template <bool POS, bool TIME>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -142,8 +188,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   for (int i = threadIdx.x; i < kThrLen; i += kThreads) s_thr[i] = a.bt.thr[i];
   for (int i = threadIdx.x; i < 64; i += kThreads) s_first[i] = a.bt.first_k[i];
-  if (TIME)
-    for (int i = threadIdx.x; i < a.nb; i += kThreads) s_rabt[i] = __ldg(a.rab_time + h * a.nb + i);
+  CandTab tab;
+  tab.oct_ = reinterpret_cast<const uint4*>(smem + kOffOct);
+  tab.thr32_ = reinterpret_cast<const unsigned*>(smem + kOffThr32);
+  tab.rabh_ = reinterpret_cast<const float*>(smem + kOffRabH);
+  if (TIME) {
+    for (int i = threadIdx.x; i < a.nb; i += kThreads) {
+      const float v = __ldg(a.rab_time + h * a.nb + i);
+      s_rabt[i] = v;
+      reinterpret_cast<float*>(smem + kOffRabH)[i] = 0.5f * v;
+    }
+    for (int i = threadIdx.x; i < 32; i += kThreads)
+      reinterpret_cast<uint4*>(smem + kOffOct)[i] = a.bt.oct[i];
+    for (int i = threadIdx.x; i < kMaxBuckets; i += kThreads)
+      reinterpret_cast<unsigned*>(smem + kOffThr32)[i] = a.bt.thr32[i];
+  }
   if (warp == 1) {
     tmem_alloc(sbase + kOffMisc, kTmemCols);
     tmem_relinquish();
@@ -257,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long my_ts = TIME ? __ldg(a.cand_ts + checked(a.status, cand, a.C, BS_CAND_ROW)) : 0ll;
     // rpos[d] = this head's position bias at relative position d >= 0
     const float* rpos = POS ? a.rab_pos + static_cast<size_t>(h) * (2 * a.L - 1) + (a.L - 1) : nullptr;
+    Stage* stg = reinterpret_cast<Stage*>(smem + kOffStage) + ew;
     bool ok = true;
     for (int n = 0; n < nt; ++n) {
       const int st = n % kStages;
@@ -274,55 +334,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32_nowait(saddr, sv);
       tmem_wait_ld_dep(sv);
       const int nvalid = nb - (128 * n + 32 * cs);   // columns of this chunk that are history keys
-      // Time bias plan of the chunk: |t_c - t_j| is monotone in t_j, so when
-      // the bucket of this row's smallest and largest |dt| over the chunk's
-      // keys agree (the usual case: the history is in time order and buckets
-      // widen logarithmically) one bias serves all 32 columns.
-      float tconst = 0.f;
-      bool cst = true;
-      if (TIME && nvalid > 0) {
-        long long kmn = jv ? kts : 0x7FFFFFFFFFFFFFFFll, kmx = jv ? kts : -0x7FFFFFFFFFFFFFFFll;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
-          kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
-        }
-        const long long dlo = my_ts - kmx, dhi = my_ts - kmn;
-        cst = false;
-        if (dlo >= 0 || dhi <= 0) {
-          const int k0 = time_bucket(dlo, s_thr, s_first), k1 = time_bucket(dhi, s_thr, s_first);
-          cst = k0 == k1;
-          tconst = s_rabt[k0];
-        }
-      }
       uint32_t packed[16];
-      if (!TIME || __all_sync(0xffffffffu, cst)) {
+      if (nvalid <= 0) {
+        // past the history: every column is masked
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float p2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 2 * i + e;
-            float x = __uint_as_float(sv[c]) + tconst;
-            if (POS) x += __shfl_sync(0xffffffffu, pb, c);
-            p2[e] = c < nvalid ? silu_t(x) : 0.f;   // keys past the history: exactly 0
-          }
-          packed[i] = pack2(p2[0], p2[1]);
-        }
+        for (int i = 0; i < 16; ++i) packed[i] = 0u;
       } else {
+        // Stage this warp's 32 keys: the half position-bias pair (pb_c, pb_c+1)
+        // lane c = 2i forms, and the timestamps, keys past the history
+        // repeating the last one (which keeps them ascending; they are masked).
+        __syncwarp();
+        if (POS) {
+          const float hb = 0.5f * pb;
+          const float nxt = __shfl_down_sync(0xffffffffu, hb, 1);
+          if ((lane & 1) == 0) stg->ppk[lane >> 1] = pack_bf16x2(hb, nxt);
+        }
+        TimePlan tp{};
+        int tb = TB_NONE;
+        if (TIME) {
+          const long long last = __shfl_sync(0xffffffffu, kts, nvalid < 32 ? nvalid - 1 : 31);
+          const long long kt = jv ? kts : last;
+          stg->ts32[lane] = static_cast<uint32_t>(kt);
+          const long long nx = __shfl_down_sync(0xffffffffu, kt, 1);
+          const bool asc = !__any_sync(0xffffffffu, lane < 31 && nx < kt);
+          long long kmn = kt, kmx = kt;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float p2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 2 * i + e;
-            float x = __uint_as_float(sv[c]);
-            if (POS) x += __shfl_sync(0xffffffffu, pb, c);
-            const long long kt = __shfl_sync(0xffffffffu, kts, c);
-            x += s_rabt[time_bucket(my_ts - kt, s_thr, s_first)];
-            p2[e] = c < nvalid ? silu_t(x) : 0.f;
+          for (int o = 16; o > 0; o >>= 1) {
+            kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+            kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
           }
-          packed[i] = pack2(p2[0], p2[1]);
+          __syncwarp();
+          tb = plan_dn(tp, my_ts, kmn, kmx, asc, stg->ts32, tab);
+        } else {
+          __syncwarp();
+        }
+        const uint32_t my32 = static_cast<uint32_t>(my_ts);
+        if (tb == TB_GEN64) {
+          // time spans of 2^31 or more: fp32 with the 64-bit bucket search
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float p2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = 2 * i + e;
+              float x = __uint_as_float(sv[c]);
+              if (POS) x += __shfl_sync(0xffffffffu, pb, c);
+              const long long kt = __shfl_sync(0xffffffffu, kts, c);
+              x += s_rabt[time_bucket(my_ts - kt, s_thr, s_first)];
+              p2[e] = c < nvalid ? silu_t(x) : 0.f;
+            }
+            packed[i] = pack2(p2[0], p2[1]);
+          }
+        } else {
+#define HSTU_CAND(TB_) cand_pairs<POS, TB_>(sv, stg, tp, my32, tab, nvalid, packed)
+          if (tb == TB_NONE) {
+            HSTU_CAND(TB_NONE);
+          } else if (tb == TB_CONST) {
+            HSTU_CAND(TB_CONST);
+          } else if (tb == TB_SPLIT) {
+            HSTU_CAND(TB_SPLIT);
+          } else if (tb == TB_MULTI) {
+            HSTU_CAND(TB_MULTI);
+          } else {
+            HSTU_CAND(TB_GEN32);
+          }
+#undef HSTU_CAND
         }
       }
       tmem_st16(saddr, packed);   // over this warp's own S columns, already read

@@ -223,4 +223,15 @@ __device__ __forceinline__ uint32_t plan_pair(const TimePlan& p, int i) {
   return __byte_perm(plan_value(p, 2 * i), plan_value(p, 2 * i + 1), 0x7610);
 }
 
+// Buckets of columns 2i, 2i+1 on the per-element 32-bit path (|dt| < 2^31),
+// from the low 32 bits of the columns' and the row's timestamps.
+template <class Tab>
+__device__ __forceinline__ int2 gen_bucket_pair(const uint32_t* ts32, int i, uint32_t my32,
+                                                const Tab& tt) {
+  const uint2 t2 = *reinterpret_cast<const uint2*>(ts32 + 2 * i);
+  const int d0 = static_cast<int>(t2.x - my32), d1 = static_cast<int>(t2.y - my32);
+  return make_int2(bucket32(static_cast<uint32_t>(d0 < 0 ? -d0 : d0), tt.oct()),
+                   bucket32(static_cast<uint32_t>(d1 < 0 ? -d1 : d1), tt.oct()));
+}
+
 }  // namespace hstu

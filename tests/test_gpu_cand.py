@@ -124,3 +124,15 @@ def test_full_size_sampled_candidates():
                         ci.cand_ts[keep_t])
     ref = oracle.mfalcon(sub)
     assert_close(y[keep_t.to(DEV)].double().cpu().numpy(), ref["y"], "bf16", "y")
+
+
+@pytest.mark.parametrize("how", ["wide", "jump"])
+def test_time_span_past_2_31(how):
+    """History timestamps whose differences reach 2^31 s and more: the chunks
+    that cross them take the 64-bit per-element search, the others the plans."""
+    sp = spec((300, 150), H=2)
+    ci = hi.make_cand_inputs(sp, (40, 130), seed=21)
+    hi.wide_time_span(ci.hist, how)
+    y = run(ci)
+    ref = oracle.mfalcon(ci)
+    assert_close(y.double().cpu().numpy(), ref["y"], "bf16", "y")
