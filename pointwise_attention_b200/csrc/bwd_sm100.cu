@@ -72,35 +72,16 @@ struct Stage {
   float w[64];
   long long ts[32];
   uint32_t ts32[32];
-  long long cmin, cmax;   // the columns' time range
-  int asc;                // the columns' timestamps ascend
   // bf16 pairs of neighbouring diagonals for the packed path: (w[k], w[k+1])
   // in the dK/dV kernel, (w[k], w[k-1]) in the dQ kernel
   uint32_t wpk[64];
 };
 
-// Stage the block's 32 column timestamps (lane c holds column c's), whether
-// they ascend, and their range.
+// Stage the block's 32 column timestamps (lane c holds column c's) for the
+// per-element paths.
 __device__ __forceinline__ void stage_time(Stage* stg, int lane, long long pt) {
   stg->ts[lane] = pt;
   stg->ts32[lane] = static_cast<uint32_t>(pt);
-  const long long nxt = __shfl_down_sync(0xffffffffu, pt, 1);
-  const bool asc = !__any_sync(0xffffffffu, lane < 31 && nxt < pt);
-  long long lo = pt, hi = pt;
-  if (!asc) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const long long x = __shfl_xor_sync(0xffffffffu, lo, o);
-      const long long y = __shfl_xor_sync(0xffffffffu, hi, o);
-      lo = x < lo ? x : lo;
-      hi = y > hi ? y : hi;
-    }
-  }
-  if (lane == 0) {
-    stg->cmin = lo;                  // ascending: lane 0 holds the minimum
-    stg->asc = asc;
-  }
-  if (lane == 31) stg->cmax = hi;    // and lane 31 the maximum
 }
 
 constexpr uint32_t kOne2 = 0x3F803F80u;     // (1, 1)
@@ -638,9 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     Stage* stg = reinterpret_cast<Stage*>(smem + kOffStage) + ew;
     float pw0 = 0.f, pw1 = 0.f;
     long long pt = 0;
+    uint32_t pw = 0, plan_w = 0;                    // time plan word: prefetched, current
     // Staged for sub-tile x: the 63 position-bias diagonals of this warp's
     // 32 x 32 block (i - j = 128 (m - n) + 64 u + 32 c2 + cl - 32 q4 - lane,
-    // index cl - lane + 31) and its 32 query timestamps.
+    // index cl - lane + 31), its 32 query timestamps and this row's plan.
     auto prefetch = [&](int x) {
       const int cbase = 128 * (x >> 1) + 64 * (x & 1) + 32 * c2;   // query - 128 n
       if (POS) {
@@ -652,6 +634,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (TIME) {
         const int i = 128 * n + cbase + lane;
         pt = a.timestamps[checked(a.status, s + (i < n_b ? i : n_b - 1), a.T, BS_BWD_TS)];
+        // this row's plan against the block (rows past the end read the last row's)
+        pw = a.plan_up[static_cast<size_t>(4 * n + (cbase >> 5)) * a.T +
+                       checked(a.status, row_ok ? t_row : s + n_b - 1, a.T, BS_BWD_TS)];
       }
     };
     auto stage = [&]() {
@@ -666,7 +651,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         stg->wpk[lane] = pack_bf16x2(w0, lane < 31 ? n0 : w32);
         stg->wpk[32 + lane] = pack_bf16x2(w1, lane < 31 ? n1 : 0.f);
       }
-      if (TIME) stage_time(stg, lane, pt);
+      if (TIME) {
+        stage_time(stg, lane, pt);
+        plan_w = pw;
+      }
       __syncwarp();
     };
     prefetch(g);
@@ -684,7 +672,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // and dA^T hides its chain of shared-memory loads there.
       const bool dead = (diag && c0 + 31 < 32 * q4) || c0 >= qlim;
       TimePlan tp{};
-      const int tb = (TIME && !dead) ? plan_up(tp, my_ts, stg->cmin, stg->cmax, stg->asc != 0, stg->ts32, tt) : TB_NONE;
+      int tb = TB_NONE;
+      if (TIME && !dead) {
+        tb = plan_unword(tp, plan_w);
+        plan_values<true>(tp, tb, tt);
+      }
       if (ok) ok = mbar_wait(bar(B_SFULL + u), k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t s_addr = tmem + lane_addr + kColS + 64u * u;
@@ -953,9 +945,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     Stage* stg = reinterpret_cast<Stage*>(smem + kOffStage) + ew;
     float pw0 = 0.f, pw1 = 0.f;
     long long pt = 0;
+    uint32_t pw = 0, plan_w = 0;                    // time plan word: prefetched, current
     // Staged for sub-tile x: the 63 diagonals of this warp's 32 x 32 block
     // (i - j = 128 m + 32 q4 + lane - (64 x + 32 c2 + cl), index
-    // lane - cl + 31) and its 32 key timestamps.
+    // lane - cl + 31), its 32 key timestamps and this row's plan.
     auto prefetch = [&](int x) {
       const int kbase = 64 * x + 32 * c2;          // first key of the warp's columns
       if (POS) {
@@ -967,6 +960,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (TIME) {
         const int j = kbase + lane;
         pt = a.timestamps[checked(a.status, s + (j < n_b ? j : n_b - 1), a.T, BS_BWD_TS)];
+        // this row's plan against the block (rows past the end read the last row's)
+        pw = a.plan_dn[static_cast<size_t>(kbase >> 5) * a.T +
+                       checked(a.status, row_ok ? t_row : s + n_b - 1, a.T, BS_BWD_TS)];
       }
     };
     auto stage = [&]() {
@@ -981,7 +977,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         stg->wpk[lane] = pack_bf16x2(w0, lane > 0 ? p0 : 0.f);
         stg->wpk[32 + lane] = pack_bf16x2(w1, lane > 0 ? p1 : w31);
       }
-      if (TIME) stage_time(stg, lane, pt);
+      if (TIME) {
+        stage_time(stg, lane, pt);
+        plan_w = pw;
+      }
       __syncwarp();
     };
     prefetch(g);
@@ -1027,7 +1026,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool dead =
           (diag && c0 > 32 * q4 + 31) || c0 >= klim || !__any_sync(0xffffffffu, row_ok);
       TimePlan tp{};
-      const int tb = (TIME && !dead) ? plan_dn(tp, my_ts, stg->cmin, stg->cmax, stg->asc != 0, stg->ts32, tt) : TB_NONE;
+      int tb = TB_NONE;
+      if (TIME && !dead) {
+        tb = plan_unword(tp, plan_w);
+        plan_values<false>(tp, tb, tt);
+      }
       if (ok) ok = mbar_wait(bar(B_SFULL + u), k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       const uint32_t s_addr = tmem + lane_addr + kColS + 64u * u;
@@ -1135,6 +1138,75 @@ cudaError_t launch_plain(K kernel, unsigned grid, const CUtensorMap* maps, const
   return cudaGetLastError();
 }
 
+// ===================================================================== time plans
+// The shapes of the time-bias plans (first bucket, split columns, kind) of
+// every row against every 32-column block it meets, for both kernels: they
+// depend on the timestamps only, so one pass serves all H heads.  CTA (row
+// tile rt, sequence b, group z of kPlanBlocks blocks); warp w takes rows
+// 128 rt + 32 w + lane, the same 32-row groups as the epilogue warps of the
+// two kernels, so the warp-level choices of kind agree with theirs.
+constexpr int kPlanThreads = 128;
+constexpr int kPlanBlocks = 8;
+
+struct PlanTab {
+  const uint4* oct_;
+  const unsigned* thr32_;
+  __device__ __forceinline__ const uint4* oct() const { return oct_; }
+  __device__ __forceinline__ const unsigned* thr32() const { return thr32_; }
+};
+
+__global__ void __launch_bounds__(kPlanThreads) bwd_time_plans(const __grid_constant__ BwdArgs a) {
+  __shared__ uint4 s_oct[32];
+  __shared__ unsigned s_thr32[kMaxBuckets];
+  __shared__ uint32_t s_ts[kPlanThreads / 32][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 32; i += kPlanThreads) s_oct[i] = a.bt.oct[i];
+  for (int i = threadIdx.x; i < kMaxBuckets; i += kPlanThreads) s_thr32[i] = a.bt.thr32[i];
+  __syncthreads();
+  const int rt = static_cast<int>(blockIdx.x), b = static_cast<int>(blockIdx.y);
+  const int s = __ldg(a.offsets + b), e = __ldg(a.offsets + b + 1);
+  const int n_b = e - s;
+  // inconsistent offsets are reported by the attention kernels
+  if (s < 0 || n_b <= 0 || e > a.T || n_b > a.max_seq_len || 128 * rt >= n_b) return;
+  const int i = 128 * rt + 32 * warp + lane;          // this thread's row of the sequence
+  const bool row_ok = i < n_b;
+  const long long my_ts = a.timestamps[checked(a.status, s + (row_ok ? i : n_b - 1), a.T, BS_BWD_TS)];
+  const int jt = 4 * ((n_b + 127) / 128);             // blocks over the sequence's tiles
+  const int j0 = static_cast<int>(blockIdx.z) * kPlanBlocks;
+  const int j1 = min(jt, j0 + kPlanBlocks);
+  const PlanTab tab{s_oct, s_thr32};
+  uint32_t* ts32 = s_ts[warp];
+  for (int jc = j0; jc < j1; ++jc) {
+    // keys at or before the row tile (dQ); queries at or after it (dK, dV)
+    const bool dn = jc < 4 * rt + 4, up = jc >= 4 * rt;
+    const int j = 32 * jc + lane;
+    const long long kt = a.timestamps[checked(a.status, s + (j < n_b ? j : n_b - 1), a.T, BS_BWD_TS)];
+    __syncwarp();
+    ts32[lane] = static_cast<uint32_t>(kt);
+    const long long nx = __shfl_down_sync(0xffffffffu, kt, 1);
+    const bool asc = !__any_sync(0xffffffffu, lane < 31 && nx < kt);
+    long long lo = kt, hi = kt;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const long long x = __shfl_xor_sync(0xffffffffu, lo, o);
+      const long long y = __shfl_xor_sync(0xffffffffu, hi, o);
+      lo = x < lo ? x : lo;
+      hi = y > hi ? y : hi;
+    }
+    __syncwarp();
+    const size_t at = static_cast<size_t>(jc) * a.T + s + (row_ok ? i : 0);
+    TimePlan p;
+    if (dn) {
+      const int tb = plan_shape_dn(p, my_ts, lo, hi, asc, ts32, tab);
+      if (row_ok) a.plan_dn[at] = plan_word(p, tb);
+    }
+    if (up) {
+      const int tb = plan_shape_up(p, my_ts, lo, hi, asc, ts32, tab);
+      if (row_ok) a.plan_up[at] = plan_word(p, tb);
+    }
+  }
+}
+
 template <bool POS, bool TIME>
 cudaError_t launch_variant(const BwdArgs& a, const CUtensorMap* maps, cudaStream_t stream) {
   static std::atomic<bool> conf_dq[64], conf_dkv[64];   // zero-initialised: false
@@ -1157,6 +1229,13 @@ cudaError_t launch_bwd_attn_bf16_sm100(const BwdArgs& a, const CUtensorMap* maps
                                        cudaStream_t stream) {
   if (a.B == 0 || a.max_tiles == 0) return cudaSuccess;
   const bool pos = a.rab_pos != nullptr, tim = a.rab_time != nullptr;
+  if (tim) {
+    if (!a.plan_dn || !a.plan_up || a.plan_j < 4 * a.max_tiles) return cudaErrorInvalidValue;
+    const dim3 grid(a.max_tiles, a.B, (a.plan_j + kPlanBlocks - 1) / kPlanBlocks);
+    bwd_time_plans<<<grid, kPlanThreads, 0, stream>>>(a);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
   if (pos && tim) return launch_variant<true, true>(a, maps, stream);
   if (pos) return launch_variant<true, false>(a, maps, stream);
   if (tim) return launch_variant<false, true>(a, maps, stream);

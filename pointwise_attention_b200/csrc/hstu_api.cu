@@ -182,8 +182,11 @@ bool f32_supported(const hstu_problem_t* p) {
 //                    B * ceil(max_seq_len/128) u32][per (token, head) row
 //                    statistics: T * H float4]
 //   backward:       [status 256 B][dO: T*H*dv in the input dtype]
+//                    and, bf16 with a time table, [time plans: 2 * J * T u32]
+//                    with J = 4 * ceil(max_seq_len / 128)
 struct WsLayout {
-  size_t cnt_off, stats_off, dO_off, total;
+  size_t cnt_off, stats_off, dO_off, plan_off, total;
+  int plan_j;
 };
 
 WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
@@ -193,6 +196,11 @@ WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
   if (is_bwd) {
     l.dO_off = off;
     off += align_up(T * p->num_heads * p->d_v * (p->dtype == HSTU_BF16 ? 2 : 4));
+    if (p->dtype == HSTU_BF16 && p->rab_time) {
+      l.plan_j = 4 * ((p->max_seq_len + 127) / 128);
+      l.plan_off = off;
+      off += align_up(2 * static_cast<size_t>(l.plan_j) * T * 4);
+    }
   } else if (p->dtype == HSTU_BF16) {
     const size_t tiles = static_cast<size_t>((p->max_seq_len + 127) / 128);
     l.cnt_off = off;
@@ -390,6 +398,11 @@ hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void*
   a.ln_weight = p->ln_weight; a.ln_bias = p->ln_bias;
   a.d_ln_weight = d_ln_weight; a.d_ln_bias = d_ln_bias;
   a.dO = ws + l.dO_off;
+  if (l.plan_j > 0) {
+    a.plan_j = l.plan_j;
+    a.plan_dn = reinterpret_cast<uint32_t*>(ws + l.plan_off);
+    a.plan_up = a.plan_dn + static_cast<size_t>(l.plan_j) * p->total_tokens;
+  }
   a.status = common.status;
   a.B = common.B; a.T = common.T; a.H = common.H; a.d_qk = common.d_qk; a.d_v = common.d_v;
   a.max_seq_len = common.max_seq_len; a.max_tiles = common.max_tiles;

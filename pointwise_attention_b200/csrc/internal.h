@@ -94,6 +94,12 @@ struct BwdArgs {
   float* d_ln_weight;       // [H*d_v] or nullptr; zeroed by the caller of the kernels
   float* d_ln_bias;
   void* dO;          // workspace: dO in the compute dtype [T, H*d_v]
+  // workspace (bf16 with timestamps): the time plans of every 32-row group and
+  // 32-column block, [plan_j][T] words each: rows = queries against earlier
+  // keys (dQ), rows = keys against later queries (dK, dV)
+  uint32_t* plan_dn;
+  uint32_t* plan_up;
+  int plan_j;        // blocks per row: 4 * max_tiles
   int* status;
   int B, T, H, d_qk, d_v;
   int max_seq_len;

@@ -130,18 +130,22 @@ __device__ __forceinline__ uint32_t bias_pair(const Tab& tt, int k) {
   return pack_bf16x2(v, v);
 }
 
+// The plan's shape: k_a, the split columns and the plan kind, which depend on
+// the timestamps only (not on the head's bias table).
+//
 // Rows at my_ts against later columns (timestamps in [cmin, cmax], low 32
 // bits in ts32): dt = t_column - my_ts rises along the columns, so the bucket
 // climbs from k_a.
 template <class Tab>
-__device__ __forceinline__ int plan_up(TimePlan& p, long long my_ts, long long cmin,
-                                       long long cmax, bool asc, const uint32_t* ts32,
-                                       const Tab& tt) {
+__device__ __forceinline__ int plan_shape_up(TimePlan& p, long long my_ts, long long cmin,
+                                             long long cmax, bool asc, const uint32_t* ts32,
+                                             const Tab& tt) {
   const long long dlo = cmin - my_ts, dhi = cmax - my_ts;
   const bool fast = dhi < 0x7FFFFFFFll && dlo > -0x7FFFFFFFll;
   const bool mono = fast && asc && dlo >= 0;
   int k_b = 0;
   p.k_a = 0;
+  p.s[0] = p.s[1] = p.s[2] = 32;
   if (mono) {
     p.k_a = bucket32(static_cast<uint32_t>(dlo), tt.oct());
     k_b = bucket32(static_cast<uint32_t>(dhi), tt.oct());
@@ -154,18 +158,10 @@ __device__ __forceinline__ int plan_up(TimePlan& p, long long my_ts, long long c
       for (int t = 0; t < 3; ++t) {
         // columns still in buckets <= k_a + t: dt < thr[k_a + t + 1]
         const int kt = p.k_a + t + 1;
-        p.s[t] = 32;
         if (t < spread)
           p.s[t] = count_below_up(ts32, my32, kt < kMaxBuckets ? tt.thr32()[kt] : 0xFFFFFFFFu);
       }
-#pragma unroll
-      for (int t = 0; t < 4; ++t) p.v[t] = bias_pair(tt, min(p.k_a + min(t, spread), kMaxBuckets - 1));
-      if (spread == 0) return TB_CONST;
-      if (spread == 1) {
-        p.t_ab = __byte_perm(p.v[0], p.v[1], 0x7610);
-        return TB_SPLIT;
-      }
-      return TB_MULTI;
+      return spread == 0 ? TB_CONST : spread == 1 ? TB_SPLIT : TB_MULTI;
     }
   }
   return __all_sync(0xffffffffu, fast) ? TB_GEN32 : TB_GEN64;
@@ -174,14 +170,15 @@ __device__ __forceinline__ int plan_up(TimePlan& p, long long my_ts, long long c
 // Rows at my_ts against earlier columns: dt = my_ts - t_column falls along
 // the columns, so the bucket drops from k_a.
 template <class Tab>
-__device__ __forceinline__ int plan_dn(TimePlan& p, long long my_ts, long long cmin,
-                                       long long cmax, bool asc, const uint32_t* ts32,
-                                       const Tab& tt) {
+__device__ __forceinline__ int plan_shape_dn(TimePlan& p, long long my_ts, long long cmin,
+                                             long long cmax, bool asc, const uint32_t* ts32,
+                                             const Tab& tt) {
   const long long dhi = my_ts - cmin, dlo = my_ts - cmax;
   const bool fast = dhi < 0x7FFFFFFFll && dlo > -0x7FFFFFFFll;
   const bool mono = fast && asc && dlo >= 0;
   int k_b = 0;
   p.k_a = 0;
+  p.s[0] = p.s[1] = p.s[2] = 32;
   if (mono) {
     p.k_a = bucket32(static_cast<uint32_t>(dhi), tt.oct());
     k_b = bucket32(static_cast<uint32_t>(dlo), tt.oct());
@@ -194,20 +191,62 @@ __device__ __forceinline__ int plan_dn(TimePlan& p, long long my_ts, long long c
       for (int t = 0; t < 3; ++t) {
         // columns still in buckets >= k_a - t: dt >= thr[k_a - t]
         const int kt = p.k_a - t;
-        p.s[t] = 32;
         if (t < spread && kt > 0) p.s[t] = count_at_least_dn(ts32, my32, tt.thr32()[kt]);
       }
-#pragma unroll
-      for (int t = 0; t < 4; ++t) p.v[t] = bias_pair(tt, max(p.k_a - min(t, spread), 0));
-      if (spread == 0) return TB_CONST;
-      if (spread == 1) {
-        p.t_ab = __byte_perm(p.v[0], p.v[1], 0x7610);
-        return TB_SPLIT;
-      }
-      return TB_MULTI;
+      return spread == 0 ? TB_CONST : spread == 1 ? TB_SPLIT : TB_MULTI;
     }
   }
   return __all_sync(0xffffffffu, fast) ? TB_GEN32 : TB_GEN64;
+}
+
+// The plan's values: the head's half bias of the buckets it passes, as pairs
+// (UP: buckets rise from k_a, else they fall).  Kinds other than TB_CONST,
+// TB_SPLIT and TB_MULTI need none.
+template <bool UP, class Tab>
+__device__ __forceinline__ void plan_values(TimePlan& p, int tb, const Tab& tt) {
+  if (tb < TB_CONST || tb > TB_MULTI) return;
+  const int n = tb == TB_CONST ? 1 : tb == TB_SPLIT ? 2 : 4;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int k = UP ? min(p.k_a + min(t, n - 1), kMaxBuckets - 1) : max(p.k_a - min(t, n - 1), 0);
+    p.v[t] = bias_pair(tt, k);
+  }
+  p.t_ab = __byte_perm(p.v[0], p.v[1], 0x7610);
+}
+
+// Shape and values together.
+template <class Tab>
+__device__ __forceinline__ int plan_up(TimePlan& p, long long my_ts, long long cmin,
+                                       long long cmax, bool asc, const uint32_t* ts32,
+                                       const Tab& tt) {
+  const int tb = plan_shape_up(p, my_ts, cmin, cmax, asc, ts32, tt);
+  plan_values<true>(p, tb, tt);
+  return tb;
+}
+
+template <class Tab>
+__device__ __forceinline__ int plan_dn(TimePlan& p, long long my_ts, long long cmin,
+                                       long long cmax, bool asc, const uint32_t* ts32,
+                                       const Tab& tt) {
+  const int tb = plan_shape_dn(p, my_ts, cmin, cmax, asc, ts32, tt);
+  plan_values<false>(p, tb, tt);
+  return tb;
+}
+
+// A plan's shape in one word: k_a (7 bits), the three split columns (6 bits
+// each, 0..32) and the kind (3 bits).
+__device__ __forceinline__ uint32_t plan_word(const TimePlan& p, int tb) {
+  return static_cast<uint32_t>(p.k_a) | (static_cast<uint32_t>(p.s[0]) << 7) |
+         (static_cast<uint32_t>(p.s[1]) << 13) | (static_cast<uint32_t>(p.s[2]) << 19) |
+         (static_cast<uint32_t>(tb) << 25);
+}
+
+__device__ __forceinline__ int plan_unword(TimePlan& p, uint32_t w) {
+  p.k_a = static_cast<int>(w & 127u);
+  p.s[0] = static_cast<int>((w >> 7) & 63u);
+  p.s[1] = static_cast<int>((w >> 13) & 63u);
+  p.s[2] = static_cast<int>((w >> 19) & 63u);
+  return static_cast<int>((w >> 25) & 7u);
 }
 
 // The plan's half bias of column c (the buckets passed before it).
