@@ -743,10 +743,27 @@ def run_gpu(args, spec):
 
 
 def run_once(args, spec):
-    """One call of the forward or the backward, run twice on one input set:
-    the launch a profiler captures (ncu -s 1 -c 1), with nothing around it."""
+    """One call of the forward, the backward or candidate scoring (the mfalcon
+    workload), run twice on one input set: the launch a profiler captures
+    (ncu -s 1 -c 1), with nothing around it."""
     import pointwise_attention_b200 as pa
     torch.cuda.set_device(0)
+    if args.once == "cand":
+        sp, ncand = hi.CAND_WORKLOADS["mfalcon"]
+        ci = hi.make_cand_inputs(sp, ncand, seed=args.seed)
+        h = ci.hist
+        d = lambda t: None if t is None else t.to("cuda").contiguous()
+        cargs = [d(h.k), d(h.v), d(h.offsets), max(h.lengths), d(ci.qc), d(ci.kc), d(ci.vc),
+                 d(ci.uc), d(ci.cand_offsets), max(ci.counts)]
+        ckw = dict(timestamps=d(h.timestamps), cand_timestamps=d(ci.cand_ts),
+                   rab_pos=d(h.rab_pos), rab_time=d(h.rab_time), norm_len=h.norm_len)
+        y = pa.hstu_cand_fwd(*cargs, **ckw)
+        for _ in range(2):
+            pa.hstu_cand_fwd(*cargs, y=y, **ckw)
+        torch.cuda.synchronize()
+        print(json.dumps({"once": "cand", "workload": "mfalcon", "users": sp.batch,
+                          "candidates": ci.total_cands}))
+        return 0
     inp = hi.make_inputs(spec, seed=args.seed)
     d = lambda t: None if t is None else t.to("cuda").contiguous()
     q, k, v, u, offs = d(inp.q), d(inp.k), d(inp.v), d(inp.u), d(inp.offsets)
@@ -784,8 +801,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (profiling a smaller case)")
-    ap.add_argument("--once", choices=["fwd", "bwd"], default=None,
-                    help="run one forward or backward call twice and exit (for ncu captures)")
+    ap.add_argument("--once", choices=["fwd", "bwd", "cand"], default=None,
+                    help="run one forward, backward or candidate-scoring call twice and exit "
+                         "(for ncu captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
