@@ -246,6 +246,8 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sp)[16], const uint32_
     const uint32_t my32 = static_cast<uint32_t>(my_ts);
     // dS' of the row, and of its columns from each split on
     float t_all = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
+    // sums of diagonals lane - 1 and lane - 33, the next lane's to take
+    float dpos1 = 0.f, dneg1 = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       // half bias pair (position + time), added before S arrives in the chain
@@ -270,10 +272,17 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sp)[16], const uint32_
       dk[i] = d;
       const float v0 = __uint_as_float(d << 16), v1 = __uint_as_float(d & 0xFFFF0000u);
       if (POS) {
-        const float w0 = __shfl_sync(0xffffffffu, v0, (lane + 2 * i) & 31);
-        if (lane + 2 * i < 32) dpos += w0; else dneg += w0;
-        const float w1 = __shfl_sync(0xffffffffu, v1, (lane + 2 * i + 1) & 31);
-        if (lane + 2 * i + 1 < 32) dpos += w1; else dneg += w1;
+        // the pair of row (lane + 2i) mod 32: its low element lies on this
+        // lane's diagonal, its high one on the next lower diagonal
+        const uint32_t pr = __shfl_sync(0xffffffffu, d, (lane + 2 * i) & 31);
+        const float lo = __uint_as_float(pr << 16), hi = __uint_as_float(pr & 0xFFFF0000u);
+        if (lane + 2 * i < 32) {
+          dpos += lo;
+          dpos1 += hi;
+        } else {
+          dneg += lo;
+          dneg1 += hi;
+        }
       }
       if (TB == TB_GEN32) {
         run_add_packed(kb.x, v0, run_k, run_s, s_dt);
@@ -291,6 +300,14 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sp)[16], const uint32_
           if (2 * i + 1 >= tp.s[2]) g3 += v1;
         }
       }
+    }
+    if (POS) {
+      // lane L takes diagonal L from lane L + 1's second sums (lane 31 takes
+      // diagonal -1 from lane 0's)
+      const float p1 = __shfl_sync(0xffffffffu, dpos1, (lane + 1) & 31);
+      const float n1 = __shfl_sync(0xffffffffu, dneg1, (lane + 1) & 31);
+      dpos += lane < 31 ? p1 : 0.f;
+      dneg += lane < 31 ? n1 : p1;
     }
     if (TB == TB_CONST || TB == TB_SPLIT || TB == TB_MULTI) {
       // The warp's 32 rows (consecutive queries) reach neighbouring buckets:
