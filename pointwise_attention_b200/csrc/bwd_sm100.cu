@@ -319,13 +319,32 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sp)[16], const uint32_
       const int kmax = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(tp.k_a));
       int kmin = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<unsigned>(tp.k_a))) - steps;
       kmin = kmin < 0 ? 0 : kmin;
+      // Each bucket's warp sum in fixed point, one integer reduction: the
+      // scale 2^(24 - e) (2^e <= the warp's largest |b| < 2^(e+1)) keeps each
+      // term below 2^25 and 32 of them inside 30 bits, and rounds each to
+      // 2^-25 of that largest term.
+      float amax = fmaxf(fmaxf(fabsf(b0), fabsf(b1)), fmaxf(fabsf(b2), fabsf(b3)));
+      const unsigned mbits = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+      const int e = static_cast<int>(mbits >> 23) - 127;
+      if (mbits != 0u && e > -100 && e < 100) {
+        const float scale = __uint_as_float(static_cast<unsigned>(127 + 24 - e) << 23);
+        const float unscale = __uint_as_float(static_cast<unsigned>(127 - 24 + e) << 23);
 #pragma unroll 1
-      for (int kb = kmax; kb >= kmin; --kb) {
-        const int t = tp.k_a - kb;
-        float v = t == 0 ? b0 : t == 1 ? b1 : t == 2 ? b2 : t == 3 ? b3 : 0.f;
+        for (int kb = kmax; kb >= kmin; --kb) {
+          const int t = tp.k_a - kb;
+          const float v = t == 0 ? b0 : t == 1 ? b1 : t == 2 ? b2 : t == 3 ? b3 : 0.f;
+          const int sum = __reduce_add_sync(0xffffffffu, __float2int_rn(v * scale));
+          if (lane == 0 && sum != 0) atomicAdd(&s_dt[kb], static_cast<float>(sum) * unscale);
+        }
+      } else if (mbits != 0u) {
+#pragma unroll 1
+        for (int kb = kmax; kb >= kmin; --kb) {
+          const int t = tp.k_a - kb;
+          float v = t == 0 ? b0 : t == 1 ? b1 : t == 2 ? b2 : t == 3 ? b3 : 0.f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0 && v != 0.f) atomicAdd(&s_dt[kb], v);
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0 && v != 0.f) atomicAdd(&s_dt[kb], v);
+        }
       }
     }
   } else {
