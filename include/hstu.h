@@ -85,9 +85,10 @@ typedef struct {
 
 /*
  * Bytes of device workspace the call needs (is_bwd = 0: forward; 1: backward).
- * The bf16 backward with a time table also keeps there the shapes of its
- * time-bias plans, 8 bytes per token and 32-column block of max_seq_len
- * (rounded up to 128): 8 * T * 4 * ceil(max_seq_len / 128) bytes.
+ * With a time table the bf16 calls also keep there the shapes of their
+ * time-bias plans, 4 bytes per token and 32-column block of max_seq_len
+ * (rounded up to 128) for the forward, twice that for the backward:
+ * 4 * T * 4 * ceil(max_seq_len / 128) bytes (forward), 8 * T * ... (backward).
  * The workspace must be 256-byte aligned and zero-filled before its first use;
  * its first word is the device status that hstu_attn_check reads and re-arms.
  * Words 16 and 17 hold the bf16 forward's work counters: each launch hands its

@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libhstu.so")
 
-SOURCES = ["hstu_api.cu", "fwd_sm100.cu", "bwd_sm100.cu", "proj_sm100.cu", "cand_sm100.cu",
+SOURCES = ["hstu_api.cu", "fwd_sm100.cu", "bwd_sm100.cu", "plans.cu", "proj_sm100.cu", "cand_sm100.cu",
            "simt.cu", "selftest.cu", "noalloc.cu"]
 HEADERS = ["internal.h", "ptx.cuh", "tile_math.cuh", "bounds.cuh"]
 # The debug build: every data-derived index checked on the device (bounds.cuh).

@@ -1174,75 +1174,6 @@ cudaError_t launch_plain(K kernel, unsigned grid, const CUtensorMap* maps, const
   return cudaGetLastError();
 }
 
-// ===================================================================== time plans
-// The shapes of the time-bias plans (first bucket, split columns, kind) of
-// every row against every 32-column block it meets, for both kernels: they
-// depend on the timestamps only, so one pass serves all H heads.  CTA (row
-// tile rt, sequence b, group z of kPlanBlocks blocks); warp w takes rows
-// 128 rt + 32 w + lane, the same 32-row groups as the epilogue warps of the
-// two kernels, so the warp-level choices of kind agree with theirs.
-constexpr int kPlanThreads = 128;
-constexpr int kPlanBlocks = 8;
-
-struct PlanTab {
-  const uint4* oct_;
-  const unsigned* thr32_;
-  __device__ __forceinline__ const uint4* oct() const { return oct_; }
-  __device__ __forceinline__ const unsigned* thr32() const { return thr32_; }
-};
-
-__global__ void __launch_bounds__(kPlanThreads) bwd_time_plans(const __grid_constant__ BwdArgs a) {
-  __shared__ uint4 s_oct[32];
-  __shared__ unsigned s_thr32[kMaxBuckets];
-  __shared__ uint32_t s_ts[kPlanThreads / 32][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < 32; i += kPlanThreads) s_oct[i] = a.bt.oct[i];
-  for (int i = threadIdx.x; i < kMaxBuckets; i += kPlanThreads) s_thr32[i] = a.bt.thr32[i];
-  __syncthreads();
-  const int rt = static_cast<int>(blockIdx.x), b = static_cast<int>(blockIdx.y);
-  const int s = __ldg(a.offsets + b), e = __ldg(a.offsets + b + 1);
-  const int n_b = e - s;
-  // inconsistent offsets are reported by the attention kernels
-  if (s < 0 || n_b <= 0 || e > a.T || n_b > a.max_seq_len || 128 * rt >= n_b) return;
-  const int i = 128 * rt + 32 * warp + lane;          // this thread's row of the sequence
-  const bool row_ok = i < n_b;
-  const long long my_ts = a.timestamps[checked(a.status, s + (row_ok ? i : n_b - 1), a.T, BS_BWD_TS)];
-  const int jt = 4 * ((n_b + 127) / 128);             // blocks over the sequence's tiles
-  const int j0 = static_cast<int>(blockIdx.z) * kPlanBlocks;
-  const int j1 = min(jt, j0 + kPlanBlocks);
-  const PlanTab tab{s_oct, s_thr32};
-  uint32_t* ts32 = s_ts[warp];
-  for (int jc = j0; jc < j1; ++jc) {
-    // keys at or before the row tile (dQ); queries at or after it (dK, dV)
-    const bool dn = jc < 4 * rt + 4, up = jc >= 4 * rt;
-    const int j = 32 * jc + lane;
-    const long long kt = a.timestamps[checked(a.status, s + (j < n_b ? j : n_b - 1), a.T, BS_BWD_TS)];
-    __syncwarp();
-    ts32[lane] = static_cast<uint32_t>(kt);
-    const long long nx = __shfl_down_sync(0xffffffffu, kt, 1);
-    const bool asc = !__any_sync(0xffffffffu, lane < 31 && nx < kt);
-    long long lo = kt, hi = kt;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const long long x = __shfl_xor_sync(0xffffffffu, lo, o);
-      const long long y = __shfl_xor_sync(0xffffffffu, hi, o);
-      lo = x < lo ? x : lo;
-      hi = y > hi ? y : hi;
-    }
-    __syncwarp();
-    const size_t at = static_cast<size_t>(jc) * a.T + s + (row_ok ? i : 0);
-    TimePlan p;
-    if (dn) {
-      const int tb = plan_shape_dn(p, my_ts, lo, hi, asc, ts32, tab);
-      if (row_ok) a.plan_dn[at] = plan_word(p, tb);
-    }
-    if (up) {
-      const int tb = plan_shape_up(p, my_ts, lo, hi, asc, ts32, tab);
-      if (row_ok) a.plan_up[at] = plan_word(p, tb);
-    }
-  }
-}
-
 template <bool POS, bool TIME>
 cudaError_t launch_variant(const BwdArgs& a, const CUtensorMap* maps, cudaStream_t stream) {
   static std::atomic<bool> conf_dq[64], conf_dkv[64];   // zero-initialised: false
@@ -1267,9 +1198,19 @@ cudaError_t launch_bwd_attn_bf16_sm100(const BwdArgs& a, const CUtensorMap* maps
   const bool pos = a.rab_pos != nullptr, tim = a.rab_time != nullptr;
   if (tim) {
     if (!a.plan_dn || !a.plan_up || a.plan_j < 4 * a.max_tiles) return cudaErrorInvalidValue;
-    const dim3 grid(a.max_tiles, a.B, (a.plan_j + kPlanBlocks - 1) / kPlanBlocks);
-    bwd_time_plans<<<grid, kPlanThreads, 0, stream>>>(a);
-    const cudaError_t err = cudaGetLastError();
+    PlanArgs pa;
+    pa.offsets = a.offsets;
+    pa.timestamps = a.timestamps;
+    pa.plan_dn = a.plan_dn;
+    pa.plan_up = a.plan_up;
+    pa.status = a.status;
+    pa.B = a.B;
+    pa.T = a.T;
+    pa.max_seq_len = a.max_seq_len;
+    pa.max_tiles = a.max_tiles;
+    pa.plan_j = a.plan_j;
+    pa.bt = a.bt;
+    const cudaError_t err = launch_time_plans(pa, stream);
     if (err != cudaSuccess) return err;
   }
   if (pos && tim) return launch_variant<true, true>(a, maps, stream);

@@ -222,12 +222,10 @@ __device__ Item claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots,
   }
 }
 
-// Time bias of one 32-key chunk for one row, as a plan the element loop uses.
-// With the chunk's keys ascending and all at or before the row (and |dt| <
-// 2^31), dt falls along the chunk and the bucket lies between the buckets k0
-// >= k1 of its two ends: one value (CONST) or two with a split column (SPLIT,
-// found by bisection).  Otherwise every element takes its own bucket (GEN32
-// with 32-bit differences, GEN64 for time spans of 2^31 or more).
+// Time bias of one 32-key chunk for one row, as the element loop takes it:
+// one value (CONST) or two with a split column (SPLIT), from the row's plan
+// word (plans.cu); every other plan kind takes each element's own bucket
+// (GEN32 with 32-bit differences, GEN64 for time spans of 2^31 or more).
 enum { T_CONST = 0, T_SPLIT = 1, T_GEN32 = 2, T_GEN64 = 3 };
 
 struct EpiShared {
@@ -596,13 +594,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Staging of this warp's 32 x 32 block of tile n: half position bias of
       // the 63 diagonals d = r - c in [32 q4 - 32 cq - 31, 32 q4 - 32 cq + 31]
       // (table index 128 (m - n) + d + L - 1), entry k as the bf16 pair
-      // (diagonal k, diagonal k-1), and the timestamps of its 32 keys (keys
-      // past the sequence end repeat its last timestamp, which keeps them
-      // ascending; those keys are masked anyway), with their minimum, maximum
-      // and whether they ascend.
+      // (diagonal k, diagonal k-1), the timestamps of its 32 keys for the
+      // per-element paths (keys past the sequence end repeat its last
+      // timestamp; those keys are masked anyway) and this row's plan word.
       const int dbase = 32 * q4 - 32 * cq - 31;
       float pre_w0 = 0.f, pre_w1 = 0.f;
       long long pre_t = 0;
+      uint32_t pre_w = 0, plan_w = 0;             // time plan word: prefetched, current
       auto prefetch = [&](int n) {
         if (POS) {
           const int t0 = kRows * (m - n) + dbase + lane + a.L - 1;
@@ -613,10 +611,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (TIME) {
           const int jj = kCols * n + 32 * cq + lane;
           pre_t = a.timestamps[checked(a.status, s + (jj < n_b ? jj : n_b - 1), a.T, BS_FWD_TS)];
+          // this row's time plan against the block (rows past the end read the last row's)
+          pre_w = a.plan_dn[static_cast<size_t>(4 * n + cq) * a.T +
+                            checked(a.status, row_ok ? t_row : s + n_b - 1, a.T, BS_FWD_TS)];
         }
       };
-      long long kmin = 0, kmax = 0;
-      bool asc = true;
       auto stage = [&]() {   // this warp's previous reads of its buffer are done
         if (POS) {
           const float v0 = 0.5f * pre_w0, v1 = 0.5f * pre_w1;
@@ -633,24 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (TIME) {
           wts[lane] = pre_t;
           wts32[lane] = static_cast<uint32_t>(pre_t);
-          const long long nx = __shfl_down_sync(0xffffffffu, pre_t, 1);
-          asc = !__any_sync(0xffffffffu, lane < 31 && nx < pre_t);
-          // ascending keys (the usual case): the ends are the extremes
-          if (asc) {
-            kmin = __shfl_sync(0xffffffffu, pre_t, 0);
-            kmax = __shfl_sync(0xffffffffu, pre_t, 31);
-          } else {
-            long long mn = pre_t, mx = pre_t;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              const long long a2 = __shfl_xor_sync(0xffffffffu, mn, o);
-              const long long b2 = __shfl_xor_sync(0xffffffffu, mx, o);
-              mn = a2 < mn ? a2 : mn;
-              mx = b2 > mx ? b2 : mx;
-            }
-            kmin = mn;
-            kmax = mx;
-          }
+          plan_w = pre_w;
         }
         __syncwarp();
       };
@@ -683,38 +665,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             chunk_pairs<POS, false, T_CONST>(sv, wp, 0u, 0u, 0u, 0u, 0, 0u, 0ll, nullptr,
                                              nullptr, es, packed);
           } else {
-            // plan of this row's 32 keys
-            const long long dmax = my64 - kmin, dmin = my64 - kmax;
-            const bool fast = dmax < 0x7FFFFFFFll && dmax > -0x7FFFFFFFll &&
-                              dmin < 0x7FFFFFFFll && dmin > -0x7FFFFFFFll;
-            const bool mono = fast && asc && dmin >= 0;
-            int k0 = 0, k1 = 0;
-            if (mono) {
-              k0 = bucket32(static_cast<uint32_t>(dmax), es.oct);
-              k1 = bucket32(static_cast<uint32_t>(dmin), es.oct);
-            }
-            if (__all_sync(0xffffffffu, mono && k0 == k1)) {
+            // this row's plan against the block's 32 keys (the time-plan pass):
+            // the first key's bucket k0, the first column of bucket k0 - 1
+            const int kind = static_cast<int>(plan_w >> 25) & 7;
+            const int k0 = static_cast<int>(plan_w & 127u);
+            if (kind == TB_CONST) {
               const float tv = es.rabt[k0];
               chunk_pairs<POS, true, T_CONST>(sv, wp, pack_bf16x2(tv, tv), 0u, 0u, 0u, 0, my32,
                                               my64, wts32, wts, es, packed);
-            } else if (__all_sync(0xffffffffu, mono && k0 - k1 <= 1)) {
-              // first column whose bucket is k1: dt < thr[k0]
-              int split = 32;
-              if (k0 != k1) {
-                // leading columns with dt >= thr[k0] (dt falls along the
-                // chunk): a fixed five-step bisection, then the last column
-                const uint32_t th = es.thr32[k0];
-                int pos = 0;
-#pragma unroll
-                for (int step = 16; step > 0; step >>= 1)
-                  if (my32 - wts32[pos + step - 1] >= th) pos += step;
-                split = pos + static_cast<int>(my32 - wts32[pos] >= th);
-              }
-              const float hv = es.rabt[k0], lv = es.rabt[k1];
+            } else if (kind == TB_SPLIT) {
+              const int split = static_cast<int>((plan_w >> 7) & 63u);
+              const float hv = es.rabt[k0], lv = es.rabt[k0 > 0 ? k0 - 1 : 0];
               chunk_pairs<POS, true, T_SPLIT>(sv, wp, 0u, pack_bf16x2(hv, hv),
                                               pack_bf16x2(lv, lv), pack_bf16x2(hv, lv), split,
                                               my32, my64, wts32, wts, es, packed);
-            } else if (__all_sync(0xffffffffu, fast)) {
+            } else if (kind != TB_GEN64) {               // multi-bucket or per element
               chunk_pairs<POS, true, T_GEN32>(sv, wp, 0u, 0u, 0u, 0u, 0, my32, my64, wts32, wts,
                                               es, packed);
             } else {

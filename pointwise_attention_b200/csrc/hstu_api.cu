@@ -180,7 +180,8 @@ bool f32_supported(const hstu_problem_t* p) {
 // Workspace layout:
 //   forward (bf16): [status 256 B][per (sequence, query tile) head counters:
 //                    B * ceil(max_seq_len/128) u32][per (token, head) row
-//                    statistics: T * H float4]
+//                    statistics: T * H float4] and, with a time table,
+//                    [time plans (queries against keys): J * T u32]
 //   backward:       [status 256 B][dO: T*H*dv in the input dtype]
 //                    and, bf16 with a time table, [time plans: 2 * J * T u32]
 //                    with J = 4 * ceil(max_seq_len / 128)
@@ -207,6 +208,11 @@ WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
     off += align_up(static_cast<size_t>(p->batch) * tiles * 4);
     l.stats_off = off;
     off += align_up(T * p->num_heads * 16);
+    if (p->rab_time) {
+      l.plan_j = 4 * static_cast<int>(tiles);
+      l.plan_off = off;
+      off += align_up(static_cast<size_t>(l.plan_j) * T * 4);
+    }
   }
   l.total = off;
   return l;
@@ -310,14 +316,32 @@ hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* 
   a.item_cnt = reinterpret_cast<unsigned*>(ws + l.cnt_off);
   a.stats = reinterpret_cast<float4*>(ws + l.stats_off);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t err;
+  cudaError_t err = cudaSuccess;
   if (p->dtype == HSTU_BF16) {
     CUtensorMap tq, tk, tv;
     if (!make_map_3d(&tq, q, p->total_tokens, p->num_heads, 128) ||
         !make_map_3d(&tk, k, p->total_tokens, p->num_heads, 128) ||
         !make_map_3d(&tv, v, p->total_tokens, p->num_heads, 128))
       return HSTU_ERR_CUDA;
-    err = launch_fwd_bf16_sm100(a, tq, tk, tv, s);
+    if (l.plan_j > 0) {
+      // the time-plan shapes, once for all heads
+      uint32_t* plans = reinterpret_cast<uint32_t*>(ws + l.plan_off);
+      a.plan_dn = plans;
+      PlanArgs pa;
+      std::memset(&pa, 0, sizeof(pa));
+      pa.offsets = a.offsets;
+      pa.timestamps = a.timestamps;
+      pa.plan_dn = plans;
+      pa.status = a.status;
+      pa.B = a.B;
+      pa.T = a.T;
+      pa.max_seq_len = a.max_seq_len;
+      pa.max_tiles = a.max_tiles;
+      pa.plan_j = l.plan_j;
+      pa.bt = a.bt;
+      err = launch_time_plans(pa, s);
+    }
+    if (err == cudaSuccess) err = launch_fwd_bf16_sm100(a, tq, tk, tv, s);
   } else {
     err = launch_fwd_f32_simt(a, s);
   }

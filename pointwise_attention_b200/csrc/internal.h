@@ -67,6 +67,9 @@ struct FwdArgs {
   // {mean, M2, shift, 0} [T * H] for the LayerNorm over heads.
   unsigned* item_cnt;
   float4* stats;
+  // bf16 forward with a time table, workspace: the time-plan shapes of every
+  // query row against every 32-key block, [4 * max_tiles][T] words
+  const uint32_t* plan_dn;
   BucketTable bt;
 };
 
@@ -108,6 +111,21 @@ struct BwdArgs {
   int nb;
   int norm_len;
   float eps;
+  BucketTable bt;
+};
+
+// Arguments of the time-plan pass: the shapes of the time-bias plans of every
+// row against every 32-column block it meets (tile_math.cuh, plan_word),
+// [plan_j][T] words each; plan_dn: rows against earlier columns (queries
+// against keys), plan_up: rows against later columns (keys against queries),
+// either may be null.
+struct PlanArgs {
+  const int32_t* offsets;
+  const int64_t* timestamps;
+  uint32_t* plan_dn;
+  uint32_t* plan_up;
+  int* status;
+  int B, T, max_seq_len, max_tiles, plan_j;
   BucketTable bt;
 };
 
@@ -178,6 +196,7 @@ cudaError_t launch_uvqk_sm100(const ProjArgs& a, const CUtensorMap& tx, const CU
                               cudaStream_t stream);
 cudaError_t launch_out_sm100(const ProjArgs& a, const CUtensorMap& ty, const CUtensorMap& tw,
                              cudaStream_t stream);
+cudaError_t launch_time_plans(const PlanArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_attn_bf16_sm100(const BwdArgs& a, const CUtensorMap* maps,
                                        cudaStream_t stream);
 

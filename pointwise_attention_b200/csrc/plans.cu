@@ -1,0 +1,95 @@
+// plans.cu -- the shapes of the time-bias plans, computed once per call.
+//
+// The time bias of "HSTU Hierarchical Sequential Transduction Units" (§1 and
+// §3: a per-head table indexed by the bucket of t_i - t_j) is applied by the
+// attention kernels per warp and 32-column block through a plan (tile_math.cuh:
+// the block's first bucket, up to three split columns, the kind).  A plan's
+// shape depends on the timestamps only, not on the head, so this pass computes
+// it once for every row and every block the row meets and the kernels of all
+// H heads read it.  CTA (row tile rt, sequence b, group z of kPlanBlocks
+// blocks); warp w takes rows 128 rt + 32 w + lane, the same 32-row groups as
+// the kernels' epilogue warps, so the warp-level choice of kind is theirs.
+#include "bounds.cuh"
+#include "internal.h"
+#include "tile_math.cuh"
+
+namespace hstu {
+namespace {
+
+constexpr int kPlanThreads = 128;
+constexpr int kPlanBlocks = 8;
+
+struct PlanTab {
+  const uint4* oct_;
+  const unsigned* thr32_;
+  __device__ __forceinline__ const uint4* oct() const { return oct_; }
+  __device__ __forceinline__ const unsigned* thr32() const { return thr32_; }
+};
+
+__global__ void __launch_bounds__(kPlanThreads) time_plans(const __grid_constant__ PlanArgs a) {
+  __shared__ uint4 s_oct[32];
+  __shared__ unsigned s_thr32[kMaxBuckets];
+  __shared__ uint32_t s_ts[kPlanThreads / 32][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 32; i += kPlanThreads) s_oct[i] = a.bt.oct[i];
+  for (int i = threadIdx.x; i < kMaxBuckets; i += kPlanThreads) s_thr32[i] = a.bt.thr32[i];
+  __syncthreads();
+  const int rt = static_cast<int>(blockIdx.x), b = static_cast<int>(blockIdx.y);
+  const int s = __ldg(a.offsets + b), e = __ldg(a.offsets + b + 1);
+  const int n_b = e - s;
+  // inconsistent offsets are reported by the attention kernels
+  if (s < 0 || n_b <= 0 || e > a.T || n_b > a.max_seq_len || 128 * rt >= n_b) return;
+  const int i = 128 * rt + 32 * warp + lane;          // this thread's row of the sequence
+  const bool row_ok = i < n_b;
+  // rows past the end take the last row's timestamp, as in the kernels
+  const long long my_ts =
+      a.timestamps[checked(a.status, s + (row_ok ? i : n_b - 1), a.T, BS_BWD_TS)];
+  const int jt = 4 * ((n_b + 127) / 128);             // blocks over the sequence's tiles
+  const int j0 = static_cast<int>(blockIdx.z) * kPlanBlocks;
+  const int j1 = min(jt, j0 + kPlanBlocks);
+  const PlanTab tab{s_oct, s_thr32};
+  uint32_t* ts32 = s_ts[warp];
+  for (int jc = j0; jc < j1; ++jc) {
+    // columns at or before the row tile (dn); at or after it (up)
+    const bool dn = a.plan_dn && jc < 4 * rt + 4, up = a.plan_up && jc >= 4 * rt;
+    if (!dn && !up) continue;
+    // the block's columns, those past the end repeating the last timestamp
+    const int j = 32 * jc + lane;
+    const long long kt = a.timestamps[checked(a.status, s + (j < n_b ? j : n_b - 1), a.T, BS_BWD_TS)];
+    __syncwarp();
+    ts32[lane] = static_cast<uint32_t>(kt);
+    const long long nx = __shfl_down_sync(0xffffffffu, kt, 1);
+    const bool asc = !__any_sync(0xffffffffu, lane < 31 && nx < kt);
+    long long lo = kt, hi = kt;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const long long x = __shfl_xor_sync(0xffffffffu, lo, o);
+      const long long y = __shfl_xor_sync(0xffffffffu, hi, o);
+      lo = x < lo ? x : lo;
+      hi = y > hi ? y : hi;
+    }
+    __syncwarp();
+    const size_t at = static_cast<size_t>(jc) * a.T + s + (row_ok ? i : 0);
+    TimePlan p;
+    if (dn) {
+      const int tb = plan_shape_dn(p, my_ts, lo, hi, asc, ts32, tab);
+      if (row_ok) a.plan_dn[at] = plan_word(p, tb);
+    }
+    if (up) {
+      const int tb = plan_shape_up(p, my_ts, lo, hi, asc, ts32, tab);
+      if (row_ok) a.plan_up[at] = plan_word(p, tb);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_time_plans(const PlanArgs& a, cudaStream_t stream) {
+  if (a.B == 0 || a.max_tiles == 0) return cudaSuccess;
+  if (a.plan_j < 4 * a.max_tiles) return cudaErrorInvalidValue;
+  const dim3 grid(a.max_tiles, a.B, (a.plan_j + kPlanBlocks - 1) / kPlanBlocks);
+  time_plans<<<grid, kPlanThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu
