@@ -226,7 +226,7 @@ __device__ Item claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots,
 // one value (CONST) or two with a split column (SPLIT), from the row's plan
 // word (plans.cu); every other plan kind takes each element's own bucket
 // (GEN32 with 32-bit differences, GEN64 for time spans of 2^31 or more).
-enum { T_CONST = 0, T_SPLIT = 1, T_GEN32 = 2, T_GEN64 = 3 };
+enum { T_CONST = 0, T_SPLIT = 1, T_GEN32 = 2, T_GEN64 = 3, T_MULTI = 4 };
 
 struct EpiShared {
   const uint4* oct;
@@ -256,6 +256,14 @@ __device__ __forceinline__ void chunk_pairs(const uint32_t (&sv)[32], const uint
         tb = tconst;
       } else if (TM == T_SPLIT) {
         tb = (2 * i + 1 < split) ? thh : ((2 * i < split) ? thl : tll);
+      } else if (TM == T_MULTI) {
+        // splits in `split` (6 bits each), the four bucket values in
+        // tconst, thh, tll, thl
+        const int s0 = split & 63, s1 = (split >> 6) & 63, s2 = (split >> 12) & 63;
+        const int c = 2 * i;
+        const uint32_t lo = c >= s2 ? thl : c >= s1 ? tll : c >= s0 ? thh : tconst;
+        const uint32_t hi = c + 1 >= s2 ? thl : c + 1 >= s1 ? tll : c + 1 >= s0 ? thh : tconst;
+        tb = __byte_perm(lo, hi, 0x7610);
       } else {
         float tv[2];
 #pragma unroll
@@ -679,7 +687,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               chunk_pairs<POS, true, T_SPLIT>(sv, wp, 0u, pack_bf16x2(hv, hv),
                                               pack_bf16x2(lv, lv), pack_bf16x2(hv, lv), split,
                                               my32, my64, wts32, wts, es, packed);
-            } else if (kind != TB_GEN64) {               // multi-bucket or per element
+            } else if (kind == TB_MULTI) {
+              // the word's three split columns and the buckets k0 .. k0 - 3
+              const float v0 = es.rabt[k0], v1 = es.rabt[max(k0 - 1, 0)];
+              const float v2 = es.rabt[max(k0 - 2, 0)], v3 = es.rabt[max(k0 - 3, 0)];
+              chunk_pairs<POS, true, T_MULTI>(sv, wp, pack_bf16x2(v0, v0), pack_bf16x2(v1, v1),
+                                              pack_bf16x2(v2, v2), pack_bf16x2(v3, v3),
+                                              static_cast<int>((plan_w >> 7) & 0x3FFFFu), my32,
+                                              my64, wts32, wts, es, packed);
+            } else if (kind != TB_GEN64) {               // per element
               chunk_pairs<POS, true, T_GEN32>(sv, wp, 0u, 0u, 0u, 0u, 0, my32, my64, wts32, wts,
                                               es, packed);
             } else {
