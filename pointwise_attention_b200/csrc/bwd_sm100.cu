@@ -1198,7 +1198,7 @@ cudaError_t launch_bwd_attn_bf16_sm100(const BwdArgs& a, const CUtensorMap* maps
   const bool pos = a.rab_pos != nullptr, tim = a.rab_time != nullptr;
   if (tim) {
     if (!a.plan_dn || !a.plan_up || a.plan_j < 4 * a.max_tiles) return cudaErrorInvalidValue;
-    PlanArgs pa;
+    PlanArgs pa{};
     pa.offsets = a.offsets;
     pa.timestamps = a.timestamps;
     pa.plan_dn = a.plan_dn;

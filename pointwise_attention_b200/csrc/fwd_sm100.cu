@@ -226,7 +226,7 @@ __device__ Item claim_item(const FwdArgs& a, unsigned* counter, unsigned nslots,
 // one value (CONST) or two with a split column (SPLIT), from the row's plan
 // word (plans.cu); every other plan kind takes each element's own bucket
 // (GEN32 with 32-bit differences, GEN64 for time spans of 2^31 or more).
-enum { T_CONST = 0, T_SPLIT = 1, T_GEN32 = 2, T_GEN64 = 3, T_MULTI = 4 };
+enum { T_CONST = 0, T_SPLIT = 1, T_GEN32 = 2, T_GEN64 = 3, T_MULTI = 4, T_BYTES = 5 };
 
 struct EpiShared {
   const uint4* oct;
@@ -245,7 +245,7 @@ __device__ __forceinline__ void chunk_pairs(const uint32_t (&sv)[32], const uint
                                             uint32_t thl, int split, uint32_t my32,
                                             long long my64, const uint32_t* kts32,
                                             const long long* kts64, const EpiShared& es,
-                                            uint32_t (&packed)[16]) {
+                                            uint32_t (&packed)[16], const uint32_t* nbw = nullptr) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const uint32_t s2 = pack_bf16x2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
@@ -264,6 +264,10 @@ __device__ __forceinline__ void chunk_pairs(const uint32_t (&sv)[32], const uint
         const uint32_t lo = c >= s2 ? thl : c >= s1 ? tll : c >= s0 ? thh : tconst;
         const uint32_t hi = c + 1 >= s2 ? thl : c + 1 >= s1 ? tll : c + 1 >= s0 ? thh : tconst;
         tb = __byte_perm(lo, hi, 0x7610);
+      } else if (TM == T_BYTES) {
+        // each element's bucket from the plan pass, one byte per column
+        const uint32_t w = nbw[i >> 1] >> (16 * (i & 1));
+        tb = pack_bf16x2(es.rabt[w & 0xFFu], es.rabt[(w >> 8) & 0xFFu]);
       } else {
         float tv[2];
 #pragma unroll
@@ -696,8 +700,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               static_cast<int>((plan_w >> 7) & 0x3FFFFu), my32,
                                               my64, wts32, wts, es, packed);
             } else if (kind != TB_GEN64) {               // per element
-              chunk_pairs<POS, true, T_GEN32>(sv, wp, 0u, 0u, 0u, 0u, 0, my32, my64, wts32, wts,
-                                              es, packed);
+              const int jd = 4 * m + q4, jc = 4 * n + cq;   // diagonal block, this block
+              if (jc == jd || jc == jd - 1) {
+                // the buckets of the two blocks nearest the diagonal, from the plan pass
+                const uint4* src = a.near_dn +
+                                   static_cast<size_t>(row_ok ? t_row : s + n_b - 1) * 4 +
+                                   (jc == jd ? 0 : 2);
+                const uint4 b0 = __ldg(src), b1 = __ldg(src + 1);
+                const uint32_t nbw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                chunk_pairs<POS, true, T_BYTES>(sv, wp, 0u, 0u, 0u, 0u, 0, my32, my64, wts32, wts,
+                                                es, packed, nbw);
+              } else {
+                chunk_pairs<POS, true, T_GEN32>(sv, wp, 0u, 0u, 0u, 0u, 0, my32, my64, wts32,
+                                                wts, es, packed);
+              }
             } else {
               chunk_pairs<POS, true, T_GEN64>(sv, wp, 0u, 0u, 0u, 0u, 0, my32, my64, wts32, wts,
                                               es, packed);

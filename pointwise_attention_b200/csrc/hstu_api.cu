@@ -182,11 +182,12 @@ bool f32_supported(const hstu_problem_t* p) {
 //                    B * ceil(max_seq_len/128) u32][per (token, head) row
 //                    statistics: T * H float4] and, with a time table,
 //                    [time plans (queries against keys): J * T u32]
+//                    [the buckets of the two blocks nearest the diagonal: T * 64 B]
 //   backward:       [status 256 B][dO: T*H*dv in the input dtype]
 //                    and, bf16 with a time table, [time plans: 2 * J * T u32]
 //                    with J = 4 * ceil(max_seq_len / 128)
 struct WsLayout {
-  size_t cnt_off, stats_off, dO_off, plan_off, total;
+  size_t cnt_off, stats_off, dO_off, plan_off, near_off, total;
   int plan_j;
 };
 
@@ -212,6 +213,8 @@ WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
       l.plan_j = 4 * static_cast<int>(tiles);
       l.plan_off = off;
       off += align_up(static_cast<size_t>(l.plan_j) * T * 4);
+      l.near_off = off;
+      off += align_up(T * 64);
     }
   }
   l.total = off;
@@ -327,11 +330,13 @@ hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* 
       // the time-plan shapes, once for all heads
       uint32_t* plans = reinterpret_cast<uint32_t*>(ws + l.plan_off);
       a.plan_dn = plans;
+      a.near_dn = reinterpret_cast<const uint4*>(ws + l.near_off);
       PlanArgs pa;
       std::memset(&pa, 0, sizeof(pa));
       pa.offsets = a.offsets;
       pa.timestamps = a.timestamps;
       pa.plan_dn = plans;
+      pa.near_dn = reinterpret_cast<uint4*>(ws + l.near_off);
       pa.status = a.status;
       pa.B = a.B;
       pa.T = a.T;

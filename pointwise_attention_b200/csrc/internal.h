@@ -68,8 +68,10 @@ struct FwdArgs {
   unsigned* item_cnt;
   float4* stats;
   // bf16 forward with a time table, workspace: the time-plan shapes of every
-  // query row against every 32-key block, [4 * max_tiles][T] words
+  // query row against every 32-key block, [4 * max_tiles][T] words, and the
+  // per-element buckets of its two blocks nearest the diagonal, [T][4] uint4
   const uint32_t* plan_dn;
+  const uint4* near_dn;
   BucketTable bt;
 };
 
@@ -124,6 +126,10 @@ struct PlanArgs {
   const int64_t* timestamps;
   uint32_t* plan_dn;
   uint32_t* plan_up;
+  // or null: per row, the buckets (one byte each) of its 32-column block that
+  // holds the diagonal and of the block before it, rows against earlier
+  // columns: [T][4] uint4, bytes 0..31 and 32..63
+  uint4* near_dn;
   int* status;
   int B, T, max_seq_len, max_tiles, plan_j;
   BucketTable bt;
