@@ -87,8 +87,10 @@ typedef struct {
  * Bytes of device workspace the call needs (is_bwd = 0: forward; 1: backward).
  * With a time table the bf16 calls also keep there the shapes of their
  * time-bias plans, 4 bytes per token and 32-column block of max_seq_len
- * (rounded up to 128) for the forward, twice that for the backward:
- * 4 * T * 4 * ceil(max_seq_len / 128) bytes (forward), 8 * T * ... (backward).
+ * (rounded up to 128) for the forward, twice that for the backward, and 96
+ * bytes per token of per-element buckets near the diagonal:
+ * T * (16 * ceil(max_seq_len / 128) + 96) bytes (forward),
+ * T * (32 * ceil(max_seq_len / 128) + 96) bytes (backward), each rounded up to 256.
  * The workspace must be 256-byte aligned and zero-filled before its first use;
  * its first word is the device status that hstu_attn_check reads and re-arms.
  * Words 16 and 17 hold the bf16 forward's work counters: each launch hands its

@@ -167,7 +167,7 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sp)[16], const uint32
                                           const Stage* stg, int lane, int r, int c0, bool diag,
                                           int qlim, const TimePlan& tp, long long my_ts,
                                           const TimeTables& tt, uint32_t (&pk)[16],
-                                          uint32_t (&dk)[16]) {
+                                          uint32_t (&dk)[16], const uint32_t* nbw = nullptr) {
   if (TB != TB_GEN64) {
     // bf16x2 arithmetic: P' and dS' are bf16 operands of the next MMAs anyway
     const uint32_t* wp = stg->wpk + 31 - lane;   // pair i: diagonals 2i - lane + 31 (+1)
@@ -176,8 +176,8 @@ __device__ __forceinline__ void dkv_chunk(const uint32_t (&sp)[16], const uint32
     for (int i = 0; i < 16; ++i) {
       // half bias pair (position + time), added before S arrives in the chain
       uint32_t hb = POS ? wp[2 * i] : 0u;
-      if (TB == TB_GEN32) {
-        const int2 kb = gen_bucket_pair(stg->ts32, i, my32, tt);
+      if (TB == TB_GEN32 || TB == TB_BYTES) {
+        const int2 kb = TB == TB_BYTES ? byte_bucket_pair(nbw, i) : gen_bucket_pair(stg->ts32, i, my32, tt);
         const uint32_t tb = pack_bf16x2(tt.rabt()[kb.x], tt.rabt()[kb.y]);
         hb = POS ? hadd2(hb, tb) : tb;
       } else if (TB != TB_NONE) {
@@ -236,7 +236,7 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sp)[16], const uint32_
                                          int klim, bool row_ok, const TimePlan& tp,
                                          long long my_ts, const TimeTables& tt, float* win,
                                          int wbase, float* s_dt, uint32_t (&dk)[16], int& run_k,
-                                         float& run_s) {
+                                         float& run_s, const uint32_t* nbw = nullptr) {
   // Diagonal sums (row - column = const) of the warp's 32 x 32 block: at
   // column cl lane L reads lane (L + cl) mod 32, so every element with
   // row - cl = L, or L - 32, passes through lane L.
@@ -253,8 +253,8 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sp)[16], const uint32_
       // half bias pair (position + time), added before S arrives in the chain
       uint32_t hb = POS ? wp[-2 * i] : 0u;
       int2 kb = make_int2(0, 0);
-      if (TB == TB_GEN32) {
-        kb = gen_bucket_pair(stg->ts32, i, my32, tt);
+      if (TB == TB_GEN32 || TB == TB_BYTES) {
+        kb = TB == TB_BYTES ? byte_bucket_pair(nbw, i) : gen_bucket_pair(stg->ts32, i, my32, tt);
         const uint32_t tb = pack_bf16x2(tt.rabt()[kb.x], tt.rabt()[kb.y]);
         hb = POS ? hadd2(hb, tb) : tb;
       } else if (TB != TB_NONE) {
@@ -284,7 +284,7 @@ __device__ __forceinline__ void dq_chunk(const uint32_t (&sp)[16], const uint32_
           dneg1 += hi;
         }
       }
-      if (TB == TB_GEN32) {
+      if (TB == TB_GEN32 || TB == TB_BYTES) {
         run_add_packed(kb.x, v0, run_k, run_s, s_dt);
         run_add_packed(kb.y, v1, run_k, run_s, s_dt);
       } else if (TB != TB_NONE) {
@@ -736,7 +736,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else if (tb == TB_MULTI) {
             HSTU_DKV(TB_MULTI, true);
           } else if (tb == TB_GEN32) {
-            HSTU_DKV(TB_GEN32, true);
+            // the diagonal block and the one after it: buckets from the plan pass
+            const int jd = 4 * n + q4, jc = 4 * m + (c0 >> 5);
+            if (jc == jd || jc == jd + 1) {
+              const uint4* src = a.near + static_cast<size_t>(row_ok ? t_row : s + n_b - 1) * 6 +
+                                 (jc == jd ? 0 : 4);
+              const uint4 b0 = __ldg(src), b1 = __ldg(src + 1);
+              const uint32_t nbw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+              dkv_chunk<POS, TB_BYTES, true>(sp, dp, stg, lane, r, c0, diag, qlim, tp, my_ts, tt,
+                                             pk, dk, nbw);
+            } else {
+              HSTU_DKV(TB_GEN32, true);
+            }
           } else {
             HSTU_DKV(TB_GEN64, true);
           }
@@ -1096,7 +1107,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else if (tb == TB_MULTI) {
             HSTU_DQ(TB_MULTI, true);
           } else if (tb == TB_GEN32) {
-            HSTU_DQ(TB_GEN32, true);
+            // the diagonal block and the one before it: buckets from the plan pass
+            const int jd = 4 * m + q4, jc = 4 * k + (c0 >> 5);
+            if (jc == jd || jc == jd - 1) {
+              const uint4* src = a.near + static_cast<size_t>(row_ok ? t_row : s + n_b - 1) * 6 +
+                                 (jc == jd ? 0 : 2);
+              const uint4 b0 = __ldg(src), b1 = __ldg(src + 1);
+              const uint32_t nbw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+              dq_chunk<POS, TB_BYTES, true>(sp, dp, stg, lane, r, c0, diag, klim, row_ok, tp, my_ts,
+                                            tt, win, wbase, s_dt, dk, run_k, run_s, nbw);
+            } else {
+              HSTU_DQ(TB_GEN32, true);
+            }
           } else {
             HSTU_DQ(TB_GEN64, true);
           }
@@ -1203,6 +1225,7 @@ cudaError_t launch_bwd_attn_bf16_sm100(const BwdArgs& a, const CUtensorMap* maps
     pa.timestamps = a.timestamps;
     pa.plan_dn = a.plan_dn;
     pa.plan_up = a.plan_up;
+    pa.near = a.near;
     pa.status = a.status;
     pa.B = a.B;
     pa.T = a.T;

@@ -266,8 +266,8 @@ __device__ __forceinline__ void chunk_pairs(const uint32_t (&sv)[32], const uint
         tb = __byte_perm(lo, hi, 0x7610);
       } else if (TM == T_BYTES) {
         // each element's bucket from the plan pass, one byte per column
-        const uint32_t w = nbw[i >> 1] >> (16 * (i & 1));
-        tb = pack_bf16x2(es.rabt[w & 0xFFu], es.rabt[(w >> 8) & 0xFFu]);
+        const int2 kb = byte_bucket_pair(nbw, i);
+        tb = pack_bf16x2(es.rabt[kb.x], es.rabt[kb.y]);
       } else {
         float tv[2];
 #pragma unroll
@@ -703,8 +703,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int jd = 4 * m + q4, jc = 4 * n + cq;   // diagonal block, this block
               if (jc == jd || jc == jd - 1) {
                 // the buckets of the two blocks nearest the diagonal, from the plan pass
-                const uint4* src = a.near_dn +
-                                   static_cast<size_t>(row_ok ? t_row : s + n_b - 1) * 4 +
+                const uint4* src = a.near +
+                                   static_cast<size_t>(row_ok ? t_row : s + n_b - 1) * 6 +
                                    (jc == jd ? 0 : 2);
                 const uint4 b0 = __ldg(src), b1 = __ldg(src + 1);
                 const uint32_t nbw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};

@@ -182,7 +182,7 @@ bool f32_supported(const hstu_problem_t* p) {
 //                    B * ceil(max_seq_len/128) u32][per (token, head) row
 //                    statistics: T * H float4] and, with a time table,
 //                    [time plans (queries against keys): J * T u32]
-//                    [the buckets of the two blocks nearest the diagonal: T * 64 B]
+//                    [the buckets of the blocks nearest the diagonal: T * 96 B]
 //   backward:       [status 256 B][dO: T*H*dv in the input dtype]
 //                    and, bf16 with a time table, [time plans: 2 * J * T u32]
 //                    with J = 4 * ceil(max_seq_len / 128)
@@ -202,6 +202,8 @@ WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
       l.plan_j = 4 * ((p->max_seq_len + 127) / 128);
       l.plan_off = off;
       off += align_up(2 * static_cast<size_t>(l.plan_j) * T * 4);
+      l.near_off = off;
+      off += align_up(T * 96);
     }
   } else if (p->dtype == HSTU_BF16) {
     const size_t tiles = static_cast<size_t>((p->max_seq_len + 127) / 128);
@@ -214,7 +216,7 @@ WsLayout ws_layout(const hstu_problem_t* p, int is_bwd) {
       l.plan_off = off;
       off += align_up(static_cast<size_t>(l.plan_j) * T * 4);
       l.near_off = off;
-      off += align_up(T * 64);
+      off += align_up(T * 96);
     }
   }
   l.total = off;
@@ -330,13 +332,13 @@ hstu_status_t hstu_attn_fwd(const hstu_problem_t* p, const void* q, const void* 
       // the time-plan shapes, once for all heads
       uint32_t* plans = reinterpret_cast<uint32_t*>(ws + l.plan_off);
       a.plan_dn = plans;
-      a.near_dn = reinterpret_cast<const uint4*>(ws + l.near_off);
+      a.near = reinterpret_cast<const uint4*>(ws + l.near_off);
       PlanArgs pa;
       std::memset(&pa, 0, sizeof(pa));
       pa.offsets = a.offsets;
       pa.timestamps = a.timestamps;
       pa.plan_dn = plans;
-      pa.near_dn = reinterpret_cast<uint4*>(ws + l.near_off);
+      pa.near = reinterpret_cast<uint4*>(ws + l.near_off);
       pa.status = a.status;
       pa.B = a.B;
       pa.T = a.T;
@@ -431,6 +433,7 @@ hstu_status_t hstu_attn_bwd(const hstu_problem_t* p, const void* dy, const void*
     a.plan_j = l.plan_j;
     a.plan_dn = reinterpret_cast<uint32_t*>(ws + l.plan_off);
     a.plan_up = a.plan_dn + static_cast<size_t>(l.plan_j) * p->total_tokens;
+    a.near = reinterpret_cast<uint4*>(ws + l.near_off);
   }
   a.status = common.status;
   a.B = common.B; a.T = common.T; a.H = common.H; a.d_qk = common.d_qk; a.d_v = common.d_v;

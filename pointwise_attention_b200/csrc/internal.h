@@ -69,9 +69,9 @@ struct FwdArgs {
   float4* stats;
   // bf16 forward with a time table, workspace: the time-plan shapes of every
   // query row against every 32-key block, [4 * max_tiles][T] words, and the
-  // per-element buckets of its two blocks nearest the diagonal, [T][4] uint4
+  // per-element buckets of its blocks nearest the diagonal, [T][6] uint4
   const uint32_t* plan_dn;
-  const uint4* near_dn;
+  const uint4* near;
   BucketTable bt;
 };
 
@@ -104,6 +104,7 @@ struct BwdArgs {
   // keys (dQ), rows = keys against later queries (dK, dV)
   uint32_t* plan_dn;
   uint32_t* plan_up;
+  uint4* near;       // per-element buckets of the blocks nearest the diagonal, [T][6] uint4
   int plan_j;        // blocks per row: 4 * max_tiles
   int* status;
   int B, T, H, d_qk, d_v;
@@ -126,10 +127,10 @@ struct PlanArgs {
   const int64_t* timestamps;
   uint32_t* plan_dn;
   uint32_t* plan_up;
-  // or null: per row, the buckets (one byte each) of its 32-column block that
-  // holds the diagonal and of the block before it, rows against earlier
-  // columns: [T][4] uint4, bytes 0..31 and 32..63
-  uint4* near_dn;
+  // or null: per row, the buckets (one byte each) of the 32-column block that
+  // holds its diagonal, of the block before and of the block after it:
+  // [T][6] uint4, 32 bytes each
+  uint4* near;
   int* status;
   int B, T, max_seq_len, max_tiles, plan_j;
   BucketTable bt;

@@ -70,32 +70,34 @@ __global__ void __launch_bounds__(kPlanThreads) time_plans(const __grid_constant
     }
     __syncwarp();
     const size_t at = static_cast<size_t>(jc) * a.T + s + (row_ok ? i : 0);
+    // The block holding this warp's diagonal, the one before and (for the
+    // rows-against-later-columns plans) the one after it: the bucket of every
+    // element, for the per-element path (32-bit differences; the kernels use
+    // these only where every |dt| of the block is below 2^31).
+    const int jd = 4 * rt + warp;
+    const int slot = jc == jd ? 0 : jc == jd - 1 ? 2 : (jc == jd + 1 && a.plan_up) ? 4 : -1;
+    if (a.near && row_ok && slot >= 0) {
+      const uint32_t my32 = static_cast<uint32_t>(my_ts);
+      uint32_t w[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const int d = static_cast<int>(my32 - ts32[4 * q + e2]);
+          const int k = bucket32(static_cast<uint32_t>(d < 0 ? -d : d), tab.oct());
+          word |= static_cast<uint32_t>(k) << (8 * e2);
+        }
+        w[q] = word;
+      }
+      uint4* dst = a.near + static_cast<size_t>(s + i) * 6 + slot;
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
     TimePlan p;
     if (dn) {
       const int tb = plan_shape_dn(p, my_ts, lo, hi, asc, ts32, tab);
       if (row_ok) a.plan_dn[at] = plan_word(p, tb);
-      // the block holding this warp's diagonal, and the one before it: the
-      // bucket of every element, for the per-element path (32-bit differences;
-      // the kernels use these only where every |dt| of the block is below 2^31)
-      const int jd = 4 * rt + warp;
-      if (a.near_dn && row_ok && (jc == jd || jc == jd - 1)) {
-        const uint32_t my32 = static_cast<uint32_t>(my_ts);
-        uint32_t w[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint32_t word = 0;
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const int d = static_cast<int>(my32 - ts32[4 * q + e2]);
-            const int k = bucket32(static_cast<uint32_t>(d < 0 ? -d : d), tab.oct());
-            word |= static_cast<uint32_t>(k) << (8 * e2);
-          }
-          w[q] = word;
-        }
-        uint4* dst = a.near_dn + static_cast<size_t>(s + i) * 4 + (jc == jd ? 0 : 2);
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      }
     }
     if (up) {
       const int tb = plan_shape_up(p, my_ts, lo, hi, asc, ts32, tab);

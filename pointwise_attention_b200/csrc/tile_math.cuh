@@ -92,6 +92,9 @@ constexpr uint32_t kHalfPair = 0x3F003F00u;   // (0.5, 0.5) in bf16
 // the span reaches 2^31.  TB_NONE: no time table (or a block that is all
 // masked).
 enum { TB_NONE = 0, TB_CONST = 1, TB_SPLIT = 2, TB_MULTI = 3, TB_GEN32 = 4, TB_GEN64 = 5 };
+// A kernel's own per-element kind: the buckets precomputed per element (one
+// byte each) for the blocks nearest the diagonal.
+constexpr int TB_BYTES = 6;
 
 // The bucket of column 0 is k_a; from column s[t] on it is t + 1 buckets
 // further (down when dt falls along the columns, up when it rises); 32: never.
@@ -260,6 +263,14 @@ __device__ __forceinline__ uint32_t plan_pair(const TimePlan& p, int i) {
   if (TB == TB_CONST) return p.v[0];
   if (TB == TB_SPLIT) return (2 * i + 1 < p.s[0]) ? p.v[0] : ((2 * i < p.s[0]) ? p.t_ab : p.v[1]);
   return __byte_perm(plan_value(p, 2 * i), plan_value(p, 2 * i + 1), 0x7610);
+}
+
+// Buckets of columns 2i, 2i+1 from a row's 32 bucket bytes (8 words); the
+// 7-bit mask keeps any word in range of the bucket tables (rows past a
+// sequence's end read words they were not written for, and mask the result).
+__device__ __forceinline__ int2 byte_bucket_pair(const uint32_t* w8, int i) {
+  const uint32_t w = w8[i >> 1] >> (16 * (i & 1));
+  return make_int2(static_cast<int>(w & 0x7Fu), static_cast<int>((w >> 8) & 0x7Fu));
 }
 
 // Buckets of columns 2i, 2i+1 on the per-element 32-bit path (|dt| < 2^31),
