@@ -256,10 +256,13 @@ HSTU_API hstu_status_t hstu_out_fwd(int32_t T, int32_t E, int32_t D, const void 
  * candidates (at most max_cands per user); cand_timestamps device int64
  * [total_cands] (required with rab_time).  q, k, v [C, H, 128], u [C, H*128]:
  * the candidates' projections; y [C, H*128] output.  Supported: bf16,
- * d_qk = d_v = 128, 1 <= H <= 16.  workspace: hstu_cand_workspace_size bytes,
- * 256-byte aligned, zero-filled before its first use (its per-micro-batch
- * counters return to zero after each call); candidate offsets found
- * inconsistent on the device are reported by hstu_attn_check.
+ * d_qk = d_v = 128, 1 <= H <= 16.  workspace: hstu_cand_workspace_size bytes
+ * for the same problem (with a time table it also holds the time-plan shape
+ * of every candidate against every 32-event block of its user's history:
+ * 16 * ceil(max_seq_len / 128) bytes per candidate), 256-byte aligned,
+ * zero-filled before its first use (its per-micro-batch counters return to
+ * zero after each call); candidate offsets found inconsistent on the device
+ * are reported by hstu_attn_check.
  */
 HSTU_API size_t hstu_cand_workspace_size(const hstu_problem_t *p, int32_t total_cands,
                                          int32_t max_cands);

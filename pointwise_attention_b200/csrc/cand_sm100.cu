@@ -325,6 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool jv = j < nb;
       const float pb = (POS && jv) ? __ldg(rpos + (nb - j)) : 0.f;
       const long long kts = (TIME && jv) ? __ldg(a.timestamps + checked(a.status, s + j, a.T, BS_CAND_TS)) : 0ll;
+      // this candidate's time plan against the chunk (the plan pass)
+      const uint32_t pw = (TIME && 128 * n + 32 * cs < nb)
+                              ? __ldg(a.plan + static_cast<size_t>(4 * n + cs) * a.C + cand)
+                              : 0u;
       if (ok) ok = checked(mbar_wait(bar(B_SFULL + st), (n / kStages) & 1, abort_flag), a.status);
       ok = __all_sync(0xffffffffu, ok);   // the TMEM accesses below are warp-collective
       if (!ok) break;
@@ -352,22 +356,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         TimePlan tp{};
         int tb = TB_NONE;
         if (TIME) {
+          // the keys' timestamps for the per-element paths (past the history:
+          // the last one; those columns are masked)
           const long long last = __shfl_sync(0xffffffffu, kts, nvalid < 32 ? nvalid - 1 : 31);
-          const long long kt = jv ? kts : last;
-          stg->ts32[lane] = static_cast<uint32_t>(kt);
-          const long long nx = __shfl_down_sync(0xffffffffu, kt, 1);
-          const bool asc = !__any_sync(0xffffffffu, lane < 31 && nx < kt);
-          long long kmn = kt, kmx = kt;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
-            kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
-          }
-          __syncwarp();
-          tb = plan_dn(tp, my_ts, kmn, kmx, asc, stg->ts32, tab);
-        } else {
-          __syncwarp();
+          stg->ts32[lane] = static_cast<uint32_t>(jv ? kts : last);
+          tb = plan_unword(tp, pw);
+          plan_values<false>(tp, tb, tab);
         }
+        __syncwarp();
         const uint32_t my32 = static_cast<uint32_t>(my_ts);
         if (tb == TB_GEN64) {
           // time spans of 2^31 or more: fp32 with the 64-bit bucket search

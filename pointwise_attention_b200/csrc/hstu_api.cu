@@ -556,10 +556,18 @@ hstu_status_t hstu_out_fwd(int32_t T, int32_t E, int32_t D, const void* y, const
 // ---------------------------------------------------------- candidate scoring
 static size_t cand_tiles(int32_t max_cands) { return (static_cast<size_t>(max_cands) + 127) / 128; }
 
+// Candidate workspace: [status][per (user, micro-batch) counters][O / N per
+// candidate, fp32][with a time table: plan words, J * C u32 with
+// J = 4 * ceil(max_seq_len / 128)]
+static size_t cand_plan_j(const hstu_problem_t* p) {
+  return p->rab_time ? 4 * static_cast<size_t>((p->max_seq_len + 127) / 128) : 0;
+}
+
 size_t hstu_cand_workspace_size(const hstu_problem_t* p, int32_t total_cands, int32_t max_cands) {
   if (check_problem(p) != HSTU_OK || total_cands < 0 || max_cands < 0) return 0;
   return kStatusBytes + align_up(static_cast<size_t>(p->batch) * cand_tiles(max_cands) * 4) +
-         align_up(static_cast<size_t>(total_cands) * p->num_heads * p->d_v * 4);
+         align_up(static_cast<size_t>(total_cands) * p->num_heads * p->d_v * 4) +
+         align_up(cand_plan_j(p) * static_cast<size_t>(total_cands) * 4);
 }
 
 hstu_status_t hstu_cand_fwd(const hstu_problem_t* p, const void* k_hist, const void* v_hist,
@@ -609,6 +617,11 @@ hstu_status_t hstu_cand_fwd(const hstu_problem_t* p, const void* k_hist, const v
   const size_t cnt_bytes = align_up(static_cast<size_t>(p->batch) * cand_tiles(max_cands) * 4);
   a.cnt = reinterpret_cast<unsigned*>(ws + kStatusBytes);
   a.o_ws = reinterpret_cast<float*>(ws + kStatusBytes + cnt_bytes);
+  a.plan_j = static_cast<int>(cand_plan_j(p));
+  if (a.plan_j > 0)
+    a.plan = reinterpret_cast<uint32_t*>(
+        ws + kStatusBytes + cnt_bytes +
+        align_up(static_cast<size_t>(total_cands) * p->num_heads * p->d_v * 4));
   a.status = static_cast<int*>(workspace);
   a.B = p->batch;
   a.T = p->total_tokens;
@@ -629,7 +642,10 @@ hstu_status_t hstu_cand_fwd(const hstu_problem_t* p, const void* k_hist, const v
       !make_map_3d(&tk, hist ? k_hist : k, hist ? p->total_tokens : total_cands, p->num_heads, 128) ||
       !make_map_3d(&tv, hist ? v_hist : v, hist ? p->total_tokens : total_cands, p->num_heads, 128))
     return HSTU_ERR_CUDA;
-  const cudaError_t err = launch_cand_sm100(a, tq, tk, tv, static_cast<cudaStream_t>(stream));
+  cudaError_t err = cudaSuccess;
+  if (a.plan && hist && total_cands > 0)   // the time-plan shapes, once for all heads
+    err = launch_cand_plans(a, static_cast<cudaStream_t>(stream));
+  if (err == cudaSuccess) err = launch_cand_sm100(a, tq, tk, tv, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 

@@ -173,6 +173,10 @@ struct CandArgs {
   const float* ln_bias;
   float* o_ws;                   // workspace: O / N per candidate [C, H*128] fp32
   unsigned* cnt;                 // workspace: head CTAs done per (user, micro-batch)
+  // workspace (with a time table): the time-plan shape of every candidate
+  // against every 32-event block of its user's history, [plan_j][C] words
+  uint32_t* plan;
+  int plan_j;
   int* status;
   int B, T, C, H;
   int max_tiles;                 // micro-batches per user in the grid
@@ -204,6 +208,7 @@ cudaError_t launch_uvqk_sm100(const ProjArgs& a, const CUtensorMap& tx, const CU
 cudaError_t launch_out_sm100(const ProjArgs& a, const CUtensorMap& ty, const CUtensorMap& tw,
                              cudaStream_t stream);
 cudaError_t launch_time_plans(const PlanArgs& a, cudaStream_t stream);
+cudaError_t launch_cand_plans(const CandArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_attn_bf16_sm100(const BwdArgs& a, const CUtensorMap* maps,
                                        cudaStream_t stream);
 

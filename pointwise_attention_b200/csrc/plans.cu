@@ -106,7 +106,68 @@ __global__ void __launch_bounds__(kPlanThreads) time_plans(const __grid_constant
   }
 }
 
+// Candidates against their user's history: CTA (micro-batch mt of 128
+// candidates, user b, group z of kPlanBlocks history blocks); warp w takes
+// candidates 128 mt + 32 w + lane, the same 32-row groups as the scoring
+// kernel's epilogue warps.  Every candidate follows the whole history, so
+// these are plans against earlier columns.
+__global__ void __launch_bounds__(kPlanThreads) cand_plans(const __grid_constant__ CandArgs a) {
+  __shared__ uint4 s_oct[32];
+  __shared__ unsigned s_thr32[kMaxBuckets];
+  __shared__ uint32_t s_ts[kPlanThreads / 32][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 32; i += kPlanThreads) s_oct[i] = a.bt.oct[i];
+  for (int i = threadIdx.x; i < kMaxBuckets; i += kPlanThreads) s_thr32[i] = a.bt.thr32[i];
+  __syncthreads();
+  const int mt = static_cast<int>(blockIdx.x), b = static_cast<int>(blockIdx.y);
+  const int c0 = __ldg(a.cand_offsets + b), cb = __ldg(a.cand_offsets + b + 1) - c0;
+  const int s = __ldg(a.offsets + b), nb = __ldg(a.offsets + b + 1) - s;
+  // inconsistent offsets are reported by the scoring kernel
+  if (c0 < 0 || cb <= 0 || c0 + cb > a.C || s < 0 || nb <= 0 || s + nb > a.T ||
+      nb > a.max_seq_len || 128 * mt >= cb)
+    return;
+  const int ci = 128 * mt + 32 * warp + lane;         // this thread's candidate of the user
+  const bool row_ok = ci < cb;
+  // candidates past the user's last take the first one's timestamp, as in the kernel
+  const int cand = c0 + (row_ok ? ci : 0);
+  const long long my_ts = a.cand_ts[checked(a.status, cand, a.C, BS_CAND_ROW)];
+  const int jt = 4 * ((nb + 127) / 128);
+  const int j0 = static_cast<int>(blockIdx.z) * kPlanBlocks;
+  const int j1 = min(jt, j0 + kPlanBlocks);
+  const PlanTab tab{s_oct, s_thr32};
+  uint32_t* ts32 = s_ts[warp];
+  for (int jc = j0; jc < j1; ++jc) {
+    if (32 * jc >= nb) break;                          // blocks past the history are skipped
+    const int j = 32 * jc + lane;
+    const long long kt = a.timestamps[checked(a.status, s + (j < nb ? j : nb - 1), a.T, BS_CAND_TS)];
+    __syncwarp();
+    ts32[lane] = static_cast<uint32_t>(kt);
+    const long long nx = __shfl_down_sync(0xffffffffu, kt, 1);
+    const bool asc = !__any_sync(0xffffffffu, lane < 31 && nx < kt);
+    long long lo = kt, hi = kt;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const long long x = __shfl_xor_sync(0xffffffffu, lo, o);
+      const long long y = __shfl_xor_sync(0xffffffffu, hi, o);
+      lo = x < lo ? x : lo;
+      hi = y > hi ? y : hi;
+    }
+    __syncwarp();
+    TimePlan p;
+    const int tb = plan_shape_dn(p, my_ts, lo, hi, asc, ts32, tab);
+    if (row_ok) a.plan[static_cast<size_t>(jc) * a.C + cand] = plan_word(p, tb);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_cand_plans(const CandArgs& a, cudaStream_t stream) {
+  if (a.B == 0 || a.max_tiles == 0 || !a.plan) return cudaSuccess;
+  if (a.plan_j < 4 * ((a.max_seq_len + 127) / 128)) return cudaErrorInvalidValue;
+  const dim3 grid(a.max_tiles, a.B, (a.plan_j + kPlanBlocks - 1) / kPlanBlocks);
+  cand_plans<<<grid, kPlanThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_time_plans(const PlanArgs& a, cudaStream_t stream) {
   if (a.B == 0 || a.max_tiles == 0) return cudaSuccess;

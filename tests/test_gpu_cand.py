@@ -29,7 +29,8 @@ def run(ci, max_cands=None, workspace=None):
     d = lambda t: None if t is None else t.to(DEV)
     mc = max_cands if max_cands is not None else max(ci.counts + [0])
     if workspace is None:
-        p = pa.make_problem(d(h.k), d(h.v), d(h.offsets), max(h.lengths + [0]))
+        p = pa.make_problem(d(h.k), d(h.v), d(h.offsets), max(h.lengths + [0]),
+                            d(h.timestamps), d(h.rab_pos), d(h.rab_time))
         n = pa.load_library().hstu_cand_workspace_size(ctypes.byref(p), ci.total_cands, mc)
         workspace = torch.zeros(max(n, 256), dtype=torch.uint8, device=DEV)
     y = pa.hstu_cand_fwd(d(h.k), d(h.v), d(h.offsets), max(h.lengths + [0]), d(ci.qc),
