@@ -153,9 +153,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_rabt = reinterpret_cast<float*>(smem + kOffRabT);
   float* s_part = reinterpret_cast<float*>(smem + kOffPart);
 
-  const int h = blockIdx.y;
-  const int b = static_cast<int>(blockIdx.x / static_cast<unsigned>(a.max_tiles));
-  const int mt = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.max_tiles));
+  // CTA (head, rank, micro-batch), the micro-batch fastest: the micro-batches
+  // of one (user, head) run together and share its history tiles in L2, and
+  // within each head the user with the longest history comes first
+  const unsigned bb = static_cast<unsigned>(a.B), tt_ = static_cast<unsigned>(a.max_tiles);
+  const int mt = static_cast<int>(blockIdx.x % tt_);
+  const int rank = static_cast<int>((blockIdx.x / tt_) % bb);
+  const int h = static_cast<int>(blockIdx.x / tt_ / bb);
+  const int b = a.order ? __ldg(a.order + rank) : rank;
   const int c0 = __ldg(a.cand_offsets + b);
   const int cb = __ldg(a.cand_offsets + b + 1) - c0;
   const int s = __ldg(a.offsets + b);
@@ -547,9 +552,29 @@ cudaError_t launch_t(const CandArgs& a, const CUtensorMap& tq, const CUtensorMap
     if (err != cudaSuccess) return err;
     if (dev >= 0 && dev < 64) configured[dev].store(true, std::memory_order_release);
   }
-  const dim3 grid(static_cast<unsigned>(a.B) * static_cast<unsigned>(a.max_tiles),
+  const dim3 grid(static_cast<unsigned>(a.B) * static_cast<unsigned>(a.max_tiles) *
                   static_cast<unsigned>(a.H));
   hstu_cand_sm100<POS, TIME><<<grid, kThreads, kSmem, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+// The users' ranks by history length (longest first, ties by index): each
+// thread counts the users that come before its own, a few thousand at most.
+__global__ void cand_order(const int32_t* offsets, int B, int* order) {
+  const int b = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+  if (b >= B) return;
+  const int n = __ldg(offsets + b + 1) - __ldg(offsets + b);
+  int rank = 0;
+  for (int o = 0; o < B; ++o) {
+    const int m = __ldg(offsets + o + 1) - __ldg(offsets + o);
+    rank += (m > n || (m == n && o < b)) ? 1 : 0;
+  }
+  order[rank] = b;
+}
+
+cudaError_t launch_cand_order(const CandArgs& a, cudaStream_t stream) {
+  if (!a.order || a.B == 0) return cudaSuccess;
+  cand_order<<<(a.B + 255) / 256, 256, 0, stream>>>(a.offsets, a.B, a.order);
   return cudaGetLastError();
 }
 

@@ -558,7 +558,9 @@ static size_t cand_tiles(int32_t max_cands) { return (static_cast<size_t>(max_ca
 
 // Candidate workspace: [status][per (user, micro-batch) counters][O / N per
 // candidate, fp32][with a time table: plan words, J * C u32 with
-// J = 4 * ceil(max_seq_len / 128)]
+// J = 4 * ceil(max_seq_len / 128)][the users' CTA order, B int32, up to
+// kCandOrderMax users]
+constexpr int kCandOrderMax = 4096;
 static size_t cand_plan_j(const hstu_problem_t* p) {
   return p->rab_time ? 4 * static_cast<size_t>((p->max_seq_len + 127) / 128) : 0;
 }
@@ -567,7 +569,8 @@ size_t hstu_cand_workspace_size(const hstu_problem_t* p, int32_t total_cands, in
   if (check_problem(p) != HSTU_OK || total_cands < 0 || max_cands < 0) return 0;
   return kStatusBytes + align_up(static_cast<size_t>(p->batch) * cand_tiles(max_cands) * 4) +
          align_up(static_cast<size_t>(total_cands) * p->num_heads * p->d_v * 4) +
-         align_up(cand_plan_j(p) * static_cast<size_t>(total_cands) * 4);
+         align_up(cand_plan_j(p) * static_cast<size_t>(total_cands) * 4) +
+         (p->batch <= kCandOrderMax ? align_up(static_cast<size_t>(p->batch) * 4) : 0);
 }
 
 hstu_status_t hstu_cand_fwd(const hstu_problem_t* p, const void* k_hist, const void* v_hist,
@@ -592,7 +595,8 @@ hstu_status_t hstu_cand_fwd(const hstu_problem_t* p, const void* k_hist, const v
     return HSTU_ERR_INVALID_ARG;
   if (p->dtype != HSTU_BF16 || p->d_qk != 128 || p->d_v != 128 || p->num_heads > 16)
     return HSTU_ERR_UNSUPPORTED;
-  if (static_cast<uint64_t>(p->batch) * cand_tiles(max_cands) > 0x7FFFFFFFull)
+  if (static_cast<uint64_t>(p->batch) * cand_tiles(max_cands) * static_cast<uint64_t>(p->num_heads) >
+      0x7FFFFFFFull)
     return HSTU_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
       workspace_bytes < hstu_cand_workspace_size(p, total_cands, max_cands))
@@ -618,10 +622,12 @@ hstu_status_t hstu_cand_fwd(const hstu_problem_t* p, const void* k_hist, const v
   a.cnt = reinterpret_cast<unsigned*>(ws + kStatusBytes);
   a.o_ws = reinterpret_cast<float*>(ws + kStatusBytes + cnt_bytes);
   a.plan_j = static_cast<int>(cand_plan_j(p));
-  if (a.plan_j > 0)
-    a.plan = reinterpret_cast<uint32_t*>(
-        ws + kStatusBytes + cnt_bytes +
-        align_up(static_cast<size_t>(total_cands) * p->num_heads * p->d_v * 4));
+  const size_t plan_off =
+      kStatusBytes + cnt_bytes + align_up(static_cast<size_t>(total_cands) * p->num_heads * p->d_v * 4);
+  if (a.plan_j > 0) a.plan = reinterpret_cast<uint32_t*>(ws + plan_off);
+  if (p->batch <= kCandOrderMax)
+    a.order = reinterpret_cast<int*>(
+        ws + plan_off + align_up(static_cast<size_t>(a.plan_j) * total_cands * 4));
   a.status = static_cast<int*>(workspace);
   a.B = p->batch;
   a.T = p->total_tokens;
@@ -645,6 +651,7 @@ hstu_status_t hstu_cand_fwd(const hstu_problem_t* p, const void* k_hist, const v
   cudaError_t err = cudaSuccess;
   if (a.plan && hist && total_cands > 0)   // the time-plan shapes, once for all heads
     err = launch_cand_plans(a, static_cast<cudaStream_t>(stream));
+  if (err == cudaSuccess) err = launch_cand_order(a, static_cast<cudaStream_t>(stream));
   if (err == cudaSuccess) err = launch_cand_sm100(a, tq, tk, tv, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }

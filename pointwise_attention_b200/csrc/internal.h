@@ -177,6 +177,9 @@ struct CandArgs {
   // against every 32-event block of its user's history, [plan_j][C] words
   uint32_t* plan;
   int plan_j;
+  // workspace or null: the users by history length, longest first (the CTA
+  // order of the scoring grid); null: in index order
+  int* order;
   int* status;
   int B, T, C, H;
   int max_tiles;                 // micro-batches per user in the grid
@@ -209,6 +212,7 @@ cudaError_t launch_out_sm100(const ProjArgs& a, const CUtensorMap& ty, const CUt
                              cudaStream_t stream);
 cudaError_t launch_time_plans(const PlanArgs& a, cudaStream_t stream);
 cudaError_t launch_cand_plans(const CandArgs& a, cudaStream_t stream);
+cudaError_t launch_cand_order(const CandArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_attn_bf16_sm100(const BwdArgs& a, const CUtensorMap* maps,
                                        cudaStream_t stream);
 
