@@ -26,41 +26,18 @@ struct PlanTab {
   __device__ __forceinline__ const unsigned* thr32() const { return thr32_; }
 };
 
-__global__ void __launch_bounds__(kPlanThreads) time_plans(const __grid_constant__ PlanArgs a) {
-  __shared__ uint4 s_oct[32];
-  __shared__ unsigned s_thr32[kMaxBuckets];
-  __shared__ uint32_t s_ts[kPlanThreads / 32][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < 32; i += kPlanThreads) s_oct[i] = a.bt.oct[i];
-  for (int i = threadIdx.x; i < kMaxBuckets; i += kPlanThreads) s_thr32[i] = a.bt.thr32[i];
-  __syncthreads();
-  const int rt = static_cast<int>(blockIdx.x), b = static_cast<int>(blockIdx.y);
-  const int s = __ldg(a.offsets + b), e = __ldg(a.offsets + b + 1);
-  const int n_b = e - s;
-  // inconsistent offsets are reported by the attention kernels
-  if (s < 0 || n_b <= 0 || e > a.T || n_b > a.max_seq_len || 128 * rt >= n_b) return;
-  const int i = 128 * rt + 32 * warp + lane;          // this thread's row of the sequence
-  const bool row_ok = i < n_b;
-  // rows past the end take the last row's timestamp, as in the kernels
-  const long long my_ts =
-      a.timestamps[checked(a.status, s + (row_ok ? i : n_b - 1), a.T, BS_BWD_TS)];
-  const int jt = 4 * ((n_b + 127) / 128);             // blocks over the sequence's tiles
-  const int j0 = static_cast<int>(blockIdx.z) * kPlanBlocks;
-  const int j1 = min(jt, j0 + kPlanBlocks);
-  const PlanTab tab{s_oct, s_thr32};
-  uint32_t* ts32 = s_ts[warp];
-  for (int jc = j0; jc < j1; ++jc) {
-    // columns at or before the row tile (dn); at or after it (up)
-    const bool dn = a.plan_dn && jc < 4 * rt + 4, up = a.plan_up && jc >= 4 * rt;
-    if (!dn && !up) continue;
-    // the block's columns, those past the end repeating the last timestamp
-    const int j = 32 * jc + lane;
-    const long long kt = a.timestamps[checked(a.status, s + (j < n_b ? j : n_b - 1), a.T, BS_BWD_TS)];
-    __syncwarp();
-    ts32[lane] = static_cast<uint32_t>(kt);
-    const long long nx = __shfl_down_sync(0xffffffffu, kt, 1);
-    const bool asc = !__any_sync(0xffffffffu, lane < 31 && nx < kt);
-    long long lo = kt, hi = kt;
+// The extremes of a warp's 32 column timestamps (lane c holds column c's):
+// the end lanes when they ascend, else a shuffle reduction.
+__device__ __forceinline__ void block_range(long long kt, int lane, bool& asc, long long& lo,
+                                            long long& hi) {
+  const long long nx = __shfl_down_sync(0xffffffffu, kt, 1);
+  asc = !__any_sync(0xffffffffu, lane < 31 && nx < kt);
+  if (asc) {
+    lo = __shfl_sync(0xffffffffu, kt, 0);
+    hi = __shfl_sync(0xffffffffu, kt, 31);
+  } else {
+    lo = kt;
+    hi = kt;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const long long x = __shfl_xor_sync(0xffffffffu, lo, o);
@@ -68,6 +45,54 @@ __global__ void __launch_bounds__(kPlanThreads) time_plans(const __grid_constant
       lo = x < lo ? x : lo;
       hi = y > hi ? y : hi;
     }
+  }
+}
+
+__global__ void __launch_bounds__(kPlanThreads) time_plans(const __grid_constant__ PlanArgs a) {
+  __shared__ uint4 s_oct[32];
+  __shared__ unsigned s_thr32[kMaxBuckets];
+  __shared__ uint32_t s_ts[kPlanThreads / 32][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rt = static_cast<int>(blockIdx.x), b = static_cast<int>(blockIdx.y);
+  const int s = __ldg(a.offsets + b), e = __ldg(a.offsets + b + 1);
+  const int n_b = e - s;
+  const int jt = 4 * ((n_b + 127) / 128);             // blocks over the sequence's tiles
+  const int j0 = static_cast<int>(blockIdx.z) * kPlanBlocks;
+  // inconsistent offsets are reported by the attention kernels; groups of
+  // blocks past the sequence, or (without the later-column plans) past the
+  // row tile, have nothing to do (a uniform exit, before any barrier)
+  if (s < 0 || n_b <= 0 || e > a.T || n_b > a.max_seq_len || 128 * rt >= n_b || j0 >= jt ||
+      (!a.plan_up && j0 >= 4 * rt + 4))
+    return;
+  for (int i = threadIdx.x; i < 32; i += kPlanThreads) s_oct[i] = a.bt.oct[i];
+  for (int i = threadIdx.x; i < kMaxBuckets; i += kPlanThreads) s_thr32[i] = a.bt.thr32[i];
+  __syncthreads();
+  const int i = 128 * rt + 32 * warp + lane;          // this thread's row of the sequence
+  const bool row_ok = i < n_b;
+  // rows past the end take the last row's timestamp, as in the kernels
+  const long long my_ts =
+      a.timestamps[checked(a.status, s + (row_ok ? i : n_b - 1), a.T, BS_BWD_TS)];
+  const int j1 = min(jt, j0 + kPlanBlocks);
+  const PlanTab tab{s_oct, s_thr32};
+  uint32_t* ts32 = s_ts[warp];
+  // the block's columns, those past the end repeating the last timestamp;
+  // the next block's load is issued before this block's plans
+  auto column_ts = [&](int jc) {
+    const int j = 32 * jc + lane;
+    return a.timestamps[checked(a.status, s + (j < n_b ? j : n_b - 1), a.T, BS_BWD_TS)];
+  };
+  long long kt_next = column_ts(j0);
+  for (int jc = j0; jc < j1; ++jc) {
+    const long long kt = kt_next;
+    if (jc + 1 < j1) kt_next = column_ts(jc + 1);
+    // columns at or before the row tile (dn); at or after it (up)
+    const bool dn = a.plan_dn && jc < 4 * rt + 4, up = a.plan_up && jc >= 4 * rt;
+    if (!dn && !up) continue;
+    __syncwarp();
+    ts32[lane] = static_cast<uint32_t>(kt);
+    bool asc;
+    long long lo, hi;
+    block_range(kt, lane, asc, lo, hi);
     __syncwarp();
     const size_t at = static_cast<size_t>(jc) * a.T + s + (row_ok ? i : 0);
     // The block holding this warp's diagonal, the one before and (for the
@@ -116,16 +141,17 @@ __global__ void __launch_bounds__(kPlanThreads) cand_plans(const __grid_constant
   __shared__ unsigned s_thr32[kMaxBuckets];
   __shared__ uint32_t s_ts[kPlanThreads / 32][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < 32; i += kPlanThreads) s_oct[i] = a.bt.oct[i];
-  for (int i = threadIdx.x; i < kMaxBuckets; i += kPlanThreads) s_thr32[i] = a.bt.thr32[i];
-  __syncthreads();
   const int mt = static_cast<int>(blockIdx.x), b = static_cast<int>(blockIdx.y);
   const int c0 = __ldg(a.cand_offsets + b), cb = __ldg(a.cand_offsets + b + 1) - c0;
   const int s = __ldg(a.offsets + b), nb = __ldg(a.offsets + b + 1) - s;
-  // inconsistent offsets are reported by the scoring kernel
+  // inconsistent offsets are reported by the scoring kernel (a uniform exit,
+  // before any barrier, as for groups of blocks past the history)
   if (c0 < 0 || cb <= 0 || c0 + cb > a.C || s < 0 || nb <= 0 || s + nb > a.T ||
-      nb > a.max_seq_len || 128 * mt >= cb)
+      nb > a.max_seq_len || 128 * mt >= cb || 32 * static_cast<int>(blockIdx.z) * kPlanBlocks >= nb)
     return;
+  for (int i = threadIdx.x; i < 32; i += kPlanThreads) s_oct[i] = a.bt.oct[i];
+  for (int i = threadIdx.x; i < kMaxBuckets; i += kPlanThreads) s_thr32[i] = a.bt.thr32[i];
+  __syncthreads();
   const int ci = 128 * mt + 32 * warp + lane;         // this thread's candidate of the user
   const bool row_ok = ci < cb;
   // candidates past the user's last take the first one's timestamp, as in the kernel
@@ -136,22 +162,20 @@ __global__ void __launch_bounds__(kPlanThreads) cand_plans(const __grid_constant
   const int j1 = min(jt, j0 + kPlanBlocks);
   const PlanTab tab{s_oct, s_thr32};
   uint32_t* ts32 = s_ts[warp];
+  auto column_ts = [&](int jc) {
+    const int j = 32 * jc + lane;
+    return a.timestamps[checked(a.status, s + (j < nb ? j : nb - 1), a.T, BS_CAND_TS)];
+  };
+  long long kt_next = column_ts(j0);
   for (int jc = j0; jc < j1; ++jc) {
     if (32 * jc >= nb) break;                          // blocks past the history are skipped
-    const int j = 32 * jc + lane;
-    const long long kt = a.timestamps[checked(a.status, s + (j < nb ? j : nb - 1), a.T, BS_CAND_TS)];
+    const long long kt = kt_next;
+    if (jc + 1 < j1 && 32 * (jc + 1) < nb) kt_next = column_ts(jc + 1);
     __syncwarp();
     ts32[lane] = static_cast<uint32_t>(kt);
-    const long long nx = __shfl_down_sync(0xffffffffu, kt, 1);
-    const bool asc = !__any_sync(0xffffffffu, lane < 31 && nx < kt);
-    long long lo = kt, hi = kt;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const long long x = __shfl_xor_sync(0xffffffffu, lo, o);
-      const long long y = __shfl_xor_sync(0xffffffffu, hi, o);
-      lo = x < lo ? x : lo;
-      hi = y > hi ? y : hi;
-    }
+    bool asc;
+    long long lo, hi;
+    block_range(kt, lane, asc, lo, hi);
     __syncwarp();
     TimePlan p;
     const int tb = plan_shape_dn(p, my_ts, lo, hi, asc, ts32, tab);
