@@ -367,8 +367,10 @@ class Workload:
                                   d_rab_time=(torch.empty_like(d["rab_time"])
                                               if d["rab_time"] is not None else None))
             self.sets.append(d)
-        # forward; the backward's LN/gate, dQ and dK/dV kernels
-        self.launches_per_step = 1 if not train else 1 + 3
+        # forward (after the time-plan pass with a bf16 time table); the
+        # backward's LN/gate kernel, its time-plan pass, dQ and dK/dV kernels
+        plans = 1 if (inp.q.dtype == torch.bfloat16 and inp.rab_time is not None) else 0
+        self.launches_per_step = (1 + plans) if not train else (1 + plans) + (3 + plans)
 
     def forward(self, i: int, stream=None):
         d, inp, pa = self.sets[i % self.R], self.inp, self.pa
@@ -505,7 +507,8 @@ def measure(spec, seed: int, steps: int, warmup: int, device, world: int, local:
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["traffic"] = None
         roof["peak_source"] = peak_kind + " burst"
-        roof["kernel"] = "hstu_attn_bwd (%s)" % BWD_KERNELS
+        roof["kernel"] = "hstu_attn_bwd (%s)" % (
+            BWD_KERNELS if inp.rab_time is None else BWD_KERNELS + ", time_plans")
         roof["algorithmic_flops"] = flops_bwd
         roof["ms_per_call"] = t_bwd * 1e3
         roof["flops_2x_fwd_tflops"] = 2.0 * flops_fwd / t_bwd / 1e12
