@@ -319,3 +319,29 @@ def test_cand_rejections(lib):
     assert call_cand(lib, p, ws=None) == 5
     assert call_cand(lib, p, ws_bytes=need - 1) == 5
     assert call_cand(lib, p, C=0) == 0                        # nothing to score
+
+
+def _al(x):
+    return (x + 255) // 256 * 256
+
+
+def test_workspace_sizes_with_a_time_table(lib):
+    """With a time table the bf16 calls keep the time-plan words and the
+    near-diagonal buckets in the workspace; the sizes follow the header's
+    formulas."""
+    so = lib.load_library()
+    T, B, L, H = 1000, 3, 300, 4
+    J = 4 * ((L + 127) // 128)
+    kw = dict(total_tokens=T, batch=B, max_seq_len=L, num_heads=H, timestamps=FAKE,
+              rab_time=FAKE, num_time_buckets=128)
+    p, _ = problem(lib, **kw)
+    q, _ = problem(lib, total_tokens=T, batch=B, max_seq_len=L, num_heads=H)
+    fwd_t, fwd_0 = lib.hstu_attn_workspace_size(p, False), lib.hstu_attn_workspace_size(q, False)
+    assert fwd_t - fwd_0 == _al(J * T * 4) + _al(T * 96)
+    bwd_t, bwd_0 = lib.hstu_attn_workspace_size(p, True), lib.hstu_attn_workspace_size(q, True)
+    assert bwd_t - bwd_0 == _al(2 * J * T * 4) + _al(T * 96)
+    assert bwd_0 == 256 + _al(T * H * 128 * 2)
+    C, M = 700, 300
+    cand_t = so.hstu_cand_workspace_size(ctypes.byref(p), C, M)
+    cand_0 = so.hstu_cand_workspace_size(ctypes.byref(q), C, M)
+    assert cand_t - cand_0 == _al(J * C * 4)
