@@ -217,25 +217,6 @@ __device__ __forceinline__ void plan_values(TimePlan& p, int tb, const Tab& tt) 
   p.t_ab = __byte_perm(p.v[0], p.v[1], 0x7610);
 }
 
-// Shape and values together.
-template <class Tab>
-__device__ __forceinline__ int plan_up(TimePlan& p, long long my_ts, long long cmin,
-                                       long long cmax, bool asc, const uint32_t* ts32,
-                                       const Tab& tt) {
-  const int tb = plan_shape_up(p, my_ts, cmin, cmax, asc, ts32, tt);
-  plan_values<true>(p, tb, tt);
-  return tb;
-}
-
-template <class Tab>
-__device__ __forceinline__ int plan_dn(TimePlan& p, long long my_ts, long long cmin,
-                                       long long cmax, bool asc, const uint32_t* ts32,
-                                       const Tab& tt) {
-  const int tb = plan_shape_dn(p, my_ts, cmin, cmax, asc, ts32, tt);
-  plan_values<false>(p, tb, tt);
-  return tb;
-}
-
 // A plan's shape in one word: k_a (7 bits), the three split columns (6 bits
 // each, 0..32) and the kind (3 bits).
 __device__ __forceinline__ uint32_t plan_word(const TimePlan& p, int tb) {
