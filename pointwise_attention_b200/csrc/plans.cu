@@ -6,7 +6,7 @@
 // the block's first bucket, up to three split columns, the kind).  A plan's
 // shape depends on the timestamps only, not on the head, so this pass computes
 // it once for every row and every block the row meets and the kernels of all
-// H heads read it.  CTA (row tile rt, sequence b, group z of kPlanBlocks
+// H heads read it.  CTA (sequence b, row tile rt; group z of kPlanBlocks
 // blocks); warp w takes rows 128 rt + 32 w + lane, the same 32-row groups as
 // the kernels' epilogue warps, so the warp-level choice of kind is theirs.
 #include "bounds.cuh"
@@ -53,11 +53,12 @@ __global__ void __launch_bounds__(kPlanThreads) time_plans(const __grid_constant
   __shared__ unsigned s_thr32[kMaxBuckets];
   __shared__ uint32_t s_ts[kPlanThreads / 32][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rt = static_cast<int>(blockIdx.x), b = static_cast<int>(blockIdx.y);
+  const unsigned tiles = static_cast<unsigned>(a.max_tiles);
+  const int rt = static_cast<int>(blockIdx.x % tiles), b = static_cast<int>(blockIdx.x / tiles);
   const int s = __ldg(a.offsets + b), e = __ldg(a.offsets + b + 1);
   const int n_b = e - s;
   const int jt = 4 * ((n_b + 127) / 128);             // blocks over the sequence's tiles
-  const int j0 = static_cast<int>(blockIdx.z) * kPlanBlocks;
+  const int j0 = static_cast<int>(blockIdx.y) * kPlanBlocks;
   // inconsistent offsets are reported by the attention kernels; groups of
   // blocks past the sequence, or (without the later-column plans) past the
   // row tile, have nothing to do (a uniform exit, before any barrier)
@@ -141,13 +142,14 @@ __global__ void __launch_bounds__(kPlanThreads) cand_plans(const __grid_constant
   __shared__ unsigned s_thr32[kMaxBuckets];
   __shared__ uint32_t s_ts[kPlanThreads / 32][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = static_cast<int>(blockIdx.x), b = static_cast<int>(blockIdx.y);
+  const unsigned tiles = static_cast<unsigned>(a.max_tiles);
+  const int mt = static_cast<int>(blockIdx.x % tiles), b = static_cast<int>(blockIdx.x / tiles);
   const int c0 = __ldg(a.cand_offsets + b), cb = __ldg(a.cand_offsets + b + 1) - c0;
   const int s = __ldg(a.offsets + b), nb = __ldg(a.offsets + b + 1) - s;
   // inconsistent offsets are reported by the scoring kernel (a uniform exit,
   // before any barrier, as for groups of blocks past the history)
   if (c0 < 0 || cb <= 0 || c0 + cb > a.C || s < 0 || nb <= 0 || s + nb > a.T ||
-      nb > a.max_seq_len || 128 * mt >= cb || 32 * static_cast<int>(blockIdx.z) * kPlanBlocks >= nb)
+      nb > a.max_seq_len || 128 * mt >= cb || 32 * static_cast<int>(blockIdx.y) * kPlanBlocks >= nb)
     return;
   for (int i = threadIdx.x; i < 32; i += kPlanThreads) s_oct[i] = a.bt.oct[i];
   for (int i = threadIdx.x; i < kMaxBuckets; i += kPlanThreads) s_thr32[i] = a.bt.thr32[i];
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kPlanThreads) cand_plans(const __grid_constant
   const int cand = c0 + (row_ok ? ci : 0);
   const long long my_ts = a.cand_ts[checked(a.status, cand, a.C, BS_CAND_ROW)];
   const int jt = 4 * ((nb + 127) / 128);
-  const int j0 = static_cast<int>(blockIdx.z) * kPlanBlocks;
+  const int j0 = static_cast<int>(blockIdx.y) * kPlanBlocks;
   const int j1 = min(jt, j0 + kPlanBlocks);
   const PlanTab tab{s_oct, s_thr32};
   uint32_t* ts32 = s_ts[warp];
@@ -188,7 +190,11 @@ __global__ void __launch_bounds__(kPlanThreads) cand_plans(const __grid_constant
 cudaError_t launch_cand_plans(const CandArgs& a, cudaStream_t stream) {
   if (a.B == 0 || a.max_tiles == 0 || !a.plan) return cudaSuccess;
   if (a.plan_j < 4 * ((a.max_seq_len + 127) / 128)) return cudaErrorInvalidValue;
-  const dim3 grid(a.max_tiles, a.B, (a.plan_j + kPlanBlocks - 1) / kPlanBlocks);
+  // (user, micro-batch) in x, the group of history blocks in y (y is limited
+  // to 65535, x is not)
+  const dim3 grid(static_cast<unsigned>(a.max_tiles) * static_cast<unsigned>(a.B),
+                  (a.plan_j + kPlanBlocks - 1) / kPlanBlocks);
+  if (grid.y > 65535u) return cudaErrorInvalidConfiguration;   // max_seq_len beyond 16.7M
   cand_plans<<<grid, kPlanThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
@@ -196,7 +202,10 @@ cudaError_t launch_cand_plans(const CandArgs& a, cudaStream_t stream) {
 cudaError_t launch_time_plans(const PlanArgs& a, cudaStream_t stream) {
   if (a.B == 0 || a.max_tiles == 0) return cudaSuccess;
   if (a.plan_j < 4 * a.max_tiles) return cudaErrorInvalidValue;
-  const dim3 grid(a.max_tiles, a.B, (a.plan_j + kPlanBlocks - 1) / kPlanBlocks);
+  // (sequence, row tile) in x, the group of column blocks in y
+  const dim3 grid(static_cast<unsigned>(a.max_tiles) * static_cast<unsigned>(a.B),
+                  (a.plan_j + kPlanBlocks - 1) / kPlanBlocks);
+  if (grid.y > 65535u) return cudaErrorInvalidConfiguration;   // max_seq_len beyond 16.7M
   time_plans<<<grid, kPlanThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
